@@ -1,0 +1,508 @@
+"""Benchmark of the gated-delta-rule tree-verify hot path on B200.
+
+One step = the whole hot path for one verification step of a DDTree budget-22
+draft tree (23 nodes: root + 22 drafts) through a 48-GDN-layer stack
+(Qwen3.5/3.6-27B geometry: 48 v-heads over 16 k-heads, d_k = d_v = 128, bf16
+q/k/v, f32 g/beta/state): gdn_tree_verify on each of the 48 layers (each with
+its own buffers), then gdn_tree_commit of the accepted root-to-leaf path on
+each layer (in place: state_out aliases the layer's recurrent state).
+
+Metric: tree-nodes/s -- draft-tree nodes carried through all 48 layers and
+committed, per second, summed over ranks (weak scaling: every rank verifies
+its own independent sequences; no data-path collective).  Also reported:
+node-layers/s and algorithmic HBM GB/s of the verify kernel against the
+measured copy bandwidth.
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                        [--state-dtype f32|f16] [--batch B] [--budget 22] [--layers 48]
+Under torchrun (N > 1) every rank runs a replica; rank 0 prints the line.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from gdn_inputs import make_problem  # noqa: E402
+
+METRIC = "GDN tree-verify nodes/s and achieved HBM GB/s (% of B200 peak) at budget 22"
+UNIT = "tree-nodes/s"
+N_K_HEADS, N_V_HEADS, D = 16, 48, 128
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ----------------------------------------------------------------------------
+# Algorithmic bytes (what the method must move, per launch; implementation
+# re-reads are not counted)
+# ----------------------------------------------------------------------------
+
+def verify_bytes(batch, n_nodes, state_dtype, qkv_bytes=2, hk=N_K_HEADS, hv=N_V_HEADS, d=D):
+    """Per verify launch: q, k, v (qkv dtype), g, beta (f32), parent (int32),
+    out (f32) and every node's persisted state, plus state_in (f32) once per tree."""
+    st = 4 if state_dtype == "f32" else 2
+    per_node = (2 * hk * d + hv * d) * qkv_bytes + 2 * hv * 4 + 4 + hv * d * 4 + hv * d * d * st
+    return batch * (n_nodes * per_node + hv * d * d * 4)
+
+
+def commit_bytes(batch, state_dtype, hv=N_V_HEADS, d=D):
+    st = 4 if state_dtype == "f32" else 2
+    return batch * hv * d * d * (st + 4)
+
+
+# ----------------------------------------------------------------------------
+# Distributed plumbing (one process per GPU; torchrun env)
+# ----------------------------------------------------------------------------
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def init_dist(ws, backend):
+    import torch.distributed as dist
+    if ws > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def aggregate(local_ms: float, local_units: float, ws: int, device=None):
+    """Max of the ranks' timed-region milliseconds and sum of their units.
+    Returns (max_ms, total_units, whole-job units/s)."""
+    if ws > 1:
+        import torch.distributed as dist
+        t = torch.tensor([local_ms], dtype=torch.float64, device=device)
+        u = torch.tensor([local_units], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.all_reduce(u, op=dist.ReduceOp.SUM)
+        local_ms, local_units = float(t.item()), float(u.item())
+    return local_ms, local_units, local_units / (local_ms / 1e3)
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ----------------------------------------------------------------------------
+# Peaks, clocks, ncu traffic record
+# ----------------------------------------------------------------------------
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_digest():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "gated_deltanet_tree_verify_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_key: str, units_per_launch: float):
+    """DRAM bytes per launch from the committed ncu record, scaled to this
+    launch by units processed; None when absent or taken on other kernel code."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)[kernel_key]
+    except Exception:
+        return None
+    if rec.get("source_digest") != kernel_source_digest():
+        return None
+    return rec["dram_bytes_per_unit"] * units_per_launch
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.05):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(device_index)
+            bus = "%08X:%02X:%02X.0" % (int(props.pci_domain_id), int(props.pci_bus_id),
+                                        int(props.pci_device_id))
+            try:
+                self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                self._h = pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(props.uuid))
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._nv = pynvml
+            self.ok = True
+        except Exception:
+            self.ok = False
+        self.period = period_s
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit and bit != 0x1:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self.ok:
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": len(self.samples)}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------
+# The workload
+# ----------------------------------------------------------------------------
+
+class Stack:
+    """Per-layer device buffers of one rank's 48-layer verify + commit step."""
+
+    def __init__(self, *, batch, budget, layers, state_dtype, seed, device):
+        import gated_deltanet_tree_verify_b200 as gdn
+        self.gdn = gdn
+        self.batch, self.n_nodes, self.layers = batch, budget + 1, layers
+        self.state_dtype = state_dtype
+        tdt = torch.float32 if state_dtype == "f32" else torch.float16
+        sd = gdn.GDN_F32 if state_dtype == "f32" else gdn.GDN_F16
+        self.host, self.dev = [], []
+        first = make_problem(batch=batch, n_nodes=self.n_nodes, n_k_heads=N_K_HEADS, n_v_heads=N_V_HEADS,
+                             d_k=D, d_v=D, tree="ddtree", seed=seed, qkv_dtype="bf16", accept="leaf")
+        self.parent = first.parent.to(device)
+        self.accept_path = first.accept_path.to(device)
+        self.accept_len = first.accept_len.to(device)
+        self.max_path_len = first.accept_path.shape[1]
+        for layer in range(layers):
+            prob = first if layer == 0 else make_problem(
+                batch=batch, n_nodes=self.n_nodes, n_k_heads=N_K_HEADS, n_v_heads=N_V_HEADS, d_k=D, d_v=D,
+                tree="given", parents=first.parent.numpy(), seed=seed * 1000 + layer, qkv_dtype="bf16",
+                accept="root")
+            self.host.append(prob)
+            self.dev.append(dict(
+                q=prob.q.to(device), k=prob.k.to(device), v=prob.v.to(device), g=prob.g.to(device),
+                beta=prob.beta.to(device), state=prob.state_in.to(device),
+                out=torch.empty(batch, self.n_nodes, N_V_HEADS, D, device=device),
+                ns=torch.empty(batch, self.n_nodes, N_V_HEADS, D, D, device=device, dtype=tdt)))
+        self.scale = first.scale
+        self.desc = gdn.make_desc(batch=batch, n_nodes=self.n_nodes, n_k_heads=N_K_HEADS,
+                                  n_v_heads=N_V_HEADS, d_k=D, d_v=D, scale=self.scale,
+                                  qkv_dtype=gdn.GDN_BF16, state_dtype=sd)
+
+    def verify_all(self, stream=None):
+        g = self.gdn
+        for d in self.dev:
+            g.gdn_tree_verify(self.desc, d["q"], d["k"], d["v"], d["g"], d["beta"], self.parent,
+                              d["state"], d["out"], d["ns"], stream=stream)
+
+    def commit_all(self, stream=None):
+        g = self.gdn
+        for d in self.dev:
+            g.gdn_tree_commit(self.desc, d["ns"], self.parent, self.accept_path, self.accept_len,
+                              self.max_path_len, d["state"], stream=stream)
+
+    def launches_per_step(self):
+        return 2 * self.layers
+
+
+def stage(msg):
+    print(f"[bench] {time.strftime('%H:%M:%S')} {msg}", file=sys.stderr, flush=True)
+
+
+def run_ours(args, ws, rank, local):
+    import gated_deltanet_tree_verify_b200 as gdn
+    gdn.load_library()  # fails loudly when the CUDA library is missing
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = init_dist(ws, "nccl")
+    stage("building the layer stack")
+    stack = Stack(batch=args.batch, budget=args.budget, layers=args.layers, state_dtype=args.state_dtype,
+                  seed=args.seed + 7919 * rank, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    # CUDA graphs of the 48 verify launches and of the 48 commit launches.
+    stage("eager warm-up")
+    stack.verify_all()
+    stack.commit_all()
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream(device)
+    s.wait_stream(stream)
+    with torch.cuda.stream(s):
+        for _ in range(2):
+            stack.verify_all()
+            stack.commit_all()
+    stream.wait_stream(s)
+    torch.cuda.synchronize()
+    stage("capturing graphs")
+    gv, gc = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gv):
+        stack.verify_all()
+    with torch.cuda.graph(gc):
+        stack.commit_all()
+    torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        gv.replay()
+        gc.replay()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    barrier(ws)
+    torch.cuda.synchronize()
+    stage("timed region")
+    sampler = ClockSampler(local)
+    with sampler:
+        for i in range(K):
+            ev[i][0].record(stream)
+            gv.replay()
+            ev[i][1].record(stream)
+            gc.replay()
+            ev[i][2].record(stream)
+        torch.cuda.synchronize()
+    barrier(ws)
+    verify_ms = sum(e[0].elapsed_time(e[1]) for e in ev)
+    commit_ms = sum(e[1].elapsed_time(e[2]) for e in ev)
+    total_ms = ev[0][0].elapsed_time(ev[-1][2])
+    nodes = args.batch * stack.n_nodes * K
+    max_ms, all_nodes, value = aggregate(total_ms, nodes, ws, device)
+
+    # Roofline of the dominant kernel (verify): algorithmic bytes per launch over
+    # its average launch duration (graph of back-to-back launches, gaps included).
+    vb = verify_bytes(args.batch, stack.n_nodes, args.state_dtype)
+    avg_verify_s = verify_ms / 1e3 / (K * args.layers)
+    achieved = vb / avg_verify_s / 1e9
+    peak, peak_kind = hbm_peak()
+    traffic = ncu_traffic(f"gdn_verify_{args.state_dtype}", args.batch * stack.n_nodes)
+    cb = commit_bytes(args.batch, args.state_dtype)
+    avg_commit_s = commit_ms / 1e3 / (K * args.layers)
+
+    # End to end through the public API with host buffers: per step the
+    # step's inputs go host->device from pinned memory, the 48 layers' outputs
+    # come back device->host; the recurrent state stays resident on the GPU.
+    stage("end-to-end leg")
+    e2e = run_e2e(stack, args, ws, device, stream)
+
+    result = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": K, "warmup": args.warmup,
+        "ms_per_step": max_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": {"workload": f"ddtree_budget{args.budget}_{args.layers}layers_b{args.batch}",
+                   "batch_per_rank": args.batch, "global_batch": args.batch * ws,
+                   "budget": args.budget, "n_nodes": stack.n_nodes, "layers": args.layers,
+                   "n_k_heads": N_K_HEADS, "n_v_heads": N_V_HEADS, "d_k": D, "d_v": D, "qkv": "bf16",
+                   "state_dtype": args.state_dtype, "parallelism": f"replicas{ws}",
+                   "l2": "inputs larger than L2: each step touches %.2f GB of distinct per-layer buffers"
+                         % ((vb + cb) * args.layers / 1e9),
+                   "timing": "CUDA graphs of 48 verify + 48 commit launches, CUDA events per step"},
+        "node_layers_per_s": value * args.layers,
+        "verify_gbps": achieved,
+        "commit_gbps": cb / avg_commit_s / 1e9,
+        "verify_us_per_launch": avg_verify_s * 1e6,
+        "commit_us_per_launch": avg_commit_s * 1e6,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "kernel": "gdn_verify_kernel", "peak_source": f"{peak_kind} copy bandwidth",
+                     "algorithmic_bytes_per_launch": vb},
+        "e2e": e2e,
+        "gpu_launches": stack.launches_per_step() * K,
+        "clocks": sampler.summary(),
+    }
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        stage("cpu baseline (oracle)")
+        result["cpu_baseline"] = cpu_baseline(args, stack)
+    if ws > 1:
+        gv.reset()
+        gc.reset()
+        dist.destroy_process_group()
+    return result if rank == 0 else None
+
+
+def run_e2e(stack, args, ws, device, stream):
+    gdn = stack.gdn
+    K = max(3, min(args.steps, args.e2e_steps))
+    pin = lambda t: t.pin_memory()  # noqa: E731
+    host = [dict(q=pin(p.q), k=pin(p.k), v=pin(p.v), g=pin(p.g), beta=pin(p.beta)) for p in stack.host]
+    host_tree = dict(parent=pin(stack.host[0].parent), ap=pin(stack.host[0].accept_path),
+                     al=pin(stack.host[0].accept_len))
+    outs = [torch.empty(d["out"].shape, dtype=torch.float32).pin_memory() for d in stack.dev]
+    h2d = sum(t.numel() * t.element_size() for h in host for t in h.values()) + \
+        sum(t.numel() * t.element_size() for t in host_tree.values())
+    d2h = sum(o.numel() * o.element_size() for o in outs)
+
+    def step():
+        stack.parent.copy_(host_tree["parent"], non_blocking=True)
+        stack.accept_path.copy_(host_tree["ap"], non_blocking=True)
+        stack.accept_len.copy_(host_tree["al"], non_blocking=True)
+        for h, d in zip(host, stack.dev):
+            for key in ("q", "k", "v", "g", "beta"):
+                d[key].copy_(h[key], non_blocking=True)
+        stack.verify_all()
+        stack.commit_all()
+        for o, d in zip(outs, stack.dev):
+            o.copy_(d["out"], non_blocking=True)
+
+    for _ in range(max(3, args.warmup // 4)):
+        step()
+    torch.cuda.synchronize()
+    barrier(ws)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    ms = e0.elapsed_time(e1)
+    max_ms, units, value = aggregate(ms, args.batch * stack.n_nodes * K, ws, device)
+    return {"value": value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "steps": K, "ms_per_step": max_ms / K,
+            "api": "gdn_tree_verify + gdn_tree_commit (eager ctypes calls), pinned host buffers"}
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle legs
+# ----------------------------------------------------------------------------
+
+def _oracle_layer_seconds(prob, nthreads, state_dtype, heads=None):
+    import oracle
+    t0 = time.perf_counter()
+    if heads is None:
+        oracle.verify_problem(prob, state_dtype=state_dtype, nthreads=nthreads)
+    else:
+        for h in heads:
+            oracle.verify_pair(prob, 0, h, state_dtype=state_dtype)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(args, stack, budget_s=12.0):
+    """The oracle as it stands, on this host's cores, over a bounded sample of
+    the same workload: as many of the 48 layers (in order) as fit in about
+    ``budget_s`` seconds, at least one.  Scaled to tree-nodes/s through 48 layers."""
+    import oracle
+    oracle._load()
+    nthreads = os.cpu_count() or 1
+    _oracle_layer_seconds(stack.host[0], nthreads, args.state_dtype)  # page in
+    done, spent = 0, 0.0
+    while done < args.layers and (done == 0 or spent < budget_s):
+        spent += _oracle_layer_seconds(stack.host[done], nthreads, args.state_dtype)
+        done += 1
+    per_layer = spent / done
+    value = args.batch * stack.n_nodes / (per_layer * args.layers)
+    return {"value": value, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+            "sample": f"{done} of {args.layers} layers of the same workload (batch {args.batch}, "
+                      f"{stack.n_nodes} nodes, 48 heads), {spent:.1f} s, scaled to 48 layers"}
+
+
+def run_reference(args, ws, rank):
+    """The oracle as the reference arm: each step is one layer's verify of the
+    same workload on a bounded slice of v-heads, sized so K + W steps end within
+    a few minutes; scaled to tree-nodes/s through 48 layers x 48 heads."""
+    if rank != 0:
+        return None
+    import oracle
+    oracle._load()
+    nthreads = os.cpu_count() or 1
+    prob = make_problem(batch=args.batch, n_nodes=args.budget + 1, n_k_heads=N_K_HEADS, n_v_heads=N_V_HEADS,
+                        d_k=D, d_v=D, tree="ddtree", seed=args.seed, qkv_dtype="bf16", accept="leaf")
+    t_head = _oracle_layer_seconds(prob, 1, args.state_dtype, heads=[0])
+    total = args.steps + args.warmup
+    budget_s = 150.0
+    heads_per_step = max(1, min(N_V_HEADS, int(budget_s / max(total * t_head, 1e-6))))
+    for i in range(args.warmup):
+        _oracle_layer_seconds(prob, 1, args.state_dtype, heads=[i % N_V_HEADS])
+    spent = 0.0
+    for i in range(args.steps):
+        heads = [(i * heads_per_step + j) % N_V_HEADS for j in range(heads_per_step)]
+        spent += _oracle_layer_seconds(prob, 1, args.state_dtype, heads=heads)
+    per_head_layer = spent / (args.steps * heads_per_step)
+    step_s = per_head_layer * N_V_HEADS * args.layers
+    value = args.batch * (args.budget + 1) / step_s
+    sample = (f"{heads_per_step} of 48 v-heads of one of {args.layers} layers per step "
+              f"(batch {args.batch}, {args.budget + 1} nodes), single thread, scaled to the full step")
+    return {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": f"ddtree_budget{args.budget}_{args.layers}layers_b{args.batch}",
+                   "batch_per_rank": args.batch, "budget": args.budget, "layers": args.layers,
+                   "state_dtype": args.state_dtype, "parallelism": "cpu"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--state-dtype", choices=["f32", "f16"], default="f32")
+    ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--budget", type=int, default=22)
+    ap.add_argument("--layers", type=int, default=48)
+    ap.add_argument("--seed", type=int, default=2)
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    ws, rank, local = dist_env()
+    if args.impl == "reference":
+        res = run_reference(args, ws, rank)
+    else:
+        res = run_ours(args, ws, rank, local)
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

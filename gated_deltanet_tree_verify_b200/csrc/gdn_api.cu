@@ -1,0 +1,237 @@
+// gdn_api.cu -- the extern "C" entry points of libgdntree: host-side argument
+// checks, then one kernel launch on the caller's stream.  See include/gdntree.h
+// for the contract of each call.
+
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+
+#include <cuda_runtime.h>
+
+#include "gdn_internal.h"
+#include "gdntree.h"
+
+namespace {
+
+thread_local char g_detail[256] = "";
+
+gdn_status fail(gdn_status s, const char* fmt, const char* what = "")
+{
+    std::snprintf(g_detail, sizeof(g_detail), fmt, what);
+    return s;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+struct Range {
+    const void* p;
+    size_t bytes;
+    const char* name;
+};
+
+bool overlap(const Range& x, const Range& y)
+{
+    if (x.p == nullptr || y.p == nullptr || x.bytes == 0 || y.bytes == 0)
+        return false;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(x.p), a1 = a0 + x.bytes;
+    const uintptr_t b0 = reinterpret_cast<uintptr_t>(y.p), b1 = b0 + y.bytes;
+    return a0 < b1 && b0 < a1;
+}
+
+size_t elem_size(int dt) { return dt == GDN_F32 ? 4 : 2; }
+
+// Shape/dtype checks shared by verify and commit.
+gdn_status check_desc(const gdn_tree_desc* d, bool need_qkv)
+{
+    if (d == nullptr)
+        return fail(GDN_ERR_INVALID_ARG, "desc is NULL%s");
+    if (d->batch < 0 || d->n_nodes < 1 || d->n_k_heads < 1 || d->n_v_heads < 1)
+        return fail(GDN_ERR_INVALID_ARG, "batch, n_nodes or head counts out of range%s");
+    if (d->n_v_heads % d->n_k_heads != 0)
+        return fail(GDN_ERR_INVALID_ARG, "n_v_heads is not a multiple of n_k_heads%s");
+    if ((d->flags & ~7u) != 0)
+        return fail(GDN_ERR_INVALID_ARG, "unknown flag bits%s");
+    const bool dk_ok = d->d_k == 32 || d->d_k == 64 || d->d_k == 128;
+    const bool dv_ok = d->d_v == 32 || d->d_v == 64 || d->d_v == 128;
+    if (!dk_ok || !dv_ok)
+        return fail(GDN_ERR_UNSUPPORTED, "d_k and d_v must each be 32, 64 or 128%s");
+    if (d->state_dtype != GDN_F32 && d->state_dtype != GDN_F16)
+        return fail(GDN_ERR_UNSUPPORTED, "state_dtype must be GDN_F32 or GDN_F16%s");
+    if (need_qkv) {
+        if (d->qkv_dtype != GDN_BF16 && d->qkv_dtype != GDN_F32)
+            return fail(GDN_ERR_UNSUPPORTED, "qkv_dtype must be GDN_BF16 or GDN_F32%s");
+        if (!std::isfinite(d->scale))
+            return fail(GDN_ERR_INVALID_ARG, "scale is not finite%s");
+    }
+    if (!(d->flags & GDN_FLAG_CHAIN) && d->n_nodes > GDN_MAX_TREE_NODES)
+        return fail(GDN_ERR_UNSUPPORTED, "tree has more than GDN_MAX_TREE_NODES nodes%s");
+    if (d->n_nodes > 0xffff)
+        return fail(GDN_ERR_UNSUPPORTED, "n_nodes above 65535%s");
+    return GDN_OK;
+}
+
+size_t node_states_bytes(const gdn_tree_desc* d)
+{
+    const size_t ns = (d->flags & GDN_FLAG_PERSIST_LAST) ? 1 : (size_t)d->n_nodes;
+    return (size_t)d->batch * ns * d->n_v_heads * d->d_v * d->d_k * elem_size(d->state_dtype);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* gdn_version(void) { return "0.1.0"; }
+
+const char* gdn_last_error_detail(void) { return g_detail; }
+
+const char* gdn_status_str(gdn_status s)
+{
+    switch (s) {
+        case GDN_OK: return "GDN_OK";
+        case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG";
+        case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED";
+        case GDN_ERR_BAD_TREE: return "GDN_ERR_BAD_TREE";
+        case GDN_ERR_BAD_PATH: return "GDN_ERR_BAD_PATH";
+        case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
+        case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT";
+    }
+    return "GDN_ERR_UNKNOWN";
+}
+
+size_t gdn_node_states_bytes(const gdn_tree_desc* desc)
+{
+    if (check_desc(desc, false) != GDN_OK)
+        return 0;
+    return node_states_bytes(desc);
+}
+
+gdn_status gdn_tree_verify(const gdn_tree_desc* desc, const void* q, const void* k, const void* v,
+                           const float* g, const float* beta, const int32_t* parent_idx,
+                           const float* state_in, float* out, void* node_states,
+                           cudaStream_t stream)
+{
+    g_detail[0] = '\0';
+    gdn_status st = check_desc(desc, true);
+    if (st != GDN_OK)
+        return st;
+    const gdn_tree_desc& d = *desc;
+    const bool chain = (d.flags & GDN_FLAG_CHAIN) != 0;
+    const bool need_parent = !chain || (d.flags & GDN_FLAG_VALIDATE);
+    if (!q || !k || !v || !g || !beta || !state_in || !out || !node_states || (need_parent && !parent_idx))
+        return fail(GDN_ERR_INVALID_ARG, "a required pointer is NULL%s");
+    const struct { const void* p; size_t a; const char* n; } al[] = {
+        {q, 16, "q"}, {k, 16, "k"}, {v, 16, "v"}, {state_in, 16, "state_in"}, {out, 16, "out"},
+        {node_states, 16, "node_states"}, {g, 4, "g"}, {beta, 4, "beta"}, {parent_idx, 4, "parent_idx"},
+        {d.status, 4, "status"}};
+    for (const auto& x : al)
+        if (x.p && !aligned(x.p, x.a))
+            return fail(GDN_ERR_INVALID_ARG, "%s is misaligned", x.n);
+    if (d.batch == 0)
+        return GDN_OK;
+    const size_t B = d.batch, N = d.n_nodes, Hk = d.n_k_heads, Hv = d.n_v_heads, dk = d.d_k, dv = d.d_v;
+    const size_t es = elem_size(d.qkv_dtype);
+    const Range ins[] = {{q, B * N * Hk * dk * es, "q"},     {k, B * N * Hk * dk * es, "k"},
+                         {v, B * N * Hv * dv * es, "v"},     {g, B * N * Hv * 4, "g"},
+                         {beta, B * N * Hv * 4, "beta"},     {parent_idx, B * N * 4, "parent_idx"},
+                         {state_in, B * Hv * dv * dk * 4, "state_in"},
+                         {d.status, 4, "status"}};
+    const Range outs[] = {{out, B * N * Hv * dv * 4, "out"},
+                          {node_states, node_states_bytes(&d), "node_states"}};
+    if (overlap(outs[0], outs[1]))
+        return fail(GDN_ERR_INVALID_ARG, "out overlaps node_states%s");
+    for (const auto& o : outs)
+        for (const auto& i : ins)
+            if (overlap(o, i))
+                return fail(GDN_ERR_INVALID_ARG, "an output overlaps input %s", i.name);
+
+    gdn::VerifyArgs a{};
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.g = g;
+    a.beta = beta;
+    a.parent = parent_idx;
+    a.state_in = state_in;
+    a.out = out;
+    a.node_states = node_states;
+    a.status = d.status;
+    a.batch = d.batch;
+    a.n_nodes = d.n_nodes;
+    a.n_k_heads = d.n_k_heads;
+    a.n_v_heads = d.n_v_heads;
+    a.d_k = d.d_k;
+    a.d_v = d.d_v;
+    a.scale = d.scale;
+    a.qkv_dtype = d.qkv_dtype;
+    a.state_dtype = d.state_dtype;
+    a.flags = d.flags;
+    const gdn::VerifyGeom geom = gdn::verify_geometry(a);
+    if (geom.tiles <= 0 || geom.smem > 227 * 1024)
+        return fail(GDN_ERR_UNSUPPORTED, "no launch geometry for this shape%s");
+    if (d.n_v_heads > 65535 || d.batch > 65535)
+        return fail(GDN_ERR_UNSUPPORTED, "batch or n_v_heads above the grid limit%s");
+    const cudaError_t e = gdn::launch_verify(a, geom, stream);
+    if (e != cudaSuccess)
+        return fail(GDN_ERR_CUDA, "verify launch failed: %s", cudaGetErrorString(e));
+    return GDN_OK;
+}
+
+gdn_status gdn_tree_commit(const gdn_tree_desc* desc, const void* node_states,
+                           const int32_t* parent_idx, const int32_t* accept_path,
+                           const int32_t* accept_len, int32_t max_path_len, float* state_out,
+                           cudaStream_t stream)
+{
+    g_detail[0] = '\0';
+    gdn_status st = check_desc(desc, false);
+    if (st != GDN_OK)
+        return st;
+    const gdn_tree_desc& d = *desc;
+    const bool chain = (d.flags & GDN_FLAG_CHAIN) != 0;
+    if (!node_states || !accept_path || !accept_len || !state_out || (!chain && !parent_idx))
+        return fail(GDN_ERR_INVALID_ARG, "a required pointer is NULL%s");
+    if (max_path_len < 1)
+        return fail(GDN_ERR_INVALID_ARG, "max_path_len < 1%s");
+    const struct { const void* p; size_t a; const char* n; } al[] = {
+        {node_states, 16, "node_states"}, {state_out, 16, "state_out"}, {parent_idx, 4, "parent_idx"},
+        {accept_path, 4, "accept_path"}, {accept_len, 4, "accept_len"}, {d.status, 4, "status"}};
+    for (const auto& x : al)
+        if (x.p && !aligned(x.p, x.a))
+            return fail(GDN_ERR_INVALID_ARG, "%s is misaligned", x.n);
+    if (d.batch == 0)
+        return GDN_OK;
+    const size_t B = d.batch;
+    const Range so{state_out, B * d.n_v_heads * d.d_v * d.d_k * 4, "state_out"};
+    const Range ins[] = {{node_states, node_states_bytes(&d), "node_states"},
+                         {parent_idx, B * d.n_nodes * 4, "parent_idx"},
+                         {accept_path, B * (size_t)max_path_len * 4, "accept_path"},
+                         {accept_len, B * 4, "accept_len"},
+                         {d.status, 4, "status"}};
+    for (const auto& i : ins)
+        if (overlap(so, i))
+            return fail(GDN_ERR_INVALID_ARG, "state_out overlaps input %s", i.name);
+    if (d.batch > 65535)
+        return fail(GDN_ERR_UNSUPPORTED, "batch above the grid limit%s");
+
+    gdn::CommitArgs a{};
+    a.node_states = node_states;
+    a.parent = parent_idx;
+    a.accept_path = accept_path;
+    a.accept_len = accept_len;
+    a.state_out = state_out;
+    a.status = d.status;
+    a.batch = d.batch;
+    a.n_nodes = d.n_nodes;
+    a.n_v_heads = d.n_v_heads;
+    a.d_k = d.d_k;
+    a.d_v = d.d_v;
+    a.max_path_len = max_path_len;
+    a.state_dtype = d.state_dtype;
+    a.flags = d.flags;
+    const cudaError_t e = gdn::launch_commit(a, stream);
+    if (e != cudaSuccess)
+        return fail(GDN_ERR_CUDA, "commit launch failed: %s", cudaGetErrorString(e));
+    return GDN_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,124 @@
+// Device helpers for libgdntree kernels (sm_100a): shared-memory barriers
+// with bounded waits, exact bf16 widening, status reporting.
+#pragma once
+
+#include <cstdint>
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+namespace gdn {
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---- mbarrier (shared::cta) -------------------------------------------------
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_init_fence()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+// Arrive with release semantics: this thread's earlier shared/global accesses
+// happen before any thread that observes the phase flip.
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar)
+{
+    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
+{
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Wait for the phase with the given parity to complete.  Bounded: gives up
+// after ~2^32 SM cycles (about two seconds at B200 clocks) and returns false,
+// so a logic error can never hang the GPU.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (clock64() - t0 > (1ll << 32))
+            return false;
+    }
+    return true;
+}
+
+// ---- status -----------------------------------------------------------------
+
+__device__ __forceinline__ void report_status(int32_t* status, int32_t code)
+{
+    if (status != nullptr)
+        atomicCAS(status, 0, code);
+}
+
+// ---- conversions ------------------------------------------------------------
+
+// Two packed bf16 (low half = first element) widened exactly to f32.
+__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t x)
+{
+    return make_float2(__uint_as_float(x << 16), __uint_as_float(x & 0xffff0000u));
+}
+
+// 16 bytes of inputs widened to f32: 8 values for bf16, 4 for f32.
+template <typename QT>
+struct Widen;
+
+template <>
+struct Widen<__nv_bfloat16> {
+    static constexpr int kPerChunk = 8;
+    __device__ __forceinline__ static void store(float* dst, uint4 x)
+    {
+        const float2 a = bf16x2_to_float2(x.x), b = bf16x2_to_float2(x.y);
+        const float2 c = bf16x2_to_float2(x.z), d = bf16x2_to_float2(x.w);
+        reinterpret_cast<float4*>(dst)[0] = make_float4(a.x, a.y, b.x, b.y);
+        reinterpret_cast<float4*>(dst)[1] = make_float4(c.x, c.y, d.x, d.y);
+    }
+    // 4 consecutive elements starting at p (8-byte aligned).
+    __device__ __forceinline__ static float4 load4(const __nv_bfloat16* p)
+    {
+        const uint2 x = __ldg(reinterpret_cast<const uint2*>(p));
+        const float2 a = bf16x2_to_float2(x.x), b = bf16x2_to_float2(x.y);
+        return make_float4(a.x, a.y, b.x, b.y);
+    }
+    __device__ __forceinline__ static float load1(const __nv_bfloat16* p)
+    {
+        const unsigned short u = __ldg(reinterpret_cast<const unsigned short*>(p));
+        return __uint_as_float(static_cast<uint32_t>(u) << 16);
+    }
+};
+
+template <>
+struct Widen<float> {
+    static constexpr int kPerChunk = 4;
+    __device__ __forceinline__ static void store(float* dst, uint4 x)
+    {
+        reinterpret_cast<uint4*>(dst)[0] = x;
+    }
+    __device__ __forceinline__ static float4 load4(const float* p)
+    {
+        return __ldg(reinterpret_cast<const float4*>(p));
+    }
+    __device__ __forceinline__ static float load1(const float* p) { return __ldg(p); }
+};
+
+}  // namespace gdn

@@ -1,0 +1,65 @@
+// Internal declarations shared by the host entry points and the kernels of
+// libgdntree.  Not part of the public ABI (see include/gdntree.h).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime_api.h>
+
+#include "gdntree.h"
+
+namespace gdn {
+
+// Device-side status written when a bounded wait on a shared-memory barrier
+// runs out (an internal error: the kernel then stops early).
+constexpr int32_t kStatusTimeout = 6;
+
+// Launch geometry of the verify kernel, chosen by the host.
+struct VerifyGeom {
+    int warps;        // compute warps per CTA (one extra producer warp is added)
+    int rows;         // d_v rows per CTA = warps * rows per warp
+    int tiles;        // d_v / rows
+    int chunk;        // tree positions per ring slot
+    int ring;         // ring slots
+    int slots;        // fp32 parent-state stack slots (tree mode)
+    size_t smem;      // dynamic shared memory bytes
+};
+
+struct VerifyArgs {
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* g;
+    const float* beta;
+    const int32_t* parent;
+    const float* state_in;
+    float* out;
+    void* node_states;
+    int32_t* status;
+    int batch, n_nodes, n_k_heads, n_v_heads, d_k, d_v;
+    float scale;
+    int qkv_dtype, state_dtype;
+    uint32_t flags;
+};
+
+struct CommitArgs {
+    const void* node_states;
+    const int32_t* parent;
+    const int32_t* accept_path;
+    const int32_t* accept_len;
+    float* state_out;
+    int32_t* status;
+    int batch, n_nodes, n_v_heads, d_k, d_v, max_path_len;
+    int state_dtype;
+    uint32_t flags;
+};
+
+// Pick the launch geometry for a verify call (host only, no CUDA calls).
+VerifyGeom verify_geometry(const VerifyArgs& a);
+
+// Launch the verify / commit kernels.  Return cudaSuccess or the launch error.
+cudaError_t launch_verify(const VerifyArgs& a, const VerifyGeom& geom, cudaStream_t stream);
+cudaError_t launch_commit(const CommitArgs& a, cudaStream_t stream);
+
+}  // namespace gdn

@@ -1,0 +1,173 @@
+"""Python binding of libgdntree (argument marshalling only).
+
+Same names as the C ABI in include/gdntree.h.  Tensors are torch CUDA tensors
+(their device pointers are passed through); every step of the computation runs
+in the library's CUDA kernels.  There is no fallback: if the shared library is
+missing or a tensor is not on a CUDA device, the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional, Union
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "lib", "libgdntree.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "gdntree.h")
+
+# gdn_dtype
+GDN_F32, GDN_F16, GDN_BF16 = 0, 1, 2
+# gdn_status
+GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_BAD_TREE, GDN_ERR_BAD_PATH, \
+    GDN_ERR_CUDA, GDN_ERR_TIMEOUT = range(7)
+# flags
+GDN_FLAG_CHAIN, GDN_FLAG_PERSIST_LAST, GDN_FLAG_VALIDATE = 1, 2, 4
+GDN_MAX_TREE_NODES = 1024
+
+_TORCH_DTYPE = {GDN_F32: torch.float32, GDN_F16: torch.float16, GDN_BF16: torch.bfloat16}
+_GDN_DTYPE = {torch.float32: GDN_F32, torch.float16: GDN_F16, torch.bfloat16: GDN_BF16}
+
+
+class GdnTreeDesc(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32),
+        ("n_nodes", ctypes.c_int32),
+        ("n_k_heads", ctypes.c_int32),
+        ("n_v_heads", ctypes.c_int32),
+        ("d_k", ctypes.c_int32),
+        ("d_v", ctypes.c_int32),
+        ("scale", ctypes.c_float),
+        ("qkv_dtype", ctypes.c_int32),
+        ("state_dtype", ctypes.c_int32),
+        ("flags", ctypes.c_uint32),
+        ("status", ctypes.c_void_p),
+    ]
+
+
+class GdnError(RuntimeError):
+    def __init__(self, status: int, detail: str = ""):
+        self.status = status
+        super().__init__(f"{gdn_status_str(status)}: {detail}" if detail else gdn_status_str(status))
+
+
+class GdnLibraryMissing(ImportError):
+    pass
+
+
+_lib = None
+
+
+def load_library() -> ctypes.CDLL:
+    """Load lib/libgdntree.so (built by gated_deltanet_tree_verify_b200.build)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise GdnLibraryMissing(
+            f"{LIB_PATH} is missing: build it with `python -m gated_deltanet_tree_verify_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32 = ctypes.c_void_p, ctypes.c_int32
+    dp = ctypes.POINTER(GdnTreeDesc)
+    lib.gdn_tree_verify.argtypes = [dp] + [vp] * 10
+    lib.gdn_tree_verify.restype = ctypes.c_int
+    lib.gdn_tree_commit.argtypes = [dp, vp, vp, vp, vp, i32, vp, vp]
+    lib.gdn_tree_commit.restype = ctypes.c_int
+    lib.gdn_status_str.argtypes = [ctypes.c_int]
+    lib.gdn_status_str.restype = ctypes.c_char_p
+    lib.gdn_last_error_detail.argtypes = []
+    lib.gdn_last_error_detail.restype = ctypes.c_char_p
+    lib.gdn_node_states_bytes.argtypes = [dp]
+    lib.gdn_node_states_bytes.restype = ctypes.c_size_t
+    lib.gdn_version.argtypes = []
+    lib.gdn_version.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def header_functions() -> list:
+    """Names of the functions include/gdntree.h declares."""
+    src = open(HEADER_PATH).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn_\w+)\s*\(", src)))
+
+
+def make_desc(*, batch: int, n_nodes: int, n_k_heads: int, n_v_heads: int, d_k: int, d_v: int,
+              scale: float, qkv_dtype: Union[int, torch.dtype] = GDN_BF16,
+              state_dtype: Union[int, torch.dtype] = GDN_F32, flags: int = 0,
+              status: Optional[torch.Tensor] = None) -> GdnTreeDesc:
+    if isinstance(qkv_dtype, torch.dtype):
+        qkv_dtype = _GDN_DTYPE[qkv_dtype]
+    if isinstance(state_dtype, torch.dtype):
+        state_dtype = _GDN_DTYPE[state_dtype]
+    d = GdnTreeDesc()
+    d.batch, d.n_nodes, d.n_k_heads, d.n_v_heads = batch, n_nodes, n_k_heads, n_v_heads
+    d.d_k, d.d_v, d.scale = d_k, d_v, float(scale)
+    d.qkv_dtype, d.state_dtype, d.flags = int(qkv_dtype), int(state_dtype), int(flags)
+    d.status = _ptr(status, "status") if status is not None else None
+    return d
+
+
+def _ptr(x, name: str):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if isinstance(x, torch.Tensor):
+        if not x.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor (got device {x.device})")
+        if not x.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        return x.data_ptr()
+    raise TypeError(f"{name}: expected a CUDA tensor, an int device pointer or None")
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(rc: int, check: bool) -> int:
+    if check and rc != GDN_OK:
+        raise GdnError(rc, load_library().gdn_last_error_detail().decode())
+    return rc
+
+
+def gdn_status_str(status: int) -> str:
+    return load_library().gdn_status_str(int(status)).decode()
+
+
+def gdn_version() -> str:
+    return load_library().gdn_version().decode()
+
+
+def gdn_node_states_bytes(desc: GdnTreeDesc) -> int:
+    return int(load_library().gdn_node_states_bytes(ctypes.byref(desc)))
+
+
+def gdn_tree_verify(desc: GdnTreeDesc, q, k, v, g, beta, parent_idx, state_in, out, node_states,
+                    stream=None, check: bool = True) -> int:
+    """Calls gdn_tree_verify (see include/gdntree.h).  Raises GdnError on a
+    non-OK host status when ``check``; device-detected errors go to desc.status."""
+    lib = load_library()
+    rc = lib.gdn_tree_verify(ctypes.byref(desc), _ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"),
+                             _ptr(g, "g"), _ptr(beta, "beta"), _ptr(parent_idx, "parent_idx"),
+                             _ptr(state_in, "state_in"), _ptr(out, "out"),
+                             _ptr(node_states, "node_states"), _stream(stream))
+    return _check(rc, check)
+
+
+def gdn_tree_commit(desc: GdnTreeDesc, node_states, parent_idx, accept_path, accept_len,
+                    max_path_len: int, state_out, stream=None, check: bool = True) -> int:
+    """Calls gdn_tree_commit (see include/gdntree.h)."""
+    lib = load_library()
+    rc = lib.gdn_tree_commit(ctypes.byref(desc), _ptr(node_states, "node_states"),
+                             _ptr(parent_idx, "parent_idx"), _ptr(accept_path, "accept_path"),
+                             _ptr(accept_len, "accept_len"), int(max_path_len),
+                             _ptr(state_out, "state_out"), _stream(stream))
+    return _check(rc, check)

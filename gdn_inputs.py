@@ -188,7 +188,8 @@ def make_problem(*, batch: int, n_nodes: int, n_k_heads: int, n_v_heads: int,
     gate: "softplus" -> g = -softplus(N(0,1)); "uniform_a" -> g = ln U(0.5, 1).
     accept: "leaf" -> root to a uniformly chosen leaf; "prefix" -> root to a
       uniformly chosen node on the chain (chains); "node" -> root to a
-      uniformly chosen node.
+      uniformly chosen node; "root" -> the root alone (no tree walk, so it
+      also works for malformed trees).
     """
     gen = torch.Generator().manual_seed(seed)
     if tree == "given":
@@ -222,6 +223,9 @@ def make_problem(*, batch: int, n_nodes: int, n_k_heads: int, n_v_heads: int,
     state_in = 0.1 * torch.randn(batch, n_v_heads, d_v, d_k, generator=gen)
     paths = []
     for b in range(batch):
+        if accept == "root":
+            paths.append([0])
+            continue
         if accept == "leaf":
             cands = tree_leaves(par[b])
         elif accept in ("prefix", "node"):

@@ -1,0 +1,179 @@
+/*
+ * gdntree.h -- C ABI of libgdntree: gated-delta-rule (Gated DeltaNet) state
+ * updates over a speculative-decoding draft tree, for NVIDIA B200 (sm_100a).
+ *
+ * The operation.  A draft tree of N nodes (node 0 is the root, i.e. the last
+ * committed token re-fed through the target; nodes 1..N-1 are the drafts, so
+ * N = budget + 1 as in the GreenGames post, "Key wins", where verify reads
+ * budget + 1 positions) is verified in one pass.  Each node n with parent p
+ * runs the gated delta rule from p's state:
+ *
+ *     a_n = exp(g_n)
+ *     S_n = a_n * S_p + beta_n * (v_n - a_n * S_p k_n) k_n^T      (d_v x d_k)
+ *     o_n = scale * S_n q_n                                          (d_v)
+ *
+ * (the Gated DeltaNet recurrence run by ggml_gated_delta_net, named in the
+ * GreenGames post, "TL;DR" and "Why the experiment exists"; applied per tree
+ * node as in the DDTree row of the dflash-caddtree-integrations README, "What's
+ * in here").  The root takes S_p = state_in.  Every node's state is persisted
+ * from inside the verify kernel (the persist-write kernel of the GreenGames
+ * post, "Key wins") in fp32 or f16 (its "f16 intermediate cache"), so that the
+ * accepted root-to-leaf path is committed by a copy, without re-running it.
+ *
+ * Conventions shared by every entry point:
+ *   - Every data pointer is a caller-owned DEVICE pointer (cudaMalloc'd, or a
+ *     framework tensor's storage).  The library allocates nothing, keeps no
+ *     state between calls and never synchronises the stream.
+ *   - Layouts are row-major with the last index contiguous.  B = batch
+ *     (independent sequences), N = n_nodes, H_k / H_v = k-heads / v-heads with
+ *     G = H_v / H_k; v-head h reads k-head h / G (contiguous groups).
+ *   - Calls are asynchronous on `stream`.  The returned status reports only
+ *     what the host can check (arguments, shapes, alignment, overlap of
+ *     outputs with inputs, launch errors).  Errors in device data (a bad tree,
+ *     a bad accept path) are reported through desc->status, see below.
+ *   - Pointers passed for q, k, v, state_in, out, node_states and state_out
+ *     must be 16-byte aligned; g, beta, parent_idx, accept_path and
+ *     accept_len 4-byte aligned.
+ */
+#ifndef GDNTREE_H
+#define GDNTREE_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Element types. */
+typedef enum {
+    GDN_F32 = 0,
+    GDN_F16 = 1,
+    GDN_BF16 = 2
+} gdn_dtype;
+
+/* Status codes (host return values and device-side desc->status words). */
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned or overlapping buffers */
+    GDN_ERR_UNSUPPORTED = 2,  /* a shape or dtype this build has no kernel for */
+    GDN_ERR_BAD_TREE = 3,     /* device-detected: parent[0] != -1 or parent[n] not in [0, n) */
+    GDN_ERR_BAD_PATH = 4,     /* device-detected: accept path/length violates the tree */
+    GDN_ERR_CUDA = 5,         /* a CUDA call failed; gdn_last_error_detail() says which */
+    GDN_ERR_TIMEOUT = 6       /* device-detected internal error: a bounded wait on an
+                                 on-chip barrier ran out and the kernel stopped early */
+} gdn_status;
+
+/* desc->flags bits. */
+enum {
+    /* The caller asserts parent[n] = n - 1 (a DFlash chain).  Same numerics as
+     * the tree path; skips the tree walk.  parent_idx may then be NULL. */
+    GDN_FLAG_CHAIN = 1,
+    /* Persist only the state of the LAST node (n = N - 1); node_states then
+     * holds one state per sequence, [B][1][H_v][d_v][d_k].  Meant for long
+     * chains (prefill-style).  Commit then accepts only paths that end at
+     * node N - 1. */
+    GDN_FLAG_PERSIST_LAST = 2,
+    /* In chain mode, check parent[n] = n - 1 on the device (needs parent_idx).
+     * The tree path always checks its tree. */
+    GDN_FLAG_VALIDATE = 4
+};
+
+/* Problem description, shared by verify and commit. */
+typedef struct gdn_tree_desc {
+    int32_t batch;       /* B >= 0 sequences (0: the call does nothing) */
+    int32_t n_nodes;     /* N >= 1 tree nodes per sequence, root included */
+    int32_t n_k_heads;   /* H_k >= 1 */
+    int32_t n_v_heads;   /* H_v >= 1, a multiple of H_k */
+    int32_t d_k;         /* key/query head dim: 32, 64 or 128 */
+    int32_t d_v;         /* value head dim: 32, 64 or 128 */
+    float scale;         /* output scale, usually 1/sqrt(d_k) */
+    int32_t qkv_dtype;   /* gdn_dtype of q, k, v: GDN_BF16 or GDN_F32 */
+    int32_t state_dtype; /* gdn_dtype of node_states: GDN_F32 or GDN_F16 */
+    uint32_t flags;      /* GDN_FLAG_* bits */
+    int32_t* status;     /* optional DEVICE int32.  A kernel that finds an error
+                            in device data stores its gdn_status here with an
+                            atomic compare-and-swap from 0 (the first error
+                            sticks; the library never clears it) and writes
+                            nothing for the affected sequence.  NULL: such
+                            sequences are skipped silently. */
+} gdn_tree_desc;
+
+/*
+ * gdn_tree_verify -- run every tree node from its parent's state, emit o_n and
+ * persist S_n.
+ *
+ *   q, k        [B][N][H_k][d_k]    qkv_dtype (bf16 or f32), read-only
+ *   v           [B][N][H_v][d_v]    qkv_dtype, read-only
+ *   g, beta     [B][N][H_v]         f32, read-only; a_n = exp(g_n), g = -inf resets
+ *   parent_idx  [B][N]              int32, parent[b][0] = -1 and
+ *                                   0 <= parent[b][n] < n; may be NULL only
+ *                                   with GDN_FLAG_CHAIN and without VALIDATE
+ *   state_in    [B][H_v][d_v][d_k]  f32, read-only; the root's parent state
+ *   out         [B][N][H_v][d_v]    f32, written: o_n
+ *   node_states [B][N][H_v][d_v][d_k] in state_dtype, written: S_n rounded to
+ *               nearest even (f16 or exact f32).  With GDN_FLAG_PERSIST_LAST:
+ *               [B][1][H_v][d_v][d_k], node N - 1 only.
+ *
+ * Children always continue from their parent's unrounded fp32 state, never
+ * from the f16 copy.  Trees: N <= GDN_MAX_TREE_NODES unless GDN_FLAG_CHAIN;
+ * any depth.  Results for a node depend only on its own root path: they do
+ * not change when other branches are added, removed or renumbered.
+ *
+ * Buffers: out and node_states must not overlap each other or any input.
+ * Errors: GDN_ERR_INVALID_ARG / GDN_ERR_UNSUPPORTED / GDN_ERR_CUDA from the
+ * host (nothing launched); GDN_ERR_BAD_TREE through desc->status.
+ */
+gdn_status gdn_tree_verify(const gdn_tree_desc* desc, const void* q, const void* k,
+                           const void* v, const float* g, const float* beta,
+                           const int32_t* parent_idx, const float* state_in, float* out,
+                           void* node_states, cudaStream_t stream);
+
+/*
+ * gdn_tree_commit -- write the accepted path's state back as the new
+ * recurrent state, without re-running the path.
+ *
+ *   node_states  as written by gdn_tree_verify with the same desc (state_dtype,
+ *                GDN_FLAG_PERSIST_LAST)
+ *   parent_idx   [B][N] int32, the tree verify ran on (may be NULL only with
+ *                GDN_FLAG_CHAIN: the path is then checked against the chain)
+ *   accept_path  [B][max_path_len] int32: node ids from the root, path[0] = 0
+ *                and parent[path[i]] = path[i - 1]; entries past the length
+ *                are ignored
+ *   accept_len   [B] int32, 1 <= len <= min(N, max_path_len)
+ *   state_out    [B][H_v][d_v][d_k] f32, written: the persisted state of node
+ *                path[len - 1], widened to f32.  It may alias state_in of the
+ *                verify call (commit reads only node_states), but must not
+ *                overlap node_states.
+ *
+ * Errors: host-side as for verify; GDN_ERR_BAD_PATH (or GDN_ERR_BAD_TREE)
+ * through desc->status, and state_out[b] is then left untouched.
+ */
+gdn_status gdn_tree_commit(const gdn_tree_desc* desc, const void* node_states,
+                           const int32_t* parent_idx, const int32_t* accept_path,
+                           const int32_t* accept_len, int32_t max_path_len, float* state_out,
+                           cudaStream_t stream);
+
+/* Largest N the tree (non-chain) path takes. */
+#define GDN_MAX_TREE_NODES 1024
+
+/* Bytes of node_states for a desc (B * N * H_v * d_v * d_k * element size, or
+ * N replaced by 1 with GDN_FLAG_PERSIST_LAST); 0 for an invalid desc. */
+size_t gdn_node_states_bytes(const gdn_tree_desc* desc);
+
+/* Static, human-readable name of a status code. */
+const char* gdn_status_str(gdn_status s);
+
+/* Detail of the last GDN_ERR_* returned on this host thread (static or
+ * thread-local storage; valid until the next call on the same thread). */
+const char* gdn_last_error_detail(void);
+
+/* Library version, e.g. "0.1.0". */
+const char* gdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDNTREE_H */

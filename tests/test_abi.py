@@ -1,0 +1,154 @@
+"""The C-ABI library loads, exports what include/gdntree.h declares, and its
+host-side checks reject bad calls before launching anything (no GPU needed:
+every call here fails validation or has batch 0, so no kernel is launched)."""
+import ctypes
+
+import pytest
+
+import gated_deltanet_tree_verify_b200 as gdn
+from gated_deltanet_tree_verify_b200.build import build
+from gated_deltanet_tree_verify_b200.gdntree import header_functions
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return gdn.load_library()
+
+
+def test_exports_every_declared_function(lib):
+    names = header_functions()
+    assert {"gdn_tree_verify", "gdn_tree_commit", "gdn_status_str"} <= set(names)
+    for name in names:
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code, name in [(0, "GDN_OK"), (1, "GDN_ERR_INVALID_ARG"), (2, "GDN_ERR_UNSUPPORTED"),
+                       (3, "GDN_ERR_BAD_TREE"), (4, "GDN_ERR_BAD_PATH"), (5, "GDN_ERR_CUDA"),
+                       (6, "GDN_ERR_TIMEOUT")]:
+        assert gdn.gdn_status_str(code) == name
+    assert gdn.gdn_status_str(99) == "GDN_ERR_UNKNOWN"
+
+
+def test_desc_struct_layout():
+    # int32 x 6, float, int32 x 2, uint32, pointer
+    assert ctypes.sizeof(gdn.GdnTreeDesc) == 48
+    assert gdn.GdnTreeDesc.status.offset == 40
+
+
+def _desc(**kw):
+    base = dict(batch=1, n_nodes=23, n_k_heads=16, n_v_heads=48, d_k=128, d_v=128, scale=0.0884,
+                qkv_dtype=gdn.GDN_BF16, state_dtype=gdn.GDN_F32, flags=0)
+    base.update(kw)
+    return gdn.make_desc(**base)
+
+
+def test_node_states_bytes(lib):
+    assert gdn.gdn_node_states_bytes(_desc()) == 23 * 48 * 128 * 128 * 4
+    assert gdn.gdn_node_states_bytes(_desc(state_dtype=gdn.GDN_F16, batch=3)) == 3 * 23 * 48 * 128 * 128 * 2
+    assert gdn.gdn_node_states_bytes(_desc(flags=gdn.GDN_FLAG_PERSIST_LAST | gdn.GDN_FLAG_CHAIN,
+                                           n_nodes=4096, batch=8)) == 8 * 48 * 128 * 128 * 4
+    assert gdn.gdn_node_states_bytes(_desc(d_k=48)) == 0
+
+
+# Fake, well-separated, aligned device addresses: validation runs on the host and
+# these calls never reach a launch.
+BASE = 1 << 40
+MB = 1 << 30
+
+
+def _ptrs(n=10):
+    return [BASE + i * MB for i in range(n)]
+
+
+def _verify(desc, ptrs=None):
+    q, k, v, g, beta, par, sin, out, ns = (ptrs or _ptrs())[:9]
+    return gdn.gdn_tree_verify(desc, q, k, v, g, beta, par, sin, out, ns, stream=0, check=False)
+
+
+def test_verify_batch_zero_is_a_noop(lib):
+    assert _verify(_desc(batch=0)) == gdn.GDN_OK
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d_k=48), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(d_v=256), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(n_v_heads=40), gdn.GDN_ERR_INVALID_ARG),
+    (dict(n_nodes=0), gdn.GDN_ERR_INVALID_ARG),
+    (dict(batch=-1), gdn.GDN_ERR_INVALID_ARG),
+    (dict(n_nodes=gdn.GDN_MAX_TREE_NODES + 1), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(qkv_dtype=gdn.GDN_F16), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(state_dtype=gdn.GDN_BF16), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(flags=8), gdn.GDN_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), gdn.GDN_ERR_INVALID_ARG),
+])
+def test_verify_rejects_bad_desc(lib, kw, code):
+    assert _verify(_desc(**kw)) == code
+
+
+def test_verify_rejects_null_desc(lib):
+    p = _ptrs()
+    rc = lib.gdn_tree_verify(None, *p[:9], None)
+    assert rc == gdn.GDN_ERR_INVALID_ARG
+
+
+def test_verify_null_and_misaligned_pointers(lib):
+    for i in range(9):
+        p = _ptrs()
+        if i == 5:  # parent_idx may be NULL only in chain mode
+            p[i] = None
+            assert _verify(_desc(), p) == gdn.GDN_ERR_INVALID_ARG
+            continue
+        p[i] = None
+        assert _verify(_desc(), p) == gdn.GDN_ERR_INVALID_ARG, i
+    for i, align in [(0, 16), (1, 16), (2, 16), (6, 16), (7, 16), (8, 16), (3, 4), (4, 4), (5, 4)]:
+        p = _ptrs()
+        p[i] += align // 2
+        assert _verify(_desc(), p) == gdn.GDN_ERR_INVALID_ARG, i
+    assert "misaligned" in lib.gdn_last_error_detail().decode()
+
+
+def test_verify_rejects_overlapping_outputs(lib):
+    p = _ptrs()
+    p[7] = p[8] + 64  # out inside node_states
+    assert _verify(_desc(), p) == gdn.GDN_ERR_INVALID_ARG
+    p = _ptrs()
+    p[8] = p[6]  # node_states on top of state_in
+    assert _verify(_desc(), p) == gdn.GDN_ERR_INVALID_ARG
+    assert "state_in" in lib.gdn_last_error_detail().decode()
+
+
+def test_chain_mode_parent_may_be_null_but_not_with_validate(lib):
+    p = _ptrs()
+    p[5] = None
+    # passes every host check, so use batch 0 to stay off the GPU
+    assert _verify(_desc(batch=0, flags=gdn.GDN_FLAG_CHAIN), p) == gdn.GDN_OK
+    assert _verify(_desc(flags=gdn.GDN_FLAG_CHAIN | gdn.GDN_FLAG_VALIDATE), p) == gdn.GDN_ERR_INVALID_ARG
+
+
+def _commit(desc, ptrs=None, max_path_len=17):
+    ns, par, ap, al, so = (ptrs or _ptrs(5))[:5]
+    return gdn.gdn_tree_commit(desc, ns, par, ap, al, max_path_len, so, stream=0, check=False)
+
+
+def test_commit_host_checks(lib):
+    assert _commit(_desc(batch=0)) == gdn.GDN_OK
+    assert _commit(_desc(), max_path_len=0) == gdn.GDN_ERR_INVALID_ARG
+    assert _commit(_desc(d_k=16)) == gdn.GDN_ERR_UNSUPPORTED
+    p = _ptrs(5)
+    p[1] = None
+    assert _commit(_desc(), p) == gdn.GDN_ERR_INVALID_ARG
+    p = _ptrs(5)
+    p[4] = p[0] + 256  # state_out inside node_states
+    assert _commit(_desc(), p) == gdn.GDN_ERR_INVALID_ARG
+    p = _ptrs(5)
+    p[4] += 8
+    assert _commit(_desc(), p) == gdn.GDN_ERR_INVALID_ARG
+
+
+def test_binding_refuses_host_tensors(lib):
+    import torch
+    t = torch.zeros(16)
+    with pytest.raises(ValueError):
+        gdn.gdn_tree_verify(_desc(), t, t, t, t, t, t, t, t, t, stream=0)
