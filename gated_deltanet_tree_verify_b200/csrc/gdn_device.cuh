@@ -48,6 +48,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
     return done != 0;
 }
 
+// As mbar_try_wait, but the hardware may suspend the thread for up to
+// `hint_ns` nanoseconds waiting for the phase, instead of returning at once,
+// so a waiting warp issues no instructions.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity,
+                                                      uint32_t hint_ns)
+{
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return done != 0;
+}
+
 // Wait for the phase with the given parity to complete.  Bounded: gives up
 // after ~2^32 SM cycles (about two seconds at B200 clocks) and returns false,
 // so a logic error can never hang the GPU.
@@ -56,7 +73,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity)
     if (mbar_try_wait(bar, parity))
         return true;
     const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_try_wait_suspend(bar, parity, 200000u)) {
         if (clock64() - t0 > (1ll << 32))
             return false;
     }
@@ -105,6 +122,18 @@ struct Widen<__nv_bfloat16> {
         const unsigned short u = __ldg(reinterpret_cast<const unsigned short*>(p));
         return __uint_as_float(static_cast<uint32_t>(u) << 16);
     }
+    // Same, from shared memory.
+    __device__ __forceinline__ static float4 lds4(const __nv_bfloat16* p)
+    {
+        const uint2 x = *reinterpret_cast<const uint2*>(p);
+        const float2 a = bf16x2_to_float2(x.x), b = bf16x2_to_float2(x.y);
+        return make_float4(a.x, a.y, b.x, b.y);
+    }
+    __device__ __forceinline__ static float lds1(const __nv_bfloat16* p)
+    {
+        const unsigned short u = *reinterpret_cast<const unsigned short*>(p);
+        return __uint_as_float(static_cast<uint32_t>(u) << 16);
+    }
 };
 
 template <>
@@ -119,6 +148,11 @@ struct Widen<float> {
         return __ldg(reinterpret_cast<const float4*>(p));
     }
     __device__ __forceinline__ static float load1(const float* p) { return __ldg(p); }
+    __device__ __forceinline__ static float4 lds4(const float* p)
+    {
+        return *reinterpret_cast<const float4*>(p);
+    }
+    __device__ __forceinline__ static float lds1(const float* p) { return *p; }
 };
 
 }  // namespace gdn

@@ -15,15 +15,20 @@ namespace gdn {
 // runs out (an internal error: the kernel then stops early).
 constexpr int32_t kStatusTimeout = 6;
 
-// Launch geometry of the verify kernel, chosen by the host.
+// Launch geometry of the verify kernels, chosen by the host.
 struct VerifyGeom {
-    int warps;        // compute warps per CTA (one extra producer warp is added)
-    int rows;         // d_v rows per CTA = warps * rows per warp
-    int tiles;        // d_v / rows
-    int chunk;        // tree positions per ring slot
-    int ring;         // ring slots
-    int slots;        // fp32 parent-state stack slots (tree mode)
-    size_t smem;      // dynamic shared memory bytes
+    bool staged;          // whole-tree staging kernel (else the producer/ring kernel)
+    bool warp_tree;       // staged tree walked from warp registers (N <= 32)
+    bool reload;          // branch parents re-read from f32 node_states (no stack)
+    int rows_per_lane;    // 1 or 2
+    int warps;            // compute warps per CTA (the ring kernel adds a producer warp)
+    int rows;             // d_v rows per CTA
+    int tiles;            // d_v / rows
+    int slots;            // f32 parent-state stack slots
+    uint32_t raw_bytes;   // one node's raw record: k row | q row | v slice
+    uint32_t rec_floats;  // the same record widened to f32
+    uint32_t off_raw, off_rec, off_ab, off_slots, off_tree;  // shared-memory layout
+    size_t smem;          // dynamic shared memory bytes
 };
 
 struct VerifyArgs {
