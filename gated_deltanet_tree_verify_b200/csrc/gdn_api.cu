@@ -177,10 +177,10 @@ gdn_status gdn_tree_verify(const gdn_tree_desc* desc, const void* q, const void*
     return GDN_OK;
 }
 
-gdn_status gdn_tree_commit(const gdn_tree_desc* desc, const void* node_states,
-                           const int32_t* parent_idx, const int32_t* accept_path,
-                           const int32_t* accept_len, int32_t max_path_len, float* state_out,
-                           cudaStream_t stream)
+gdn_status gdn_tree_commit_layers(const gdn_tree_desc* desc, int32_t n_layers,
+                                  const void* const* node_states, const int32_t* parent_idx,
+                                  const int32_t* accept_path, const int32_t* accept_len,
+                                  int32_t max_path_len, float* const* state_out, cudaStream_t stream)
 {
     g_detail[0] = '\0';
     gdn_status st = check_desc(desc, false);
@@ -188,37 +188,57 @@ gdn_status gdn_tree_commit(const gdn_tree_desc* desc, const void* node_states,
         return st;
     const gdn_tree_desc& d = *desc;
     const bool chain = (d.flags & GDN_FLAG_CHAIN) != 0;
-    if (!node_states || !accept_path || !accept_len || !state_out || (!chain && !parent_idx))
+    if (n_layers < 0)
+        return fail(GDN_ERR_INVALID_ARG, "n_layers < 0%s");
+    if (n_layers > 0 && (!node_states || !state_out))
+        return fail(GDN_ERR_INVALID_ARG, "node_states or state_out array is NULL%s");
+    if (!accept_path || !accept_len || (!chain && !parent_idx))
         return fail(GDN_ERR_INVALID_ARG, "a required pointer is NULL%s");
     if (max_path_len < 1)
         return fail(GDN_ERR_INVALID_ARG, "max_path_len < 1%s");
     const struct { const void* p; size_t a; const char* n; } al[] = {
-        {node_states, 16, "node_states"}, {state_out, 16, "state_out"}, {parent_idx, 4, "parent_idx"},
-        {accept_path, 4, "accept_path"}, {accept_len, 4, "accept_len"}, {d.status, 4, "status"}};
+        {parent_idx, 4, "parent_idx"}, {accept_path, 4, "accept_path"}, {accept_len, 4, "accept_len"},
+        {d.status, 4, "status"}};
     for (const auto& x : al)
         if (x.p && !aligned(x.p, x.a))
             return fail(GDN_ERR_INVALID_ARG, "%s is misaligned", x.n);
-    if (d.batch == 0)
+    for (int l = 0; l < n_layers; ++l) {
+        if (!node_states[l] || !state_out[l])
+            return fail(GDN_ERR_INVALID_ARG, "a per-layer pointer is NULL%s");
+        if (!aligned(node_states[l], 16) || !aligned(state_out[l], 16))
+            return fail(GDN_ERR_INVALID_ARG, "a per-layer pointer is misaligned%s");
+    }
+    if (d.batch == 0 || n_layers == 0)
         return GDN_OK;
     const size_t B = d.batch;
-    const Range so{state_out, B * d.n_v_heads * d.d_v * d.d_k * 4, "state_out"};
-    const Range ins[] = {{node_states, node_states_bytes(&d), "node_states"},
-                         {parent_idx, B * d.n_nodes * 4, "parent_idx"},
-                         {accept_path, B * (size_t)max_path_len * 4, "accept_path"},
-                         {accept_len, B * 4, "accept_len"},
-                         {d.status, 4, "status"}};
-    for (const auto& i : ins)
-        if (overlap(so, i))
-            return fail(GDN_ERR_INVALID_ARG, "state_out overlaps input %s", i.name);
+    const size_t so_bytes = B * d.n_v_heads * d.d_v * d.d_k * 4;
+    const Range shared_in[] = {{parent_idx, B * d.n_nodes * 4, "parent_idx"},
+                               {accept_path, B * (size_t)max_path_len * 4, "accept_path"},
+                               {accept_len, B * 4, "accept_len"},
+                               {d.status, 4, "status"}};
+    for (int l = 0; l < n_layers; ++l) {
+        const Range so{state_out[l], so_bytes, "state_out"};
+        for (const auto& i : shared_in)
+            if (overlap(so, i))
+                return fail(GDN_ERR_INVALID_ARG, "state_out overlaps input %s", i.name);
+        for (int m = 0; m < n_layers; ++m) {
+            const Range ns{node_states[m], node_states_bytes(&d), "node_states"};
+            if (overlap(so, ns))
+                return fail(GDN_ERR_INVALID_ARG, "state_out overlaps node_states%s");
+            if (m != l && overlap(so, Range{state_out[m], so_bytes, "state_out"}))
+                return fail(GDN_ERR_INVALID_ARG, "two layers' state_out overlap%s");
+        }
+    }
     if (d.batch > 65535)
         return fail(GDN_ERR_UNSUPPORTED, "batch above the grid limit%s");
 
     gdn::CommitArgs a{};
+    a.n_layers = n_layers;
     a.node_states = node_states;
+    a.state_out = state_out;
     a.parent = parent_idx;
     a.accept_path = accept_path;
     a.accept_len = accept_len;
-    a.state_out = state_out;
     a.status = d.status;
     a.batch = d.batch;
     a.n_nodes = d.n_nodes;
@@ -232,6 +252,22 @@ gdn_status gdn_tree_commit(const gdn_tree_desc* desc, const void* node_states,
     if (e != cudaSuccess)
         return fail(GDN_ERR_CUDA, "commit launch failed: %s", cudaGetErrorString(e));
     return GDN_OK;
+}
+
+gdn_status gdn_tree_commit(const gdn_tree_desc* desc, const void* node_states,
+                           const int32_t* parent_idx, const int32_t* accept_path,
+                           const int32_t* accept_len, int32_t max_path_len, float* state_out,
+                           cudaStream_t stream)
+{
+    if (!node_states || !state_out) {
+        g_detail[0] = '\0';
+        const gdn_status st = check_desc(desc, false);
+        if (st != GDN_OK)
+            return st;
+        return fail(GDN_ERR_INVALID_ARG, "a required pointer is NULL%s");
+    }
+    return gdn_tree_commit_layers(desc, 1, &node_states, parent_idx, accept_path, accept_len,
+                                  max_path_len, &state_out, stream);
 }
 
 }  // extern "C"

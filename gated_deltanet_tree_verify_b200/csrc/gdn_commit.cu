@@ -4,10 +4,16 @@
 // its state persisted by the verify kernel (the GreenGames post, "Key wins":
 // the persist-write kernel, so no state copy or re-run is needed at verify
 // time).  Committing is therefore a bandwidth copy of one node's state per
-// sequence into the recurrent state buffer, widened from f16 when the
-// persisted dtype is f16.  Each CTA first checks the sequence's accept path
-// against the tree (path[0] = 0, parent[path[i]] = path[i-1]) and copies
-// nothing for a bad path.
+// sequence and layer into the recurrent state buffer, widened from f16 when
+// the persisted dtype is f16.  One launch covers up to kMaxCommitLayers
+// layers (an engine commits every GDN layer of the model after the forward
+// pass).
+//
+// Each CTA copies 4096 elements of one (layer, sequence).  Its threads load
+// the path's last node id and start loading their part of that node's state
+// right away (from a clamped, always in-bounds address), while warp 0 checks
+// the whole path against the tree (path[0] = 0, parent[path[i]] = path[i-1]);
+// the stores happen only for a valid path.
 
 #include <cstdint>
 
@@ -22,13 +28,14 @@ namespace {
 
 constexpr int kCommitThreads = 256;
 constexpr int kCommitElems = 4096;  // elements per CTA (16 KB of f32 output)
+constexpr int kPerThread = kCommitElems / (4 * kCommitThreads);
 
 struct CParams {
-    const void* node_states;
+    const void* node_states[kMaxCommitLayers];
+    float* state_out[kMaxCommitLayers];
     const int32_t* parent;
     const int32_t* accept_path;
     const int32_t* accept_len;
-    float* state_out;
     int32_t* status;
     int N, P, NS;
     int persist_last;
@@ -60,53 +67,62 @@ struct Load4<__half> {
 template <typename ST>
 __global__ void __launch_bounds__(kCommitThreads) gdn_commit_kernel(const CParams p)
 {
-    __shared__ int s_ok, s_last;
-    const int b = blockIdx.y;
+    __shared__ int s_ok;
+    const int b = blockIdx.y, layer = blockIdx.z;
     const int tid = threadIdx.x;
+    const int32_t* path = p.accept_path + (size_t)b * p.P;
+    pdl_wait_then_release();
+    const int len = __ldg(p.accept_len + b);
+    const bool len_ok = len >= 1 && len <= p.N && len <= p.P;
+
+    // speculative: the state of the path's last node (clamped in bounds)
+    int last = len_ok ? __ldg(path + len - 1) : 0;
+    last = last < 0 ? 0 : (last >= p.N ? p.N - 1 : last);
+    const ST* src = static_cast<const ST*>(p.node_states[layer]) +
+                    ((size_t)b * p.NS + (p.persist_last ? 0 : last)) * p.per_seq;
+    const size_t e0 = (size_t)blockIdx.x * kCommitElems;
+    float4 x[kPerThread];
+#pragma unroll
+    for (int it = 0; it < kPerThread; ++it) {
+        const size_t e = e0 + (size_t)(it * kCommitThreads + tid) * 4;
+        if (e < p.per_seq)
+            x[it] = Load4<ST>::load(src + e);
+    }
+
     if (tid < 32) {
-        const int len = __ldg(p.accept_len + b);
-        const int32_t* path = p.accept_path + (size_t)b * p.P;
-        bool ok = len >= 1 && len <= p.N && len <= p.P;
+        bool ok = len_ok;
         if (ok) {
             for (int i = tid; i < len; i += 32) {
-                const int x = __ldg(path + i);
+                const int xi = __ldg(path + i);
                 if (i == 0) {
-                    ok &= (x == 0);
+                    ok &= (xi == 0);
                 } else {
                     const int prev = __ldg(path + i - 1);
-                    const bool in_range = x > prev && x < p.N;
-                    const int px = (in_range && p.parent) ? __ldg(p.parent + (size_t)b * p.N + x) : x - 1;
+                    const bool in_range = xi > prev && xi < p.N;
+                    const int px =
+                        (in_range && p.parent) ? __ldg(p.parent + (size_t)b * p.N + xi) : xi - 1;
                     ok &= in_range && px == prev;
                 }
             }
         }
         ok = __all_sync(0xffffffffu, ok);
-        int last = 0;
-        if (ok) {
-            last = __ldg(path + len - 1);
-            if (p.persist_last && last != p.N - 1)
-                ok = false;
-        }
-        if (tid == 0) {
+        if (ok && p.persist_last && __ldg(path + len - 1) != p.N - 1)
+            ok = false;
+        if (tid == 0)
             s_ok = ok ? 1 : 0;
-            s_last = last;
-        }
     }
     __syncthreads();
     if (!s_ok) {
-        if (blockIdx.x == 0 && tid == 0)
+        if (blockIdx.x == 0 && layer == 0 && tid == 0)
             report_status(p.status, GDN_ERR_BAD_PATH);
         return;
     }
-    const ST* src = static_cast<const ST*>(p.node_states) +
-                    ((size_t)b * p.NS + (p.persist_last ? 0 : s_last)) * p.per_seq;
-    float* dst = p.state_out + (size_t)b * p.per_seq;
-    const size_t e0 = (size_t)blockIdx.x * kCommitElems;
+    float* dst = p.state_out[layer] + (size_t)b * p.per_seq;
 #pragma unroll
-    for (int it = 0; it < kCommitElems / (4 * kCommitThreads); ++it) {
+    for (int it = 0; it < kPerThread; ++it) {
         const size_t e = e0 + (size_t)(it * kCommitThreads + tid) * 4;
         if (e < p.per_seq)
-            *reinterpret_cast<float4*>(dst + e) = Load4<ST>::load(src + e);
+            *reinterpret_cast<float4*>(dst + e) = x[it];
     }
 }
 
@@ -115,23 +131,31 @@ __global__ void __launch_bounds__(kCommitThreads) gdn_commit_kernel(const CParam
 cudaError_t launch_commit(const CommitArgs& a, cudaStream_t stream)
 {
     CParams p{};
-    p.node_states = a.node_states;
     p.parent = a.parent;
     p.accept_path = a.accept_path;
     p.accept_len = a.accept_len;
-    p.state_out = a.state_out;
     p.status = a.status;
     p.N = a.n_nodes;
     p.P = a.max_path_len;
     p.persist_last = (a.flags & GDN_FLAG_PERSIST_LAST) ? 1 : 0;
     p.NS = p.persist_last ? 1 : a.n_nodes;
     p.per_seq = (size_t)a.n_v_heads * a.d_v * a.d_k;
-    dim3 grid((unsigned)((p.per_seq + kCommitElems - 1) / kCommitElems), a.batch);
-    if (a.state_dtype == GDN_F16)
-        gdn_commit_kernel<__half><<<grid, kCommitThreads, 0, stream>>>(p);
-    else
-        gdn_commit_kernel<float><<<grid, kCommitThreads, 0, stream>>>(p);
-    return cudaGetLastError();
+    const unsigned chunks = (unsigned)((p.per_seq + kCommitElems - 1) / kCommitElems);
+    for (int l0 = 0; l0 < a.n_layers; l0 += kMaxCommitLayers) {
+        const int nl = a.n_layers - l0 < kMaxCommitLayers ? a.n_layers - l0 : kMaxCommitLayers;
+        for (int l = 0; l < nl; ++l) {
+            p.node_states[l] = a.node_states[l0 + l];
+            p.state_out[l] = a.state_out[l0 + l];
+        }
+        dim3 grid(chunks, a.batch, nl);
+        const cudaError_t e =
+            a.state_dtype == GDN_F16
+                ? launch_pdl(gdn_commit_kernel<__half>, grid, dim3(kCommitThreads), 0, stream, p)
+                : launch_pdl(gdn_commit_kernel<float>, grid, dim3(kCommitThreads), 0, stream, p);
+        if (e != cudaSuccess)
+            return e;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace gdn

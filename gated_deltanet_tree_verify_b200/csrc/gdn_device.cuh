@@ -80,6 +80,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity)
     return true;
 }
 
+// ---- programmatic dependent launch -------------------------------------------
+
+// Kernels are launched with programmatic stream serialization: the next
+// kernel in the stream may become resident before this one finishes.  Every
+// kernel first waits for the grid it depends on to complete (and its memory
+// to be visible) before touching global memory, then lets its own dependents
+// launch.  Without the launch attribute both are no-ops.
+__device__ __forceinline__ void pdl_wait_then_release()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---- status -----------------------------------------------------------------
 
 __device__ __forceinline__ void report_status(int32_t* status, int32_t code)

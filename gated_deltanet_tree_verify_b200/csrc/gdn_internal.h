@@ -5,7 +5,7 @@
 #include <cstddef>
 #include <cstdint>
 
-#include <cuda_runtime_api.h>
+#include <cuda_runtime.h>
 
 #include "gdntree.h"
 
@@ -48,17 +48,40 @@ struct VerifyArgs {
     uint32_t flags;
 };
 
+// Layers one commit launch covers (more are split over several launches).
+constexpr int kMaxCommitLayers = 64;
+
 struct CommitArgs {
-    const void* node_states;
+    int n_layers;
+    const void* const* node_states;  // host array [n_layers] of device pointers
+    float* const* state_out;         // host array [n_layers] of device pointers
     const int32_t* parent;
     const int32_t* accept_path;
     const int32_t* accept_len;
-    float* state_out;
     int32_t* status;
     int batch, n_nodes, n_v_heads, d_k, d_v, max_path_len;
     int state_dtype;
     uint32_t flags;
 };
+
+// Launches kernel(args...) with programmatic stream serialization allowed (see
+// pdl_wait_then_release in gdn_device.cuh).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
 
 // Pick the launch geometry for a verify call (host only, no CUDA calls).
 VerifyGeom verify_geometry(const VerifyArgs& a);

@@ -64,7 +64,13 @@ VerifyGeom verify_geometry(const VerifyArgs& a)
         size_t off_raw = 0, off_rec = 0, off_ab = 0, off_slots = 0;
         if (staged) {
             const size_t stage_raw = align16((size_t)a.n_nodes * raw_bytes);
-            if (es == 2) {
+            if (es == 2 && g.rows_per_lane == 1) {
+                // raw bf16 records are read by the node loop itself
+                off_raw = off_rec = off;
+                off += stage_raw;
+                off_slots = off;
+                off += align16(slot_bytes);
+            } else if (es == 2) {
                 // raw rows are dead once widened: they share space with the stack
                 off_raw = off_slots = off;
                 off += stage_raw > slot_bytes ? stage_raw : align16(slot_bytes);

@@ -57,6 +57,7 @@
 
 #include <atomic>
 #include <cstdint>
+#include <type_traits>
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -299,28 +300,29 @@ __device__ __forceinline__ void save_state(const StateT<RL>& S, float* base, con
     }
 }
 
-// k and the v slice of one node from its widened record [k | q | v slice].
-template <int DK, int RL>
-__device__ __forceinline__ void load_k(const float* rec, const LaneMap<DK, RL>& L, float2 (&k2)[8],
+// k and the v slice of one node from its shared-memory record [k | q | v
+// slice], stored either widened (RT = float) or raw (RT = bf16: widened here).
+template <int DK, int RL, typename RT>
+__device__ __forceinline__ void load_k(const RT* rec, const LaneMap<DK, RL>& L, float2 (&k2)[8],
                                        float (&vr)[RL])
 {
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
-        const float4 x = *reinterpret_cast<const float4*>(rec + L.col(m));
+        const float4 x = Widen<RT>::lds4(rec + L.col(m));
         k2[2 * m] = make_float2(x.x, x.y);
         k2[2 * m + 1] = make_float2(x.z, x.w);
     }
 #pragma unroll
     for (int r = 0; r < RL; ++r)
-        vr[r] = rec[2 * DK + L.rloc[r]];
+        vr[r] = Widen<RT>::lds1(rec + 2 * DK + L.rloc[r]);
 }
 
-template <int DK, int RL>
-__device__ __forceinline__ void load_q(const float* rec, const LaneMap<DK, RL>& L, float2 (&q2)[8])
+template <int DK, int RL, typename RT>
+__device__ __forceinline__ void load_q(const RT* rec, const LaneMap<DK, RL>& L, float2 (&q2)[8])
 {
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
-        const float4 y = *reinterpret_cast<const float4*>(rec + DK + L.col(m));
+        const float4 y = Widen<RT>::lds4(rec + DK + L.col(m));
         q2[2 * m] = make_float2(y.x, y.y);
         q2[2 * m + 1] = make_float2(y.z, y.w);
     }
@@ -704,7 +706,7 @@ __device__ __forceinline__ void walk(StateT<RL>& S, const KParams& p, const Tree
                         source_parent<DK, RL>(S, m, pp, rs, p, tree, slotbuf, sin_head, b, h, row0, L,
                                               ctx.fetcher());
                 }
-                const float* rec = ctx.rec(pos, n);
+                const auto* rec = ctx.rec(pos, n);
                 float2 k2[8], q2[8];
                 float vr[RL];
                 load_k<DK, RL>(rec, L, k2, vr);
@@ -736,43 +738,44 @@ __device__ __forceinline__ void walk(StateT<RL>& S, const KParams& p, const Tree
 // Staged kernel: every node's inputs copied into shared memory at start
 // ---------------------------------------------------------------------------
 
-template <int DK, int RL>
+// Staged records: RT = float (widened once) or the raw input type.
+template <int DK, int RL, typename RT>
 struct StagedFetch {
-    const float* recs;
+    const RT* recs;
     const float* ab;
-    uint32_t rec_floats;
+    uint32_t rec_elems;
     int N;
     LaneMap<DK, RL> L;
     __device__ __forceinline__ void operator()(int y, float2 (&k2)[8], float (&vr)[RL], float& a,
                                                float& be) const
     {
-        load_k<DK, RL>(recs + (size_t)y * rec_floats, L, k2, vr);
+        load_k<DK, RL>(recs + (size_t)y * rec_elems, L, k2, vr);
         a = ab[y];
         be = ab[N + y];
     }
 };
 
-template <int DK, int RL>
+template <int DK, int RL, typename RT>
 struct StagedCtx {
-    const float* recs;
+    const RT* recs;
     const float* ab_;
-    uint32_t rec_floats;
+    uint32_t rec_elems;
     int N;
     LaneMap<DK, RL> L;
     __device__ __forceinline__ bool begin(int) { return true; }
     __device__ __forceinline__ void end(int) {}
-    __device__ __forceinline__ const float* rec(int, int n) const
+    __device__ __forceinline__ const RT* rec(int, int n) const
     {
-        return recs + (size_t)n * rec_floats;
+        return recs + (size_t)n * rec_elems;
     }
     __device__ __forceinline__ void ab(int, int n, float& a, float& be) const
     {
         a = ab_[n];
         be = ab_[N + n];
     }
-    __device__ __forceinline__ StagedFetch<DK, RL> fetcher() const
+    __device__ __forceinline__ StagedFetch<DK, RL, RT> fetcher() const
     {
-        return StagedFetch<DK, RL>{recs, ab_, rec_floats, N, L};
+        return StagedFetch<DK, RL, RT>{recs, ab_, rec_elems, N, L};
     }
 };
 
@@ -816,6 +819,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32) gdn_verify_staged(const KParam
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
     const int nwarps = blockDim.x >> 5;
     const int32_t* prow = p.parent + (size_t)b * N;
+    pdl_wait_then_release();
 
     // 1. the parent array (index order keeps it in shared memory; chain
     //    validation only checks it)
@@ -890,8 +894,12 @@ __global__ void __launch_bounds__(kMaxWarps * 32) gdn_verify_staged(const KParam
             report_status(p.status, GDN_ERR_BAD_TREE);
         return;
     }
-    // 6. widen the raw records to f32 (bf16 inputs; f32 inputs are used as is)
-    if constexpr (sizeof(QT) == 2) {
+    // 6. widen the raw records to f32 once (bf16 inputs, two rows per lane);
+    //    with one row per lane the node loop widens its own k, q, v instead
+    //    (small grids: the loop is store-bound and the prologue is not)
+    constexpr bool kWiden = sizeof(QT) == 2 && RL == 2;
+    using RT = typename std::conditional<kWiden, float, QT>::type;
+    if constexpr (kWiden) {
         for (int n = warp; n < N; n += nwarps) {
             const unsigned char* src = raw + (size_t)n * p.raw_bytes;
             float* dst = recs + (size_t)n * p.rec_floats;
@@ -900,8 +908,10 @@ __global__ void __launch_bounds__(kMaxWarps * 32) gdn_verify_staged(const KParam
         }
         __syncthreads();
     }
+    const RT* rt = kWiden ? reinterpret_cast<const RT*>(recs) : reinterpret_cast<const RT*>(raw);
+    const uint32_t rt_elems = kWiden ? p.rec_floats : p.raw_bytes / (uint32_t)sizeof(QT);
 
-    StagedCtx<DK, RL> ctx{recs, ab, p.rec_floats, N, L};
+    StagedCtx<DK, RL, RT> ctx{rt, ab, rt_elems, N, L};
     if constexpr (TREE == kTreeChain)
         walk<DK, RL, ST, true>(S, p, NoTree{}, slotbuf, sin_head, b, h, row0, L, ctx);
     else if constexpr (TREE == kTreeIndex)
@@ -1019,6 +1029,7 @@ __global__ void __launch_bounds__((kMaxWarps + 1) * 32) gdn_verify_ring(const KP
     const QT* kg = static_cast<const QT*>(p.k);
     const QT* qg = static_cast<const QT*>(p.q);
     const QT* vg = static_cast<const QT*>(p.v);
+    pdl_wait_then_release();
 
     if (tid == 0) {
         for (int i = 0; i < kRing; ++i) {
@@ -1158,8 +1169,8 @@ cudaError_t launch_staged(const KParams& kp, const VerifyArgs& a, const VerifyGe
     cudaError_t e = grant_smem<gdn_verify_staged<DK, RL, QT, ST, TREE>>(geom.smem);
     if (e != cudaSuccess)
         return e;
-    gdn_verify_staged<DK, RL, QT, ST, TREE><<<grid, geom.warps * 32, geom.smem, stream>>>(kp);
-    return cudaGetLastError();
+    return launch_pdl(gdn_verify_staged<DK, RL, QT, ST, TREE>, grid, dim3(geom.warps * 32), geom.smem,
+                      stream, kp);
 }
 
 template <int DK, int RL, typename QT, typename ST, int TREE>
@@ -1170,8 +1181,8 @@ cudaError_t launch_ring(const KParams& kp, const VerifyArgs& a, const VerifyGeom
     cudaError_t e = grant_smem<gdn_verify_ring<DK, RL, QT, ST, TREE>>(geom.smem);
     if (e != cudaSuccess)
         return e;
-    gdn_verify_ring<DK, RL, QT, ST, TREE><<<grid, (geom.warps + 1) * 32, geom.smem, stream>>>(kp);
-    return cudaGetLastError();
+    return launch_pdl(gdn_verify_ring<DK, RL, QT, ST, TREE>, grid, dim3((geom.warps + 1) * 32),
+                      geom.smem, stream, kp);
 }
 
 template <int DK, int RL, typename QT, typename ST, bool CHAIN>

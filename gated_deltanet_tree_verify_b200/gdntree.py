@@ -75,6 +75,9 @@ def load_library() -> ctypes.CDLL:
     lib.gdn_tree_verify.restype = ctypes.c_int
     lib.gdn_tree_commit.argtypes = [dp, vp, vp, vp, vp, i32, vp, vp]
     lib.gdn_tree_commit.restype = ctypes.c_int
+    lib.gdn_tree_commit_layers.argtypes = [dp, i32, ctypes.POINTER(vp), vp, vp, vp, i32,
+                                           ctypes.POINTER(vp), vp]
+    lib.gdn_tree_commit_layers.restype = ctypes.c_int
     lib.gdn_status_str.argtypes = [ctypes.c_int]
     lib.gdn_status_str.restype = ctypes.c_char_p
     lib.gdn_last_error_detail.argtypes = []
@@ -170,4 +173,21 @@ def gdn_tree_commit(desc: GdnTreeDesc, node_states, parent_idx, accept_path, acc
                              _ptr(parent_idx, "parent_idx"), _ptr(accept_path, "accept_path"),
                              _ptr(accept_len, "accept_len"), int(max_path_len),
                              _ptr(state_out, "state_out"), _stream(stream))
+    return _check(rc, check)
+
+
+def gdn_tree_commit_layers(desc: GdnTreeDesc, node_states, parent_idx, accept_path, accept_len,
+                           max_path_len: int, state_out, stream=None, check: bool = True) -> int:
+    """Calls gdn_tree_commit_layers (see include/gdntree.h): ``node_states`` and
+    ``state_out`` are equal-length sequences of per-layer CUDA tensors (or int
+    device pointers)."""
+    lib = load_library()
+    if len(node_states) != len(state_out):
+        raise ValueError("node_states and state_out must have one entry per layer")
+    n = len(node_states)
+    ns = (ctypes.c_void_p * max(n, 1))(*[_ptr(t, "node_states") for t in node_states])
+    so = (ctypes.c_void_p * max(n, 1))(*[_ptr(t, "state_out") for t in state_out])
+    rc = lib.gdn_tree_commit_layers(ctypes.byref(desc), n, ns, _ptr(parent_idx, "parent_idx"),
+                                    _ptr(accept_path, "accept_path"), _ptr(accept_len, "accept_len"),
+                                    int(max_path_len), so, _stream(stream))
     return _check(rc, check)

@@ -155,6 +155,28 @@ gdn_status gdn_tree_commit(const gdn_tree_desc* desc, const void* node_states,
                            const int32_t* accept_len, int32_t max_path_len, float* state_out,
                            cudaStream_t stream);
 
+/*
+ * gdn_tree_commit_layers -- gdn_tree_commit for n_layers layers in one launch
+ * (an engine commits the accepted path of every GDN layer at once, after the
+ * verification forward pass).  The tree, accept paths and desc are shared by
+ * all layers; each layer has its own node_states and state_out.
+ *
+ *   n_layers     >= 0 (0: nothing to do)
+ *   node_states  HOST array [n_layers] of DEVICE pointers, each as for
+ *                gdn_tree_commit
+ *   state_out    HOST array [n_layers] of DEVICE pointers, each as for
+ *                gdn_tree_commit; no two may overlap, and none may overlap
+ *                any layer's node_states
+ *
+ * The host arrays are read during the call only.  Errors as for
+ * gdn_tree_commit (a bad path leaves every layer's state_out[b] untouched).
+ */
+gdn_status gdn_tree_commit_layers(const gdn_tree_desc* desc, int32_t n_layers,
+                                  const void* const* node_states, const int32_t* parent_idx,
+                                  const int32_t* accept_path, const int32_t* accept_len,
+                                  int32_t max_path_len, float* const* state_out,
+                                  cudaStream_t stream);
+
 /* Largest N the tree (non-chain) path takes. */
 #define GDN_MAX_TREE_NODES 1024
 

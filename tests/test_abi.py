@@ -152,3 +152,23 @@ def test_binding_refuses_host_tensors(lib):
     t = torch.zeros(16)
     with pytest.raises(ValueError):
         gdn.gdn_tree_verify(_desc(), t, t, t, t, t, t, t, t, t, stream=0)
+
+
+def _commit_layers(desc, ns, so, max_path_len=17, par=BASE + 60 * MB, ap=BASE + 61 * MB, al=BASE + 62 * MB):
+    return gdn.gdn_tree_commit_layers(desc, ns, par, ap, al, max_path_len, so, stream=0, check=False)
+
+
+def test_commit_layers_host_checks(lib):
+    ns = [BASE + i * MB for i in range(3)]
+    so = [BASE + (10 + i) * MB for i in range(3)]
+    assert _commit_layers(_desc(batch=0), ns, so) == gdn.GDN_OK
+    assert _commit_layers(_desc(), [], []) == gdn.GDN_OK          # no layers: nothing to do
+    assert lib.gdn_tree_commit_layers(ctypes.byref(_desc()), -1, None, BASE, BASE, BASE, 4, None,
+                                      None) == gdn.GDN_ERR_INVALID_ARG
+    assert _commit_layers(_desc(), ns, [so[0], 0, so[2]]) == gdn.GDN_ERR_INVALID_ARG
+    assert _commit_layers(_desc(), ns, [so[0], so[1] + 8, so[2]]) == gdn.GDN_ERR_INVALID_ARG
+    assert _commit_layers(_desc(), ns, [so[0], so[0] + 1024, so[2]]) == gdn.GDN_ERR_INVALID_ARG
+    assert "overlap" in lib.gdn_last_error_detail().decode()
+    assert _commit_layers(_desc(), ns, [so[0], ns[2] + 4096, so[2]]) == gdn.GDN_ERR_INVALID_ARG
+    with pytest.raises(ValueError):
+        gdn.gdn_tree_commit_layers(_desc(), ns, 0, 0, 0, 4, so[:2], stream=0)
