@@ -234,12 +234,20 @@ class Stack:
         self.desc = gdn.make_desc(batch=batch, n_nodes=self.n_nodes, n_k_heads=N_K_HEADS,
                                   n_v_heads=N_V_HEADS, d_k=D, d_v=D, scale=self.scale,
                                   qkv_dtype=gdn.GDN_BF16, state_dtype=sd)
+        # Layers after the first: the tree and the layer's recurrent state were
+        # written before the preceding kernel (the previous layer's verify)
+        # was launched, so they may be read while it still runs.
+        self.desc_next = gdn.make_desc(batch=batch, n_nodes=self.n_nodes, n_k_heads=N_K_HEADS,
+                                       n_v_heads=N_V_HEADS, d_k=D, d_v=D, scale=self.scale,
+                                       qkv_dtype=gdn.GDN_BF16, state_dtype=sd,
+                                       flags=gdn.GDN_FLAG_EARLY_TREE)
 
     def verify_all(self, stream=None):
         g = self.gdn
-        for d in self.dev:
-            g.gdn_tree_verify(self.desc, d["q"], d["k"], d["v"], d["g"], d["beta"], self.parent,
-                              d["state"], d["out"], d["ns"], stream=stream)
+        for layer, d in enumerate(self.dev):
+            g.gdn_tree_verify(self.desc if layer == 0 else self.desc_next, d["q"], d["k"], d["v"],
+                              d["g"], d["beta"], self.parent, d["state"], d["out"], d["ns"],
+                              stream=stream)
 
     def commit_all(self, stream=None):
         # one launch commits the accepted path on every layer

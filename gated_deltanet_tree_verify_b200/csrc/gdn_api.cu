@@ -50,7 +50,7 @@ gdn_status check_desc(const gdn_tree_desc* d, bool need_qkv)
         return fail(GDN_ERR_INVALID_ARG, "batch, n_nodes or head counts out of range%s");
     if (d->n_v_heads % d->n_k_heads != 0)
         return fail(GDN_ERR_INVALID_ARG, "n_v_heads is not a multiple of n_k_heads%s");
-    if ((d->flags & ~7u) != 0)
+    if ((d->flags & ~15u) != 0)
         return fail(GDN_ERR_INVALID_ARG, "unknown flag bits%s");
     const bool dk_ok = d->d_k == 32 || d->d_k == 64 || d->d_k == 128;
     const bool dv_ok = d->d_v == 32 || d->d_v == 64 || d->d_v == 128;

@@ -147,6 +147,7 @@ cudaError_t launch_verify(const VerifyArgs& a, const VerifyGeom& geom, cudaStrea
     kp.persist_last = (a.flags & GDN_FLAG_PERSIST_LAST) ? 1 : 0;
     kp.validate = (a.flags & GDN_FLAG_VALIDATE) ? 1 : 0;
     kp.reload = geom.reload ? 1 : 0;
+    kp.early_tree = (a.flags & GDN_FLAG_EARLY_TREE) ? 1 : 0;
     kp.raw_bytes = geom.raw_bytes;
     kp.rec_floats = geom.rec_floats;
     kp.off_raw = geom.off_raw;

@@ -105,7 +105,7 @@ struct KParams {
     int N, Hk, Hv, dv, G;
     float scale;
     int rows, warps, slots;
-    int persist_last, validate, reload;
+    int persist_last, validate, reload, early_tree;
     uint32_t raw_bytes;   // one node's raw record (k | q | v slice) in bytes
     uint32_t rec_floats;  // one node's widened record in floats
     uint32_t off_raw, off_rec, off_ab, off_slots, off_tree;
@@ -819,7 +819,11 @@ __global__ void __launch_bounds__(kMaxWarps * 32) gdn_verify_staged(const KParam
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
     const int nwarps = blockDim.x >> 5;
     const int32_t* prow = p.parent + (size_t)b * N;
-    pdl_wait_then_release();
+    // Everything that reads q, k, v, g, beta waits for the preceding kernel;
+    // with GDN_FLAG_EARLY_TREE the tree and the root's parent state are read
+    // before that (they were written before the preceding kernel started).
+    if (!p.early_tree)
+        pdl_wait_then_release();
 
     // 1. the parent array (index order keeps it in shared memory; chain
     //    validation only checks it)
@@ -836,7 +840,32 @@ __global__ void __launch_bounds__(kMaxWarps * 32) gdn_verify_staged(const KParam
                 bad |= __ldg(prow + n) != n - 1;
         }
     }
-    // 2. every node's raw k row, q row and v slice -> shared memory (async);
+    // 2. the root's parent state
+    const LaneMap<DK, RL> L(warp, lane);
+    const float* sin_head = p.state_in + ((size_t)b * p.Hv + h) * p.dv * DK + (size_t)row0 * DK;
+    StateT<RL> S;
+    load_state<DK, RL>(S, sin_head, L);
+    // 3. the walk: warp 0 builds it for trees of <= 32 nodes (the other warps
+    //    go on to the copies); all threads for larger trees
+    const TreeView tv(tsm, N);
+    if constexpr (TREE == kTreeWarp) {
+        if (warp == 0) {
+            WarpTree wt{};
+            if (build_warp_walk(prow, N, p.slots, p.reload != 0, wt)) {
+                tsm[lane] = wt.meta_l;
+                tsm[32 + lane] = wt.rstart_l;
+                tsm[64 + lane] = wt.par_l;
+                tsm[96 + lane] = static_cast<int>(wt.mask_l);
+            } else {
+                bad = true;
+            }
+        }
+    } else if constexpr (TREE == kTreeSmem) {
+        bad = !build_walk(prow, N, p.slots, p.reload != 0, tv);
+    }
+    if (p.early_tree)
+        pdl_wait_then_release();
+    // 4. every node's raw k row, q row and v slice -> shared memory (async);
     //    warp w copies nodes w, w + warps, ...
     const int per_node = p.raw_bytes / 16;  // 16-byte chunks per node
     {
@@ -858,35 +887,13 @@ __global__ void __launch_bounds__(kMaxWarps * 32) gdn_verify_staged(const KParam
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
     }
-    // 3. gates and the root's parent state
+    // 5. gates
     for (int n = tid; n < N; n += blockDim.x) {
         const size_t gi = ((size_t)b * N + n) * p.Hv + h;
         ab[n] = gdn_gate(__ldg(p.g + gi));
         ab[N + n] = __ldg(p.beta + gi);
     }
-    const LaneMap<DK, RL> L(warp, lane);
-    const float* sin_head = p.state_in + ((size_t)b * p.Hv + h) * p.dv * DK + (size_t)row0 * DK;
-    StateT<RL> S;
-    load_state<DK, RL>(S, sin_head, L);
-    // 4. the walk: warp 0 builds it for trees of <= 32 nodes (the other warps
-    //    go on to the copies); all threads for larger trees
-    const TreeView tv(tsm, N);
-    if constexpr (TREE == kTreeWarp) {
-        if (warp == 0) {
-            WarpTree wt{};
-            if (build_warp_walk(prow, N, p.slots, p.reload != 0, wt)) {
-                tsm[lane] = wt.meta_l;
-                tsm[32 + lane] = wt.rstart_l;
-                tsm[64 + lane] = wt.par_l;
-                tsm[96 + lane] = static_cast<int>(wt.mask_l);
-            } else {
-                bad = true;
-            }
-        }
-    } else if constexpr (TREE == kTreeSmem) {
-        bad = !build_walk(prow, N, p.slots, p.reload != 0, tv);
-    }
-    // 5. the copies target this CTA's shared memory: wait for them even when
+    // 6. the copies target this CTA's shared memory: wait for them even when
     //    the tree is rejected
     asm volatile("cp.async.wait_all;" ::: "memory");
     if (__syncthreads_or(bad)) {
@@ -894,7 +901,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32) gdn_verify_staged(const KParam
             report_status(p.status, GDN_ERR_BAD_TREE);
         return;
     }
-    // 6. widen the raw records to f32 once (bf16 inputs, two rows per lane);
+    // 7. widen the raw records to f32 once (bf16 inputs, two rows per lane);
     //    with one row per lane the node loop widens its own k, q, v instead
     //    (small grids: the loop is store-bound and the prologue is not)
     constexpr bool kWiden = sizeof(QT) == 2 && RL == 2;
@@ -1029,7 +1036,8 @@ __global__ void __launch_bounds__((kMaxWarps + 1) * 32) gdn_verify_ring(const KP
     const QT* kg = static_cast<const QT*>(p.k);
     const QT* qg = static_cast<const QT*>(p.q);
     const QT* vg = static_cast<const QT*>(p.v);
-    pdl_wait_then_release();
+    if (!p.early_tree)
+        pdl_wait_then_release();
 
     if (tid == 0) {
         for (int i = 0; i < kRing; ++i) {
@@ -1057,6 +1065,8 @@ __global__ void __launch_bounds__((kMaxWarps + 1) * 32) gdn_verify_ring(const KP
         __syncthreads();
         ok = build_walk(p.parent + (size_t)b * N, N, p.slots, p.reload != 0, T);
     }
+    if (p.early_tree)
+        pdl_wait_then_release();
     if (!ok) {
         if (tid == 0)
             report_status(p.status, GDN_ERR_BAD_TREE);

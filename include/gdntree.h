@@ -77,7 +77,17 @@ enum {
     GDN_FLAG_PERSIST_LAST = 2,
     /* In chain mode, check parent[n] = n - 1 on the device (needs parent_idx).
      * The tree path always checks its tree. */
-    GDN_FLAG_VALIDATE = 4
+    GDN_FLAG_VALIDATE = 4,
+    /* Verify only.  The caller asserts that parent_idx and state_in were
+     * written before the kernel that precedes this call in the stream was
+     * launched (e.g. the draft tree is built once per step, the recurrent
+     * state by the previous step's commit, and this is any layer but the
+     * first of a layer stack).  The kernels are launched with programmatic
+     * dependent launch; with this flag they read parent_idx and state_in and
+     * build the tree walk while the preceding kernel may still run, and wait
+     * for it only before reading q, k, v, g, beta.  Without the flag every
+     * global read waits for the preceding kernel to complete. */
+    GDN_FLAG_EARLY_TREE = 8
 };
 
 /* Problem description, shared by verify and commit. */
