@@ -488,6 +488,112 @@ def run_reference(args, ws, rank):
     }
 
 
+# ----------------------------------------------------------------------------
+# Sweep (not the default line): single-layer verify timings over the pages'
+# workload shapes, one JSON line per point
+# ----------------------------------------------------------------------------
+
+FP32_LANES_PER_SM = 128  # FP32 CUDA-core lanes per SM (B200); 148 SMs
+
+
+def _verify_point(*, batch, n_nodes, tree, state_dtype, flags=0, gate="softplus", reps=20,
+                  min_bytes=512 << 20, seed=11):
+    """Mean time of one verify launch, over graph replays of R launches on R
+    distinct buffer sets (R sized so the sets together exceed min_bytes)."""
+    import gated_deltanet_tree_verify_b200 as gdn
+    persist_last = bool(flags & gdn.GDN_FLAG_PERSIST_LAST)
+    tdt = torch.float32 if state_dtype == "f32" else torch.float16
+    es = 4 if state_dtype == "f32" else 2
+    ns_bytes = batch * (1 if persist_last else n_nodes) * N_V_HEADS * D * D * es
+    io_bytes = batch * n_nodes * (45444 - 4) + batch * N_V_HEADS * D * D * 4
+    R = max(2, min(16, -(-min_bytes // max(1, ns_bytes + io_bytes))))
+    sets = []
+    for r in range(R):
+        prob = make_problem(batch=batch, n_nodes=n_nodes, n_k_heads=N_K_HEADS, n_v_heads=N_V_HEADS,
+                            d_k=D, d_v=D, tree=tree, seed=seed + 1000 * r, qkv_dtype="bf16", gate=gate,
+                            accept="root")
+        dev = {k: getattr(prob, k).cuda() for k in ("q", "k", "v", "g", "beta", "parent", "state_in")}
+        dev["out"] = torch.empty(batch, n_nodes, N_V_HEADS, D, device="cuda")
+        dev["ns"] = torch.empty(batch, 1 if persist_last else n_nodes, N_V_HEADS, D, D, device="cuda",
+                                dtype=tdt)
+        sets.append((prob, dev))
+    desc = gdn.make_desc(batch=batch, n_nodes=n_nodes, n_k_heads=N_K_HEADS, n_v_heads=N_V_HEADS, d_k=D,
+                         d_v=D, scale=sets[0][0].scale, qkv_dtype=gdn.GDN_BF16,
+                         state_dtype=gdn.GDN_F32 if state_dtype == "f32" else gdn.GDN_F16, flags=flags)
+
+    def run_all():
+        for _, d in sets:
+            gdn.gdn_tree_verify(desc, d["q"], d["k"], d["v"], d["g"], d["beta"], d["parent"], d["state_in"],
+                                d["out"], d["ns"])
+
+    run_all()
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        run_all()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        run_all()
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    per_launch_s = e0.elapsed_time(e1) / 1e3 / (reps * R)
+    del graph
+    return per_launch_s, R
+
+
+def run_sweep(args):
+    import gated_deltanet_tree_verify_b200 as gdn
+    gdn.load_library()
+    torch.cuda.set_device(0)
+    peak, peak_kind = hbm_peak()
+    points = []
+    for budget in (8, 15, 22, 32, 64, 128):
+        for batch in (1, 8, 32):
+            for sd in ("f32", "f16"):
+                points.append(dict(kind="tree", budget=budget, batch=batch, state_dtype=sd))
+    for sd in ("f32", "f16"):
+        points.append(dict(kind="chain16", budget=15, batch=1, state_dtype=sd))
+    points.append(dict(kind="chain4096", budget=4095, batch=8, state_dtype="f32"))
+    for pt in points:
+        n = pt["budget"] + 1
+        if pt["kind"] == "chain4096":
+            flags = gdn.GDN_FLAG_CHAIN | gdn.GDN_FLAG_PERSIST_LAST
+            t, R = _verify_point(batch=pt["batch"], n_nodes=n, tree="chain", state_dtype="f32", flags=flags,
+                                 gate="uniform_a", reps=3, min_bytes=0)
+            tokens = pt["batch"] * n
+            io = tokens * (45444 - 4) + 2 * pt["batch"] * N_V_HEADS * D * D * 4
+            flops = tokens * N_V_HEADS * D * D * 7.0  # dot S k, a S, u k^T, S q: 7 flops per element
+            clock = args.sm_mhz * 1e6
+            alu_peak = 148 * FP32_LANES_PER_SM * 2 * clock / 1e12
+            line = {"sweep": "chain4096_persist_last", "batch": pt["batch"], "tokens": n,
+                    "state_dtype": "f32", "verify_ms": t * 1e3, "tokens_per_s": tokens / t,
+                    "roofline": {"bound": "alu", "achieved": flops / t / 1e12, "unit": "TFLOP/s",
+                                 "peak": alu_peak, "frac": flops / t / 1e12 / alu_peak,
+                                 "peak_source": f"148 SMs x 128 FP32 lanes x 2 x {args.sm_mhz:.0f} MHz"},
+                    "hbm_gbps": io / t / 1e9}
+        else:
+            tree = "ddtree" if pt["kind"] == "tree" else "chain"
+            flags = 0 if pt["kind"] == "tree" else gdn.GDN_FLAG_CHAIN
+            t, R = _verify_point(batch=pt["batch"], n_nodes=n, tree=tree, state_dtype=pt["state_dtype"],
+                                 flags=flags)
+            vb = verify_bytes(pt["batch"], n, pt["state_dtype"])
+            line = {"sweep": pt["kind"], "budget": pt["budget"], "batch": pt["batch"],
+                    "state_dtype": pt["state_dtype"], "verify_us": t * 1e6,
+                    "node_layers_per_s": pt["batch"] * n / t, "gbps": vb / t / 1e9,
+                    "frac_of_hbm": vb / t / 1e9 / peak, "buffer_sets": R}
+        print(json.dumps(line), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -501,7 +607,15 @@ def main(argv=None):
     ap.add_argument("--seed", type=int, default=2)
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="single-layer verify timings over budgets, batches, dtypes and the long chain "
+                         "(one JSON line per point; not the benchmark line)")
+    ap.add_argument("--sm-mhz", type=float, default=1965.0,
+                    help="SM clock for the sweep's FP32 ALU roofline (default: the B200 maximum)")
     args = ap.parse_args(argv)
+    if args.sweep:
+        run_sweep(args)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     ws, rank, local = dist_env()

@@ -83,10 +83,10 @@ VerifyGeom verify_geometry(const VerifyArgs& a)
                 off += align16(slot_bytes);
             }
             off_ab = off;
-            off += align16((size_t)2 * a.n_nodes * 4);
+            off += align16((size_t)3 * a.n_nodes * 4);  // a | beta | k.q per node
         } else {
             off_rec = off;
-            off += (size_t)kRing * align16((kChunk * rec_floats + 2 * kChunk) * 4);
+            off += (size_t)kRing * align16((kChunk * rec_floats + 3 * kChunk) * 4);
             off_slots = off;
             off += align16(slot_bytes);
         }

@@ -73,7 +73,6 @@ constexpr int kColsPerLane = 16;  // 4 chunks of 4 consecutive columns
 constexpr int kMaxWarps = 4;      // compute warps per CTA
 constexpr int kChunk = 8;         // walk positions per ring slot
 constexpr int kRing = 3;          // ring slots
-constexpr int kOutBatch = 4;      // nodes whose outputs are reduced together
 constexpr int kMaxDevices = 64;
 constexpr int kStagedMaxSmem = 100 * 1024;
 
@@ -139,9 +138,13 @@ struct StateT {
 
 // One node's state update on a lane's RL rows x 16 columns.  Shared by the
 // walk and the recompute path; explicit intrinsics keep both bit-identical.
-template <int LR, int RL>
-__device__ __forceinline__ void gdn_step(StateT<RL>& S, const float2 (&k2)[8], const float (&vr)[RL],
-                                         float a, float beta)
+// With WITH_Q it also reduces this node's output read of the pre-update state,
+// pq = S_p q, in the same butterfly as S_p k, and returns u: the output is
+// then o = scale * (a * pq + u * (k . q)) = scale * S_n q (S_n = a S_p + u k^T).
+template <int LR, int RL, bool WITH_Q>
+__device__ __forceinline__ void gdn_step(StateT<RL>& S, const float2 (&k2)[8], const float2 (&q2)[8],
+                                         const float (&vr)[RL], float a, float beta, float (&pq)[RL],
+                                         float (&uo)[RL])
 {
     float w[RL];
 #pragma unroll
@@ -153,17 +156,30 @@ __device__ __forceinline__ void gdn_step(StateT<RL>& S, const float2 (&k2)[8], c
             acc1 = __ffma2_rn(S.s[r][t + 1], k2[t + 1], acc1);
         }
         w[r] = __fadd_rn(__fadd_rn(acc0.x, acc0.y), __fadd_rn(acc1.x, acc1.y));
+        if constexpr (WITH_Q) {
+            float2 b0 = make_float2(0.f, 0.f), b1 = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int t = 0; t < 8; t += 2) {
+                b0 = __ffma2_rn(S.s[r][t], q2[t], b0);
+                b1 = __ffma2_rn(S.s[r][t + 1], q2[t + 1], b1);
+            }
+            pq[r] = __fadd_rn(__fadd_rn(b0.x, b0.y), __fadd_rn(b1.x, b1.y));
+        }
     }
 #pragma unroll
     for (int off = 1; off < LR; off <<= 1) {
 #pragma unroll
-        for (int r = 0; r < RL; ++r)
+        for (int r = 0; r < RL; ++r) {
             w[r] = __fadd_rn(w[r], __shfl_xor_sync(0xffffffffu, w[r], off));
+            if constexpr (WITH_Q)
+                pq[r] = __fadd_rn(pq[r], __shfl_xor_sync(0xffffffffu, pq[r], off));
+        }
     }
     const float2 a2 = make_float2(a, a);
 #pragma unroll
     for (int r = 0; r < RL; ++r) {
         const float u = __fmul_rn(beta, __fsub_rn(vr[r], __fmul_rn(a, w[r])));
+        uo[r] = u;
         const float2 u2 = make_float2(u, u);
 #pragma unroll
         for (int t = 0; t < 8; ++t)
@@ -171,80 +187,27 @@ __device__ __forceinline__ void gdn_step(StateT<RL>& S, const float2 (&k2)[8], c
     }
 }
 
-// This lane's partial of (S q) for each of its rows.
-template <int RL>
-__device__ __forceinline__ void partial_out(const StateT<RL>& S, const float2 (&q2)[8], float* o)
+// State update only (recompute path): the same instructions on S.
+template <int LR, int RL>
+__device__ __forceinline__ void gdn_update(StateT<RL>& S, const float2 (&k2)[8], const float (&vr)[RL],
+                                           float a, float beta)
 {
-#pragma unroll
-    for (int r = 0; r < RL; ++r) {
-        float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int t = 0; t < 8; t += 2) {
-            acc0 = __ffma2_rn(S.s[r][t], q2[t], acc0);
-            acc1 = __ffma2_rn(S.s[r][t + 1], q2[t + 1], acc1);
-        }
-        o[r] = __fadd_rn(__fadd_rn(acc0.x, acc0.y), __fadd_rn(acc1.x, acc1.y));
-    }
+    float pq[RL], uo[RL];
+    gdn_step<LR, RL, false>(S, k2, k2, vr, a, beta, pq, uo);
 }
 
-// a[i] for a lane-dependent i, by selects (no local-memory array).
-template <int K>
-__device__ __forceinline__ int pick(const int (&a)[K], int i)
+// k . q of one node's record, the same reduction wherever it is computed.
+template <int DK, typename RT>
+__device__ __forceinline__ float node_kq(const RT* rec, int lane)
 {
-    int x = a[0];
+    float acc = 0.f;
 #pragma unroll
-    for (int t = 1; t < K; ++t)
-        x = (i == t) ? a[t] : x;
-    return x;
-}
-
-// Reduces V = kOutBatch * RL partial values per lane over the LR lanes of a
-// row and stores scale * sum for every (batch node i, row r) value j = i*RL+r.
-// Every level adds the partials of the two lanes that differ in one lane bit
-// (bits from high to low); while a lane still holds several values it keeps
-// half of them (a transpose-reduce), else both lanes keep the sum.  Every
-// value goes through the same additions in the same order.
-template <int DK, int RL>
-__device__ __forceinline__ void flush_out(float (&v)[kOutBatch * RL], const int (&nodes)[kOutBatch],
-                                          int count, const KParams& p, int b, int h, int row0,
-                                          const LaneMap<DK, RL>& L)
-{
-    constexpr int LR = LaneMap<DK, RL>::LR;
-    constexpr int V = kOutBatch * RL;
-    int c = V, base = 0, dup_mask = 0;
+    for (int j = lane; j < DK; j += 32)
+        acc = __fmaf_rn(Widen<RT>::lds1(rec + j), Widen<RT>::lds1(rec + DK + j), acc);
 #pragma unroll
-    for (int o = LR / 2; o >= 1; o >>= 1) {
-        if (c >= 2) {
-            const int half = c / 2;
-            const bool upper = (L.cl & o) != 0;
-#pragma unroll
-            for (int t = 0; t < V / 2; ++t) {
-                if (t < half) {
-                    const float send = upper ? v[t] : v[t + half];
-                    const float keep = upper ? v[t + half] : v[t];
-                    v[t] = __fadd_rn(keep, __shfl_xor_sync(0xffffffffu, send, o));
-                }
-            }
-            if (upper)
-                base += half;
-            c = half;
-        } else {
-            v[0] = __fadd_rn(v[0], __shfl_xor_sync(0xffffffffu, v[0], o));
-            dup_mask |= o;
-        }
-    }
-    if ((L.cl & dup_mask) == 0) {
-#pragma unroll
-        for (int t = 0; t < V; ++t) {
-            if (t < c) {
-                const int j = base + t;
-                const int i = j / RL, r = j % RL;
-                if (i < count)
-                    p.out[(((size_t)b * p.N + pick(nodes, i)) * p.Hv + h) * p.dv + row0 +
-                          pick(L.rloc, r)] = __fmul_rn(p.scale, v[t]);
-            }
-        }
-    }
+    for (int off = 16; off >= 1; off >>= 1)
+        acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, off));
+    return acc;
 }
 
 template <typename ST>
@@ -632,27 +595,50 @@ __device__ __forceinline__ void source_parent(StateT<RL>& S, int m, int pp, int 
             float vr[RL];
             float a, be;
             fetch(y, k2, vr, a, be);
-            gdn_step<LR, RL>(S, k2, vr, a, be);
+            gdn_update<LR, RL>(S, k2, vr, a, be);
         });
     }
 }
 
+// Where this lane's rows of node n's state and output live: one 64-bit base
+// per node plus per-lane 32-bit offsets computed once.
 template <int DK, int RL, typename ST>
-__device__ __forceinline__ void persist(const StateT<RL>& S, int n, int pos, const KParams& p, int b,
-                                        int h, int row0, const LaneMap<DK, RL>& L)
+struct OutPtrs {
+    ST* ns_head;          // node_states of (b, h) at node 0
+    size_t ns_stride;     // elements between consecutive nodes' states
+    float* out_head;      // out of (b, h) at node 0, row row0
+    size_t out_stride;    // elements between consecutive nodes' outputs
+    uint32_t ns_off[RL];  // (row0 + row) * DK + 4 * cl
+    uint32_t out_off[RL];
+    __device__ __forceinline__ OutPtrs(const KParams& p, int b, int h, int row0, const LaneMap<DK, RL>& L)
+    {
+        const int NS = p.persist_last ? 1 : p.N;
+        ns_stride = (size_t)p.Hv * p.dv * DK;
+        ns_head = static_cast<ST*>(p.node_states) + (size_t)b * NS * ns_stride + (size_t)h * p.dv * DK;
+        out_stride = (size_t)p.Hv * p.dv;
+        out_head = p.out + (size_t)b * p.N * out_stride + (size_t)h * p.dv + row0;
+#pragma unroll
+        for (int r = 0; r < RL; ++r) {
+            ns_off[r] = (uint32_t)((row0 + L.rloc[r]) * DK + 4 * L.cl);
+            out_off[r] = (uint32_t)L.rloc[r];
+        }
+    }
+};
+
+template <int DK, int RL, typename ST>
+__device__ __forceinline__ void persist(const StateT<RL>& S, int n, int pos, const KParams& p,
+                                        const OutPtrs<DK, RL, ST>& P)
 {
+    constexpr int LR = DK / kColsPerLane;
     if (p.persist_last && pos != p.N - 1)
         return;
-    const int ni = p.persist_last ? 0 : n;
-    const int NS = p.persist_last ? 1 : p.N;
-    ST* dst = static_cast<ST*>(p.node_states) + (((size_t)b * NS + ni) * p.Hv + h) * p.dv * DK +
-              (size_t)row0 * DK;
+    ST* node = P.ns_head + (size_t)(p.persist_last ? 0 : n) * P.ns_stride;
 #pragma unroll
     for (int r = 0; r < RL; ++r) {
-        ST* row = dst + (size_t)L.rloc[r] * DK;
+        ST* row = node + P.ns_off[r];
 #pragma unroll
         for (int m = 0; m < 4; ++m)
-            Persist<ST>::store(row + L.col(m), S.s[r][2 * m], S.s[r][2 * m + 1]);
+            Persist<ST>::store(row + 4 * m * LR, S.s[r][2 * m], S.s[r][2 * m + 1]);
     }
 }
 
@@ -668,69 +654,58 @@ __device__ __forceinline__ void walk(StateT<RL>& S, const KParams& p, const Tree
 {
     constexpr int LR = LaneMap<DK, RL>::LR;
     const int N = p.N;
-    float ov[kOutBatch * RL];
-    int onodes[kOutBatch];
+    const OutPtrs<DK, RL, ST> P(p, b, h, row0, L);
     StateT<RL> Sn;  // index order: the next position's parent state, prefetched
     const float* nsf = static_cast<const float*>(p.node_states) +
                        ((size_t)b * p.N * p.Hv + h) * p.dv * DK + (size_t)row0 * DK;
     const size_t node_stride = (size_t)p.Hv * p.dv * DK;
-    for (int pos0 = 0; pos0 < N; pos0 += kOutBatch) {
-#pragma unroll
-        for (int i = 0; i < kOutBatch; ++i) {
-            const int pos = pos0 + i;
-            onodes[i] = 0;
+    for (int pos = 0; pos < N; ++pos) {
+        if (!ctx.begin(pos))
+            return;
+        int n = pos, save = -1;
+        bool next_reload = false;
+        if constexpr (Tree::kIndex) {
+            // issue the loads of the next position's parent state now; it was
+            // persisted by this thread at an earlier position
+            if (pos + 1 < N) {
+                const int pn = tree.parent(pos + 1);
+                next_reload = pn != pos;
+                if (next_reload)
+                    load_state<DK, RL>(Sn, nsf + (size_t)pn * node_stride, L);
+            }
+        } else if constexpr (!CHAIN) {
+            const int m = tree.meta(pos);
+            n = meta_node(m);
+            save = meta_save(m);
+            const int rs = tree.rstart(pos);
+            const int pp = tree.parent(n);
+            if (meta_src(m) != kSrcCont && meta_src(m) != kSrcRoot)
+                source_parent<DK, RL>(S, m, pp, rs, p, tree, slotbuf, sin_head, b, h, row0, L,
+                                      ctx.fetcher());
+        }
+        const auto* rec = ctx.rec(pos, n);
+        float2 k2[8], q2[8];
+        float vr[RL];
+        load_k<DK, RL>(rec, L, k2, vr);
+        load_q<DK, RL>(rec, L, q2);
+        float a, be, kq;
+        ctx.ab(pos, n, a, be, kq);
+        float pq[RL], u[RL];
+        gdn_step<LR, RL, true>(S, k2, q2, vr, a, be, pq, u);
+        if (L.cl == 0) {
+            float* o = P.out_head + (size_t)n * P.out_stride;
 #pragma unroll
             for (int r = 0; r < RL; ++r)
-                ov[i * RL + r] = 0.f;
-            if (pos < N) {
-                if (!ctx.begin(pos))
-                    return;
-                int n = pos, save = -1;
-                bool next_reload = false;
-                if constexpr (Tree::kIndex) {
-                    // issue the loads of the next position's parent state now;
-                    // it was persisted by this thread at an earlier position
-                    if (pos + 1 < N) {
-                        const int pn = tree.parent(pos + 1);
-                        next_reload = pn != pos;
-                        if (next_reload)
-                            load_state<DK, RL>(Sn, nsf + (size_t)pn * node_stride, L);
-                    }
-                } else if constexpr (!CHAIN) {
-                    const int m = tree.meta(pos);
-                    n = meta_node(m);
-                    save = meta_save(m);
-                    const int rs = tree.rstart(pos);
-                    const int pp = tree.parent(n);
-                    if (meta_src(m) != kSrcCont && meta_src(m) != kSrcRoot)
-                        source_parent<DK, RL>(S, m, pp, rs, p, tree, slotbuf, sin_head, b, h, row0, L,
-                                              ctx.fetcher());
-                }
-                const auto* rec = ctx.rec(pos, n);
-                float2 k2[8], q2[8];
-                float vr[RL];
-                load_k<DK, RL>(rec, L, k2, vr);
-                float a, be;
-                ctx.ab(pos, n, a, be);
-                gdn_step<LR, RL>(S, k2, vr, a, be);
-                load_q<DK, RL>(rec, L, q2);
-                float o[RL];
-                partial_out<RL>(S, q2, o);
-#pragma unroll
-                for (int r = 0; r < RL; ++r)
-                    ov[i * RL + r] = o[r];
-                onodes[i] = n;
-                persist<DK, RL, ST>(S, n, pos, p, b, h, row0, L);
-                if (save >= 0)
-                    save_state<DK, RL>(S, slotbuf + (size_t)save * p.rows * DK, L);
-                if constexpr (Tree::kIndex) {
-                    if (next_reload)
-                        S = Sn;
-                }
-                ctx.end(pos);
-            }
+                o[P.out_off[r]] = __fmul_rn(p.scale, __fmaf_rn(u[r], kq, __fmul_rn(a, pq[r])));
         }
-        flush_out<DK, RL>(ov, onodes, min(kOutBatch, N - pos0), p, b, h, row0, L);
+        persist<DK, RL, ST>(S, n, pos, p, P);
+        if (save >= 0)
+            save_state<DK, RL>(S, slotbuf + (size_t)save * p.rows * DK, L);
+        if constexpr (Tree::kIndex) {
+            if (next_reload)
+                S = Sn;
+        }
+        ctx.end(pos);
     }
 }
 
@@ -768,10 +743,11 @@ struct StagedCtx {
     {
         return recs + (size_t)n * rec_elems;
     }
-    __device__ __forceinline__ void ab(int, int n, float& a, float& be) const
+    __device__ __forceinline__ void ab(int, int n, float& a, float& be, float& kq) const
     {
         a = ab_[n];
         be = ab_[N + n];
+        kq = ab_[2 * N + n];
     }
     __device__ __forceinline__ StagedFetch<DK, RL, RT> fetcher() const
     {
@@ -917,6 +893,13 @@ __global__ void __launch_bounds__(kMaxWarps * 32) gdn_verify_staged(const KParam
     }
     const RT* rt = kWiden ? reinterpret_cast<const RT*>(recs) : reinterpret_cast<const RT*>(raw);
     const uint32_t rt_elems = kWiden ? p.rec_floats : p.raw_bytes / (uint32_t)sizeof(QT);
+    // 8. k . q of every node (outputs read the pre-update state)
+    for (int n = warp; n < N; n += nwarps) {
+        const float kq = node_kq<DK, RT>(rt + (size_t)n * rt_elems, lane);
+        if (lane == 0)
+            ab[2 * N + n] = kq;
+    }
+    __syncthreads();
 
     StagedCtx<DK, RL, RT> ctx{rt, ab, rt_elems, N, L};
     if constexpr (TREE == kTreeChain)
@@ -965,7 +948,7 @@ template <int DK, int RL, typename QT>
 struct RingCtx {
     uint64_t* full;
     uint64_t* empty;
-    const float* ring;  // kRing slots of [kChunk records | a[kChunk] | beta[kChunk]]
+    const float* ring;  // kRing slots of [kChunk records | a | beta | k.q, kChunk each]
     uint32_t rec_floats;
     uint32_t slot_floats;
     int32_t* status;
@@ -1000,11 +983,12 @@ struct RingCtx {
     {
         return slot(pos) + (size_t)(pos % kChunk) * rec_floats;
     }
-    __device__ __forceinline__ void ab(int pos, int, float& a, float& be) const
+    __device__ __forceinline__ void ab(int pos, int, float& a, float& be, float& kq) const
     {
         const float* s = slot(pos) + (size_t)kChunk * rec_floats;
         a = s[pos % kChunk];
         be = s[kChunk + pos % kChunk];
+        kq = s[2 * kChunk + pos % kChunk];
     }
     __device__ __forceinline__ GlobalFetch<DK, RL, QT> fetcher() const { return gf; }
 };
@@ -1024,7 +1008,7 @@ __global__ void __launch_bounds__((kMaxWarps + 1) * 32) gdn_verify_ring(const KP
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + kRing;
     float* ring = reinterpret_cast<float*>(smem + p.off_rec);
-    const uint32_t slot_floats = kChunk * p.rec_floats + 2 * kChunk;
+    const uint32_t slot_floats = kChunk * p.rec_floats + 3 * kChunk;
     float* slotbuf = reinterpret_cast<float*>(smem + p.off_slots);
     const TreeView T(reinterpret_cast<int*>(smem + p.off_tree), p.N);
 
@@ -1121,6 +1105,12 @@ __global__ void __launch_bounds__((kMaxWarps + 1) * 32) gdn_verify_ring(const KP
                     const int i = idx / per_pos, j = idx - i * per_pos;
                     Widen<QT>::store(base + (size_t)i * p.rec_floats + j * EPC, regs[t]);
                 }
+            }
+            __syncwarp();
+            for (int i = 0; i < cnt; ++i) {
+                const float kq = node_kq<DK, float>(base + (size_t)i * p.rec_floats, lane);
+                if (lane == 0)
+                    base[kChunk * p.rec_floats + 2 * kChunk + i] = kq;
             }
             mbar_arrive(&full[s]);
         }
