@@ -121,8 +121,8 @@ gdn_status gdn_tree_verify(const gdn_tree_desc* desc, const void* q, const void*
     if (!q || !k || !v || !g || !beta || !state_in || !out || !node_states || (need_parent && !parent_idx))
         return fail(GDN_ERR_INVALID_ARG, "a required pointer is NULL%s");
     const struct { const void* p; size_t a; const char* n; } al[] = {
-        {q, 16, "q"}, {k, 16, "k"}, {v, 16, "v"}, {state_in, 16, "state_in"}, {out, 16, "out"},
-        {node_states, 16, "node_states"}, {g, 4, "g"}, {beta, 4, "beta"}, {parent_idx, 4, "parent_idx"},
+        {q, 16, "q"}, {k, 16, "k"}, {v, 16, "v"}, {state_in, 32, "state_in"}, {out, 16, "out"},
+        {node_states, 32, "node_states"}, {g, 4, "g"}, {beta, 4, "beta"}, {parent_idx, 4, "parent_idx"},
         {d.status, 4, "status"}};
     for (const auto& x : al)
         if (x.p && !aligned(x.p, x.a))

@@ -93,6 +93,26 @@ __device__ __forceinline__ void pdl_wait_then_release()
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// ---- 256-bit global accesses ---------------------------------------------------
+
+// 8 floats at a 32-byte-aligned global address in one access.  The load is a
+// plain (coherent) load, so it sees this thread's earlier stores.
+__device__ __forceinline__ void ld_global_v8(const float* p, float4& lo, float4& hi)
+{
+    asm volatile("ld.global.v8.f32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=f"(lo.x), "=f"(lo.y), "=f"(lo.z), "=f"(lo.w), "=f"(hi.x), "=f"(hi.y), "=f"(hi.z),
+                   "=f"(hi.w)
+                 : "l"(p)
+                 : "memory");
+}
+
+__device__ __forceinline__ void st_global_v8(float* p, float4 lo, float4 hi)
+{
+    asm volatile("st.global.v8.f32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "f"(lo.x), "f"(lo.y),
+                 "f"(lo.z), "f"(lo.w), "f"(hi.x), "f"(hi.y), "f"(hi.z), "f"(hi.w)
+                 : "memory");
+}
+
 // ---- status -----------------------------------------------------------------
 
 __device__ __forceinline__ void report_status(int32_t* status, int32_t code)
@@ -147,6 +167,23 @@ struct Widen<__nv_bfloat16> {
         const unsigned short u = *reinterpret_cast<const unsigned short*>(p);
         return __uint_as_float(static_cast<uint32_t>(u) << 16);
     }
+    // 8 consecutive elements starting at p (16-byte aligned) as 4 pairs, from
+    // shared memory (lds8) or global memory (ldg8).
+    __device__ __forceinline__ static void pairs(uint4 u, float2 (&x)[4])
+    {
+        x[0] = bf16x2_to_float2(u.x);
+        x[1] = bf16x2_to_float2(u.y);
+        x[2] = bf16x2_to_float2(u.z);
+        x[3] = bf16x2_to_float2(u.w);
+    }
+    __device__ __forceinline__ static void lds8(const __nv_bfloat16* p, float2 (&x)[4])
+    {
+        pairs(*reinterpret_cast<const uint4*>(p), x);
+    }
+    __device__ __forceinline__ static void ldg8(const __nv_bfloat16* p, float2 (&x)[4])
+    {
+        pairs(__ldg(reinterpret_cast<const uint4*>(p)), x);
+    }
 };
 
 template <>
@@ -166,6 +203,21 @@ struct Widen<float> {
         return *reinterpret_cast<const float4*>(p);
     }
     __device__ __forceinline__ static float lds1(const float* p) { return *p; }
+    __device__ __forceinline__ static void pairs(float4 a, float4 b, float2 (&x)[4])
+    {
+        x[0] = make_float2(a.x, a.y);
+        x[1] = make_float2(a.z, a.w);
+        x[2] = make_float2(b.x, b.y);
+        x[3] = make_float2(b.z, b.w);
+    }
+    __device__ __forceinline__ static void lds8(const float* p, float2 (&x)[4])
+    {
+        pairs(reinterpret_cast<const float4*>(p)[0], reinterpret_cast<const float4*>(p)[1], x);
+    }
+    __device__ __forceinline__ static void ldg8(const float* p, float2 (&x)[4])
+    {
+        pairs(__ldg(reinterpret_cast<const float4*>(p)), __ldg(reinterpret_cast<const float4*>(p) + 1), x);
+    }
 };
 
 }  // namespace gdn

@@ -20,14 +20,14 @@ struct VerifyGeom {
     bool staged;          // whole-tree staging kernel (else the producer/ring kernel)
     bool warp_tree;       // staged tree walked from warp registers (N <= 32)
     bool reload;          // branch parents re-read from f32 node_states (no stack)
-    int rows_per_lane;    // 1 or 2
+    int chunks;           // lane shape: chunks of 8 state columns per lane and row (1 or 2)
+    int rows_per_lane;    // lane shape: rows per lane (1 or 2)
     int warps;            // compute warps per CTA (the ring kernel adds a producer warp)
     int rows;             // d_v rows per CTA
     int tiles;            // d_v / rows
     int slots;            // f32 parent-state stack slots
-    uint32_t raw_bytes;   // one node's raw record: k row | q row | v slice
-    uint32_t rec_floats;  // the same record widened to f32
-    uint32_t off_raw, off_rec, off_ab, off_slots, off_tree;  // shared-memory layout
+    uint32_t raw_bytes;   // one node's record: k row | q row | v slice, input type
+    uint32_t off_raw, off_desc, off_ab, off_slots, off_tree;  // shared-memory layout
     size_t smem;          // dynamic shared memory bytes
 };
 

@@ -1,5 +1,6 @@
 // gdn_verify.cu -- launch geometry and dispatch of the verify kernels (the
-// kernels themselves are in gdn_verify.cuh).
+// kernels themselves are in gdn_verify.cuh, instantiated per head dim and
+// lane shape in gdn_verify_d*_c*r*.cu).
 
 #include <cstdint>
 
@@ -10,16 +11,34 @@
 
 namespace gdn {
 namespace verify {
-extern template cudaError_t launch_dk<32>(const KParams&, const VerifyArgs&, const VerifyGeom&,
-                                          cudaStream_t);
-extern template cudaError_t launch_dk<64>(const KParams&, const VerifyArgs&, const VerifyGeom&,
-                                          cudaStream_t);
-extern template cudaError_t launch_dk<128>(const KParams&, const VerifyArgs&, const VerifyGeom&,
-                                           cudaStream_t);
+#define GDN_EXTERN_SHAPE(DK, C, RL)                                                                \
+    extern template cudaError_t launch_dk<DK, C, RL>(const KParams&, const VerifyArgs&,          \
+                                                     const VerifyGeom&, cudaStream_t);
+GDN_EXTERN_SHAPE(32, 2, 2)
+GDN_EXTERN_SHAPE(32, 2, 1)
+GDN_EXTERN_SHAPE(64, 2, 2)
+GDN_EXTERN_SHAPE(64, 2, 1)
+GDN_EXTERN_SHAPE(128, 2, 2)
+GDN_EXTERN_SHAPE(128, 2, 1)
+#undef GDN_EXTERN_SHAPE
 }  // namespace verify
 
 namespace {
 size_t align16(size_t x) { return (x + 15) & ~size_t(15); }
+
+// Warps per SM below which a launch uses the lane shape with one row per
+// lane (twice the warps, to hide the per-node dependency chain).
+constexpr long long kWarpsPerSmTarget = 16;
+constexpr long long kSms = 148;
+
+template <int DK>
+cudaError_t launch_shapes(const verify::KParams& kp, const VerifyArgs& a, const VerifyGeom& g,
+                          cudaStream_t s)
+{
+    if (g.rows_per_lane == 2)
+        return verify::launch_dk<DK, 2, 2>(kp, a, g, s);
+    return verify::launch_dk<DK, 2, 1>(kp, a, g, s);
+}
 }  // namespace
 
 using namespace verify;
@@ -29,7 +48,6 @@ VerifyGeom verify_geometry(const VerifyArgs& a)
     VerifyGeom g{};
     const bool chain = (a.flags & GDN_FLAG_CHAIN) != 0;
     const bool persist_last = (a.flags & GDN_FLAG_PERSIST_LAST) != 0;
-    const int lr = a.d_k / kColsPerLane;
     const size_t es = a.qkv_dtype == GDN_BF16 ? 2 : 4;
     g.reload = !chain && a.state_dtype == GDN_F32 && !persist_last;
     if (chain || g.reload) {
@@ -43,11 +61,17 @@ VerifyGeom verify_geometry(const VerifyArgs& a)
         const int cap = a.n_nodes <= 32 ? 2 : (a.n_nodes <= 96 ? 3 : 4);
         g.slots = k < 1 ? 1 : (k > cap ? cap : k);
     }
-    // One row per lane when two would leave fewer than 8 warps per SM (148
-    // SMs): more warps hide the per-node dependency chain of small batches.
-    const long long warps_rl2 = (long long)a.batch * a.n_v_heads * a.d_v / (2 * 32 / lr);
-    g.rows_per_lane = warps_rl2 < 8 * 148 ? 1 : 2;
-    const int rpw = g.rows_per_lane * 32 / lr;
+    // Lane shape: C = 2 chunks of 8 columns and RL rows per lane; two rows
+    // (fewer instructions per row) unless that leaves fewer than
+    // kWarpsPerSmTarget warps per SM.  (One chunk per lane, twice the warps
+    // again, measured slower at every batch: the per-node overhead doubles.)
+    auto rows_per_warp = [&](int c, int rl) { return rl * 32 * 8 * c / a.d_k; };
+    auto total_warps = [&](int c, int rl) {
+        return (long long)a.batch * a.n_v_heads * a.d_v / rows_per_warp(c, rl);
+    };
+    g.chunks = 2;
+    g.rows_per_lane = total_warps(2, 2) >= kWarpsPerSmTarget * kSms ? 2 : 1;
+    const int rpw = rows_per_warp(g.chunks, g.rows_per_lane);
     // Staged kernel first, else the ring kernel (which adds a producer warp).
     for (int pass = 0; pass < 2; ++pass) {
         const bool staged = pass == 0;
@@ -58,40 +82,24 @@ VerifyGeom verify_geometry(const VerifyArgs& a)
         if (a.d_v % rows != 0 || (rows * es) % 16 != 0)
             continue;
         const size_t raw_bytes = (size_t)(2 * a.d_k + rows) * es;
-        const size_t rec_floats = (size_t)(2 * a.d_k + rows);
         const size_t slot_bytes = (size_t)g.slots * rows * a.d_k * 4;
         size_t off = 64;  // mbarriers
-        size_t off_raw = 0, off_rec = 0, off_ab = 0, off_slots = 0;
+        size_t off_raw = 0, off_desc = 0, off_ab = 0, off_slots = 0;
         if (staged) {
-            const size_t stage_raw = align16((size_t)a.n_nodes * raw_bytes);
-            if (es == 2 && g.rows_per_lane == 1) {
-                // raw bf16 records are read by the node loop itself
-                off_raw = off_rec = off;
-                off += stage_raw;
-                off_slots = off;
-                off += align16(slot_bytes);
-            } else if (es == 2) {
-                // raw rows are dead once widened: they share space with the stack
-                off_raw = off_slots = off;
-                off += stage_raw > slot_bytes ? stage_raw : align16(slot_bytes);
-                off_rec = off;
-                off += align16((size_t)a.n_nodes * rec_floats * 4);
-            } else {
-                off_raw = off_rec = off;  // f32 rows are the records
-                off += stage_raw;
-                off_slots = off;
-                off += align16(slot_bytes);
-            }
+            off_raw = off;
+            off += align16((size_t)a.n_nodes * raw_bytes);
+            off_desc = off;
+            off += (size_t)a.n_nodes * sizeof(PosDesc);
             off_ab = off;
-            off += align16((size_t)3 * a.n_nodes * 4);  // a | beta | k.q per node
+            off += align16((size_t)2 * a.n_nodes * 4);  // g (then a) | beta, by node
         } else {
-            off_rec = off;
-            off += (size_t)kRing * align16((kChunk * rec_floats + 3 * kChunk) * 4);
-            off_slots = off;
-            off += align16(slot_bytes);
+            off_raw = off;
+            off += (size_t)kRing * (align16(kChunk * raw_bytes) + kChunk * sizeof(PosDesc));
         }
+        off_slots = off;
+        off += align16(slot_bytes);
         // tree area: none for chains, the parent array for index order, the
-        // register-built walk's 4 x 32 ints, else the shared-memory walk
+        // warp-built walk (kWarpTreeInts ints), else the shared-memory walk
         const size_t off_tree = off;
         const bool warp_tree = staged && !chain && !g.reload && a.n_nodes <= 32;
         if (chain)
@@ -99,7 +107,7 @@ VerifyGeom verify_geometry(const VerifyArgs& a)
         else if (g.reload)
             off += align16((size_t)a.n_nodes * 4);
         else if (warp_tree)
-            off += 4 * 32 * 4;
+            off += kWarpTreeInts * 4;
         else
             off += (size_t)(kTreeArrays + warps) * a.n_nodes * 4;
         if (staged && off > (size_t)kStagedMaxSmem)
@@ -110,9 +118,8 @@ VerifyGeom verify_geometry(const VerifyArgs& a)
         g.rows = rows;
         g.tiles = a.d_v / rows;
         g.raw_bytes = (uint32_t)raw_bytes;
-        g.rec_floats = (uint32_t)rec_floats;
         g.off_raw = (uint32_t)off_raw;
-        g.off_rec = (uint32_t)off_rec;
+        g.off_desc = (uint32_t)off_desc;
         g.off_ab = (uint32_t)off_ab;
         g.off_slots = (uint32_t)off_slots;
         g.off_tree = (uint32_t)off_tree;
@@ -146,19 +153,17 @@ cudaError_t launch_verify(const VerifyArgs& a, const VerifyGeom& geom, cudaStrea
     kp.slots = geom.slots;
     kp.persist_last = (a.flags & GDN_FLAG_PERSIST_LAST) ? 1 : 0;
     kp.validate = (a.flags & GDN_FLAG_VALIDATE) ? 1 : 0;
-    kp.reload = geom.reload ? 1 : 0;
     kp.early_tree = (a.flags & GDN_FLAG_EARLY_TREE) ? 1 : 0;
     kp.raw_bytes = geom.raw_bytes;
-    kp.rec_floats = geom.rec_floats;
     kp.off_raw = geom.off_raw;
-    kp.off_rec = geom.off_rec;
+    kp.off_desc = geom.off_desc;
     kp.off_ab = geom.off_ab;
     kp.off_slots = geom.off_slots;
     kp.off_tree = geom.off_tree;
     switch (a.d_k) {
-        case 32: return launch_dk<32>(kp, a, geom, stream);
-        case 64: return launch_dk<64>(kp, a, geom, stream);
-        case 128: return launch_dk<128>(kp, a, geom, stream);
+        case 32: return launch_shapes<32>(kp, a, geom, stream);
+        case 64: return launch_shapes<64>(kp, a, geom, stream);
+        case 128: return launch_shapes<128>(kp, a, geom, stream);
         default: return cudaErrorInvalidValue;
     }
 }

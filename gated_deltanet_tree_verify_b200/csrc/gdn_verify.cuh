@@ -2,9 +2,7 @@
 // templates; gdn_verify_d{32,64,128}.cu instantiate them per head dim.
 //
 // One CTA per (sequence b, v-head h, tile of d_v rows).  The CTA walks the
-// tree's nodes in depth-first preorder, a topological order, visiting each
-// node's children by increasing subtree size (ties by index) so that the
-// largest child subtree comes last, and for each node applies the gated
+// tree's nodes in a topological order and for each node applies the gated
 // delta rule (Gated DeltaNet; the ggml_gated_delta_net recurrence named in
 // the GreenGames post, "TL;DR"):
 //
@@ -12,35 +10,44 @@
 //     S_n = a * S_p + u k_n^T;         o_n = scale * S_n q_n
 //
 // and persists S_n from inside the kernel (the GreenGames post, "Key wins":
-// persist-write kernel, f16 intermediate cache).
+// persist-write kernel, f16 intermediate cache).  The output is formed from
+// the parent state, o_n = scale * (a * (S_p q_n) + u * (k_n . q_n)), so S_p q
+// is reduced together with S_p k.
 //
-// Compute layout: LR = d_k / 16 lanes share a state row, each holding 16
-// columns (4 chunks of 4 at columns 4 * (c + m * LR)); a lane holds RL rows
-// (RL = 1 or 2), so a warp owns RL * 32 / LR rows (4 or 8 at d_k = 128).
-// S k is a packed-fp32 (FFMA2) partial dot plus an xor-butterfly over the
-// row's LR lanes; the rank-1 update is packed fp32.  The partial S q dots of
-// four consecutive nodes are reduced together by a transpose-reduce and
-// stored as one vector.  Each node's state leaves as 16-byte (f32) or 8-byte
-// (f16) stores that cover whole 128-byte lines of a row.  Which rows a lane
-// holds (RL, warps per CTA) never changes a row's arithmetic.
+// Compute layout.  A state row of d_k columns is split into chunks of 8
+// consecutive columns; a lane holds C chunks of each of its RL rows (C = 1 or
+// 2, RL = 1 or 2), so LR = d_k / (8 C) lanes share a row and a warp owns
+// RL * 32 / LR rows.  The shape is picked per launch from the size of the
+// grid: (C, RL) = (2, 2) for large batches, (2, 1) for small ones (twice the
+// warps to hide the per-node dependency chain); the templates also take
+// C = 1, which is not instantiated.  A row's arithmetic is the same in every
+// shape:
+// each chunk's partial dot product is a chain of four packed-fp32 (FFMA2)
+// steps, chunks c and c + d_k / 16 are added next, then an xor butterfly
+// adds the rest in a fixed order.  So results never depend on the shape.
 //
-// Inputs are widened to f32 once per CTA into shared-memory records
-// (k_n | q_n | the CTA's slice of v_n).  Two kernels:
-//   * gdn_verify_staged: trees and chains small enough to stage whole.  All
-//     threads issue 16-byte asynchronous copies (cp.async) of every node's
-//     raw rows at kernel start, so they overlap the tree walk and the
-//     state_in load; all threads then widen them; all warps compute.  Trees
-//     of up to 32 nodes are walked from warp registers (each warp builds the
-//     walk with shuffles and ballots, no shared memory, no block barrier).
-//   * gdn_verify_ring: anything larger (long chains).  A producer warp loads,
-//     widens and streams chunks of walk positions through a ring of
-//     mbarrier-guarded slots.
+// Node inputs stay in their storage type in shared memory: each node's
+// record is its k row, its q row and the CTA's slice of v, copied with
+// 16-byte cp.async; the node loop widens each lane's 16-byte chunks (exact
+// for bf16).  Two kernels:
+//   * gdn_verify_staged: trees and chains small enough to stage whole.  The
+//     copies of every node's record are issued at kernel start and overlap
+//     the tree work and the state_in load; a prologue pass then writes one
+//     32-byte descriptor per walk position (node, tree metadata, a, beta,
+//     k . q).  Trees of up to 32 nodes have their walk built by one warp
+//     (build_warp_walk), larger ones by the whole CTA (build_walk).
+//   * gdn_verify_ring: anything larger (long chains, large trees).  A
+//     producer warp streams records and descriptors of chunks of walk
+//     positions through a ring of mbarrier-guarded slots.
 //
 // Parents that are not the previous node of the walk: with exact f32
-// persistence the parent's state is re-read from node_states (written by the
-// same thread, bit-exact).  Otherwise a node with two or more children saves
-// its f32 state in a shared-memory stack slot, and a later child reloads it.
-// The slot index is the number of edges on the node's root path that enter a
+// persistence the walk goes in index order and the parent's state is re-read
+// from node_states (written by the same thread, bit-exact), prefetched one
+// node ahead.  Otherwise the walk is a depth-first preorder visiting each
+// node's children by increasing subtree size (ties by index), so the largest
+// child subtree comes last; a node with two or more children saves its f32
+// state in a shared-memory stack slot, and a later child reloads it.  The
+// slot index is the number of edges on the node's root path that enter a
 // child other than the last one visited; since every such child's subtree
 // holds at most half of its parent's, floor(log2 N) slots always suffice.  If
 // fewer slots are configured and a tree needs more, the parent's state is
@@ -69,10 +76,9 @@
 namespace gdn {
 namespace verify {
 
-constexpr int kColsPerLane = 16;  // 4 chunks of 4 consecutive columns
-constexpr int kMaxWarps = 4;      // compute warps per CTA
-constexpr int kChunk = 8;         // walk positions per ring slot
-constexpr int kRing = 3;          // ring slots
+constexpr int kMaxWarps = 4;  // compute warps per CTA
+constexpr int kChunk = 8;     // walk positions per ring slot
+constexpr int kRing = 3;      // ring slots
 constexpr int kMaxDevices = 64;
 constexpr int kStagedMaxSmem = 100 * 1024;
 
@@ -104,70 +110,94 @@ struct KParams {
     int N, Hk, Hv, dv, G;
     float scale;
     int rows, warps, slots;
-    int persist_last, validate, reload, early_tree;
-    uint32_t raw_bytes;   // one node's raw record (k | q | v slice) in bytes
-    uint32_t rec_floats;  // one node's widened record in floats
-    uint32_t off_raw, off_rec, off_ab, off_slots, off_tree;
+    int persist_last, validate, early_tree;
+    uint32_t raw_bytes;  // one node's record (k row | q row | v slice) in bytes
+    uint32_t off_raw, off_desc, off_ab, off_slots, off_tree;
+};
+
+// One walk position: its node and tree metadata, and the node's scalars.
+struct PosDesc {
+    int4 i;    // node, metadata, recomputation start, parent
+    float4 f;  // a = exp(g), beta, k . q, unused
 };
 
 // ---------------------------------------------------------------------------
 // Lane geometry and per-node arithmetic
 // ---------------------------------------------------------------------------
 
-template <int DK, int RL>
+template <int DK, int C, int RL>
 struct LaneMap {
-    static constexpr int LR = DK / kColsPerLane;  // lanes per row
-    static constexpr int RG = 32 / LR;            // row groups per warp
-    static constexpr int RPW = RL * RG;           // rows per warp
-    int cl;
-    int rloc[RL];
-    __device__ __forceinline__ LaneMap(int warp, int lane)
+    static constexpr int E = 8 * C;     // state columns per lane and row
+    static constexpr int LR = DK / E;   // lanes per row
+    static constexpr int RG = 32 / LR;  // row groups per warp
+    static constexpr int RPW = RL * RG; // rows per warp
+    int cl;                             // lane within its row: chunks cl, cl + LR
+    int row;                            // the lane's first row in the tile; then every RG rows
+    __device__ __forceinline__ LaneMap(int warp, int lane) : cl(lane % LR), row(warp * RPW + lane / LR)
     {
-        cl = lane % LR;
-#pragma unroll
-        for (int r = 0; r < RL; ++r)
-            rloc[r] = warp * RPW + lane / LR + r * RG;
     }
-    __device__ __forceinline__ int col(int m) const { return 4 * (cl + m * LR); }
+    // first column of chunk c of this lane
+    __device__ __forceinline__ int col(int c) const { return 8 * (cl + c * LR); }
+    // offset of this lane's first element in a [rows][DK] row-major tile
+    __device__ __forceinline__ int tile_offset() const { return row * DK + 8 * cl; }
 };
 
-template <int RL>
+template <int C, int RL>
 struct StateT {
-    float2 s[RL][8];
+    float2 s[RL][4 * C];
 };
 
-// One node's state update on a lane's RL rows x 16 columns.  Shared by the
+// Sum of one chunk's 8 products x * y (pairs t = 0..3): a chain of packed
+// FMAs, then the two halves.
+__device__ __forceinline__ float chunk_dot(const float2* x, const float2* y)
+{
+    float2 acc = __fmul2_rn(x[0], y[0]);
+    acc = __ffma2_rn(x[1], y[1], acc);
+    acc = __ffma2_rn(x[2], y[2], acc);
+    acc = __ffma2_rn(x[3], y[3], acc);
+    return __fadd_rn(acc.x, acc.y);
+}
+
+// Adds up the chunk sums of a row across its LR lanes.  C = 2: the lane's two
+// chunks (cl, cl + LR) first, then lanes xor 1, 2, .. LR / 2.  C = 1: lanes
+// xor LR / 2 first (chunks c and c + LR / 2, the same pair), then 1, 2, ...
+// LR / 4.  Both orders add the same operands in the same sequence.
+template <int LR, int C>
+__device__ __forceinline__ float row_sum_first(const float (&cs)[C])
+{
+    if constexpr (C == 2)
+        return __fadd_rn(cs[0], cs[1]);
+    else
+        return __fadd_rn(cs[0], __shfl_xor_sync(0xffffffffu, cs[0], LR / 2));
+}
+
+// One node's state update on a lane's RL rows x 8C columns.  Shared by the
 // walk and the recompute path; explicit intrinsics keep both bit-identical.
-// With WITH_Q it also reduces this node's output read of the pre-update state,
-// pq = S_p q, in the same butterfly as S_p k, and returns u: the output is
-// then o = scale * (a * pq + u * (k . q)) = scale * S_n q (S_n = a S_p + u k^T).
-template <int LR, int RL, bool WITH_Q>
-__device__ __forceinline__ void gdn_step(StateT<RL>& S, const float2 (&k2)[8], const float2 (&q2)[8],
-                                         const float (&vr)[RL], float a, float beta, float (&pq)[RL],
-                                         float (&uo)[RL])
+// With WITH_Q it also returns pq = S_p q (reduced in the same butterfly as
+// S_p k) and u: the output is then o = scale * (a * pq + u * (k . q)) =
+// scale * S_n q, with S_n = a S_p + u k^T.
+template <int LR, int C, int RL, bool WITH_Q>
+__device__ __forceinline__ void gdn_step(StateT<C, RL>& S, const float2 (&k2)[4 * C],
+                                         const float2 (&q2)[4 * C], const float (&vr)[RL], float a,
+                                         float beta, float (&pq)[RL], float (&uo)[RL])
 {
     float w[RL];
 #pragma unroll
     for (int r = 0; r < RL; ++r) {
-        float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+        float cw[C], cq[C];
 #pragma unroll
-        for (int t = 0; t < 8; t += 2) {
-            acc0 = __ffma2_rn(S.s[r][t], k2[t], acc0);
-            acc1 = __ffma2_rn(S.s[r][t + 1], k2[t + 1], acc1);
+        for (int c = 0; c < C; ++c) {
+            cw[c] = chunk_dot(&S.s[r][4 * c], &k2[4 * c]);
+            if constexpr (WITH_Q)
+                cq[c] = chunk_dot(&S.s[r][4 * c], &q2[4 * c]);
         }
-        w[r] = __fadd_rn(__fadd_rn(acc0.x, acc0.y), __fadd_rn(acc1.x, acc1.y));
-        if constexpr (WITH_Q) {
-            float2 b0 = make_float2(0.f, 0.f), b1 = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int t = 0; t < 8; t += 2) {
-                b0 = __ffma2_rn(S.s[r][t], q2[t], b0);
-                b1 = __ffma2_rn(S.s[r][t + 1], q2[t + 1], b1);
-            }
-            pq[r] = __fadd_rn(__fadd_rn(b0.x, b0.y), __fadd_rn(b1.x, b1.y));
-        }
+        w[r] = row_sum_first<LR, C>(cw);
+        if constexpr (WITH_Q)
+            pq[r] = row_sum_first<LR, C>(cq);
     }
+    constexpr int BL = C == 2 ? LR : LR / 2;  // lanes still to be added after the first step
 #pragma unroll
-    for (int off = 1; off < LR; off <<= 1) {
+    for (int off = 1; off < BL; off <<= 1) {
 #pragma unroll
         for (int r = 0; r < RL; ++r) {
             w[r] = __fadd_rn(w[r], __shfl_xor_sync(0xffffffffu, w[r], off));
@@ -182,114 +212,174 @@ __device__ __forceinline__ void gdn_step(StateT<RL>& S, const float2 (&k2)[8], c
         uo[r] = u;
         const float2 u2 = make_float2(u, u);
 #pragma unroll
-        for (int t = 0; t < 8; ++t)
+        for (int t = 0; t < 4 * C; ++t)
             S.s[r][t] = __ffma2_rn(u2, k2[t], __fmul2_rn(a2, S.s[r][t]));
     }
 }
 
 // State update only (recompute path): the same instructions on S.
-template <int LR, int RL>
-__device__ __forceinline__ void gdn_update(StateT<RL>& S, const float2 (&k2)[8], const float (&vr)[RL],
-                                           float a, float beta)
+template <int LR, int C, int RL>
+__device__ __forceinline__ void gdn_update(StateT<C, RL>& S, const float2 (&k2)[4 * C],
+                                           const float (&vr)[RL], float a, float beta)
 {
     float pq[RL], uo[RL];
-    gdn_step<LR, RL, false>(S, k2, k2, vr, a, beta, pq, uo);
+    gdn_step<LR, C, RL, false>(S, k2, k2, vr, a, beta, pq, uo);
 }
 
-// k . q of one node's record, the same reduction wherever it is computed.
+// k . q of one node's record, reduced by a group of 8 lanes (sub = lane % 8;
+// a warp handles four nodes at once; every lane of the warp must call it).
+// The same reduction wherever it is computed.
 template <int DK, typename RT>
-__device__ __forceinline__ float node_kq(const RT* rec, int lane)
+__device__ __forceinline__ float node_kq8(const RT* rec, int sub)
 {
-    float acc = 0.f;
+    float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-    for (int j = lane; j < DK; j += 32)
-        acc = __fmaf_rn(Widen<RT>::lds1(rec + j), Widen<RT>::lds1(rec + DK + j), acc);
+    for (int j = sub; j < DK; j += 16) {
+        acc0 = __fmaf_rn(Widen<RT>::lds1(rec + j), Widen<RT>::lds1(rec + DK + j), acc0);
+        acc1 = __fmaf_rn(Widen<RT>::lds1(rec + j + 8), Widen<RT>::lds1(rec + DK + j + 8), acc1);
+    }
+    float acc = __fadd_rn(acc0, acc1);
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1)
+    for (int off = 4; off >= 1; off >>= 1)
         acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, off));
     return acc;
 }
 
+// ---------------------------------------------------------------------------
+// State and record access.  Row-layout accesses take a pointer already at
+// the lane's first element (LaneMap::tile_offset), so every other offset is
+// a compile-time constant.
+// ---------------------------------------------------------------------------
+
+// S <- this lane's part of a row-major f32 tile in global memory (32-byte
+// aligned): one 32-byte plain load per chunk, so a state this thread stored
+// earlier in the kernel is seen.
+template <int DK, int C, int RL>
+__device__ __forceinline__ void load_rows(StateT<C, RL>& S, const float* lane_ptr)
+{
+    using LM = LaneMap<DK, C, RL>;
+#pragma unroll
+    for (int r = 0; r < RL; ++r) {
+#pragma unroll
+        for (int c = 0; c < C; ++c) {
+            float4 x, y;
+            ld_global_v8(lane_ptr + r * LM::RG * DK + c * 8 * LM::LR, x, y);
+            S.s[r][4 * c + 0] = make_float2(x.x, x.y);
+            S.s[r][4 * c + 1] = make_float2(x.z, x.w);
+            S.s[r][4 * c + 2] = make_float2(y.x, y.y);
+            S.s[r][4 * c + 3] = make_float2(y.z, y.w);
+        }
+    }
+}
+
+// Persisted-state stores of one chunk (8 values) in f32 (one 32-byte store)
+// or f16 (RNE, one 16-byte store): the lanes of a row cover whole sectors.
 template <typename ST>
 struct Persist;
 
 template <>
 struct Persist<float> {
-    __device__ __forceinline__ static void store(float* dst, float2 lo, float2 hi)
+    __device__ __forceinline__ static void store8(float* dst, const float2* x)
     {
-        *reinterpret_cast<float4*>(dst) = make_float4(lo.x, lo.y, hi.x, hi.y);
+        st_global_v8(dst, make_float4(x[0].x, x[0].y, x[1].x, x[1].y), make_float4(x[2].x, x[2].y, x[3].x, x[3].y));
     }
 };
 
 template <>
 struct Persist<__half> {
-    __device__ __forceinline__ static void store(__half* dst, float2 lo, float2 hi)
+    __device__ __forceinline__ static void store8(__half* dst, const float2* x)
     {
-        const __half2 a = __float22half2_rn(lo);
-        const __half2 b = __float22half2_rn(hi);
-        uint2 u;
-        u.x = *reinterpret_cast<const uint32_t*>(&a);
-        u.y = *reinterpret_cast<const uint32_t*>(&b);
-        *reinterpret_cast<uint2*>(dst) = u;
+        uint4 u;
+        __half2 h;
+        h = __float22half2_rn(x[0]);
+        u.x = *reinterpret_cast<const uint32_t*>(&h);
+        h = __float22half2_rn(x[1]);
+        u.y = *reinterpret_cast<const uint32_t*>(&h);
+        h = __float22half2_rn(x[2]);
+        u.z = *reinterpret_cast<const uint32_t*>(&h);
+        h = __float22half2_rn(x[3]);
+        u.w = *reinterpret_cast<const uint32_t*>(&h);
+        *reinterpret_cast<uint4*>(dst) = u;
     }
 };
 
-// S <- this lane's part of a [rows][DK] f32 matrix (plain loads, so a state
-// this thread stored earlier in the kernel is seen).
-template <int DK, int RL>
-__device__ __forceinline__ void load_state(StateT<RL>& S, const float* base, const LaneMap<DK, RL>& L)
+template <int DK, int C, int RL, typename ST>
+__device__ __forceinline__ void persist(const StateT<C, RL>& S, ST* lane_ptr)
+{
+    using LM = LaneMap<DK, C, RL>;
+#pragma unroll
+    for (int r = 0; r < RL; ++r) {
+#pragma unroll
+        for (int c = 0; c < C; ++c)
+            Persist<ST>::store8(lane_ptr + r * LM::RG * DK + c * 8 * LM::LR, &S.s[r][4 * c]);
+    }
+}
+
+// Stack slots in shared memory are private to each lane: its 2 C RL float4
+// lie `stride` floats apart (the CTA's thread count x 4), consecutive lanes
+// in consecutive 16-byte words.
+template <int C, int RL>
+__device__ __forceinline__ void save_slot(const StateT<C, RL>& S, float* lane_slot, int stride)
 {
 #pragma unroll
     for (int r = 0; r < RL; ++r) {
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const float4 x = *reinterpret_cast<const float4*>(base + (size_t)L.rloc[r] * DK + L.col(m));
-            S.s[r][2 * m] = make_float2(x.x, x.y);
-            S.s[r][2 * m + 1] = make_float2(x.z, x.w);
+        for (int j = 0; j < 2 * C; ++j)
+            *reinterpret_cast<float4*>(lane_slot + (r * 2 * C + j) * stride) =
+                make_float4(S.s[r][2 * j].x, S.s[r][2 * j].y, S.s[r][2 * j + 1].x, S.s[r][2 * j + 1].y);
+    }
+}
+
+template <int C, int RL>
+__device__ __forceinline__ void load_slot(StateT<C, RL>& S, const float* lane_slot, int stride)
+{
+#pragma unroll
+    for (int r = 0; r < RL; ++r) {
+#pragma unroll
+        for (int j = 0; j < 2 * C; ++j) {
+            const float4 x = *reinterpret_cast<const float4*>(lane_slot + (r * 2 * C + j) * stride);
+            S.s[r][2 * j] = make_float2(x.x, x.y);
+            S.s[r][2 * j + 1] = make_float2(x.z, x.w);
         }
     }
 }
 
-template <int DK, int RL>
-__device__ __forceinline__ void save_state(const StateT<RL>& S, float* base, const LaneMap<DK, RL>& L)
-{
-#pragma unroll
-    for (int r = 0; r < RL; ++r) {
-#pragma unroll
-        for (int m = 0; m < 4; ++m)
-            *reinterpret_cast<float4*>(base + (size_t)L.rloc[r] * DK + L.col(m)) =
-                make_float4(S.s[r][2 * m].x, S.s[r][2 * m].y, S.s[r][2 * m + 1].x,
-                            S.s[r][2 * m + 1].y);
-    }
-}
-
-// k and the v slice of one node from its shared-memory record [k | q | v
-// slice], stored either widened (RT = float) or raw (RT = bf16: widened here).
-template <int DK, int RL, typename RT>
-__device__ __forceinline__ void load_k(const RT* rec, const LaneMap<DK, RL>& L, float2 (&k2)[8],
+// k, q and the v slice of one node from its shared-memory record
+// [k | q | v slice] in the input type, widened here.
+template <int DK, int C, int RL, typename QT>
+__device__ __forceinline__ void load_k(const QT* rec, const LaneMap<DK, C, RL>& L, float2 (&k2)[4 * C],
                                        float (&vr)[RL])
 {
+    using LM = LaneMap<DK, C, RL>;
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-        const float4 x = Widen<RT>::lds4(rec + L.col(m));
-        k2[2 * m] = make_float2(x.x, x.y);
-        k2[2 * m + 1] = make_float2(x.z, x.w);
+    for (int c = 0; c < C; ++c) {
+        float2 x[4];
+        Widen<QT>::lds8(rec + L.col(c), x);
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+            k2[4 * c + t] = x[t];
     }
 #pragma unroll
     for (int r = 0; r < RL; ++r)
-        vr[r] = Widen<RT>::lds1(rec + 2 * DK + L.rloc[r]);
+        vr[r] = Widen<QT>::lds1(rec + 2 * DK + L.row + r * LM::RG);
 }
 
-template <int DK, int RL, typename RT>
-__device__ __forceinline__ void load_q(const RT* rec, const LaneMap<DK, RL>& L, float2 (&q2)[8])
+template <int DK, int C, int RL, typename QT>
+__device__ __forceinline__ void load_q(const QT* rec, const LaneMap<DK, C, RL>& L, float2 (&q2)[4 * C])
 {
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-        const float4 y = Widen<RT>::lds4(rec + DK + L.col(m));
-        q2[2 * m] = make_float2(y.x, y.y);
-        q2[2 * m + 1] = make_float2(y.z, y.w);
+    for (int c = 0; c < C; ++c) {
+        float2 x[4];
+        Widen<QT>::lds8(rec + DK + L.col(c), x);
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+            q2[4 * c + t] = x[t];
     }
 }
+
+// ---------------------------------------------------------------------------
+// Tree walks
+// ---------------------------------------------------------------------------
 
 // Shared-memory tree arrays (tree mode), each [N] int:
 //   par | ord | meta | rstart | nch | sz | lt | off | last | path scratch [warps][N]
@@ -307,8 +397,8 @@ struct TreeView {
 // node: O(depth) to walk up its root path, O(N) to rank it among its
 // siblings).  Siblings are visited by increasing (subtree size, index).
 // Returns false on every thread if the tree is malformed.  K: shared-memory
-// stack slots; reload: parents come from node_states instead of slots.
-static __device__ bool build_walk(const int32_t* prow, int N, int K, bool reload, const TreeView& T)
+// stack slots.
+static __device__ bool build_walk(const int32_t* prow, int N, int K, const TreeView& T)
 {
     const int tid = threadIdx.x, nthr = blockDim.x;
     bool bad = false;
@@ -369,8 +459,6 @@ static __device__ bool build_walk(const int32_t* prow, int N, int K, bool reload
             src = kSrcRoot;
         } else if (pp == T.ord[pos - 1]) {
             src = kSrcCont;
-        } else if (reload) {
-            src = kSrcReload;
         } else if (T.lt[pp] < K) {
             src = kSrcSlot;
             ld = T.lt[pp];
@@ -383,7 +471,7 @@ static __device__ bool build_walk(const int32_t* prow, int N, int K, bool reload
                 x = T.par[x];
             start = x;
         }
-        if (!reload && T.nch[n] >= 2 && T.lt[n] < K)
+        if (T.nch[n] >= 2 && T.lt[n] < K)
             save = T.lt[n] + 1;
         T.meta[pos] = n | (src << 16) | (save << 19) | (ld << 24);
         T.rstart[pos] = start;
@@ -394,7 +482,6 @@ static __device__ bool build_walk(const int32_t* prow, int N, int K, bool reload
 
 // Tree metadata held in shared memory (any N).
 struct SmemTree {
-    static constexpr bool kIndex = false;
     TreeView T;
     int N, warp;
     __device__ __forceinline__ int meta(int pos) const { return T.meta[pos]; }
@@ -416,18 +503,11 @@ struct SmemTree {
     }
 };
 
-// Walk of a tree of N <= 32 nodes as built in one warp's registers: lane n
-// holds node n's parent and ancestor-or-self bitmask, lane p walk position
-// p's metadata.
-struct WarpTree {
-    int par_l, meta_l, rstart_l;
-    unsigned mask_l;
-};
-
-// The same walk published in shared memory for every warp of the CTA:
-// [meta | rstart | par | mask] x 32.
+// Walk of a tree of N <= 32 nodes as built by one warp (build_warp_walk) in
+// shared memory: [meta | rstart | par | mask] x 32, followed by the
+// builder's scratch.
+constexpr int kWarpTreeInts = 10 * 32;
 struct MaskTree {
-    static constexpr bool kIndex = false;
     const int* a;
     __device__ __forceinline__ int meta(int pos) const { return a[pos]; }
     __device__ __forceinline__ int rstart(int pos) const { return a[32 + pos]; }
@@ -452,7 +532,6 @@ struct MaskTree {
 // not the previous node is re-read from node_states, prefetched one node
 // ahead.  par: the tree's parent array in shared memory.
 struct IndexTree {
-    static constexpr bool kIndex = true;
     const int* par;
     __device__ __forceinline__ int meta(int pos) const
     {
@@ -467,19 +546,35 @@ struct IndexTree {
     }
 };
 
-// Builds the walk of a tree of N <= 32 nodes in the registers of the calling
-// warp (same order and metadata as build_walk, no shared memory, no block
-// barrier).  Returns false if the tree is malformed (the same on every lane).
-static __device__ bool build_warp_walk(const int32_t* prow, int N, int K, bool reload, WarpTree& W)
+// Builds the walk of a tree of N <= 32 nodes with the calling warp, lane j
+// standing for node j, into ws[kWarpTreeInts] (same order and metadata as
+// build_walk).  Ancestor masks and path sums use pointer jumping (5 rounds
+// cover depth < 32), descendant masks a transpose of the 32 x 32 bit matrix
+// of ancestor masks, siblings __match_any_sync; per-node values are exchanged
+// through ws.  Returns false if the tree is malformed (the same on every
+// lane).
+static __device__ bool build_warp_walk(const int32_t* prow, int N, int K, int* ws)
 {
     const unsigned full = 0xffffffffu;
     const int lane = threadIdx.x & 31;
+    int* const w_meta = ws;
+    int* const w_rstart = ws + 32;
+    int* const w_par = ws + 64;
+    int* const w_mask = ws + 96;
+    int* const w_sz = ws + 128;
+    int* const w_ord = ws + 160;
+    int* const w_lt = ws + 192;
+    int* const w_nch = ws + 224;
+    int* const w_kids = ws + 256;
     const bool valid = lane < N;
     const int par = valid ? __ldg(prow + lane) : -1;
     const bool bad = valid && ((lane == 0) ? par != -1 : (par < 0 || par >= lane));
     if (__any_sync(full, bad))
         return false;
-    // ancestor-or-self bitmask by pointer jumping (depth < 32)
+    w_par[lane] = par;
+    w_kids[lane] = 0;
+    w_ord[lane] = 0;
+    // ancestor-or-self mask
     unsigned mask = valid ? (1u << lane) : 0u;
     int jump = valid ? par : -1;
 #pragma unroll
@@ -491,64 +586,79 @@ static __device__ bool build_warp_walk(const int32_t* prow, int N, int K, bool r
             jump = pj;
         }
     }
-    // child counts and subtree sizes
-    int nch = 0, sz = 0;
+    // descendant-or-self mask (column `lane` of the mask matrix) and subtree
+    // size: swap the off-diagonal blocks at widths 16, 8, 4, 2, 1
+    unsigned desc = mask;
 #pragma unroll
-    for (int k = 0; k < 32; ++k) {
-        const unsigned bp = __ballot_sync(full, valid && par == k);
-        const unsigned bm = __ballot_sync(full, (mask >> k) & 1u);
-        if (lane == k) {
-            nch = __popc(bp);
-            sz = __popc(bm);
-        }
+    for (int sh = 16, k = 0; sh >= 1; sh >>= 1, ++k) {
+        const unsigned lo = k == 0 ? 0x0000ffffu
+                          : k == 1 ? 0x00ff00ffu
+                          : k == 2 ? 0x0f0f0f0fu
+                          : k == 3 ? 0x33333333u
+                                   : 0x55555555u;
+        const unsigned y = __shfl_xor_sync(full, desc, sh);
+        desc = (lane & sh) ? ((desc & ~lo) | ((y & ~lo) >> sh)) : ((desc & lo) | ((y & lo) << sh));
     }
-    // offset among siblings visited by increasing (subtree size, index), and
-    // whether the node is its parent's last-visited child
-    int off = (valid && lane > 0) ? 1 : 0, last = 1;
-#pragma unroll
-    for (int s = 0; s < 32; ++s) {
-        const int ps = __shfl_sync(full, par, s);
-        const int zs = __shfl_sync(full, sz, s);
-        if (valid && lane > 0 && s < N && s != lane && ps == par) {
-            if (zs < sz || (zs == sz && s < lane))
-                off += zs;
+    const int sz = __popc(desc);
+    w_mask[lane] = static_cast<int>(mask);
+    w_sz[lane] = sz;
+    // siblings (lanes with the same parent) and child sets
+    const unsigned sib = __match_any_sync(full, valid ? par : 64 + lane);
+    __syncwarp();
+    if (valid && lane > 0)
+        w_kids[par] = static_cast<int>(sib);  // every child writes the same set
+    // offset among the siblings visited by increasing (subtree size, index),
+    // and whether the node is its parent's last-visited child
+    int off = 0, last = 1;
+    if (valid && lane > 0) {
+        off = 1;
+        unsigned bits = sib & ~(1u << lane);
+        while (bits) {
+            const int t = __ffs(bits) - 1;
+            bits &= bits - 1;
+            const int zt = w_sz[t];
+            if (zt < sz || (zt == sz && t < lane))
+                off += zt;
             else
                 last = 0;
         }
     }
-    // preorder position and stack slot: sums along the root path
-    int pos = 0, lt = 0;
+    __syncwarp();
+    const int nch = __popc(static_cast<unsigned>(w_kids[lane]));
+    // preorder position and stack slot: sums of (off, not-last) along the
+    // root path, packed in one int
+    int acc = (valid && lane > 0) ? (off | ((last ? 0 : 1) << 16)) : 0;
+    jump = valid ? par : -1;
 #pragma unroll
-    for (int x = 1; x < 32; ++x) {
-        const int ox = __shfl_sync(full, off, x);
-        const int lx = __shfl_sync(full, last, x);
-        if ((mask >> x) & 1u) {
-            pos += ox;
-            lt += lx ? 0 : 1;
+    for (int it = 0; it < 5; ++it) {
+        const int pa = __shfl_sync(full, acc, jump & 31);
+        const int pj = __shfl_sync(full, jump, jump & 31);
+        if (jump >= 0) {
+            acc += pa;
+            jump = pj;
         }
     }
-    // lane p: the node at walk position p
-    int ord = 0;
-#pragma unroll
-    for (int k = 0; k < 32; ++k) {
-        const unsigned bb = __ballot_sync(full, valid && pos == k);
-        if (lane == k && bb)
-            ord = __ffs(bb) - 1;
-    }
-    const int pp = __shfl_sync(full, par, ord);
-    const int prev = __shfl_sync(full, ord, (lane + 31) & 31);
-    const int lt_pp = __shfl_sync(full, lt, pp & 31);
-    const int lt_n = __shfl_sync(full, lt, ord);
-    const int nch_n = __shfl_sync(full, nch, ord);
-    const unsigned mask_pp = __shfl_sync(full, mask, pp & 31);
+    const int pos = acc & 0xffff, lt = acc >> 16;
+    __syncwarp();
+    if (valid)
+        w_ord[pos] = lane;  // a permutation of [0, N) for a valid tree
+    w_lt[lane] = lt;
+    w_nch[lane] = nch;
     const unsigned cand_all = __ballot_sync(full, valid && nch >= 2 && lt == K - 1);
+    __syncwarp();
+    // lane p: the metadata of walk position p
+    const int ord = w_ord[lane];
+    const int pp = w_par[ord];
+    const int prev = lane > 0 ? w_ord[lane - 1] : -1;
+    const int lt_pp = pp >= 0 ? w_lt[pp] : 0;
+    const int lt_n = w_lt[ord];
+    const int nch_n = w_nch[ord];
+    const unsigned mask_pp = pp >= 0 ? static_cast<unsigned>(w_mask[pp]) : 0u;
     int src, ld = 0, start = -1, save = 0;
     if (lane == 0) {
         src = kSrcRoot;
     } else if (pp == prev) {
         src = kSrcCont;
-    } else if (reload) {
-        src = kSrcReload;
     } else if (lt_pp < K) {
         src = kSrcSlot;
         ld = lt_pp;
@@ -559,149 +669,109 @@ static __device__ bool build_warp_walk(const int32_t* prow, int N, int K, bool r
         const unsigned cand = cand_all & mask_pp & ~(1u << (pp & 31));
         start = cand ? 31 - __clz(cand) : -1;
     }
-    if (!reload && nch_n >= 2 && lt_n < K)
+    if (nch_n >= 2 && lt_n < K)
         save = lt_n + 1;
-    W.par_l = par;
-    W.mask_l = mask;
-    W.meta_l = ord | (src << 16) | (save << 19) | (ld << 24);
-    W.rstart_l = start;
+    w_meta[lane] = ord | (src << 16) | (save << 19) | (ld << 24);
+    w_rstart[lane] = start;
     return true;
 }
 
 // Makes S the exact f32 state of node pp, the parent of the node at a walk
-// position whose metadata says the state is not already in registers.
-// fetch(y, k2, vr, a, beta) supplies node y's inputs for the recompute path.
-template <int DK, int RL, class Tree, class Fetch>
-__device__ __forceinline__ void source_parent(StateT<RL>& S, int m, int pp, int start, const KParams& p,
-                                              const Tree& tree, const float* slotbuf,
-                                              const float* sin_head, int b, int h, int row0,
-                                              const LaneMap<DK, RL>& L, Fetch fetch)
+// position whose metadata says the state is not already in registers: a
+// stack slot, or recomputation from the deepest saved ancestor (start; -1:
+// from state_in).  fetch(y, k2, vr, a, beta) supplies node y's inputs.
+template <int DK, int C, int RL, class Tree, class Fetch>
+__device__ __forceinline__ void source_parent(StateT<C, RL>& S, int m, int pp, int start, const KParams& p,
+                                              const Tree& tree, const float* lane_slot, int slot_floats,
+                                              int stride, const float* sin_lane, Fetch fetch)
 {
-    constexpr int LR = LaneMap<DK, RL>::LR;
+    constexpr int LR = LaneMap<DK, C, RL>::LR;
     const int src = meta_src(m);
-    if (src == kSrcReload) {
-        const float* ns = static_cast<const float*>(p.node_states) +
-                          (((size_t)b * p.N + pp) * p.Hv + h) * p.dv * DK + (size_t)row0 * DK;
-        load_state<DK, RL>(S, ns, L);
-    } else if (src == kSrcSlot) {
-        load_state<DK, RL>(S, slotbuf + (size_t)meta_load(m) * p.rows * DK, L);
+    if (src == kSrcSlot) {
+        load_slot<C, RL>(S, lane_slot + (size_t)meta_load(m) * slot_floats, stride);
     } else if (src == kSrcRecompute) {
         if (start >= 0)
-            load_state<DK, RL>(S, slotbuf + (size_t)(p.slots - 1) * p.rows * DK, L);
+            load_slot<C, RL>(S, lane_slot + (size_t)(p.slots - 1) * slot_floats, stride);
         else
-            load_state<DK, RL>(S, sin_head, L);
+            load_rows<DK, C, RL>(S, sin_lane);
         tree.for_path(pp, start, [&](int y) {
-            float2 k2[8];
+            float2 k2[4 * C];
             float vr[RL];
             float a, be;
             fetch(y, k2, vr, a, be);
-            gdn_update<LR, RL>(S, k2, vr, a, be);
+            gdn_update<LR, C, RL>(S, k2, vr, a, be);
         });
     }
 }
 
-// Where this lane's rows of node n's state and output live: one 64-bit base
-// per node plus per-lane 32-bit offsets computed once.
-template <int DK, int RL, typename ST>
-struct OutPtrs {
-    ST* ns_head;          // node_states of (b, h) at node 0
-    size_t ns_stride;     // elements between consecutive nodes' states
-    float* out_head;      // out of (b, h) at node 0, row row0
-    size_t out_stride;    // elements between consecutive nodes' outputs
-    uint32_t ns_off[RL];  // (row0 + row) * DK + 4 * cl
-    uint32_t out_off[RL];
-    __device__ __forceinline__ OutPtrs(const KParams& p, int b, int h, int row0, const LaneMap<DK, RL>& L)
-    {
-        const int NS = p.persist_last ? 1 : p.N;
-        ns_stride = (size_t)p.Hv * p.dv * DK;
-        ns_head = static_cast<ST*>(p.node_states) + (size_t)b * NS * ns_stride + (size_t)h * p.dv * DK;
-        out_stride = (size_t)p.Hv * p.dv;
-        out_head = p.out + (size_t)b * p.N * out_stride + (size_t)h * p.dv + row0;
-#pragma unroll
-        for (int r = 0; r < RL; ++r) {
-            ns_off[r] = (uint32_t)((row0 + L.rloc[r]) * DK + 4 * L.cl);
-            out_off[r] = (uint32_t)L.rloc[r];
-        }
-    }
-};
-
-template <int DK, int RL, typename ST>
-__device__ __forceinline__ void persist(const StateT<RL>& S, int n, int pos, const KParams& p,
-                                        const OutPtrs<DK, RL, ST>& P)
-{
-    constexpr int LR = DK / kColsPerLane;
-    if (p.persist_last && pos != p.N - 1)
-        return;
-    ST* node = P.ns_head + (size_t)(p.persist_last ? 0 : n) * P.ns_stride;
-#pragma unroll
-    for (int r = 0; r < RL; ++r) {
-        ST* row = node + P.ns_off[r];
-#pragma unroll
-        for (int m = 0; m < 4; ++m)
-            Persist<ST>::store(row + 4 * m * LR, S.s[r][2 * m], S.s[r][2 * m + 1]);
-    }
-}
+enum : int { kTreeChain = 0, kTreeWarp = 1, kTreeSmem = 2, kTreeIndex = 3 };
 
 // The walk over positions [0, N): per position, find the parent state,
-// update, persist, and batch the outputs.  The context supplies each
-// position's widened record, gate and decay (ctx.rec, ctx.ab), the walk's
-// input fetcher for recomputation, and the ring handshakes (ctx.begin /
-// ctx.end; trivial when everything is staged).
-template <int DK, int RL, typename ST, bool CHAIN, class Tree, class Ctx>
-__device__ __forceinline__ void walk(StateT<RL>& S, const KParams& p, const Tree& tree,
-                                     float* slotbuf, const float* sin_head, int b, int h, int row0,
-                                     const LaneMap<DK, RL>& L, Ctx& ctx)
+// update, write the output and persist.  The context supplies each
+// position's descriptor and record (ctx.desc, ctx.rec), the input fetcher
+// for recomputation, and the ring handshakes (ctx.begin / ctx.end; trivial
+// when everything is staged).
+template <int DK, int C, int RL, typename QT, typename ST, int TREE, class Tree, class Ctx>
+__device__ __forceinline__ void walk(StateT<C, RL>& S, const KParams& p, const Tree& tree, float* lane_slot,
+                                     const float* sin_lane, int b, int h, int row0,
+                                     const LaneMap<DK, C, RL>& L, Ctx& ctx)
 {
-    constexpr int LR = LaneMap<DK, RL>::LR;
+    using LM = LaneMap<DK, C, RL>;
+    constexpr bool CHAIN = TREE == kTreeChain;
+    constexpr bool INDEX = TREE == kTreeIndex;
     const int N = p.N;
-    const OutPtrs<DK, RL, ST> P(p, b, h, row0, L);
-    StateT<RL> Sn;  // index order: the next position's parent state, prefetched
-    const float* nsf = static_cast<const float*>(p.node_states) +
-                       ((size_t)b * p.N * p.Hv + h) * p.dv * DK + (size_t)row0 * DK;
-    const size_t node_stride = (size_t)p.Hv * p.dv * DK;
+    const int NS = p.persist_last ? 1 : N;
+    const size_t ns_stride = (size_t)p.Hv * p.dv * DK;  // elements between nodes' states
+    ST* const ns_lane = static_cast<ST*>(p.node_states) + (size_t)b * NS * ns_stride +
+                        (size_t)h * p.dv * DK + (size_t)row0 * DK + L.tile_offset();
+    const size_t out_stride = (size_t)p.Hv * p.dv;
+    float* const out_lane = p.out + (size_t)b * N * out_stride + (size_t)h * p.dv + row0 + L.row;
+    const int slot_floats = p.rows * DK;
+    const int stride = p.warps * 32 * 4;
+    StateT<C, RL> Sn;  // index order: the next position's parent state, prefetched
     for (int pos = 0; pos < N; ++pos) {
         if (!ctx.begin(pos))
             return;
-        int n = pos, save = -1;
+        const PosDesc d = ctx.desc(pos);
+        const int n = CHAIN ? pos : d.i.x;
         bool next_reload = false;
-        if constexpr (Tree::kIndex) {
+        if constexpr (INDEX) {
             // issue the loads of the next position's parent state now; it was
             // persisted by this thread at an earlier position
             if (pos + 1 < N) {
                 const int pn = tree.parent(pos + 1);
                 next_reload = pn != pos;
                 if (next_reload)
-                    load_state<DK, RL>(Sn, nsf + (size_t)pn * node_stride, L);
+                    load_rows<DK, C, RL>(Sn, reinterpret_cast<const float*>(ns_lane) + (size_t)pn * ns_stride);
             }
         } else if constexpr (!CHAIN) {
-            const int m = tree.meta(pos);
-            n = meta_node(m);
-            save = meta_save(m);
-            const int rs = tree.rstart(pos);
-            const int pp = tree.parent(n);
-            if (meta_src(m) != kSrcCont && meta_src(m) != kSrcRoot)
-                source_parent<DK, RL>(S, m, pp, rs, p, tree, slotbuf, sin_head, b, h, row0, L,
-                                      ctx.fetcher());
+            const int src = meta_src(d.i.y);
+            if (src != kSrcCont && src != kSrcRoot)
+                source_parent<DK, C, RL>(S, d.i.y, d.i.w, d.i.z, p, tree, lane_slot, slot_floats, stride,
+                                         sin_lane, ctx.fetcher());
         }
-        const auto* rec = ctx.rec(pos, n);
-        float2 k2[8], q2[8];
+        const QT* rec = ctx.rec(pos, n);
+        float2 k2[4 * C], q2[4 * C];
         float vr[RL];
-        load_k<DK, RL>(rec, L, k2, vr);
-        load_q<DK, RL>(rec, L, q2);
-        float a, be, kq;
-        ctx.ab(pos, n, a, be, kq);
+        load_k<DK, C, RL, QT>(rec, L, k2, vr);
+        load_q<DK, C, RL, QT>(rec, L, q2);
+        const float a = d.f.x;
         float pq[RL], u[RL];
-        gdn_step<LR, RL, true>(S, k2, q2, vr, a, be, pq, u);
+        gdn_step<LM::LR, C, RL, true>(S, k2, q2, vr, a, d.f.y, pq, u);
         if (L.cl == 0) {
-            float* o = P.out_head + (size_t)n * P.out_stride;
+            float* o = out_lane + (size_t)n * out_stride;
 #pragma unroll
             for (int r = 0; r < RL; ++r)
-                o[P.out_off[r]] = __fmul_rn(p.scale, __fmaf_rn(u[r], kq, __fmul_rn(a, pq[r])));
+                o[r * LM::RG] = __fmul_rn(p.scale, __fmaf_rn(u[r], d.f.z, __fmul_rn(a, pq[r])));
         }
-        persist<DK, RL, ST>(S, n, pos, p, P);
-        if (save >= 0)
-            save_state<DK, RL>(S, slotbuf + (size_t)save * p.rows * DK, L);
-        if constexpr (Tree::kIndex) {
+        if (!p.persist_last || pos == N - 1)
+            persist<DK, C, RL, ST>(S, ns_lane + (size_t)(p.persist_last ? 0 : n) * ns_stride);
+        if constexpr (!CHAIN && !INDEX) {
+            const int save = meta_save(d.i.y);
+            if (save >= 0)
+                save_slot<C, RL>(S, lane_slot + (size_t)save * slot_floats, stride);
+        }
+        if constexpr (INDEX) {
             if (next_reload)
                 S = Sn;
         }
@@ -709,64 +779,52 @@ __device__ __forceinline__ void walk(StateT<RL>& S, const KParams& p, const Tree
     }
 }
 
-// ---------------------------------------------------------------------------
-// Staged kernel: every node's inputs copied into shared memory at start
-// ---------------------------------------------------------------------------
-
-// Staged records: RT = float (widened once) or the raw input type.
-template <int DK, int RL, typename RT>
-struct StagedFetch {
-    const RT* recs;
-    const float* ab;
-    uint32_t rec_elems;
-    int N;
-    LaneMap<DK, RL> L;
-    __device__ __forceinline__ void operator()(int y, float2 (&k2)[8], float (&vr)[RL], float& a,
-                                               float& be) const
-    {
-        load_k<DK, RL>(recs + (size_t)y * rec_elems, L, k2, vr);
-        a = ab[y];
-        be = ab[N + y];
-    }
-};
-
-template <int DK, int RL, typename RT>
-struct StagedCtx {
-    const RT* recs;
-    const float* ab_;
-    uint32_t rec_elems;
-    int N;
-    LaneMap<DK, RL> L;
-    __device__ __forceinline__ bool begin(int) { return true; }
-    __device__ __forceinline__ void end(int) {}
-    __device__ __forceinline__ const RT* rec(int, int n) const
-    {
-        return recs + (size_t)n * rec_elems;
-    }
-    __device__ __forceinline__ void ab(int, int n, float& a, float& be, float& kq) const
-    {
-        a = ab_[n];
-        be = ab_[N + n];
-        kq = ab_[2 * N + n];
-    }
-    __device__ __forceinline__ StagedFetch<DK, RL, RT> fetcher() const
-    {
-        return StagedFetch<DK, RL, RT>{recs, ab_, rec_elems, N, L};
-    }
-};
-
-// Tree policy of the staged kernel: chain, walk in warp registers (N <= 32)
-// or walk in shared memory.
-enum : int { kTreeChain = 0, kTreeWarp = 1, kTreeSmem = 2, kTreeIndex = 3 };
-
+// Chain mode: position p is node p.
 struct NoTree {
-    static constexpr bool kIndex = false;
-    __device__ __forceinline__ int meta(int pos) const { return pos; }
+    __device__ __forceinline__ int meta(int pos) const { return pos | ((pos == 0 ? kSrcRoot : kSrcCont) << 16); }
     __device__ __forceinline__ int rstart(int) const { return -1; }
     __device__ __forceinline__ int parent(int n) const { return n - 1; }
     template <class F>
     __device__ __forceinline__ void for_path(int, int, F&&) const
     {
+    }
+};
+
+// ---------------------------------------------------------------------------
+// Staged kernel: every node's record copied into shared memory at start
+// ---------------------------------------------------------------------------
+
+template <int DK, int C, int RL, typename QT>
+struct StagedFetch {
+    const QT* recs;
+    const float* ab;  // a | beta, by node
+    uint32_t rec_elems;
+    int N;
+    LaneMap<DK, C, RL> L;
+    __device__ __forceinline__ void operator()(int y, float2 (&k2)[4 * C], float (&vr)[RL], float& a,
+                                               float& be) const
+    {
+        load_k<DK, C, RL, QT>(recs + (size_t)y * rec_elems, L, k2, vr);
+        a = ab[y];
+        be = ab[N + y];
+    }
+};
+
+template <int DK, int C, int RL, typename QT>
+struct StagedCtx {
+    const QT* recs;
+    const PosDesc* desc_;
+    const float* ab;
+    uint32_t rec_elems;
+    int N;
+    LaneMap<DK, C, RL> L;
+    __device__ __forceinline__ bool begin(int) { return true; }
+    __device__ __forceinline__ void end(int) {}
+    __device__ __forceinline__ PosDesc desc(int pos) const { return desc_[pos]; }
+    __device__ __forceinline__ const QT* rec(int, int n) const { return recs + (size_t)n * rec_elems; }
+    __device__ __forceinline__ StagedFetch<DK, C, RL, QT> fetcher() const
+    {
+        return StagedFetch<DK, C, RL, QT>{recs, ab, rec_elems, N, L};
     }
 };
 
@@ -776,14 +834,58 @@ __device__ __forceinline__ void cp_async16(void* dst_smem, const void* src_gmem)
                  : "memory");
 }
 
-template <int DK, int RL, typename QT, typename ST, int TREE>
+__device__ __forceinline__ void cp_async4(void* dst_smem, const void* src_gmem)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(dst_smem)), "l"(src_gmem)
+                 : "memory");
+}
+
+// Prologue pass of the staged kernel over walk positions, four per warp and
+// pass: converts g to a = exp(g) in place (ab holds g | beta by node), and
+// writes each position's descriptor with k . q of its node.
+template <int DK, typename QT, class Tree>
+__device__ __forceinline__ void write_descs(const Tree& tree, const unsigned char* raw, uint32_t raw_bytes,
+                                            float* ab, PosDesc* desc, int N)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+    for (int p0 = 4 * warp; p0 < N; p0 += 4 * nwarps) {
+        const int pos = min(p0 + (lane >> 3), N - 1);
+        const int m = tree.meta(pos);
+        const int n = meta_node(m);
+        const float kq = node_kq8<DK, QT>(reinterpret_cast<const QT*>(raw + (size_t)n * raw_bytes), lane & 7);
+        if ((lane & 7) == 0 && p0 + (lane >> 3) < N) {
+            const float a = gdn_gate(ab[n]);
+            ab[n] = a;
+            PosDesc d;
+            d.i = make_int4(n, m, tree.rstart(pos), tree.parent(n));
+            d.f = make_float4(a, ab[N + n], kq, 0.f);
+            desc[pos] = d;
+        }
+    }
+}
+
+template <int DK, int C, int RL, typename QT, typename ST, int TREE, class Tree>
+__device__ __forceinline__ void staged_finish(StateT<C, RL>& S, const KParams& p, const Tree& tree,
+                                              const unsigned char* raw, float* ab, PosDesc* desc,
+                                              float* slotbuf, const float* sin_lane, int b, int h, int row0,
+                                              const LaneMap<DK, C, RL>& L)
+{
+    write_descs<DK, QT>(tree, raw, p.raw_bytes, ab, desc, p.N);
+    __syncthreads();
+    const uint32_t rec_elems = p.raw_bytes / (uint32_t)sizeof(QT);
+    StagedCtx<DK, C, RL, QT> ctx{reinterpret_cast<const QT*>(raw), desc, ab, rec_elems, p.N, L};
+    float* lane_slot = slotbuf + 4 * threadIdx.x;
+    walk<DK, C, RL, QT, ST, TREE>(S, p, tree, lane_slot, sin_lane, b, h, row0, L, ctx);
+}
+
+template <int DK, int C, int RL, typename QT, typename ST, int TREE>
 __global__ void __launch_bounds__(kMaxWarps * 32) gdn_verify_staged(const KParams p)
 {
     constexpr int EPC = 16 / sizeof(QT);  // elements per 16-byte chunk
     constexpr int QKCH = DK / EPC;        // chunks per k (or q) row
     extern __shared__ __align__(16) unsigned char smem[];
     unsigned char* raw = smem + p.off_raw;
-    float* recs = reinterpret_cast<float*>(smem + p.off_rec);
+    PosDesc* desc = reinterpret_cast<PosDesc*>(smem + p.off_desc);
     float* ab = reinterpret_cast<float*>(smem + p.off_ab);
     float* slotbuf = reinterpret_cast<float*>(smem + p.off_slots);
     int* tsm = reinterpret_cast<int*>(smem + p.off_tree);
@@ -798,8 +900,39 @@ __global__ void __launch_bounds__(kMaxWarps * 32) gdn_verify_staged(const KParam
     // Everything that reads q, k, v, g, beta waits for the preceding kernel;
     // with GDN_FLAG_EARLY_TREE the tree and the root's parent state are read
     // before that (they were written before the preceding kernel started).
-    if (!p.early_tree)
+    // Every node's raw k row, q row and v slice, and its g and beta, are
+    // copied to shared memory asynchronously (warp w copies nodes w,
+    // w + warps, ...); the tree work overlaps the copies unless it already ran
+    // before the wait.
+    const int per_node = p.raw_bytes / 16;  // 16-byte chunks per node
+    auto stage = [&]() {
+        const QT* kg = static_cast<const QT*>(p.k);
+        const QT* qg = static_cast<const QT*>(p.q);
+        const QT* vg = static_cast<const QT*>(p.v);
+        for (int n = warp; n < N; n += nwarps) {
+            const size_t node = (size_t)b * N + n;
+            const QT* krow = kg + (node * p.Hk + hk) * DK;
+            const QT* qrow = qg + (node * p.Hk + hk) * DK;
+            const QT* vrow = vg + (node * p.Hv + h) * p.dv + row0;
+            unsigned char* dst = raw + (size_t)n * p.raw_bytes;
+            for (int c = lane; c < per_node; c += 32) {
+                const QT* src = c < QKCH ? krow + c * EPC
+                                         : (c < 2 * QKCH ? qrow + (c - QKCH) * EPC
+                                                         : vrow + (c - 2 * QKCH) * EPC);
+                cp_async16(dst + 16 * c, src);
+            }
+        }
+        for (int n = tid; n < N; n += blockDim.x) {
+            const size_t gi = ((size_t)b * N + n) * p.Hv + h;
+            cp_async4(ab + n, p.g + gi);
+            cp_async4(ab + N + n, p.beta + gi);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    if (!p.early_tree) {
         pdl_wait_then_release();
+        stage();
+    }
 
     // 1. the parent array (index order keeps it in shared memory; chain
     //    validation only checks it)
@@ -817,59 +950,25 @@ __global__ void __launch_bounds__(kMaxWarps * 32) gdn_verify_staged(const KParam
         }
     }
     // 2. the root's parent state
-    const LaneMap<DK, RL> L(warp, lane);
-    const float* sin_head = p.state_in + ((size_t)b * p.Hv + h) * p.dv * DK + (size_t)row0 * DK;
-    StateT<RL> S;
-    load_state<DK, RL>(S, sin_head, L);
-    // 3. the walk: warp 0 builds it for trees of <= 32 nodes (the other warps
-    //    go on to the copies); all threads for larger trees
+    const LaneMap<DK, C, RL> L(warp, lane);
+    const float* sin_lane =
+        p.state_in + ((size_t)b * p.Hv + h) * p.dv * DK + (size_t)row0 * DK + L.tile_offset();
+    StateT<C, RL> S;
+    load_rows<DK, C, RL>(S, sin_lane);
+    // 3. the walk: warp 0 builds it for trees of <= 32 nodes; all threads for
+    //    larger trees
     const TreeView tv(tsm, N);
     if constexpr (TREE == kTreeWarp) {
-        if (warp == 0) {
-            WarpTree wt{};
-            if (build_warp_walk(prow, N, p.slots, p.reload != 0, wt)) {
-                tsm[lane] = wt.meta_l;
-                tsm[32 + lane] = wt.rstart_l;
-                tsm[64 + lane] = wt.par_l;
-                tsm[96 + lane] = static_cast<int>(wt.mask_l);
-            } else {
-                bad = true;
-            }
-        }
+        if (warp == 0 && !build_warp_walk(prow, N, p.slots, tsm))
+            bad = true;
     } else if constexpr (TREE == kTreeSmem) {
-        bad = !build_walk(prow, N, p.slots, p.reload != 0, tv);
+        bad = !build_walk(prow, N, p.slots, tv);
     }
-    if (p.early_tree)
+    if (p.early_tree) {
         pdl_wait_then_release();
-    // 4. every node's raw k row, q row and v slice -> shared memory (async);
-    //    warp w copies nodes w, w + warps, ...
-    const int per_node = p.raw_bytes / 16;  // 16-byte chunks per node
-    {
-        const QT* kg = static_cast<const QT*>(p.k);
-        const QT* qg = static_cast<const QT*>(p.q);
-        const QT* vg = static_cast<const QT*>(p.v);
-        for (int n = warp; n < N; n += nwarps) {
-            const size_t node = (size_t)b * N + n;
-            const QT* krow = kg + (node * p.Hk + hk) * DK;
-            const QT* qrow = qg + (node * p.Hk + hk) * DK;
-            const QT* vrow = vg + (node * p.Hv + h) * p.dv + row0;
-            unsigned char* dst = raw + (size_t)n * p.raw_bytes;
-            for (int c = lane; c < per_node; c += 32) {
-                const QT* src = c < QKCH ? krow + c * EPC
-                                         : (c < 2 * QKCH ? qrow + (c - QKCH) * EPC
-                                                         : vrow + (c - 2 * QKCH) * EPC);
-                cp_async16(dst + 16 * c, src);
-            }
-        }
-        asm volatile("cp.async.commit_group;" ::: "memory");
+        stage();
     }
-    // 5. gates
-    for (int n = tid; n < N; n += blockDim.x) {
-        const size_t gi = ((size_t)b * N + n) * p.Hv + h;
-        ab[n] = gdn_gate(__ldg(p.g + gi));
-        ab[N + n] = __ldg(p.beta + gi);
-    }
-    // 6. the copies target this CTA's shared memory: wait for them even when
+    // 4. the copies target this CTA's shared memory: wait for them even when
     //    the tree is rejected
     asm volatile("cp.async.wait_all;" ::: "memory");
     if (__syncthreads_or(bad)) {
@@ -877,46 +976,25 @@ __global__ void __launch_bounds__(kMaxWarps * 32) gdn_verify_staged(const KParam
             report_status(p.status, GDN_ERR_BAD_TREE);
         return;
     }
-    // 7. widen the raw records to f32 once (bf16 inputs, two rows per lane);
-    //    with one row per lane the node loop widens its own k, q, v instead
-    //    (small grids: the loop is store-bound and the prologue is not)
-    constexpr bool kWiden = sizeof(QT) == 2 && RL == 2;
-    using RT = typename std::conditional<kWiden, float, QT>::type;
-    if constexpr (kWiden) {
-        for (int n = warp; n < N; n += nwarps) {
-            const unsigned char* src = raw + (size_t)n * p.raw_bytes;
-            float* dst = recs + (size_t)n * p.rec_floats;
-            for (int c = lane; c < per_node; c += 32)
-                Widen<QT>::store(dst + 8 * c, *reinterpret_cast<const uint4*>(src + 16 * c));
-        }
-        __syncthreads();
-    }
-    const RT* rt = kWiden ? reinterpret_cast<const RT*>(recs) : reinterpret_cast<const RT*>(raw);
-    const uint32_t rt_elems = kWiden ? p.rec_floats : p.raw_bytes / (uint32_t)sizeof(QT);
-    // 8. k . q of every node (outputs read the pre-update state)
-    for (int n = warp; n < N; n += nwarps) {
-        const float kq = node_kq<DK, RT>(rt + (size_t)n * rt_elems, lane);
-        if (lane == 0)
-            ab[2 * N + n] = kq;
-    }
-    __syncthreads();
-
-    StagedCtx<DK, RL, RT> ctx{rt, ab, rt_elems, N, L};
+    // 5. descriptors, then the walk
     if constexpr (TREE == kTreeChain)
-        walk<DK, RL, ST, true>(S, p, NoTree{}, slotbuf, sin_head, b, h, row0, L, ctx);
+        staged_finish<DK, C, RL, QT, ST, TREE>(S, p, NoTree{}, raw, ab, desc, slotbuf, sin_lane, b, h, row0, L);
     else if constexpr (TREE == kTreeIndex)
-        walk<DK, RL, ST, false>(S, p, IndexTree{tsm}, slotbuf, sin_head, b, h, row0, L, ctx);
+        staged_finish<DK, C, RL, QT, ST, TREE>(S, p, IndexTree{tsm}, raw, ab, desc, slotbuf, sin_lane, b, h,
+                                               row0, L);
     else if constexpr (TREE == kTreeWarp)
-        walk<DK, RL, ST, false>(S, p, MaskTree{tsm}, slotbuf, sin_head, b, h, row0, L, ctx);
+        staged_finish<DK, C, RL, QT, ST, TREE>(S, p, MaskTree{tsm}, raw, ab, desc, slotbuf, sin_lane, b, h,
+                                               row0, L);
     else
-        walk<DK, RL, ST, false>(S, p, SmemTree{tv, N, warp}, slotbuf, sin_head, b, h, row0, L, ctx);
+        staged_finish<DK, C, RL, QT, ST, TREE>(S, p, SmemTree{tv, N, warp}, raw, ab, desc, slotbuf, sin_lane,
+                                               b, h, row0, L);
 }
 
 // ---------------------------------------------------------------------------
 // Ring kernel: a producer warp streams chunks of walk positions
 // ---------------------------------------------------------------------------
 
-template <int DK, int RL, typename QT>
+template <int DK, int C, int RL, typename QT>
 struct GlobalFetch {
     const QT* kg;
     const QT* vg;
@@ -924,39 +1002,44 @@ struct GlobalFetch {
     const float* beta;
     size_t bN;  // b * N
     int Hk, Hv, dv, hk, h, row0;
-    LaneMap<DK, RL> L;
-    __device__ __forceinline__ void operator()(int y, float2 (&k2)[8], float (&vr)[RL], float& a,
+    LaneMap<DK, C, RL> L;
+    __device__ __forceinline__ void operator()(int y, float2 (&k2)[4 * C], float (&vr)[RL], float& a,
                                                float& be) const
     {
+        using LM = LaneMap<DK, C, RL>;
         const size_t node = bN + y;
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const float4 x = Widen<QT>::load4(kg + (node * Hk + hk) * DK + L.col(m));
-            k2[2 * m] = make_float2(x.x, x.y);
-            k2[2 * m + 1] = make_float2(x.z, x.w);
+        for (int c = 0; c < C; ++c) {
+            float2 x[4];
+            Widen<QT>::ldg8(kg + (node * Hk + hk) * DK + L.col(c), x);
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+                k2[4 * c + t] = x[t];
         }
 #pragma unroll
         for (int r = 0; r < RL; ++r)
-            vr[r] = Widen<QT>::load1(vg + (node * Hv + h) * dv + row0 + L.rloc[r]);
+            vr[r] = Widen<QT>::load1(vg + (node * Hv + h) * dv + row0 + L.row + r * LM::RG);
         const size_t gi = node * Hv + h;
         a = gdn_gate(__ldg(g + gi));
         be = __ldg(beta + gi);
     }
 };
 
-template <int DK, int RL, typename QT>
+// A ring slot: kChunk records (raw_bytes each) then kChunk descriptors.
+template <int DK, int C, int RL, typename QT>
 struct RingCtx {
     uint64_t* full;
     uint64_t* empty;
-    const float* ring;  // kRing slots of [kChunk records | a | beta | k.q, kChunk each]
-    uint32_t rec_floats;
-    uint32_t slot_floats;
+    const unsigned char* ring;
+    uint32_t raw_bytes;
+    uint32_t slot_bytes;
+    uint32_t desc_off;  // offset of the descriptors inside a slot
     int32_t* status;
     int lane;
-    GlobalFetch<DK, RL, QT> gf;
-    __device__ __forceinline__ const float* slot(int pos) const
+    GlobalFetch<DK, C, RL, QT> gf;
+    __device__ __forceinline__ const unsigned char* slot(int pos) const
     {
-        return ring + (size_t)((pos / kChunk) % kRing) * slot_floats;
+        return ring + (size_t)((pos / kChunk) % kRing) * slot_bytes;
     }
     __device__ __forceinline__ bool begin(int pos)
     {
@@ -979,36 +1062,34 @@ struct RingCtx {
                 mbar_arrive(&empty[(pos / kChunk) % kRing]);
         }
     }
-    __device__ __forceinline__ const float* rec(int pos, int) const
+    __device__ __forceinline__ PosDesc desc(int pos) const
     {
-        return slot(pos) + (size_t)(pos % kChunk) * rec_floats;
+        return reinterpret_cast<const PosDesc*>(slot(pos) + desc_off)[pos % kChunk];
     }
-    __device__ __forceinline__ void ab(int pos, int, float& a, float& be, float& kq) const
+    __device__ __forceinline__ const QT* rec(int pos, int) const
     {
-        const float* s = slot(pos) + (size_t)kChunk * rec_floats;
-        a = s[pos % kChunk];
-        be = s[kChunk + pos % kChunk];
-        kq = s[2 * kChunk + pos % kChunk];
+        return reinterpret_cast<const QT*>(slot(pos) + (size_t)(pos % kChunk) * raw_bytes);
     }
-    __device__ __forceinline__ GlobalFetch<DK, RL, QT> fetcher() const { return gf; }
+    __device__ __forceinline__ GlobalFetch<DK, C, RL, QT> fetcher() const { return gf; }
 };
 
-template <int DK, int RL, typename QT, typename ST, int TREE>
+template <int DK, int C, int RL, typename QT, typename ST, int TREE>
 __global__ void __launch_bounds__((kMaxWarps + 1) * 32) gdn_verify_ring(const KParams p)
 {
     constexpr bool CHAIN = TREE == kTreeChain;
     constexpr bool INDEX = TREE == kTreeIndex;
-    constexpr int EPC = 16 / sizeof(QT);            // elements per 16-byte chunk
-    constexpr int QKCH = DK / EPC;                  // chunks per k (or q) row
-    constexpr int RPW = LaneMap<DK, RL>::RPW;
-    constexpr int VCH_MAX = kMaxWarps * RPW / EPC;  // chunks per v slice, upper bound
+    constexpr int EPC = 16 / sizeof(QT);  // elements per 16-byte chunk
+    constexpr int QKCH = DK / EPC;        // chunks per k (or q) row
+    using LM = LaneMap<DK, C, RL>;
+    constexpr int VCH_MAX = (kMaxWarps * LM::RPW + EPC - 1) / EPC;  // chunks per v slice, upper bound
     constexpr int MAXT = (kChunk * (2 * QKCH + VCH_MAX) + 31) / 32;
 
     extern __shared__ __align__(16) unsigned char smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + kRing;
-    float* ring = reinterpret_cast<float*>(smem + p.off_rec);
-    const uint32_t slot_floats = kChunk * p.rec_floats + 3 * kChunk;
+    unsigned char* ring = smem + p.off_raw;
+    const uint32_t desc_off = (kChunk * p.raw_bytes + 15u) & ~15u;
+    const uint32_t slot_bytes = desc_off + kChunk * (uint32_t)sizeof(PosDesc);
     float* slotbuf = reinterpret_cast<float*>(smem + p.off_slots);
     const TreeView T(reinterpret_cast<int*>(smem + p.off_tree), p.N);
 
@@ -1047,7 +1128,7 @@ __global__ void __launch_bounds__((kMaxWarps + 1) * 32) gdn_verify_ring(const KP
         ok = !__syncthreads_or(bad);
     } else {
         __syncthreads();
-        ok = build_walk(p.parent + (size_t)b * N, N, p.slots, p.reload != 0, T);
+        ok = build_walk(p.parent + (size_t)b * N, N, p.slots, T);
     }
     if (p.early_tree)
         pdl_wait_then_release();
@@ -1068,7 +1149,8 @@ __global__ void __launch_bounds__((kMaxWarps + 1) * 32) gdn_verify_ring(const KP
                 report_status(p.status, kStatusTimeout);
                 return;
             }
-            float* base = ring + (size_t)s * slot_floats;
+            unsigned char* base = ring + (size_t)s * slot_bytes;
+            PosDesc* sdesc = reinterpret_cast<PosDesc*>(base + desc_off);
             const int p0 = c * kChunk;
             const int cnt = min(kChunk, N - p0);
             const int total = cnt * per_pos;
@@ -1091,26 +1173,52 @@ __global__ void __launch_bounds__((kMaxWarps + 1) * 32) gdn_verify_ring(const KP
                     regs[t] = __ldg(reinterpret_cast<const uint4*>(src));
                 }
             }
+            // lane i < cnt: position p0 + i's node, metadata and scalars
+            int dn = 0, dm = 0, drs = -1, dpp = -1;
+            float da = 0.f, dbe = 0.f;
             if (lane < cnt) {
                 const int pos = p0 + lane;
-                const int n = (CHAIN || INDEX) ? pos : meta_node(T.meta[pos]);
-                const size_t gi = ((size_t)b * N + n) * p.Hv + h;
-                base[kChunk * p.rec_floats + lane] = gdn_gate(__ldg(p.g + gi));
-                base[kChunk * p.rec_floats + kChunk + lane] = __ldg(p.beta + gi);
+                if constexpr (CHAIN) {
+                    dm = NoTree{}.meta(pos);
+                } else if constexpr (INDEX) {
+                    dm = IndexTree{T.par}.meta(pos);
+                } else {
+                    dm = T.meta[pos];
+                    drs = T.rstart[pos];
+                }
+                dn = meta_node(dm);
+                dpp = CHAIN ? dn - 1 : T.par[dn];
+                const size_t gi = ((size_t)b * N + dn) * p.Hv + h;
+                da = gdn_gate(__ldg(p.g + gi));
+                dbe = __ldg(p.beta + gi);
             }
 #pragma unroll
             for (int t = 0; t < MAXT; ++t) {
                 const int idx = lane + 32 * t;
                 if (idx < total) {
                     const int i = idx / per_pos, j = idx - i * per_pos;
-                    Widen<QT>::store(base + (size_t)i * p.rec_floats + j * EPC, regs[t]);
+                    *reinterpret_cast<uint4*>(base + (size_t)i * p.raw_bytes + 16 * j) = regs[t];
                 }
             }
             __syncwarp();
-            for (int i = 0; i < cnt; ++i) {
-                const float kq = node_kq<DK, float>(base + (size_t)i * p.rec_floats, lane);
-                if (lane == 0)
-                    base[kChunk * p.rec_floats + 2 * kChunk + i] = kq;
+            for (int i0 = 0; i0 < cnt; i0 += 4) {
+                const int gi = i0 + (lane >> 3);
+                const int i = min(gi, cnt - 1);
+                const float kq =
+                    node_kq8<DK, QT>(reinterpret_cast<const QT*>(base + (size_t)i * p.raw_bytes), lane & 7);
+                const int src_lane = i;
+                const int n = __shfl_sync(0xffffffffu, dn, src_lane);
+                const int m = __shfl_sync(0xffffffffu, dm, src_lane);
+                const int rs = __shfl_sync(0xffffffffu, drs, src_lane);
+                const int pp = __shfl_sync(0xffffffffu, dpp, src_lane);
+                const float a = __shfl_sync(0xffffffffu, da, src_lane);
+                const float be = __shfl_sync(0xffffffffu, dbe, src_lane);
+                if ((lane & 7) == 0 && gi < cnt) {
+                    PosDesc d;
+                    d.i = make_int4(n, m, rs, pp);
+                    d.f = make_float4(a, be, kq, 0.f);
+                    sdesc[i] = d;
+                }
             }
             mbar_arrive(&full[s]);
         }
@@ -1118,18 +1226,20 @@ __global__ void __launch_bounds__((kMaxWarps + 1) * 32) gdn_verify_ring(const KP
     }
 
     // ---------------------------------------------------------------- compute
-    const LaneMap<DK, RL> L(warp, lane);
-    const float* sin_head = p.state_in + ((size_t)b * p.Hv + h) * p.dv * DK + (size_t)row0 * DK;
-    StateT<RL> S;
-    load_state<DK, RL>(S, sin_head, L);
-    const GlobalFetch<DK, RL, QT> gf{kg, vg, p.g, p.beta, (size_t)b * N, p.Hk, p.Hv, p.dv, hk, h, row0, L};
-    RingCtx<DK, RL, QT> ctx{full, empty, ring, p.rec_floats, slot_floats, p.status, lane, gf};
+    const LM L(warp, lane);
+    const float* sin_lane =
+        p.state_in + ((size_t)b * p.Hv + h) * p.dv * DK + (size_t)row0 * DK + L.tile_offset();
+    StateT<C, RL> S;
+    load_rows<DK, C, RL>(S, sin_lane);
+    const GlobalFetch<DK, C, RL, QT> gf{kg, vg, p.g, p.beta, (size_t)b * N, p.Hk, p.Hv, p.dv, hk, h, row0, L};
+    RingCtx<DK, C, RL, QT> ctx{full, empty, ring, p.raw_bytes, slot_bytes, desc_off, p.status, lane, gf};
+    float* lane_slot = slotbuf + 4 * threadIdx.x;
     if constexpr (CHAIN)
-        walk<DK, RL, ST, true>(S, p, NoTree{}, slotbuf, sin_head, b, h, row0, L, ctx);
+        walk<DK, C, RL, QT, ST, TREE>(S, p, NoTree{}, lane_slot, sin_lane, b, h, row0, L, ctx);
     else if constexpr (INDEX)
-        walk<DK, RL, ST, false>(S, p, IndexTree{T.par}, slotbuf, sin_head, b, h, row0, L, ctx);
+        walk<DK, C, RL, QT, ST, TREE>(S, p, IndexTree{T.par}, lane_slot, sin_lane, b, h, row0, L, ctx);
     else
-        walk<DK, RL, ST, false>(S, p, SmemTree{T, N, warp}, slotbuf, sin_head, b, h, row0, L, ctx);
+        walk<DK, C, RL, QT, ST, TREE>(S, p, SmemTree{T, N, warp}, lane_slot, sin_lane, b, h, row0, L, ctx);
 }
 
 // ---------------------------------------------------------------------------
@@ -1161,84 +1271,81 @@ cudaError_t grant_smem(size_t smem)
     return cudaSuccess;
 }
 
-template <int DK, int RL, typename QT, typename ST, int TREE>
+template <int DK, int C, int RL, typename QT, typename ST, int TREE>
 cudaError_t launch_staged(const KParams& kp, const VerifyArgs& a, const VerifyGeom& geom,
                           cudaStream_t stream)
 {
     dim3 grid(geom.tiles, a.n_v_heads, a.batch);
-    cudaError_t e = grant_smem<gdn_verify_staged<DK, RL, QT, ST, TREE>>(geom.smem);
+    cudaError_t e = grant_smem<gdn_verify_staged<DK, C, RL, QT, ST, TREE>>(geom.smem);
     if (e != cudaSuccess)
         return e;
-    return launch_pdl(gdn_verify_staged<DK, RL, QT, ST, TREE>, grid, dim3(geom.warps * 32), geom.smem,
+    return launch_pdl(gdn_verify_staged<DK, C, RL, QT, ST, TREE>, grid, dim3(geom.warps * 32), geom.smem,
                       stream, kp);
 }
 
-template <int DK, int RL, typename QT, typename ST, int TREE>
+template <int DK, int C, int RL, typename QT, typename ST, int TREE>
 cudaError_t launch_ring(const KParams& kp, const VerifyArgs& a, const VerifyGeom& geom,
                         cudaStream_t stream)
 {
     dim3 grid(geom.tiles, a.n_v_heads, a.batch);
-    cudaError_t e = grant_smem<gdn_verify_ring<DK, RL, QT, ST, TREE>>(geom.smem);
+    cudaError_t e = grant_smem<gdn_verify_ring<DK, C, RL, QT, ST, TREE>>(geom.smem);
     if (e != cudaSuccess)
         return e;
-    return launch_pdl(gdn_verify_ring<DK, RL, QT, ST, TREE>, grid, dim3((geom.warps + 1) * 32),
+    return launch_pdl(gdn_verify_ring<DK, C, RL, QT, ST, TREE>, grid, dim3((geom.warps + 1) * 32),
                       geom.smem, stream, kp);
 }
 
-template <int DK, int RL, typename QT, typename ST, bool CHAIN>
+template <int DK, int C, int RL, typename QT, typename ST, bool CHAIN>
 cudaError_t launch_one(const KParams& kp, const VerifyArgs& a, const VerifyGeom& geom,
                        cudaStream_t stream)
 {
     if (geom.staged) {
         if (CHAIN)
-            return launch_staged<DK, RL, QT, ST, kTreeChain>(kp, a, geom, stream);
+            return launch_staged<DK, C, RL, QT, ST, kTreeChain>(kp, a, geom, stream);
         if (geom.reload)
-            return launch_staged<DK, RL, QT, ST, kTreeIndex>(kp, a, geom, stream);
+            return launch_staged<DK, C, RL, QT, ST, kTreeIndex>(kp, a, geom, stream);
         if (geom.warp_tree)
-            return launch_staged<DK, RL, QT, ST, kTreeWarp>(kp, a, geom, stream);
-        return launch_staged<DK, RL, QT, ST, kTreeSmem>(kp, a, geom, stream);
+            return launch_staged<DK, C, RL, QT, ST, kTreeWarp>(kp, a, geom, stream);
+        return launch_staged<DK, C, RL, QT, ST, kTreeSmem>(kp, a, geom, stream);
     }
     if (CHAIN)
-        return launch_ring<DK, RL, QT, ST, kTreeChain>(kp, a, geom, stream);
+        return launch_ring<DK, C, RL, QT, ST, kTreeChain>(kp, a, geom, stream);
     if (geom.reload)
-        return launch_ring<DK, RL, QT, ST, kTreeIndex>(kp, a, geom, stream);
-    return launch_ring<DK, RL, QT, ST, kTreeSmem>(kp, a, geom, stream);
+        return launch_ring<DK, C, RL, QT, ST, kTreeIndex>(kp, a, geom, stream);
+    return launch_ring<DK, C, RL, QT, ST, kTreeSmem>(kp, a, geom, stream);
 }
 
-template <int DK, int RL, typename QT, typename ST>
+template <int DK, int C, int RL, typename QT, typename ST>
 cudaError_t launch_mode(const KParams& kp, const VerifyArgs& a, const VerifyGeom& g, cudaStream_t s)
 {
     if (a.flags & GDN_FLAG_CHAIN)
-        return launch_one<DK, RL, QT, ST, true>(kp, a, g, s);
-    return launch_one<DK, RL, QT, ST, false>(kp, a, g, s);
+        return launch_one<DK, C, RL, QT, ST, true>(kp, a, g, s);
+    return launch_one<DK, C, RL, QT, ST, false>(kp, a, g, s);
 }
 
-template <int DK, int RL, typename QT>
+template <int DK, int C, int RL, typename QT>
 cudaError_t launch_state(const KParams& kp, const VerifyArgs& a, const VerifyGeom& g, cudaStream_t s)
 {
     if (a.state_dtype == GDN_F16)
-        return launch_mode<DK, RL, QT, __half>(kp, a, g, s);
-    return launch_mode<DK, RL, QT, float>(kp, a, g, s);
+        return launch_mode<DK, C, RL, QT, __half>(kp, a, g, s);
+    return launch_mode<DK, C, RL, QT, float>(kp, a, g, s);
 }
 
-template <int DK, int RL>
-cudaError_t launch_qkv(const KParams& kp, const VerifyArgs& a, const VerifyGeom& g, cudaStream_t s)
+template <int DK, int C, int RL>
+cudaError_t launch_shape(const KParams& kp, const VerifyArgs& a, const VerifyGeom& g, cudaStream_t s)
 {
     if (a.qkv_dtype == GDN_BF16)
-        return launch_state<DK, RL, __nv_bfloat16>(kp, a, g, s);
-    return launch_state<DK, RL, float>(kp, a, g, s);
+        return launch_state<DK, C, RL, __nv_bfloat16>(kp, a, g, s);
+    return launch_state<DK, C, RL, float>(kp, a, g, s);
 }
 
-// Launches the verify kernel for head dim DK (instantiated once per DK, in
-// gdn_verify_d{32,64,128}.cu).
-template <int DK>
+// Launches the verify kernel for head dim DK and lane shape (C, RL); each
+// shape is instantiated in its own translation unit.
+template <int DK, int C, int RL>
 cudaError_t launch_dk(const KParams& kp, const VerifyArgs& a, const VerifyGeom& g, cudaStream_t s)
 {
-    if (g.rows_per_lane == 1)
-        return launch_qkv<DK, 1>(kp, a, g, s);
-    return launch_qkv<DK, 2>(kp, a, g, s);
+    return launch_shape<DK, C, RL>(kp, a, g, s);
 }
-
 
 }  // namespace verify
 }  // namespace gdn

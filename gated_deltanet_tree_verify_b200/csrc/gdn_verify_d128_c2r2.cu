@@ -1,0 +1,11 @@
+// gdn_verify_d128_c2r2.cu -- the verify kernels instantiated for d_k = 128
+// and lane shape C = 2 chunks, RL = 2 rows per lane.
+
+#include "gdn_verify.cuh"
+
+namespace gdn {
+namespace verify {
+template cudaError_t launch_dk<128, 2, 2>(const KParams&, const VerifyArgs&, const VerifyGeom&,
+                                           cudaStream_t);
+}  // namespace verify
+}  // namespace gdn

@@ -31,9 +31,10 @@
  *     what the host can check (arguments, shapes, alignment, overlap of
  *     outputs with inputs, launch errors).  Errors in device data (a bad tree,
  *     a bad accept path) are reported through desc->status, see below.
- *   - Pointers passed for q, k, v, state_in, out, node_states and state_out
- *     must be 16-byte aligned; g, beta, parent_idx, accept_path and
- *     accept_len 4-byte aligned.
+ *   - Pointers passed for q, k, v, out and state_out must be 16-byte
+ *     aligned; state_in and node_states 32-byte aligned for gdn_tree_verify
+ *     (states move in 32-byte accesses) and 16-byte aligned for the commit
+ *     calls; g, beta, parent_idx, accept_path and accept_len 4-byte aligned.
  */
 #ifndef GDNTREE_H
 #define GDNTREE_H
