@@ -50,17 +50,7 @@ VerifyGeom verify_geometry(const VerifyArgs& a)
     const bool persist_last = (a.flags & GDN_FLAG_PERSIST_LAST) != 0;
     const size_t es = a.qkv_dtype == GDN_BF16 ? 2 : 4;
     g.reload = !chain && a.state_dtype == GDN_F32 && !persist_last;
-    if (chain || g.reload) {
-        g.slots = 0;
-    } else {
-        // floor(log2 N) slots make recomputation impossible; fewer keep more
-        // CTAs resident.  Draft trees of budget <= 31 need at most 2.
-        int k = 0;
-        while ((2 << k) <= a.n_nodes)
-            ++k;
-        const int cap = a.n_nodes <= 32 ? 2 : (a.n_nodes <= 96 ? 3 : 4);
-        g.slots = k < 1 ? 1 : (k > cap ? cap : k);
-    }
+
     // Lane shape: C = 2 chunks of 8 columns and RL rows per lane; two rows
     // (fewer instructions per row) unless that leaves fewer than
     // kWarpsPerSmTarget warps per SM.  (One chunk per lane, twice the warps
@@ -71,6 +61,19 @@ VerifyGeom verify_geometry(const VerifyArgs& a)
     };
     g.chunks = 2;
     g.rows_per_lane = total_warps(2, 2) >= kWarpsPerSmTarget * kSms ? 2 : 1;
+    if (chain || g.reload) {
+        g.slots = 0;
+    } else {
+        // floor(log2 N) slots make recomputation impossible; fewer keep more
+        // CTAs resident.  Draft trees of budget <= 31 need at most 2; with
+        // one, about one node per tree is recomputed, which pays off on
+        // large grids (more resident CTAs) but not on small ones.
+        int k = 0;
+        while ((2 << k) <= a.n_nodes)
+            ++k;
+        const int cap = a.n_nodes <= 32 ? (g.rows_per_lane == 2 ? 1 : 2) : (a.n_nodes <= 96 ? 3 : 4);
+        g.slots = k < 1 ? 1 : (k > cap ? cap : k);
+    }
     const int rpw = rows_per_warp(g.chunks, g.rows_per_lane);
     // Staged kernel first, else the ring kernel (which adds a producer warp).
     for (int pass = 0; pass < 2; ++pass) {

@@ -140,7 +140,22 @@ struct LaneMap {
     __device__ __forceinline__ int col(int c) const { return 8 * (cl + c * LR); }
     // offset of this lane's first element in a [rows][DK] row-major tile
     __device__ __forceinline__ int tile_offset() const { return row * DK + 8 * cl; }
+    // f32 records (see swz_pos): where the low and high 16-byte halves of
+    // this lane's chunks sit, relative to the chunk start of chunk cl
+    __device__ __forceinline__ int swz_lo() const { return 8 * cl + 4 * ((cl >> 2) & 1); }
+    __device__ __forceinline__ int swz_hi() const { return 8 * cl + 4 * (((cl >> 2) & 1) ^ 1); }
 };
+
+// f32 records in shared memory: chunk j (8 floats) of a k or q row has its
+// two 16-byte halves swapped when bit 2 of (j mod LR) is set, so the 8 lanes
+// of a quarter warp, which read chunks cl = 0..7 of a row, hit 8 distinct
+// 4-bank groups.  Position of element e of a row:
+template <int LR>
+__device__ __forceinline__ int swz_pos(int e)
+{
+    const int j = e >> 3, w = e & 7;
+    return 8 * j + ((((w >> 2) ^ (((j % LR) >> 2) & 1))) << 2) + (w & 3);
+}
 
 template <int C, int RL>
 struct StateT {
@@ -226,17 +241,30 @@ __device__ __forceinline__ void gdn_update(StateT<C, RL>& S, const float2 (&k2)[
     gdn_step<LR, C, RL, false>(S, k2, k2, vr, a, beta, pq, uo);
 }
 
+// Element e of the k (part 0) or q (part DK) row of a shared-memory record:
+// raw bf16 rows are plain, f32 rows swizzled (swz_pos).
+template <int DK, int LR>
+__device__ __forceinline__ float rec_elem(const __nv_bfloat16* rec, int part, int e)
+{
+    return Widen<__nv_bfloat16>::lds1(rec + part + e);
+}
+template <int DK, int LR>
+__device__ __forceinline__ float rec_elem(const float* rec, int part, int e)
+{
+    return rec[part + swz_pos<LR>(e)];
+}
+
 // k . q of one node's record, reduced by a group of 8 lanes (sub = lane % 8;
 // a warp handles four nodes at once; every lane of the warp must call it).
 // The same reduction wherever it is computed.
-template <int DK, typename RT>
+template <int DK, int LR, typename RT>
 __device__ __forceinline__ float node_kq8(const RT* rec, int sub)
 {
     float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
     for (int j = sub; j < DK; j += 16) {
-        acc0 = __fmaf_rn(Widen<RT>::lds1(rec + j), Widen<RT>::lds1(rec + DK + j), acc0);
-        acc1 = __fmaf_rn(Widen<RT>::lds1(rec + j + 8), Widen<RT>::lds1(rec + DK + j + 8), acc1);
+        acc0 = __fmaf_rn(rec_elem<DK, LR>(rec, 0, j), rec_elem<DK, LR>(rec, DK, j), acc0);
+        acc1 = __fmaf_rn(rec_elem<DK, LR>(rec, 0, j + 8), rec_elem<DK, LR>(rec, DK, j + 8), acc1);
     }
     float acc = __fadd_rn(acc0, acc1);
 #pragma unroll
@@ -344,38 +372,140 @@ __device__ __forceinline__ void load_slot(StateT<C, RL>& S, const float* lane_sl
     }
 }
 
-// k, q and the v slice of one node from its shared-memory record
-// [k | q | v slice] in the input type, widened here.
-template <int DK, int C, int RL, typename QT>
-__device__ __forceinline__ void load_k(const QT* rec, const LaneMap<DK, C, RL>& L, float2 (&k2)[4 * C],
-                                       float (&vr)[RL])
+// This lane's chunks of the k (part 0) or q (part DK) row of a shared-memory
+// record: raw bf16 (widened here) or swizzled f32.
+template <int DK, int C, int RL>
+__device__ __forceinline__ void load_row8(const __nv_bfloat16* rec, int part, const LaneMap<DK, C, RL>& L,
+                                          float2 (&x2)[4 * C])
+{
+#pragma unroll
+    for (int c = 0; c < C; ++c) {
+        float2 x[4];
+        Widen<__nv_bfloat16>::lds8(rec + part + L.col(c), x);
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+            x2[4 * c + t] = x[t];
+    }
+}
+
+template <int DK, int C, int RL>
+__device__ __forceinline__ void load_row8(const float* rec, int part, const LaneMap<DK, C, RL>& L,
+                                          float2 (&x2)[4 * C])
+{
+    using LM = LaneMap<DK, C, RL>;
+    const float* lo = rec + part + L.swz_lo();
+    const float* hi = rec + part + L.swz_hi();
+#pragma unroll
+    for (int c = 0; c < C; ++c) {
+        const float4 a = *reinterpret_cast<const float4*>(lo + c * 8 * LM::LR);
+        const float4 b = *reinterpret_cast<const float4*>(hi + c * 8 * LM::LR);
+        x2[4 * c + 0] = make_float2(a.x, a.y);
+        x2[4 * c + 1] = make_float2(a.z, a.w);
+        x2[4 * c + 2] = make_float2(b.x, b.y);
+        x2[4 * c + 3] = make_float2(b.z, b.w);
+    }
+}
+
+// One node's inputs for this lane as loaded from its shared-memory record,
+// before widening: k and q chunks and the v values of the lane's rows.
+template <typename RT, int C, int RL>
+struct RawRec;
+
+template <int C, int RL>
+struct RawRec<__nv_bfloat16, C, RL> {
+    uint4 k[C], q[C];
+    uint32_t v[RL];
+};
+
+template <int C, int RL>
+struct RawRec<float, C, RL> {
+    float4 k[2 * C], q[2 * C];
+    float v[RL];
+};
+
+template <int DK, int C, int RL>
+__device__ __forceinline__ void fetch_raw(const __nv_bfloat16* rec, const LaneMap<DK, C, RL>& L,
+                                          RawRec<__nv_bfloat16, C, RL>& R)
 {
     using LM = LaneMap<DK, C, RL>;
 #pragma unroll
     for (int c = 0; c < C; ++c) {
-        float2 x[4];
-        Widen<QT>::lds8(rec + L.col(c), x);
-#pragma unroll
-        for (int t = 0; t < 4; ++t)
-            k2[4 * c + t] = x[t];
+        R.k[c] = *reinterpret_cast<const uint4*>(rec + L.col(c));
+        R.q[c] = *reinterpret_cast<const uint4*>(rec + DK + L.col(c));
     }
 #pragma unroll
     for (int r = 0; r < RL; ++r)
-        vr[r] = Widen<QT>::lds1(rec + 2 * DK + L.row + r * LM::RG);
+        R.v[r] = *reinterpret_cast<const unsigned short*>(rec + 2 * DK + L.row + r * LM::RG);
 }
 
-template <int DK, int C, int RL, typename QT>
-__device__ __forceinline__ void load_q(const QT* rec, const LaneMap<DK, C, RL>& L, float2 (&q2)[4 * C])
+template <int DK, int C, int RL>
+__device__ __forceinline__ void fetch_raw(const float* rec, const LaneMap<DK, C, RL>& L,
+                                          RawRec<float, C, RL>& R)
+{
+    using LM = LaneMap<DK, C, RL>;
+    const float* lo = rec + L.swz_lo();
+    const float* hi = rec + L.swz_hi();
+#pragma unroll
+    for (int c = 0; c < C; ++c) {
+        R.k[2 * c] = *reinterpret_cast<const float4*>(lo + c * 8 * LM::LR);
+        R.k[2 * c + 1] = *reinterpret_cast<const float4*>(hi + c * 8 * LM::LR);
+        R.q[2 * c] = *reinterpret_cast<const float4*>(lo + DK + c * 8 * LM::LR);
+        R.q[2 * c + 1] = *reinterpret_cast<const float4*>(hi + DK + c * 8 * LM::LR);
+    }
+#pragma unroll
+    for (int r = 0; r < RL; ++r)
+        R.v[r] = rec[2 * DK + L.row + r * LM::RG];
+}
+
+template <int C, int RL>
+__device__ __forceinline__ void widen_raw(const RawRec<__nv_bfloat16, C, RL>& R, float2 (&k2)[4 * C],
+                                          float2 (&q2)[4 * C], float (&vr)[RL])
 {
 #pragma unroll
     for (int c = 0; c < C; ++c) {
-        float2 x[4];
-        Widen<QT>::lds8(rec + DK + L.col(c), x);
+        float2 x[4], y[4];
+        Widen<__nv_bfloat16>::pairs(R.k[c], x);
+        Widen<__nv_bfloat16>::pairs(R.q[c], y);
 #pragma unroll
-        for (int t = 0; t < 4; ++t)
-            q2[4 * c + t] = x[t];
+        for (int t = 0; t < 4; ++t) {
+            k2[4 * c + t] = x[t];
+            q2[4 * c + t] = y[t];
+        }
     }
+#pragma unroll
+    for (int r = 0; r < RL; ++r)
+        vr[r] = __uint_as_float(R.v[r] << 16);
 }
+
+template <int C, int RL>
+__device__ __forceinline__ void widen_raw(const RawRec<float, C, RL>& R, float2 (&k2)[4 * C],
+                                          float2 (&q2)[4 * C], float (&vr)[RL])
+{
+#pragma unroll
+    for (int c = 0; c < 2 * C; ++c) {
+        k2[2 * c] = make_float2(R.k[c].x, R.k[c].y);
+        k2[2 * c + 1] = make_float2(R.k[c].z, R.k[c].w);
+        q2[2 * c] = make_float2(R.q[c].x, R.q[c].y);
+        q2[2 * c + 1] = make_float2(R.q[c].z, R.q[c].w);
+    }
+#pragma unroll
+    for (int r = 0; r < RL; ++r)
+        vr[r] = R.v[r];
+}
+
+// k and the v slice of one node from its shared-memory record
+// [k | q | v slice] (RT: raw bf16 or swizzled f32).
+template <int DK, int C, int RL, typename RT>
+__device__ __forceinline__ void load_k(const RT* rec, const LaneMap<DK, C, RL>& L, float2 (&k2)[4 * C],
+                                       float (&vr)[RL])
+{
+    using LM = LaneMap<DK, C, RL>;
+    load_row8<DK, C, RL>(rec, 0, L, k2);
+#pragma unroll
+    for (int r = 0; r < RL; ++r)
+        vr[r] = Widen<RT>::lds1(rec + 2 * DK + L.row + r * LM::RG);
+}
+
 
 // ---------------------------------------------------------------------------
 // Tree walks
@@ -711,7 +841,7 @@ enum : int { kTreeChain = 0, kTreeWarp = 1, kTreeSmem = 2, kTreeIndex = 3 };
 // position's descriptor and record (ctx.desc, ctx.rec), the input fetcher
 // for recomputation, and the ring handshakes (ctx.begin / ctx.end; trivial
 // when everything is staged).
-template <int DK, int C, int RL, typename QT, typename ST, int TREE, class Tree, class Ctx>
+template <int DK, int C, int RL, typename RT, typename ST, int TREE, class Tree, class Ctx>
 __device__ __forceinline__ void walk(StateT<C, RL>& S, const KParams& p, const Tree& tree, float* lane_slot,
                                      const float* sin_lane, int b, int h, int row0,
                                      const LaneMap<DK, C, RL>& L, Ctx& ctx)
@@ -729,11 +859,16 @@ __device__ __forceinline__ void walk(StateT<C, RL>& S, const KParams& p, const T
     const int slot_floats = p.rows * DK;
     const int stride = p.warps * 32 * 4;
     StateT<C, RL> Sn;  // index order: the next position's parent state, prefetched
+    // (Loading the next position's record a node ahead as well costs ~30
+    // registers per thread; on small grids that keeps the next layer's CTAs
+    // from becoming resident early, which costs more than it saves.)
     for (int pos = 0; pos < N; ++pos) {
         if (!ctx.begin(pos))
             return;
         const PosDesc d = ctx.desc(pos);
         const int n = CHAIN ? pos : d.i.x;
+        RawRec<RT, C, RL> R;
+        fetch_raw<DK, C, RL>(ctx.rec(pos, n), L, R);
         bool next_reload = false;
         if constexpr (INDEX) {
             // issue the loads of the next position's parent state now; it was
@@ -750,11 +885,9 @@ __device__ __forceinline__ void walk(StateT<C, RL>& S, const KParams& p, const T
                 source_parent<DK, C, RL>(S, d.i.y, d.i.w, d.i.z, p, tree, lane_slot, slot_floats, stride,
                                          sin_lane, ctx.fetcher());
         }
-        const QT* rec = ctx.rec(pos, n);
         float2 k2[4 * C], q2[4 * C];
         float vr[RL];
-        load_k<DK, C, RL, QT>(rec, L, k2, vr);
-        load_q<DK, C, RL, QT>(rec, L, q2);
+        widen_raw<C, RL>(R, k2, q2, vr);
         const float a = d.f.x;
         float pq[RL], u[RL];
         gdn_step<LM::LR, C, RL, true>(S, k2, q2, vr, a, d.f.y, pq, u);
@@ -794,9 +927,9 @@ struct NoTree {
 // Staged kernel: every node's record copied into shared memory at start
 // ---------------------------------------------------------------------------
 
-template <int DK, int C, int RL, typename QT>
+template <int DK, int C, int RL, typename RT>
 struct StagedFetch {
-    const QT* recs;
+    const RT* recs;
     const float* ab;  // a | beta, by node
     uint32_t rec_elems;
     int N;
@@ -804,15 +937,15 @@ struct StagedFetch {
     __device__ __forceinline__ void operator()(int y, float2 (&k2)[4 * C], float (&vr)[RL], float& a,
                                                float& be) const
     {
-        load_k<DK, C, RL, QT>(recs + (size_t)y * rec_elems, L, k2, vr);
+        load_k<DK, C, RL, RT>(recs + (size_t)y * rec_elems, L, k2, vr);
         a = ab[y];
         be = ab[N + y];
     }
 };
 
-template <int DK, int C, int RL, typename QT>
+template <int DK, int C, int RL, typename RT>
 struct StagedCtx {
-    const QT* recs;
+    const RT* recs;
     const PosDesc* desc_;
     const float* ab;
     uint32_t rec_elems;
@@ -821,10 +954,10 @@ struct StagedCtx {
     __device__ __forceinline__ bool begin(int) { return true; }
     __device__ __forceinline__ void end(int) {}
     __device__ __forceinline__ PosDesc desc(int pos) const { return desc_[pos]; }
-    __device__ __forceinline__ const QT* rec(int, int n) const { return recs + (size_t)n * rec_elems; }
-    __device__ __forceinline__ StagedFetch<DK, C, RL, QT> fetcher() const
+    __device__ __forceinline__ const RT* rec(int, int n) const { return recs + (size_t)n * rec_elems; }
+    __device__ __forceinline__ StagedFetch<DK, C, RL, RT> fetcher() const
     {
-        return StagedFetch<DK, C, RL, QT>{recs, ab, rec_elems, N, L};
+        return StagedFetch<DK, C, RL, RT>{recs, ab, rec_elems, N, L};
     }
 };
 
@@ -841,19 +974,22 @@ __device__ __forceinline__ void cp_async4(void* dst_smem, const void* src_gmem)
 }
 
 // Prologue pass of the staged kernel over walk positions, four per warp and
-// pass: converts g to a = exp(g) in place (ab holds g | beta by node), and
-// writes each position's descriptor with k . q of its node.
-template <int DK, typename QT, class Tree>
+// pass (8 lanes each): converts g to a = exp(g) in place (ab holds g | beta by
+// node) and writes each position's descriptor with k . q of its node.
+template <int DK, int LR, typename QT, class Tree>
 __device__ __forceinline__ void write_descs(const Tree& tree, const unsigned char* raw, uint32_t raw_bytes,
                                             float* ab, PosDesc* desc, int N)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+    const int sub = lane & 7;
     for (int p0 = 4 * warp; p0 < N; p0 += 4 * nwarps) {
         const int pos = min(p0 + (lane >> 3), N - 1);
         const int m = tree.meta(pos);
         const int n = meta_node(m);
-        const float kq = node_kq8<DK, QT>(reinterpret_cast<const QT*>(raw + (size_t)n * raw_bytes), lane & 7);
-        if ((lane & 7) == 0 && p0 + (lane >> 3) < N) {
+        const QT* rrec = reinterpret_cast<const QT*>(raw + (size_t)n * raw_bytes);
+        const bool valid = p0 + (lane >> 3) < N;
+        const float kq = node_kq8<DK, LR>(rrec, sub);
+        if (sub == 0 && valid) {
             const float a = gdn_gate(ab[n]);
             ab[n] = a;
             PosDesc d;
@@ -866,11 +1002,12 @@ __device__ __forceinline__ void write_descs(const Tree& tree, const unsigned cha
 
 template <int DK, int C, int RL, typename QT, typename ST, int TREE, class Tree>
 __device__ __forceinline__ void staged_finish(StateT<C, RL>& S, const KParams& p, const Tree& tree,
-                                              const unsigned char* raw, float* ab, PosDesc* desc,
-                                              float* slotbuf, const float* sin_lane, int b, int h, int row0,
+                                              const unsigned char* raw, float* ab, PosDesc* desc, float* slotbuf,
+                                              const float* sin_lane, int b, int h, int row0,
                                               const LaneMap<DK, C, RL>& L)
 {
-    write_descs<DK, QT>(tree, raw, p.raw_bytes, ab, desc, p.N);
+    constexpr int LR = LaneMap<DK, C, RL>::LR;
+    write_descs<DK, LR, QT>(tree, raw, p.raw_bytes, ab, desc, p.N);
     __syncthreads();
     const uint32_t rec_elems = p.raw_bytes / (uint32_t)sizeof(QT);
     StagedCtx<DK, C, RL, QT> ctx{reinterpret_cast<const QT*>(raw), desc, ab, rec_elems, p.N, L};
@@ -905,6 +1042,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32) gdn_verify_staged(const KParam
     // w + warps, ...); the tree work overlaps the copies unless it already ran
     // before the wait.
     const int per_node = p.raw_bytes / 16;  // 16-byte chunks per node
+    constexpr int LR = LaneMap<DK, C, RL>::LR;
     auto stage = [&]() {
         const QT* kg = static_cast<const QT*>(p.k);
         const QT* qg = static_cast<const QT*>(p.q);
@@ -919,7 +1057,17 @@ __global__ void __launch_bounds__(kMaxWarps * 32) gdn_verify_staged(const KParam
                 const QT* src = c < QKCH ? krow + c * EPC
                                          : (c < 2 * QKCH ? qrow + (c - QKCH) * EPC
                                                          : vrow + (c - 2 * QKCH) * EPC);
-                cp_async16(dst + 16 * c, src);
+                int off = 16 * c;
+                if constexpr (sizeof(QT) == 4) {
+                    // f32 k and q rows land swizzled (swz_pos): 16-byte half
+                    // h of 8-column chunk j
+                    if (c < 2 * QKCH) {
+                        const int part = c < QKCH ? 0 : QKCH;
+                        const int j = (c - part) >> 1, hh = (c - part) & 1;
+                        off = 16 * part + 32 * j + 16 * (hh ^ (((j % LR) >> 2) & 1));
+                    }
+                }
+                cp_async16(dst + off, src);
             }
         }
         for (int n = tid; n < N; n += blockDim.x) {
@@ -978,16 +1126,17 @@ __global__ void __launch_bounds__(kMaxWarps * 32) gdn_verify_staged(const KParam
     }
     // 5. descriptors, then the walk
     if constexpr (TREE == kTreeChain)
-        staged_finish<DK, C, RL, QT, ST, TREE>(S, p, NoTree{}, raw, ab, desc, slotbuf, sin_lane, b, h, row0, L);
+        staged_finish<DK, C, RL, QT, ST, TREE>(S, p, NoTree{}, raw, ab, desc, slotbuf, sin_lane, b, h,
+                                               row0, L);
     else if constexpr (TREE == kTreeIndex)
-        staged_finish<DK, C, RL, QT, ST, TREE>(S, p, IndexTree{tsm}, raw, ab, desc, slotbuf, sin_lane, b, h,
-                                               row0, L);
+        staged_finish<DK, C, RL, QT, ST, TREE>(S, p, IndexTree{tsm}, raw, ab, desc, slotbuf, sin_lane, b,
+                                               h, row0, L);
     else if constexpr (TREE == kTreeWarp)
-        staged_finish<DK, C, RL, QT, ST, TREE>(S, p, MaskTree{tsm}, raw, ab, desc, slotbuf, sin_lane, b, h,
-                                               row0, L);
+        staged_finish<DK, C, RL, QT, ST, TREE>(S, p, MaskTree{tsm}, raw, ab, desc, slotbuf, sin_lane, b,
+                                               h, row0, L);
     else
-        staged_finish<DK, C, RL, QT, ST, TREE>(S, p, SmemTree{tv, N, warp}, raw, ab, desc, slotbuf, sin_lane,
-                                               b, h, row0, L);
+        staged_finish<DK, C, RL, QT, ST, TREE>(S, p, SmemTree{tv, N, warp}, raw, ab, desc, slotbuf,
+                                               sin_lane, b, h, row0, L);
 }
 
 // ---------------------------------------------------------------------------
@@ -1197,7 +1346,16 @@ __global__ void __launch_bounds__((kMaxWarps + 1) * 32) gdn_verify_ring(const KP
                 const int idx = lane + 32 * t;
                 if (idx < total) {
                     const int i = idx / per_pos, j = idx - i * per_pos;
-                    *reinterpret_cast<uint4*>(base + (size_t)i * p.raw_bytes + 16 * j) = regs[t];
+                    int off = 16 * j;
+                    if constexpr (sizeof(QT) == 4) {
+                        // f32 k and q rows land swizzled (swz_pos)
+                        if (j < 2 * QKCH) {
+                            const int part = j < QKCH ? 0 : QKCH;
+                            const int jj = (j - part) >> 1, hh = (j - part) & 1;
+                            off = 16 * part + 32 * jj + 16 * (hh ^ (((jj % LM::LR) >> 2) & 1));
+                        }
+                    }
+                    *reinterpret_cast<uint4*>(base + (size_t)i * p.raw_bytes + off) = regs[t];
                 }
             }
             __syncwarp();
@@ -1205,7 +1363,7 @@ __global__ void __launch_bounds__((kMaxWarps + 1) * 32) gdn_verify_ring(const KP
                 const int gi = i0 + (lane >> 3);
                 const int i = min(gi, cnt - 1);
                 const float kq =
-                    node_kq8<DK, QT>(reinterpret_cast<const QT*>(base + (size_t)i * p.raw_bytes), lane & 7);
+                    node_kq8<DK, LM::LR>(reinterpret_cast<const QT*>(base + (size_t)i * p.raw_bytes), lane & 7);
                 const int src_lane = i;
                 const int n = __shfl_sync(0xffffffffu, dn, src_lane);
                 const int m = __shfl_sync(0xffffffffu, dm, src_lane);

@@ -102,7 +102,7 @@ def test_verify_null_and_misaligned_pointers(lib):
             continue
         p[i] = None
         assert _verify(_desc(), p) == gdn.GDN_ERR_INVALID_ARG, i
-    for i, align in [(0, 16), (1, 16), (2, 16), (6, 16), (7, 16), (8, 16), (3, 4), (4, 4), (5, 4)]:
+    for i, align in [(0, 16), (1, 16), (2, 16), (6, 32), (7, 16), (8, 32), (3, 4), (4, 4), (5, 4)]:
         p = _ptrs()
         p[i] += align // 2
         assert _verify(_desc(), p) == gdn.GDN_ERR_INVALID_ARG, i
