@@ -497,9 +497,10 @@ FP32_LANES_PER_SM = 128  # FP32 CUDA-core lanes per SM (B200); 148 SMs
 
 
 def _verify_point(*, batch, n_nodes, tree, state_dtype, flags=0, gate="softplus", reps=20,
-                  min_bytes=512 << 20, seed=11):
+                  min_bytes=512 << 20, seed=11, workspace=False):
     """Mean time of one verify launch, over graph replays of R launches on R
-    distinct buffer sets (R sized so the sets together exceed min_bytes)."""
+    distinct buffer sets (R sized so the sets together exceed min_bytes).
+    With ``workspace``, through gdn_tree_verify_ws (one workspace per set)."""
     import gated_deltanet_tree_verify_b200 as gdn
     persist_last = bool(flags & gdn.GDN_FLAG_PERSIST_LAST)
     tdt = torch.float32 if state_dtype == "f32" else torch.float16
@@ -520,11 +521,18 @@ def _verify_point(*, batch, n_nodes, tree, state_dtype, flags=0, gate="softplus"
     desc = gdn.make_desc(batch=batch, n_nodes=n_nodes, n_k_heads=N_K_HEADS, n_v_heads=N_V_HEADS, d_k=D,
                          d_v=D, scale=sets[0][0].scale, qkv_dtype=gdn.GDN_BF16,
                          state_dtype=gdn.GDN_F32 if state_dtype == "f32" else gdn.GDN_F16, flags=flags)
+    ws_bytes = gdn.gdn_tree_verify_workspace_bytes(desc) if workspace else 0
+    for _, d in sets:
+        d["ws"] = torch.empty(max(ws_bytes, 16) // 4, device="cuda") if ws_bytes else None
 
     def run_all():
         for _, d in sets:
-            gdn.gdn_tree_verify(desc, d["q"], d["k"], d["v"], d["g"], d["beta"], d["parent"], d["state_in"],
-                                d["out"], d["ns"])
+            if d["ws"] is not None:
+                gdn.gdn_tree_verify_ws(desc, d["q"], d["k"], d["v"], d["g"], d["beta"], d["parent"],
+                                       d["state_in"], d["out"], d["ns"], d["ws"], ws_bytes)
+            else:
+                gdn.gdn_tree_verify(desc, d["q"], d["k"], d["v"], d["g"], d["beta"], d["parent"],
+                                    d["state_in"], d["out"], d["ns"])
 
     run_all()
     torch.cuda.synchronize()
@@ -561,6 +569,8 @@ def run_sweep(args):
         for batch in (1, 8, 32):
             for sd in ("f32", "f16"):
                 points.append(dict(kind="tree", budget=budget, batch=batch, state_dtype=sd))
+                if sd == "f16":
+                    points.append(dict(kind="tree", budget=budget, batch=batch, state_dtype=sd, ws=True))
     for sd in ("f32", "f16"):
         points.append(dict(kind="chain16", budget=15, batch=1, state_dtype=sd))
     points.append(dict(kind="chain4096", budget=4095, batch=8, state_dtype="f32"))
@@ -585,10 +595,10 @@ def run_sweep(args):
             tree = "ddtree" if pt["kind"] == "tree" else "chain"
             flags = 0 if pt["kind"] == "tree" else gdn.GDN_FLAG_CHAIN
             t, R = _verify_point(batch=pt["batch"], n_nodes=n, tree=tree, state_dtype=pt["state_dtype"],
-                                 flags=flags)
+                                 flags=flags, workspace=pt.get("ws", False))
             vb = verify_bytes(pt["batch"], n, pt["state_dtype"])
             line = {"sweep": pt["kind"], "budget": pt["budget"], "batch": pt["batch"],
-                    "state_dtype": pt["state_dtype"], "verify_us": t * 1e6,
+                    "state_dtype": pt["state_dtype"], "workspace": pt.get("ws", False), "verify_us": t * 1e6,
                     "node_layers_per_s": pt["batch"] * n / t, "gbps": vb / t / 1e9,
                     "frac_of_hbm": vb / t / 1e9 / peak, "buffer_sets": R}
         print(json.dumps(line), flush=True)

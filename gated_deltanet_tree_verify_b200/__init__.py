@@ -9,5 +9,5 @@ from .gdntree import (  # noqa: F401
     GDN_ERR_TIMEOUT, GDN_ERR_UNSUPPORTED, GDN_F16, GDN_F32, GDN_FLAG_CHAIN,
     GDN_FLAG_EARLY_TREE, GDN_FLAG_PERSIST_LAST, GDN_FLAG_VALIDATE, GDN_MAX_TREE_NODES, GDN_OK, GdnError,
     GdnLibraryMissing, GdnTreeDesc, gdn_node_states_bytes, gdn_status_str, gdn_tree_commit, gdn_tree_commit_layers,
-    gdn_tree_verify, gdn_version, load_library, make_desc,
+    gdn_tree_verify, gdn_tree_verify_workspace_bytes, gdn_tree_verify_ws, gdn_version, load_library, make_desc,
 )

@@ -106,10 +106,32 @@ size_t gdn_node_states_bytes(const gdn_tree_desc* desc)
     return node_states_bytes(desc);
 }
 
-gdn_status gdn_tree_verify(const gdn_tree_desc* desc, const void* q, const void* k, const void* v,
-                           const float* g, const float* beta, const int32_t* parent_idx,
-                           const float* state_in, float* out, void* node_states,
-                           cudaStream_t stream)
+}  // extern "C"
+
+namespace {
+
+// VerifyArgs for a desc and buffers (no checks).
+gdn::VerifyArgs verify_args(const gdn_tree_desc& d)
+{
+    gdn::VerifyArgs a{};
+    a.status = d.status;
+    a.batch = d.batch;
+    a.n_nodes = d.n_nodes;
+    a.n_k_heads = d.n_k_heads;
+    a.n_v_heads = d.n_v_heads;
+    a.d_k = d.d_k;
+    a.d_v = d.d_v;
+    a.scale = d.scale;
+    a.qkv_dtype = d.qkv_dtype;
+    a.state_dtype = d.state_dtype;
+    a.flags = d.flags;
+    return a;
+}
+
+gdn_status verify_impl(const gdn_tree_desc* desc, const void* q, const void* k, const void* v,
+                       const float* g, const float* beta, const int32_t* parent_idx, const float* state_in,
+                       float* out, void* node_states, void* workspace, size_t workspace_bytes,
+                       cudaStream_t stream)
 {
     g_detail[0] = '\0';
     gdn_status st = check_desc(desc, true);
@@ -123,29 +145,13 @@ gdn_status gdn_tree_verify(const gdn_tree_desc* desc, const void* q, const void*
     const struct { const void* p; size_t a; const char* n; } al[] = {
         {q, 16, "q"}, {k, 16, "k"}, {v, 16, "v"}, {state_in, 32, "state_in"}, {out, 16, "out"},
         {node_states, 32, "node_states"}, {g, 4, "g"}, {beta, 4, "beta"}, {parent_idx, 4, "parent_idx"},
-        {d.status, 4, "status"}};
+        {d.status, 4, "status"}, {workspace, 16, "workspace"}};
     for (const auto& x : al)
         if (x.p && !aligned(x.p, x.a))
             return fail(GDN_ERR_INVALID_ARG, "%s is misaligned", x.n);
     if (d.batch == 0)
         return GDN_OK;
-    const size_t B = d.batch, N = d.n_nodes, Hk = d.n_k_heads, Hv = d.n_v_heads, dk = d.d_k, dv = d.d_v;
-    const size_t es = elem_size(d.qkv_dtype);
-    const Range ins[] = {{q, B * N * Hk * dk * es, "q"},     {k, B * N * Hk * dk * es, "k"},
-                         {v, B * N * Hv * dv * es, "v"},     {g, B * N * Hv * 4, "g"},
-                         {beta, B * N * Hv * 4, "beta"},     {parent_idx, B * N * 4, "parent_idx"},
-                         {state_in, B * Hv * dv * dk * 4, "state_in"},
-                         {d.status, 4, "status"}};
-    const Range outs[] = {{out, B * N * Hv * dv * 4, "out"},
-                          {node_states, node_states_bytes(&d), "node_states"}};
-    if (overlap(outs[0], outs[1]))
-        return fail(GDN_ERR_INVALID_ARG, "out overlaps node_states%s");
-    for (const auto& o : outs)
-        for (const auto& i : ins)
-            if (overlap(o, i))
-                return fail(GDN_ERR_INVALID_ARG, "an output overlaps input %s", i.name);
-
-    gdn::VerifyArgs a{};
+    gdn::VerifyArgs a = verify_args(d);
     a.q = q;
     a.k = k;
     a.v = v;
@@ -155,26 +161,66 @@ gdn_status gdn_tree_verify(const gdn_tree_desc* desc, const void* q, const void*
     a.state_in = state_in;
     a.out = out;
     a.node_states = node_states;
-    a.status = d.status;
-    a.batch = d.batch;
-    a.n_nodes = d.n_nodes;
-    a.n_k_heads = d.n_k_heads;
-    a.n_v_heads = d.n_v_heads;
-    a.d_k = d.d_k;
-    a.d_v = d.d_v;
-    a.scale = d.scale;
-    a.qkv_dtype = d.qkv_dtype;
-    a.state_dtype = d.state_dtype;
-    a.flags = d.flags;
-    const gdn::VerifyGeom geom = gdn::verify_geometry(a);
+    a.workspace = static_cast<float*>(workspace);
+    const gdn::VerifyGeom geom = gdn::verify_geometry(a, workspace != nullptr);
     if (geom.tiles <= 0 || geom.smem > 227 * 1024)
         return fail(GDN_ERR_UNSUPPORTED, "no launch geometry for this shape%s");
     if (d.n_v_heads > 65535 || d.batch > 65535)
         return fail(GDN_ERR_UNSUPPORTED, "batch or n_v_heads above the grid limit%s");
+    if (geom.gslots && workspace_bytes < geom.ws_bytes)
+        return fail(GDN_ERR_INVALID_ARG, "workspace smaller than gdn_tree_verify_workspace_bytes()%s");
+
+    const size_t B = d.batch, N = d.n_nodes, Hk = d.n_k_heads, Hv = d.n_v_heads, dk = d.d_k, dv = d.d_v;
+    const size_t es = elem_size(d.qkv_dtype);
+    const Range ins[] = {{q, B * N * Hk * dk * es, "q"},     {k, B * N * Hk * dk * es, "k"},
+                         {v, B * N * Hv * dv * es, "v"},     {g, B * N * Hv * 4, "g"},
+                         {beta, B * N * Hv * 4, "beta"},     {parent_idx, B * N * 4, "parent_idx"},
+                         {state_in, B * Hv * dv * dk * 4, "state_in"},
+                         {d.status, 4, "status"}};
+    const Range outs[] = {{out, B * N * Hv * dv * 4, "out"},
+                          {node_states, node_states_bytes(&d), "node_states"},
+                          {geom.gslots ? workspace : nullptr, geom.ws_bytes, "workspace"}};
+    for (int i = 0; i < 3; ++i)
+        for (int j = i + 1; j < 3; ++j)
+            if (overlap(outs[i], outs[j]))
+                return fail(GDN_ERR_INVALID_ARG, "%s overlaps another output", outs[j].name);
+    for (const auto& o : outs)
+        for (const auto& i : ins)
+            if (overlap(o, i))
+                return fail(GDN_ERR_INVALID_ARG, "an output overlaps input %s", i.name);
     const cudaError_t e = gdn::launch_verify(a, geom, stream);
     if (e != cudaSuccess)
         return fail(GDN_ERR_CUDA, "verify launch failed: %s", cudaGetErrorString(e));
     return GDN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+gdn_status gdn_tree_verify(const gdn_tree_desc* desc, const void* q, const void* k, const void* v,
+                           const float* g, const float* beta, const int32_t* parent_idx,
+                           const float* state_in, float* out, void* node_states,
+                           cudaStream_t stream)
+{
+    return verify_impl(desc, q, k, v, g, beta, parent_idx, state_in, out, node_states, nullptr, 0, stream);
+}
+
+gdn_status gdn_tree_verify_ws(const gdn_tree_desc* desc, const void* q, const void* k, const void* v,
+                              const float* g, const float* beta, const int32_t* parent_idx,
+                              const float* state_in, float* out, void* node_states, void* workspace,
+                              size_t workspace_bytes, cudaStream_t stream)
+{
+    return verify_impl(desc, q, k, v, g, beta, parent_idx, state_in, out, node_states, workspace,
+                       workspace_bytes, stream);
+}
+
+size_t gdn_tree_verify_workspace_bytes(const gdn_tree_desc* desc)
+{
+    if (check_desc(desc, true) != GDN_OK)
+        return 0;
+    const gdn::VerifyGeom geom = gdn::verify_geometry(verify_args(*desc), true);
+    return geom.tiles > 0 ? geom.ws_bytes : 0;
 }
 
 gdn_status gdn_tree_commit_layers(const gdn_tree_desc* desc, int32_t n_layers,

@@ -20,6 +20,8 @@ struct VerifyGeom {
     bool staged;          // whole-tree staging kernel (else the producer/ring kernel)
     bool warp_tree;       // staged tree walked from warp registers (N <= 32)
     bool reload;          // branch parents re-read from f32 node_states (no stack)
+    bool gslots;          // stack slots in the caller's workspace (global memory)
+    size_t ws_bytes;      // workspace the launch needs (gslots), else 0
     int chunks;           // lane shape: chunks of 8 state columns per lane and row (1 or 2)
     int rows_per_lane;    // lane shape: rows per lane (1 or 2)
     int warps;            // compute warps per CTA (the ring kernel adds a producer warp)
@@ -46,6 +48,7 @@ struct VerifyArgs {
     float scale;
     int qkv_dtype, state_dtype;
     uint32_t flags;
+    float* workspace;  // optional: stack slots in global memory
 };
 
 // Layers one commit launch covers (more are split over several launches).
@@ -84,7 +87,9 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 }
 
 // Pick the launch geometry for a verify call (host only, no CUDA calls).
-VerifyGeom verify_geometry(const VerifyArgs& a);
+// With use_workspace, walks that keep stack slots keep them in global memory
+// (VerifyGeom::gslots, ws_bytes).
+VerifyGeom verify_geometry(const VerifyArgs& a, bool use_workspace);
 
 // Launch the verify / commit kernels.  Return cudaSuccess or the launch error.
 cudaError_t launch_verify(const VerifyArgs& a, const VerifyGeom& geom, cudaStream_t stream);

@@ -43,7 +43,7 @@ cudaError_t launch_shapes(const verify::KParams& kp, const VerifyArgs& a, const 
 
 using namespace verify;
 
-VerifyGeom verify_geometry(const VerifyArgs& a)
+VerifyGeom verify_geometry(const VerifyArgs& a, bool use_workspace)
 {
     VerifyGeom g{};
     const bool chain = (a.flags & GDN_FLAG_CHAIN) != 0;
@@ -64,14 +64,17 @@ VerifyGeom verify_geometry(const VerifyArgs& a)
     if (chain || g.reload) {
         g.slots = 0;
     } else {
-        // floor(log2 N) slots make recomputation impossible; fewer keep more
-        // CTAs resident.  Draft trees of budget <= 31 need at most 2; with
-        // one, about one node per tree is recomputed, which pays off on
-        // large grids (more resident CTAs) but not on small ones.
+        // floor(log2 N) slots make recomputation impossible.  In shared
+        // memory fewer keep more CTAs resident: draft trees of budget <= 31
+        // need at most 2, and with one about one node per tree is recomputed,
+        // which pays off on large grids (more resident CTAs) but not on small
+        // ones.  In a workspace only the size counts.
         int k = 0;
         while ((2 << k) <= a.n_nodes)
             ++k;
-        const int cap = a.n_nodes <= 32 ? (g.rows_per_lane == 2 ? 1 : 2) : (a.n_nodes <= 96 ? 3 : 4);
+        g.gslots = use_workspace;
+        const int cap = g.gslots ? 4
+                                 : (a.n_nodes <= 32 ? (g.rows_per_lane == 2 ? 1 : 2) : (a.n_nodes <= 96 ? 3 : 4));
         g.slots = k < 1 ? 1 : (k > cap ? cap : k);
     }
     const int rpw = rows_per_warp(g.chunks, g.rows_per_lane);
@@ -85,7 +88,7 @@ VerifyGeom verify_geometry(const VerifyArgs& a)
         if (a.d_v % rows != 0 || (rows * es) % 16 != 0)
             continue;
         const size_t raw_bytes = (size_t)(2 * a.d_k + rows) * es;
-        const size_t slot_bytes = (size_t)g.slots * rows * a.d_k * 4;
+        const size_t slot_bytes = g.gslots ? 0 : (size_t)g.slots * rows * a.d_k * 4;
         size_t off = 64;  // mbarriers
         size_t off_raw = 0, off_desc = 0, off_ab = 0, off_slots = 0;
         if (staged) {
@@ -127,6 +130,7 @@ VerifyGeom verify_geometry(const VerifyArgs& a)
         g.off_slots = (uint32_t)off_slots;
         g.off_tree = (uint32_t)off_tree;
         g.smem = off;
+        g.ws_bytes = g.gslots ? (size_t)a.batch * a.n_v_heads * a.d_v * a.d_k * g.slots * 4 : 0;
         break;
     }
     return g;
@@ -157,6 +161,7 @@ cudaError_t launch_verify(const VerifyArgs& a, const VerifyGeom& geom, cudaStrea
     kp.persist_last = (a.flags & GDN_FLAG_PERSIST_LAST) ? 1 : 0;
     kp.validate = (a.flags & GDN_FLAG_VALIDATE) ? 1 : 0;
     kp.early_tree = (a.flags & GDN_FLAG_EARLY_TREE) ? 1 : 0;
+    kp.ws = geom.gslots ? a.workspace : nullptr;
     kp.raw_bytes = geom.raw_bytes;
     kp.off_raw = geom.off_raw;
     kp.off_desc = geom.off_desc;

@@ -111,6 +111,7 @@ struct KParams {
     float scale;
     int rows, warps, slots;
     int persist_last, validate, early_tree;
+    float* ws;           // global stack slots (kTreeGlobal kinds): slots x rows x d_k per CTA
     uint32_t raw_bytes;  // one node's record (k row | q row | v slice) in bytes
     uint32_t off_raw, off_desc, off_ab, off_slots, off_tree;
 };
@@ -834,7 +835,10 @@ __device__ __forceinline__ void source_parent(StateT<C, RL>& S, int m, int pp, i
     }
 }
 
-enum : int { kTreeChain = 0, kTreeWarp = 1, kTreeSmem = 2, kTreeIndex = 3 };
+// Walk kinds.  kTreeGlobal added to kTreeWarp or kTreeSmem: the stack slots
+// live in a caller workspace in global memory (L2) instead of shared memory,
+// and a slot the next position needs is loaded one node ahead.
+enum : int { kTreeChain = 0, kTreeWarp = 1, kTreeSmem = 2, kTreeIndex = 3, kTreeGlobal = 4 };
 
 // The walk over positions [0, N): per position, find the parent state,
 // update, write the output and persist.  The context supplies each
@@ -849,6 +853,7 @@ __device__ __forceinline__ void walk(StateT<C, RL>& S, const KParams& p, const T
     using LM = LaneMap<DK, C, RL>;
     constexpr bool CHAIN = TREE == kTreeChain;
     constexpr bool INDEX = TREE == kTreeIndex;
+    constexpr bool GSLOT = TREE >= kTreeGlobal;
     const int N = p.N;
     const int NS = p.persist_last ? 1 : N;
     const size_t ns_stride = (size_t)p.Hv * p.dv * DK;  // elements between nodes' states
@@ -858,7 +863,12 @@ __device__ __forceinline__ void walk(StateT<C, RL>& S, const KParams& p, const T
     float* const out_lane = p.out + (size_t)b * N * out_stride + (size_t)h * p.dv + row0 + L.row;
     const int slot_floats = p.rows * DK;
     const int stride = p.warps * 32 * 4;
-    StateT<C, RL> Sn;  // index order: the next position's parent state, prefetched
+    // Index order and workspace slots: the next position's parent state,
+    // loaded one node ahead.  (Asking for it in L1 instead, with prefetch
+    // hints and a load where it is needed, saves ~40 registers but was
+    // measured slower.)
+    StateT<C, RL> Sn;
+    bool have_next = false;
     // (Loading the next position's record a node ahead as well costs ~30
     // registers per thread; on small grids that keeps the next layer's CTAs
     // from becoming resident early, which costs more than it saves.)
@@ -869,21 +879,37 @@ __device__ __forceinline__ void walk(StateT<C, RL>& S, const KParams& p, const T
         const int n = CHAIN ? pos : d.i.x;
         RawRec<RT, C, RL> R;
         fetch_raw<DK, C, RL>(ctx.rec(pos, n), L, R);
-        bool next_reload = false;
         if constexpr (INDEX) {
-            // issue the loads of the next position's parent state now; it was
-            // persisted by this thread at an earlier position
+            // the next position's parent state, persisted by this thread at
+            // an earlier position, unless it is this position's
+            have_next = false;
             if (pos + 1 < N) {
                 const int pn = tree.parent(pos + 1);
-                next_reload = pn != pos;
-                if (next_reload)
+                if (pn != pos) {
                     load_rows<DK, C, RL>(Sn, reinterpret_cast<const float*>(ns_lane) + (size_t)pn * ns_stride);
+                    have_next = true;
+                }
             }
         } else if constexpr (!CHAIN) {
             const int src = meta_src(d.i.y);
-            if (src != kSrcCont && src != kSrcRoot)
+            if (GSLOT && have_next)
+                S = Sn;  // this position's slot, loaded at the previous one
+            else if (src != kSrcCont && src != kSrcRoot)
                 source_parent<DK, C, RL>(S, d.i.y, d.i.w, d.i.z, p, tree, lane_slot, slot_floats, stride,
                                          sin_lane, ctx.fetcher());
+            if constexpr (GSLOT) {
+                // the next position's slot.  A node whose successor in the
+                // walk reloads a slot is a leaf, so this position saves
+                // nothing into it.
+                have_next = false;
+                if (pos + 1 < N && ctx.ahead(pos + 1)) {
+                    const int mn = ctx.desc(pos + 1).i.y;
+                    if (meta_src(mn) == kSrcSlot) {
+                        load_slot<C, RL>(Sn, lane_slot + (size_t)meta_load(mn) * slot_floats, stride);
+                        have_next = true;
+                    }
+                }
+            }
         }
         float2 k2[4 * C], q2[4 * C];
         float vr[RL];
@@ -905,7 +931,7 @@ __device__ __forceinline__ void walk(StateT<C, RL>& S, const KParams& p, const T
                 save_slot<C, RL>(S, lane_slot + (size_t)save * slot_floats, stride);
         }
         if constexpr (INDEX) {
-            if (next_reload)
+            if (have_next)
                 S = Sn;
         }
         ctx.end(pos);
@@ -953,6 +979,8 @@ struct StagedCtx {
     LaneMap<DK, C, RL> L;
     __device__ __forceinline__ bool begin(int) { return true; }
     __device__ __forceinline__ void end(int) {}
+    // whether position pos's descriptor may be read before begin(pos)
+    __device__ __forceinline__ bool ahead(int) const { return true; }
     __device__ __forceinline__ PosDesc desc(int pos) const { return desc_[pos]; }
     __device__ __forceinline__ const RT* rec(int, int n) const { return recs + (size_t)n * rec_elems; }
     __device__ __forceinline__ StagedFetch<DK, C, RL, RT> fetcher() const
@@ -971,6 +999,18 @@ __device__ __forceinline__ void cp_async4(void* dst_smem, const void* src_gmem)
 {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(dst_smem)), "l"(src_gmem)
                  : "memory");
+}
+
+// This CTA's stack slots: shared memory, or its region of the workspace.
+template <int DK, int TREE>
+__device__ __forceinline__ float* cta_slots(const KParams& p, float* slotbuf)
+{
+    if constexpr (TREE >= kTreeGlobal) {
+        const size_t cta = ((size_t)blockIdx.z * p.Hv + blockIdx.y) * gridDim.x + blockIdx.x;
+        return p.ws + cta * (size_t)p.slots * p.rows * DK;
+    } else {
+        return slotbuf;
+    }
 }
 
 // Prologue pass of the staged kernel over walk positions, four per warp and
@@ -1011,7 +1051,7 @@ __device__ __forceinline__ void staged_finish(StateT<C, RL>& S, const KParams& p
     __syncthreads();
     const uint32_t rec_elems = p.raw_bytes / (uint32_t)sizeof(QT);
     StagedCtx<DK, C, RL, QT> ctx{reinterpret_cast<const QT*>(raw), desc, ab, rec_elems, p.N, L};
-    float* lane_slot = slotbuf + 4 * threadIdx.x;
+    float* lane_slot = cta_slots<DK, TREE>(p, slotbuf) + 4 * threadIdx.x;
     walk<DK, C, RL, QT, ST, TREE>(S, p, tree, lane_slot, sin_lane, b, h, row0, L, ctx);
 }
 
@@ -1027,6 +1067,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32) gdn_verify_staged(const KParam
     float* slotbuf = reinterpret_cast<float*>(smem + p.off_slots);
     int* tsm = reinterpret_cast<int*>(smem + p.off_tree);
 
+    constexpr int TK = TREE % kTreeGlobal;  // walk kind without the slot placement
     const int N = p.N;
     const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int hk = h / p.G;
@@ -1085,13 +1126,13 @@ __global__ void __launch_bounds__(kMaxWarps * 32) gdn_verify_staged(const KParam
     // 1. the parent array (index order keeps it in shared memory; chain
     //    validation only checks it)
     bool bad = false;
-    if constexpr (TREE == kTreeIndex) {
+    if constexpr (TK == kTreeIndex) {
         for (int n = tid; n < N; n += blockDim.x) {
             const int pn = __ldg(prow + n);
             tsm[n] = pn;
             bad |= (n == 0) ? (pn != -1) : (pn < 0 || pn >= n);
         }
-    } else if constexpr (TREE == kTreeChain) {
+    } else if constexpr (TK == kTreeChain) {
         if (p.validate) {
             for (int n = tid; n < N; n += blockDim.x)
                 bad |= __ldg(prow + n) != n - 1;
@@ -1106,10 +1147,10 @@ __global__ void __launch_bounds__(kMaxWarps * 32) gdn_verify_staged(const KParam
     // 3. the walk: warp 0 builds it for trees of <= 32 nodes; all threads for
     //    larger trees
     const TreeView tv(tsm, N);
-    if constexpr (TREE == kTreeWarp) {
+    if constexpr (TK == kTreeWarp) {
         if (warp == 0 && !build_warp_walk(prow, N, p.slots, tsm))
             bad = true;
-    } else if constexpr (TREE == kTreeSmem) {
+    } else if constexpr (TK == kTreeSmem) {
         bad = !build_walk(prow, N, p.slots, tv);
     }
     if (p.early_tree) {
@@ -1125,13 +1166,13 @@ __global__ void __launch_bounds__(kMaxWarps * 32) gdn_verify_staged(const KParam
         return;
     }
     // 5. descriptors, then the walk
-    if constexpr (TREE == kTreeChain)
+    if constexpr (TK == kTreeChain)
         staged_finish<DK, C, RL, QT, ST, TREE>(S, p, NoTree{}, raw, ab, desc, slotbuf, sin_lane, b, h,
                                                row0, L);
-    else if constexpr (TREE == kTreeIndex)
+    else if constexpr (TK == kTreeIndex)
         staged_finish<DK, C, RL, QT, ST, TREE>(S, p, IndexTree{tsm}, raw, ab, desc, slotbuf, sin_lane, b,
                                                h, row0, L);
-    else if constexpr (TREE == kTreeWarp)
+    else if constexpr (TK == kTreeWarp)
         staged_finish<DK, C, RL, QT, ST, TREE>(S, p, MaskTree{tsm}, raw, ab, desc, slotbuf, sin_lane, b,
                                                h, row0, L);
     else
@@ -1215,6 +1256,8 @@ struct RingCtx {
     {
         return reinterpret_cast<const PosDesc*>(slot(pos) + desc_off)[pos % kChunk];
     }
+    // only within the chunk already waited for
+    __device__ __forceinline__ bool ahead(int pos) const { return pos % kChunk != 0; }
     __device__ __forceinline__ const QT* rec(int pos, int) const
     {
         return reinterpret_cast<const QT*>(slot(pos) + (size_t)(pos % kChunk) * raw_bytes);
@@ -1391,7 +1434,7 @@ __global__ void __launch_bounds__((kMaxWarps + 1) * 32) gdn_verify_ring(const KP
     load_rows<DK, C, RL>(S, sin_lane);
     const GlobalFetch<DK, C, RL, QT> gf{kg, vg, p.g, p.beta, (size_t)b * N, p.Hk, p.Hv, p.dv, hk, h, row0, L};
     RingCtx<DK, C, RL, QT> ctx{full, empty, ring, p.raw_bytes, slot_bytes, desc_off, p.status, lane, gf};
-    float* lane_slot = slotbuf + 4 * threadIdx.x;
+    float* lane_slot = cta_slots<DK, TREE>(p, slotbuf) + 4 * threadIdx.x;
     if constexpr (CHAIN)
         walk<DK, C, RL, QT, ST, TREE>(S, p, NoTree{}, lane_slot, sin_lane, b, h, row0, L, ctx);
     else if constexpr (INDEX)
@@ -1463,14 +1506,17 @@ cudaError_t launch_one(const KParams& kp, const VerifyArgs& a, const VerifyGeom&
         if (geom.reload)
             return launch_staged<DK, C, RL, QT, ST, kTreeIndex>(kp, a, geom, stream);
         if (geom.warp_tree)
-            return launch_staged<DK, C, RL, QT, ST, kTreeWarp>(kp, a, geom, stream);
-        return launch_staged<DK, C, RL, QT, ST, kTreeSmem>(kp, a, geom, stream);
+            return geom.gslots ? launch_staged<DK, C, RL, QT, ST, kTreeWarp + kTreeGlobal>(kp, a, geom, stream)
+                               : launch_staged<DK, C, RL, QT, ST, kTreeWarp>(kp, a, geom, stream);
+        return geom.gslots ? launch_staged<DK, C, RL, QT, ST, kTreeSmem + kTreeGlobal>(kp, a, geom, stream)
+                           : launch_staged<DK, C, RL, QT, ST, kTreeSmem>(kp, a, geom, stream);
     }
     if (CHAIN)
         return launch_ring<DK, C, RL, QT, ST, kTreeChain>(kp, a, geom, stream);
     if (geom.reload)
         return launch_ring<DK, C, RL, QT, ST, kTreeIndex>(kp, a, geom, stream);
-    return launch_ring<DK, C, RL, QT, ST, kTreeSmem>(kp, a, geom, stream);
+    return geom.gslots ? launch_ring<DK, C, RL, QT, ST, kTreeSmem + kTreeGlobal>(kp, a, geom, stream)
+                       : launch_ring<DK, C, RL, QT, ST, kTreeSmem>(kp, a, geom, stream);
 }
 
 template <int DK, int C, int RL, typename QT, typename ST>

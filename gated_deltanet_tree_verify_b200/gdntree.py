@@ -73,6 +73,10 @@ def load_library() -> ctypes.CDLL:
     dp = ctypes.POINTER(GdnTreeDesc)
     lib.gdn_tree_verify.argtypes = [dp] + [vp] * 10
     lib.gdn_tree_verify.restype = ctypes.c_int
+    lib.gdn_tree_verify_ws.argtypes = [dp] + [vp] * 10 + [ctypes.c_size_t, vp]
+    lib.gdn_tree_verify_ws.restype = ctypes.c_int
+    lib.gdn_tree_verify_workspace_bytes.argtypes = [dp]
+    lib.gdn_tree_verify_workspace_bytes.restype = ctypes.c_size_t
     lib.gdn_tree_commit.argtypes = [dp, vp, vp, vp, vp, i32, vp, vp]
     lib.gdn_tree_commit.restype = ctypes.c_int
     lib.gdn_tree_commit_layers.argtypes = [dp, i32, ctypes.POINTER(vp), vp, vp, vp, i32,
@@ -162,6 +166,25 @@ def gdn_tree_verify(desc: GdnTreeDesc, q, k, v, g, beta, parent_idx, state_in, o
                              _ptr(g, "g"), _ptr(beta, "beta"), _ptr(parent_idx, "parent_idx"),
                              _ptr(state_in, "state_in"), _ptr(out, "out"),
                              _ptr(node_states, "node_states"), _stream(stream))
+    return _check(rc, check)
+
+
+def gdn_tree_verify_workspace_bytes(desc: GdnTreeDesc) -> int:
+    return int(load_library().gdn_tree_verify_workspace_bytes(ctypes.byref(desc)))
+
+
+def gdn_tree_verify_ws(desc: GdnTreeDesc, q, k, v, g, beta, parent_idx, state_in, out, node_states,
+                       workspace, workspace_bytes: Optional[int] = None, stream=None, check: bool = True) -> int:
+    """Calls gdn_tree_verify_ws (see include/gdntree.h).  ``workspace_bytes``
+    defaults to the tensor's size in bytes."""
+    lib = load_library()
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size() if isinstance(workspace, torch.Tensor) else 0
+    rc = lib.gdn_tree_verify_ws(ctypes.byref(desc), _ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"),
+                                _ptr(g, "g"), _ptr(beta, "beta"), _ptr(parent_idx, "parent_idx"),
+                                _ptr(state_in, "state_in"), _ptr(out, "out"),
+                                _ptr(node_states, "node_states"), _ptr(workspace, "workspace"),
+                                int(workspace_bytes), _stream(stream))
     return _check(rc, check)
 
 

@@ -142,6 +142,40 @@ gdn_status gdn_tree_verify(const gdn_tree_desc* desc, const void* q, const void*
                            void* node_states, cudaStream_t stream);
 
 /*
+ * gdn_tree_verify_ws -- gdn_tree_verify with a caller-owned device workspace
+ * for the walk's stack of branch states.
+ *
+ * With state_dtype f16 (or GDN_FLAG_PERSIST_LAST) a tree walk keeps the f32
+ * states of branching nodes until their later children run.  Without a
+ * workspace they live in shared memory, which caps the resident CTAs per SM
+ * for trees above ~32 nodes; with one they live in global memory (mostly
+ * L2), each loaded one node ahead of its use.  Results are bit-identical
+ * either way (the walk order and arithmetic do not change).
+ *
+ *   workspace        DEVICE buffer, 16-byte aligned, or NULL (then exactly
+ *                    gdn_tree_verify); contents on entry are ignored and on
+ *                    return undefined; it must not overlap any other buffer
+ *                    of the call, and a call in flight owns it
+ *   workspace_bytes  its size; at least gdn_tree_verify_workspace_bytes(desc)
+ *                    when that is nonzero (else GDN_ERR_INVALID_ARG)
+ *
+ * The other arguments, layouts and errors are those of gdn_tree_verify.
+ * The pages define no workspace: it is this library's placement of the
+ * walk's branch states, not part of the method.
+ */
+gdn_status gdn_tree_verify_ws(const gdn_tree_desc* desc, const void* q, const void* k,
+                              const void* v, const float* g, const float* beta,
+                              const int32_t* parent_idx, const float* state_in, float* out,
+                              void* node_states, void* workspace, size_t workspace_bytes,
+                              cudaStream_t stream);
+
+/* Workspace bytes gdn_tree_verify_ws needs for a desc: B * H_v * d_v * d_k *
+ * 4 * (stack slots, at most 4) for walks that keep branch states, 0 for
+ * chains, f32 trees (their branch states are re-read from node_states) and
+ * invalid descs.  Independent of the buffers' addresses. */
+size_t gdn_tree_verify_workspace_bytes(const gdn_tree_desc* desc);
+
+/*
  * gdn_tree_commit -- write the accepted path's state back as the new
  * recurrent state, without re-running the path.
  *

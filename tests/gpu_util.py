@@ -24,8 +24,10 @@ def to_dev(prob):
             ("q", "k", "v", "g", "beta", "parent", "state_in", "accept_path", "accept_len")}
 
 
-def run(prob, state_dtype="f32", flags=0, parent=True, commit=True, dev=None, stream=None):
-    """Verify (+ commit) on the GPU.  Unwritten outputs stay NaN."""
+def run(prob, state_dtype="f32", flags=0, parent=True, commit=True, dev=None, stream=None, workspace=False):
+    """Verify (+ commit) on the GPU.  Unwritten outputs stay NaN.  With
+    ``workspace``, through gdn_tree_verify_ws with a NaN-filled workspace of
+    exactly gdn_tree_verify_workspace_bytes."""
     d = dev or to_dev(prob)
     B, N, Hk, dk = prob.q.shape
     Hv, dv = prob.v.shape[2], prob.v.shape[3]
@@ -39,8 +41,14 @@ def run(prob, state_dtype="f32", flags=0, parent=True, commit=True, dev=None, st
                          scale=prob.scale, qkv_dtype=prob.q.dtype, state_dtype=sd, flags=flags,
                          status=status)
     par = d["parent"] if parent else None
-    gdn.gdn_tree_verify(desc, d["q"], d["k"], d["v"], d["g"], d["beta"], par, d["state_in"], out, ns,
-                        stream=stream)
+    if workspace:
+        nbytes = gdn.gdn_tree_verify_workspace_bytes(desc)
+        ws = torch.full((max(nbytes, 16) // 4,), float("nan"), device="cuda")
+        gdn.gdn_tree_verify_ws(desc, d["q"], d["k"], d["v"], d["g"], d["beta"], par, d["state_in"], out, ns,
+                               ws, nbytes, stream=stream)
+    else:
+        gdn.gdn_tree_verify(desc, d["q"], d["k"], d["v"], d["g"], d["beta"], par, d["state_in"], out, ns,
+                            stream=stream)
     if commit:
         gdn.gdn_tree_commit(desc, ns, par, d["accept_path"], d["accept_len"], d["accept_path"].shape[1],
                             so, stream=stream)

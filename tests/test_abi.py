@@ -172,3 +172,35 @@ def test_commit_layers_host_checks(lib):
     assert _commit_layers(_desc(), ns, [so[0], ns[2] + 4096, so[2]]) == gdn.GDN_ERR_INVALID_ARG
     with pytest.raises(ValueError):
         gdn.gdn_tree_commit_layers(_desc(), ns, 0, 0, 0, 4, so[:2], stream=0)
+
+
+def test_verify_workspace_bytes(lib):
+    # f16 tree: B * Hv * dv * dk * 4 bytes per stack slot, floor(log2 N) slots capped at 4
+    d = _desc(state_dtype=gdn.GDN_F16)                      # N = 23: 4 slots
+    assert gdn.gdn_tree_verify_workspace_bytes(d) == 48 * 128 * 128 * 4 * 4
+    assert gdn.gdn_tree_verify_workspace_bytes(_desc(state_dtype=gdn.GDN_F16, n_nodes=3)) == 48 * 128 * 128 * 4
+    assert gdn.gdn_tree_verify_workspace_bytes(_desc(state_dtype=gdn.GDN_F16, batch=3, n_nodes=129)) == \
+        3 * 48 * 128 * 128 * 4 * 4
+    # f32 trees re-read branch states from node_states; chains keep none
+    assert gdn.gdn_tree_verify_workspace_bytes(_desc()) == 0
+    assert gdn.gdn_tree_verify_workspace_bytes(_desc(state_dtype=gdn.GDN_F16, flags=gdn.GDN_FLAG_CHAIN)) == 0
+    assert gdn.gdn_tree_verify_workspace_bytes(_desc(flags=gdn.GDN_FLAG_PERSIST_LAST)) > 0
+    assert gdn.gdn_tree_verify_workspace_bytes(_desc(d_k=48)) == 0
+
+
+def _verify_ws(desc, ws, nbytes, ptrs=None):
+    q, k, v, g, beta, par, sin, out, ns = (ptrs or _ptrs())[:9]
+    return gdn.gdn_tree_verify_ws(desc, q, k, v, g, beta, par, sin, out, ns, ws, nbytes, stream=0, check=False)
+
+
+def test_verify_ws_host_checks(lib):
+    d = _desc(state_dtype=gdn.GDN_F16)
+    need = gdn.gdn_tree_verify_workspace_bytes(d)
+    ws = BASE + 20 * MB
+    assert _verify_ws(d, ws, need - 1) == gdn.GDN_ERR_INVALID_ARG
+    assert "workspace" in lib.gdn_last_error_detail().decode()
+    assert _verify_ws(d, ws + 8, need) == gdn.GDN_ERR_INVALID_ARG      # misaligned
+    assert _verify_ws(_desc(batch=0, state_dtype=gdn.GDN_F16), ws, 0) == gdn.GDN_OK
+    p = _ptrs()
+    assert _verify_ws(d, p[8] + 64, need, p) == gdn.GDN_ERR_INVALID_ARG  # inside node_states
+    assert _verify_ws(d, p[0], need, p) == gdn.GDN_ERR_INVALID_ARG       # on top of q
