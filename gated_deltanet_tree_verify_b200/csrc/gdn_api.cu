@@ -2,6 +2,7 @@
 // checks, then one kernel launch on the caller's stream.  See include/gdntree.h
 // for the contract of each call.
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
@@ -314,6 +315,71 @@ gdn_status gdn_tree_commit(const gdn_tree_desc* desc, const void* node_states,
     }
     return gdn_tree_commit_layers(desc, 1, &node_states, parent_idx, accept_path, accept_len,
                                   max_path_len, &state_out, stream);
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// gdn_tree_verify_static_ws: the workspace path with a library-owned static
+// device buffer, for callers that allocate nothing per call.
+// ---------------------------------------------------------------------------
+
+namespace {
+
+constexpr size_t kStaticWorkspaceBytes = size_t(32) << 20;
+constexpr int kMaxStaticDevices = 64;
+
+// One buffer per device context, shared by every call in the process.
+__device__ __align__(256) unsigned char g_static_ws[kStaticWorkspaceBytes];
+
+// Device address of g_static_ws per device, looked up on first use there.
+std::atomic<void*> g_static_ws_addr[kMaxStaticDevices];
+
+gdn_status static_ws_address(void** out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return fail(GDN_ERR_CUDA, "cudaGetDevice failed: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxStaticDevices)
+        return fail(GDN_ERR_UNSUPPORTED, "device ordinal above the static workspace table%s");
+    void* p = g_static_ws_addr[dev].load(std::memory_order_acquire);
+    if (p == nullptr) {
+        e = cudaGetSymbolAddress(&p, g_static_ws);
+        if (e != cudaSuccess)
+            return fail(GDN_ERR_CUDA, "cudaGetSymbolAddress failed: %s", cudaGetErrorString(e));
+        g_static_ws_addr[dev].store(p, std::memory_order_release);
+    }
+    *out = p;
+    return GDN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t gdn_static_workspace_capacity(void) { return kStaticWorkspaceBytes; }
+
+gdn_status gdn_tree_verify_static_ws(const gdn_tree_desc* desc, const void* q, const void* k,
+                                     const void* v, const float* g, const float* beta,
+                                     const int32_t* parent_idx, const float* state_in, float* out,
+                                     void* node_states, cudaStream_t stream)
+{
+    g_detail[0] = '\0';
+    gdn_status st = check_desc(desc, true);
+    if (st != GDN_OK)
+        return st;
+    const size_t need = gdn_tree_verify_workspace_bytes(desc);
+    if (need == 0 || desc->batch == 0)
+        return verify_impl(desc, q, k, v, g, beta, parent_idx, state_in, out, node_states, nullptr, 0, stream);
+    if (need > kStaticWorkspaceBytes)
+        return fail(GDN_ERR_UNSUPPORTED, "workspace needed exceeds gdn_static_workspace_capacity()%s");
+    void* ws = nullptr;
+    st = static_ws_address(&ws);
+    if (st != GDN_OK)
+        return st;
+    return verify_impl(desc, q, k, v, g, beta, parent_idx, state_in, out, node_states, ws,
+                       kStaticWorkspaceBytes, stream);
 }
 
 }  // extern "C"

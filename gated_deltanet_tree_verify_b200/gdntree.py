@@ -77,6 +77,10 @@ def load_library() -> ctypes.CDLL:
     lib.gdn_tree_verify_ws.restype = ctypes.c_int
     lib.gdn_tree_verify_workspace_bytes.argtypes = [dp]
     lib.gdn_tree_verify_workspace_bytes.restype = ctypes.c_size_t
+    lib.gdn_tree_verify_static_ws.argtypes = [dp] + [vp] * 10
+    lib.gdn_tree_verify_static_ws.restype = ctypes.c_int
+    lib.gdn_static_workspace_capacity.argtypes = []
+    lib.gdn_static_workspace_capacity.restype = ctypes.c_size_t
     lib.gdn_tree_commit.argtypes = [dp, vp, vp, vp, vp, i32, vp, vp]
     lib.gdn_tree_commit.restype = ctypes.c_int
     lib.gdn_tree_commit_layers.argtypes = [dp, i32, ctypes.POINTER(vp), vp, vp, vp, i32,
@@ -185,6 +189,22 @@ def gdn_tree_verify_ws(desc: GdnTreeDesc, q, k, v, g, beta, parent_idx, state_in
                                 _ptr(state_in, "state_in"), _ptr(out, "out"),
                                 _ptr(node_states, "node_states"), _ptr(workspace, "workspace"),
                                 int(workspace_bytes), _stream(stream))
+    return _check(rc, check)
+
+
+def gdn_static_workspace_capacity() -> int:
+    return int(load_library().gdn_static_workspace_capacity())
+
+
+def gdn_tree_verify_static_ws(desc: GdnTreeDesc, q, k, v, g, beta, parent_idx, state_in, out, node_states,
+                              stream=None, check: bool = True) -> int:
+    """Calls gdn_tree_verify_static_ws (see include/gdntree.h): the library's
+    static device workspace, shared by every call on the device."""
+    lib = load_library()
+    rc = lib.gdn_tree_verify_static_ws(ctypes.byref(desc), _ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"),
+                                       _ptr(g, "g"), _ptr(beta, "beta"), _ptr(parent_idx, "parent_idx"),
+                                       _ptr(state_in, "state_in"), _ptr(out, "out"),
+                                       _ptr(node_states, "node_states"), _stream(stream))
     return _check(rc, check)
 
 

@@ -176,6 +176,32 @@ gdn_status gdn_tree_verify_ws(const gdn_tree_desc* desc, const void* q, const vo
 size_t gdn_tree_verify_workspace_bytes(const gdn_tree_desc* desc);
 
 /*
+ * gdn_tree_verify_static_ws -- gdn_tree_verify_ws without a caller
+ * workspace: the library keeps one static device buffer of
+ * gdn_static_workspace_capacity() bytes per device (a __device__ array,
+ * resolved with cudaGetSymbolAddress on first use on each device) and
+ * allocates nothing per call.  The source pages describe no counterpart; it
+ * exists for callers that cannot allocate on the hot path.
+ *
+ * Same arguments, layouts and results as gdn_tree_verify.  When the desc
+ * needs no workspace (gdn_tree_verify_workspace_bytes(desc) == 0) this is
+ * gdn_tree_verify.  When it needs more than the capacity:
+ * GDN_ERR_UNSUPPORTED, nothing launched.
+ *
+ * Races: the buffer is shared by every call in the process on that device.
+ * Calls on one device must be ordered (one stream, or events between
+ * streams); two calls in flight at once on different streams or host
+ * threads overwrite each other's branch states and give wrong results.
+ */
+gdn_status gdn_tree_verify_static_ws(const gdn_tree_desc* desc, const void* q, const void* k,
+                                     const void* v, const float* g, const float* beta,
+                                     const int32_t* parent_idx, const float* state_in, float* out,
+                                     void* node_states, cudaStream_t stream);
+
+/* Bytes of the static workspace behind gdn_tree_verify_static_ws. */
+size_t gdn_static_workspace_capacity(void);
+
+/*
  * gdn_tree_commit -- write the accepted path's state back as the new
  * recurrent state, without re-running the path.
  *
