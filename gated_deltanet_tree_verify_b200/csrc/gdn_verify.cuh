@@ -1227,10 +1227,8 @@ struct RingCtx {
     int32_t* status;
     int lane;
     GlobalFetch<DK, C, RL, QT> gf;
-    __device__ __forceinline__ const unsigned char* slot(int pos) const
-    {
-        return ring + (size_t)((pos / kChunk) % kRing) * slot_bytes;
-    }
+    const unsigned char* cur = nullptr;  // the slot of the current chunk
+    __device__ __forceinline__ const unsigned char* slot(int) const { return cur; }
     __device__ __forceinline__ bool begin(int pos)
     {
         if (pos % kChunk == 0) {
@@ -1239,6 +1237,7 @@ struct RingCtx {
                 report_status(status, kStatusTimeout);
                 return false;
             }
+            cur = ring + (size_t)(c % kRing) * slot_bytes;
         }
         return true;
     }
