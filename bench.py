@@ -31,6 +31,7 @@ import sys
 import threading
 import time
 
+import numpy as np
 import torch
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -559,6 +560,64 @@ def _verify_point(*, batch, n_nodes, tree, state_dtype, flags=0, gate="softplus"
     return per_launch_s, R
 
 
+def _varlen_point(*, budgets, state_dtype, workspace=False, reps=20, min_bytes=512 << 20, seed=21):
+    """Mean time of one gdn_tree_verify_varlen launch over len(budgets)
+    DDTree-style trees of those budgets, packed along the node dimension."""
+    import gated_deltanet_tree_verify_b200 as gdn
+    tdt = torch.float32 if state_dtype == "f32" else torch.float16
+    sizes = [b + 1 for b in budgets]
+    T, B, Nmax = sum(sizes), len(sizes), max(sizes)
+    one = verify_bytes(1, 1, state_dtype) - N_V_HEADS * D * D * 4  # per node
+    R = max(2, min(16, -(-min_bytes // (T * one + B * N_V_HEADS * D * D * 4))))
+    sets = []
+    for r in range(R):
+        seqs = [make_problem(batch=1, n_nodes=n, n_k_heads=N_K_HEADS, n_v_heads=N_V_HEADS, d_k=D, d_v=D,
+                             tree="ddtree", seed=seed + 1000 * r + i, qkv_dtype="bf16", accept="root")
+                for i, n in enumerate(sizes)]
+        cat = lambda key: torch.cat([getattr(x, key)[0] for x in seqs]).contiguous().cuda()  # noqa: E731
+        d = dict(q=cat("q"), k=cat("k"), v=cat("v"), g=cat("g"), beta=cat("beta"), parent=cat("parent"),
+                 state_in=torch.cat([x.state_in for x in seqs]).contiguous().cuda(),
+                 cu=torch.tensor([0] + list(np.cumsum(sizes)), dtype=torch.int32).cuda())
+        d["out"] = torch.empty(T, N_V_HEADS, D, device="cuda")
+        d["ns"] = torch.empty(T, N_V_HEADS, D, D, device="cuda", dtype=tdt)
+        sets.append(d)
+    desc = gdn.make_desc(batch=B, n_nodes=Nmax, n_k_heads=N_K_HEADS, n_v_heads=N_V_HEADS, d_k=D, d_v=D,
+                         scale=float(D) ** -0.5, qkv_dtype=gdn.GDN_BF16,
+                         state_dtype=gdn.GDN_F32 if state_dtype == "f32" else gdn.GDN_F16)
+    ws_bytes = gdn.gdn_tree_verify_workspace_bytes(desc) if workspace else 0
+    for d in sets:
+        d["ws"] = torch.empty(max(ws_bytes, 16) // 4, device="cuda") if ws_bytes else None
+
+    def run_all():
+        for d in sets:
+            gdn.gdn_tree_verify_varlen(desc, d["cu"], T, d["q"], d["k"], d["v"], d["g"], d["beta"], d["parent"],
+                                       d["state_in"], d["out"], d["ns"], d["ws"], ws_bytes)
+
+    run_all()
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        run_all()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        run_all()
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    t = e0.elapsed_time(e1) / 1e3 / (reps * R)
+    del graph
+    return t, T * one + B * N_V_HEADS * D * D * 4, T
+
+
 def run_sweep(args):
     import gated_deltanet_tree_verify_b200 as gdn
     gdn.load_library()
@@ -573,9 +632,19 @@ def run_sweep(args):
                     points.append(dict(kind="tree", budget=budget, batch=batch, state_dtype=sd, ws=True))
     for sd in ("f32", "f16"):
         points.append(dict(kind="chain16", budget=15, batch=1, state_dtype=sd))
+    # varlen: 8 trees of budgets 8..64 in one launch
+    for sd, ws in (("f32", False), ("f16", False), ("f16", True)):
+        points.append(dict(kind="varlen", budget=0, batch=8, state_dtype=sd, ws=ws))
     points.append(dict(kind="chain4096", budget=4095, batch=8, state_dtype="f32"))
+    varlen_budgets = [8, 64, 22, 15, 32, 22, 48, 8]
     for pt in points:
         n = pt["budget"] + 1
+        if pt["kind"] == "varlen":
+            t, vb, T = _varlen_point(budgets=varlen_budgets, state_dtype=pt["state_dtype"], workspace=pt["ws"])
+            print(json.dumps({"sweep": "varlen", "budgets": varlen_budgets, "state_dtype": pt["state_dtype"],
+                              "workspace": pt["ws"], "verify_us": t * 1e6, "node_layers_per_s": T / t,
+                              "gbps": vb / t / 1e9, "frac_of_hbm": vb / t / 1e9 / peak}), flush=True)
+            continue
         if pt["kind"] == "chain4096":
             flags = gdn.GDN_FLAG_CHAIN | gdn.GDN_FLAG_PERSIST_LAST
             t, R = _verify_point(batch=pt["batch"], n_nodes=n, tree="chain", state_dtype="f32", flags=flags,

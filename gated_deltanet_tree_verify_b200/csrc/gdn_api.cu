@@ -78,6 +78,32 @@ size_t node_states_bytes(const gdn_tree_desc* d)
     return (size_t)d->batch * ns * d->n_v_heads * d->d_v * d->d_k * elem_size(d->state_dtype);
 }
 
+// Nodes of the node dimension: B N, or the varlen total.
+size_t total_nodes(const gdn_tree_desc& d, const int32_t* cu, int32_t total)
+{
+    return cu ? (size_t)total : (size_t)d.batch * d.n_nodes;
+}
+
+// node_states bytes for a fixed or varlen layout.
+size_t node_states_bytes_v(const gdn_tree_desc& d, const int32_t* cu, int32_t total)
+{
+    const size_t ns = (d.flags & GDN_FLAG_PERSIST_LAST) ? (size_t)d.batch : total_nodes(d, cu, total);
+    return ns * d.n_v_heads * d.d_v * d.d_k * elem_size(d.state_dtype);
+}
+
+// Host checks of the varlen arguments (cu_nodes itself is device memory;
+// the kernels check its entries).
+gdn_status check_varlen(const gdn_tree_desc& d, const int32_t* cu, int32_t total)
+{
+    if (!cu)
+        return fail(GDN_ERR_INVALID_ARG, "cu_nodes is NULL%s");
+    if (!aligned(cu, 4))
+        return fail(GDN_ERR_INVALID_ARG, "cu_nodes is misaligned%s");
+    if (total < d.batch || (long long)total > (long long)d.batch * d.n_nodes)
+        return fail(GDN_ERR_INVALID_ARG, "total_nodes outside [batch, batch * n_nodes]%s");
+    return GDN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -129,16 +155,18 @@ gdn::VerifyArgs verify_args(const gdn_tree_desc& d)
     return a;
 }
 
-gdn_status verify_impl(const gdn_tree_desc* desc, const void* q, const void* k, const void* v,
-                       const float* g, const float* beta, const int32_t* parent_idx, const float* state_in,
-                       float* out, void* node_states, void* workspace, size_t workspace_bytes,
-                       cudaStream_t stream)
+gdn_status verify_impl(const gdn_tree_desc* desc, const int32_t* cu, int32_t total, const void* q,
+                       const void* k, const void* v, const float* g, const float* beta,
+                       const int32_t* parent_idx, const float* state_in, float* out, void* node_states,
+                       void* workspace, size_t workspace_bytes, cudaStream_t stream, bool varlen)
 {
     g_detail[0] = '\0';
     gdn_status st = check_desc(desc, true);
     if (st != GDN_OK)
         return st;
     const gdn_tree_desc& d = *desc;
+    if (varlen && (st = check_varlen(d, cu, total)) != GDN_OK)
+        return st;
     const bool chain = (d.flags & GDN_FLAG_CHAIN) != 0;
     const bool need_parent = !chain || (d.flags & GDN_FLAG_VALIDATE);
     if (!q || !k || !v || !g || !beta || !state_in || !out || !node_states || (need_parent && !parent_idx))
@@ -163,6 +191,8 @@ gdn_status verify_impl(const gdn_tree_desc* desc, const void* q, const void* k, 
     a.out = out;
     a.node_states = node_states;
     a.workspace = static_cast<float*>(workspace);
+    a.cu_nodes = varlen ? cu : nullptr;
+    a.total_nodes = varlen ? total : 0;
     const gdn::VerifyGeom geom = gdn::verify_geometry(a, workspace != nullptr);
     if (geom.tiles <= 0 || geom.smem > 227 * 1024)
         return fail(GDN_ERR_UNSUPPORTED, "no launch geometry for this shape%s");
@@ -171,15 +201,16 @@ gdn_status verify_impl(const gdn_tree_desc* desc, const void* q, const void* k, 
     if (geom.gslots && workspace_bytes < geom.ws_bytes)
         return fail(GDN_ERR_INVALID_ARG, "workspace smaller than gdn_tree_verify_workspace_bytes()%s");
 
-    const size_t B = d.batch, N = d.n_nodes, Hk = d.n_k_heads, Hv = d.n_v_heads, dk = d.d_k, dv = d.d_v;
+    const size_t B = d.batch, T = total_nodes(d, a.cu_nodes, total), Hk = d.n_k_heads, Hv = d.n_v_heads,
+                 dk = d.d_k, dv = d.d_v;
     const size_t es = elem_size(d.qkv_dtype);
-    const Range ins[] = {{q, B * N * Hk * dk * es, "q"},     {k, B * N * Hk * dk * es, "k"},
-                         {v, B * N * Hv * dv * es, "v"},     {g, B * N * Hv * 4, "g"},
-                         {beta, B * N * Hv * 4, "beta"},     {parent_idx, B * N * 4, "parent_idx"},
+    const Range ins[] = {{q, T * Hk * dk * es, "q"},     {k, T * Hk * dk * es, "k"},
+                         {v, T * Hv * dv * es, "v"},     {g, T * Hv * 4, "g"},
+                         {beta, T * Hv * 4, "beta"},     {parent_idx, T * 4, "parent_idx"},
                          {state_in, B * Hv * dv * dk * 4, "state_in"},
-                         {d.status, 4, "status"}};
-    const Range outs[] = {{out, B * N * Hv * dv * 4, "out"},
-                          {node_states, node_states_bytes(&d), "node_states"},
+                         {d.status, 4, "status"},       {a.cu_nodes, (B + 1) * 4, "cu_nodes"}};
+    const Range outs[] = {{out, T * Hv * dv * 4, "out"},
+                          {node_states, node_states_bytes_v(d, a.cu_nodes, total), "node_states"},
                           {geom.gslots ? workspace : nullptr, geom.ws_bytes, "workspace"}};
     for (int i = 0; i < 3; ++i)
         for (int j = i + 1; j < 3; ++j)
@@ -204,7 +235,8 @@ gdn_status gdn_tree_verify(const gdn_tree_desc* desc, const void* q, const void*
                            const float* state_in, float* out, void* node_states,
                            cudaStream_t stream)
 {
-    return verify_impl(desc, q, k, v, g, beta, parent_idx, state_in, out, node_states, nullptr, 0, stream);
+    return verify_impl(desc, nullptr, 0, q, k, v, g, beta, parent_idx, state_in, out, node_states, nullptr, 0, stream,
+                       false);
 }
 
 gdn_status gdn_tree_verify_ws(const gdn_tree_desc* desc, const void* q, const void* k, const void* v,
@@ -212,8 +244,18 @@ gdn_status gdn_tree_verify_ws(const gdn_tree_desc* desc, const void* q, const vo
                               const float* state_in, float* out, void* node_states, void* workspace,
                               size_t workspace_bytes, cudaStream_t stream)
 {
-    return verify_impl(desc, q, k, v, g, beta, parent_idx, state_in, out, node_states, workspace,
-                       workspace_bytes, stream);
+    return verify_impl(desc, nullptr, 0, q, k, v, g, beta, parent_idx, state_in, out, node_states, workspace,
+                       workspace_bytes, stream, false);
+}
+
+gdn_status gdn_tree_verify_varlen(const gdn_tree_desc* desc, const int32_t* cu_nodes, int32_t total_nodes,
+                                  const void* q, const void* k, const void* v, const float* g,
+                                  const float* beta, const int32_t* parent_idx, const float* state_in,
+                                  float* out, void* node_states, void* workspace, size_t workspace_bytes,
+                                  cudaStream_t stream)
+{
+    return verify_impl(desc, cu_nodes, total_nodes, q, k, v, g, beta, parent_idx, state_in, out, node_states,
+                       workspace, workspace_bytes, stream, true);
 }
 
 size_t gdn_tree_verify_workspace_bytes(const gdn_tree_desc* desc)
@@ -224,16 +266,24 @@ size_t gdn_tree_verify_workspace_bytes(const gdn_tree_desc* desc)
     return geom.tiles > 0 ? geom.ws_bytes : 0;
 }
 
-gdn_status gdn_tree_commit_layers(const gdn_tree_desc* desc, int32_t n_layers,
-                                  const void* const* node_states, const int32_t* parent_idx,
-                                  const int32_t* accept_path, const int32_t* accept_len,
-                                  int32_t max_path_len, float* const* state_out, cudaStream_t stream)
+}  // extern "C"
+
+namespace {
+
+gdn_status commit_impl(const gdn_tree_desc* desc, const int32_t* cu, int32_t total, int32_t n_layers,
+                       const void* const* node_states, const int32_t* parent_idx, const int32_t* accept_path,
+                       const int32_t* accept_len, int32_t max_path_len, float* const* state_out,
+                       cudaStream_t stream, bool varlen)
 {
     g_detail[0] = '\0';
     gdn_status st = check_desc(desc, false);
     if (st != GDN_OK)
         return st;
     const gdn_tree_desc& d = *desc;
+    if (varlen && (st = check_varlen(d, cu, total)) != GDN_OK)
+        return st;
+    if (!varlen)
+        cu = nullptr;
     const bool chain = (d.flags & GDN_FLAG_CHAIN) != 0;
     if (n_layers < 0)
         return fail(GDN_ERR_INVALID_ARG, "n_layers < 0%s");
@@ -259,17 +309,18 @@ gdn_status gdn_tree_commit_layers(const gdn_tree_desc* desc, int32_t n_layers,
         return GDN_OK;
     const size_t B = d.batch;
     const size_t so_bytes = B * d.n_v_heads * d.d_v * d.d_k * 4;
-    const Range shared_in[] = {{parent_idx, B * d.n_nodes * 4, "parent_idx"},
+    const Range shared_in[] = {{parent_idx, total_nodes(d, cu, total) * 4, "parent_idx"},
                                {accept_path, B * (size_t)max_path_len * 4, "accept_path"},
                                {accept_len, B * 4, "accept_len"},
-                               {d.status, 4, "status"}};
+                               {d.status, 4, "status"},
+                               {cu, (B + 1) * 4, "cu_nodes"}};
     for (int l = 0; l < n_layers; ++l) {
         const Range so{state_out[l], so_bytes, "state_out"};
         for (const auto& i : shared_in)
             if (overlap(so, i))
                 return fail(GDN_ERR_INVALID_ARG, "state_out overlaps input %s", i.name);
         for (int m = 0; m < n_layers; ++m) {
-            const Range ns{node_states[m], node_states_bytes(&d), "node_states"};
+            const Range ns{node_states[m], node_states_bytes_v(d, cu, total), "node_states"};
             if (overlap(so, ns))
                 return fail(GDN_ERR_INVALID_ARG, "state_out overlaps node_states%s");
             if (m != l && overlap(so, Range{state_out[m], so_bytes, "state_out"}))
@@ -295,10 +346,34 @@ gdn_status gdn_tree_commit_layers(const gdn_tree_desc* desc, int32_t n_layers,
     a.max_path_len = max_path_len;
     a.state_dtype = d.state_dtype;
     a.flags = d.flags;
+    a.cu_nodes = cu;
+    a.total_nodes = varlen ? total : 0;
     const cudaError_t e = gdn::launch_commit(a, stream);
     if (e != cudaSuccess)
         return fail(GDN_ERR_CUDA, "commit launch failed: %s", cudaGetErrorString(e));
     return GDN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+gdn_status gdn_tree_commit_layers(const gdn_tree_desc* desc, int32_t n_layers,
+                                  const void* const* node_states, const int32_t* parent_idx,
+                                  const int32_t* accept_path, const int32_t* accept_len,
+                                  int32_t max_path_len, float* const* state_out, cudaStream_t stream)
+{
+    return commit_impl(desc, nullptr, 0, n_layers, node_states, parent_idx, accept_path, accept_len, max_path_len,
+                       state_out, stream, false);
+}
+
+gdn_status gdn_tree_commit_varlen(const gdn_tree_desc* desc, const int32_t* cu_nodes, int32_t total_nodes,
+                                  int32_t n_layers, const void* const* node_states, const int32_t* parent_idx,
+                                  const int32_t* accept_path, const int32_t* accept_len, int32_t max_path_len,
+                                  float* const* state_out, cudaStream_t stream)
+{
+    return commit_impl(desc, cu_nodes, total_nodes, n_layers, node_states, parent_idx, accept_path, accept_len,
+                       max_path_len, state_out, stream, true);
 }
 
 gdn_status gdn_tree_commit(const gdn_tree_desc* desc, const void* node_states,
@@ -371,15 +446,16 @@ gdn_status gdn_tree_verify_static_ws(const gdn_tree_desc* desc, const void* q, c
         return st;
     const size_t need = gdn_tree_verify_workspace_bytes(desc);
     if (need == 0 || desc->batch == 0)
-        return verify_impl(desc, q, k, v, g, beta, parent_idx, state_in, out, node_states, nullptr, 0, stream);
+        return verify_impl(desc, nullptr, 0, q, k, v, g, beta, parent_idx, state_in, out, node_states, nullptr, 0,
+                           stream, false);
     if (need > kStaticWorkspaceBytes)
         return fail(GDN_ERR_UNSUPPORTED, "workspace needed exceeds gdn_static_workspace_capacity()%s");
     void* ws = nullptr;
     st = static_ws_address(&ws);
     if (st != GDN_OK)
         return st;
-    return verify_impl(desc, q, k, v, g, beta, parent_idx, state_in, out, node_states, ws,
-                       kStaticWorkspaceBytes, stream);
+    return verify_impl(desc, nullptr, 0, q, k, v, g, beta, parent_idx, state_in, out, node_states, ws,
+                       kStaticWorkspaceBytes, stream, false);
 }
 
 }  // extern "C"

@@ -37,7 +37,9 @@ struct CParams {
     const int32_t* accept_path;
     const int32_t* accept_len;
     int32_t* status;
-    int N, P, NS;
+    const int32_t* cu;  // varlen node offsets, or NULL
+    int total;
+    int N, P;
     int persist_last;
     size_t per_seq;  // H_v * d_v * d_k
 };
@@ -72,14 +74,26 @@ __global__ void __launch_bounds__(kCommitThreads) gdn_commit_kernel(const CParam
     const int tid = threadIdx.x;
     const int32_t* path = p.accept_path + (size_t)b * p.P;
     pdl_wait_then_release();
+    // the sequence's nodes: n0 .. n0 + N - 1 (varlen offsets checked)
+    int n0 = b * p.N, N = p.N;
+    bool seq_ok = true;
+    if (p.cu != nullptr) {
+        n0 = __ldg(p.cu + b);
+        N = __ldg(p.cu + b + 1) - n0;
+        seq_ok = n0 >= 0 && N >= 1 && N <= p.N && n0 <= p.total - N;
+        if (!seq_ok) {
+            n0 = 0;
+            N = 1;
+        }
+    }
     const int len = __ldg(p.accept_len + b);
-    const bool len_ok = len >= 1 && len <= p.N && len <= p.P;
+    const bool len_ok = seq_ok && len >= 1 && len <= N && len <= p.P;
 
     // speculative: the state of the path's last node (clamped in bounds)
     int last = len_ok ? __ldg(path + len - 1) : 0;
-    last = last < 0 ? 0 : (last >= p.N ? p.N - 1 : last);
+    last = last < 0 ? 0 : (last >= N ? N - 1 : last);
     const ST* src = static_cast<const ST*>(p.node_states[layer]) +
-                    ((size_t)b * p.NS + (p.persist_last ? 0 : last)) * p.per_seq;
+                    (p.persist_last ? (size_t)b : (size_t)n0 + last) * p.per_seq;
     const size_t e0 = (size_t)blockIdx.x * kCommitElems;
     float4 x[kPerThread];
 #pragma unroll
@@ -98,15 +112,14 @@ __global__ void __launch_bounds__(kCommitThreads) gdn_commit_kernel(const CParam
                     ok &= (xi == 0);
                 } else {
                     const int prev = __ldg(path + i - 1);
-                    const bool in_range = xi > prev && xi < p.N;
-                    const int px =
-                        (in_range && p.parent) ? __ldg(p.parent + (size_t)b * p.N + xi) : xi - 1;
+                    const bool in_range = xi > prev && xi < N;
+                    const int px = (in_range && p.parent) ? __ldg(p.parent + (size_t)n0 + xi) : xi - 1;
                     ok &= in_range && px == prev;
                 }
             }
         }
         ok = __all_sync(0xffffffffu, ok);
-        if (ok && p.persist_last && __ldg(path + len - 1) != p.N - 1)
+        if (ok && p.persist_last && __ldg(path + len - 1) != N - 1)
             ok = false;
         if (tid == 0)
             s_ok = ok ? 1 : 0;
@@ -114,7 +127,7 @@ __global__ void __launch_bounds__(kCommitThreads) gdn_commit_kernel(const CParam
     __syncthreads();
     if (!s_ok) {
         if (blockIdx.x == 0 && layer == 0 && tid == 0)
-            report_status(p.status, GDN_ERR_BAD_PATH);
+            report_status(p.status, seq_ok ? GDN_ERR_BAD_PATH : GDN_ERR_BAD_TREE);
         return;
     }
     float* dst = p.state_out[layer] + (size_t)b * p.per_seq;
@@ -138,7 +151,8 @@ cudaError_t launch_commit(const CommitArgs& a, cudaStream_t stream)
     p.N = a.n_nodes;
     p.P = a.max_path_len;
     p.persist_last = (a.flags & GDN_FLAG_PERSIST_LAST) ? 1 : 0;
-    p.NS = p.persist_last ? 1 : a.n_nodes;
+    p.cu = a.cu_nodes;
+    p.total = a.total_nodes;
     p.per_seq = (size_t)a.n_v_heads * a.d_v * a.d_k;
     const unsigned chunks = (unsigned)((p.per_seq + kCommitElems - 1) / kCommitElems);
     for (int l0 = 0; l0 < a.n_layers; l0 += kMaxCommitLayers) {

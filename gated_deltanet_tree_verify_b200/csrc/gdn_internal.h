@@ -49,6 +49,8 @@ struct VerifyArgs {
     int qkv_dtype, state_dtype;
     uint32_t flags;
     float* workspace;  // optional: stack slots in global memory
+    const int32_t* cu_nodes;  // optional (varlen): [batch + 1] node offsets; n_nodes = the most per sequence
+    int total_nodes;          // varlen: cu_nodes[batch]
 };
 
 // Layers one commit launch covers (more are split over several launches).
@@ -65,6 +67,8 @@ struct CommitArgs {
     int batch, n_nodes, n_v_heads, d_k, d_v, max_path_len;
     int state_dtype;
     uint32_t flags;
+    const int32_t* cu_nodes;  // optional (varlen), as in VerifyArgs
+    int total_nodes;
 };
 
 // Launches kernel(args...) with programmatic stream serialization allowed (see

@@ -162,6 +162,8 @@ cudaError_t launch_verify(const VerifyArgs& a, const VerifyGeom& geom, cudaStrea
     kp.validate = (a.flags & GDN_FLAG_VALIDATE) ? 1 : 0;
     kp.early_tree = (a.flags & GDN_FLAG_EARLY_TREE) ? 1 : 0;
     kp.ws = geom.gslots ? a.workspace : nullptr;
+    kp.cu = a.cu_nodes;
+    kp.total = a.total_nodes;
     kp.raw_bytes = geom.raw_bytes;
     kp.off_raw = geom.off_raw;
     kp.off_desc = geom.off_desc;

@@ -112,9 +112,31 @@ struct KParams {
     int rows, warps, slots;
     int persist_last, validate, early_tree;
     float* ws;           // global stack slots (kTreeGlobal kinds): slots x rows x d_k per CTA
+    const int32_t* cu;   // varlen: [B + 1] node offsets of the packed layout (N: the most per sequence)
+    int total;           // varlen: nodes in the packed layout
     uint32_t raw_bytes;  // one node's record (k row | q row | v slice) in bytes
     uint32_t off_raw, off_desc, off_ab, off_slots, off_tree;
 };
+
+// The nodes of sequence b: n0 .. n0 + N - 1 of the node dimension (N = p.N
+// and n0 = b N, or from the varlen offsets).
+struct Seq {
+    int n0, N;
+};
+
+// Reads sequence b's node range; false (on every thread) if the varlen
+// offsets are out of range.
+__device__ __forceinline__ bool seq_of(const KParams& p, int b, Seq& q)
+{
+    if (p.cu == nullptr) {
+        q.n0 = b * p.N;
+        q.N = p.N;
+        return true;
+    }
+    q.n0 = __ldg(p.cu + b);
+    q.N = __ldg(p.cu + b + 1) - q.n0;
+    return q.n0 >= 0 && q.N >= 1 && q.N <= p.N && q.n0 <= p.total - q.N;
+}
 
 // One walk position: its node and tree metadata, and the node's scalars.
 struct PosDesc {
@@ -846,21 +868,20 @@ enum : int { kTreeChain = 0, kTreeWarp = 1, kTreeSmem = 2, kTreeIndex = 3, kTree
 // for recomputation, and the ring handshakes (ctx.begin / ctx.end; trivial
 // when everything is staged).
 template <int DK, int C, int RL, typename RT, typename ST, int TREE, class Tree, class Ctx>
-__device__ __forceinline__ void walk(StateT<C, RL>& S, const KParams& p, const Tree& tree, float* lane_slot,
-                                     const float* sin_lane, int b, int h, int row0,
+__device__ __forceinline__ void walk(StateT<C, RL>& S, const KParams& p, const Seq& sq, const Tree& tree,
+                                     float* lane_slot, const float* sin_lane, int b, int h, int row0,
                                      const LaneMap<DK, C, RL>& L, Ctx& ctx)
 {
     using LM = LaneMap<DK, C, RL>;
     constexpr bool CHAIN = TREE == kTreeChain;
     constexpr bool INDEX = TREE == kTreeIndex;
     constexpr bool GSLOT = TREE >= kTreeGlobal;
-    const int N = p.N;
-    const int NS = p.persist_last ? 1 : N;
+    const int N = sq.N;
     const size_t ns_stride = (size_t)p.Hv * p.dv * DK;  // elements between nodes' states
-    ST* const ns_lane = static_cast<ST*>(p.node_states) + (size_t)b * NS * ns_stride +
+    ST* const ns_lane = static_cast<ST*>(p.node_states) + (size_t)(p.persist_last ? b : sq.n0) * ns_stride +
                         (size_t)h * p.dv * DK + (size_t)row0 * DK + L.tile_offset();
     const size_t out_stride = (size_t)p.Hv * p.dv;
-    float* const out_lane = p.out + (size_t)b * N * out_stride + (size_t)h * p.dv + row0 + L.row;
+    float* const out_lane = p.out + (size_t)sq.n0 * out_stride + (size_t)h * p.dv + row0 + L.row;
     const int slot_floats = p.rows * DK;
     const int stride = p.warps * 32 * 4;
     // Index order and workspace slots: the next position's parent state,
@@ -1041,18 +1062,18 @@ __device__ __forceinline__ void write_descs(const Tree& tree, const unsigned cha
 }
 
 template <int DK, int C, int RL, typename QT, typename ST, int TREE, class Tree>
-__device__ __forceinline__ void staged_finish(StateT<C, RL>& S, const KParams& p, const Tree& tree,
+__device__ __forceinline__ void staged_finish(StateT<C, RL>& S, const KParams& p, const Seq& sq, const Tree& tree,
                                               const unsigned char* raw, float* ab, PosDesc* desc, float* slotbuf,
                                               const float* sin_lane, int b, int h, int row0,
                                               const LaneMap<DK, C, RL>& L)
 {
     constexpr int LR = LaneMap<DK, C, RL>::LR;
-    write_descs<DK, LR, QT>(tree, raw, p.raw_bytes, ab, desc, p.N);
+    write_descs<DK, LR, QT>(tree, raw, p.raw_bytes, ab, desc, sq.N);
     __syncthreads();
     const uint32_t rec_elems = p.raw_bytes / (uint32_t)sizeof(QT);
-    StagedCtx<DK, C, RL, QT> ctx{reinterpret_cast<const QT*>(raw), desc, ab, rec_elems, p.N, L};
+    StagedCtx<DK, C, RL, QT> ctx{reinterpret_cast<const QT*>(raw), desc, ab, rec_elems, sq.N, L};
     float* lane_slot = cta_slots<DK, TREE>(p, slotbuf) + 4 * threadIdx.x;
-    walk<DK, C, RL, QT, ST, TREE>(S, p, tree, lane_slot, sin_lane, b, h, row0, L, ctx);
+    walk<DK, C, RL, QT, ST, TREE>(S, p, sq, tree, lane_slot, sin_lane, b, h, row0, L, ctx);
 }
 
 template <int DK, int C, int RL, typename QT, typename ST, int TREE>
@@ -1068,20 +1089,28 @@ __global__ void __launch_bounds__(kMaxWarps * 32) gdn_verify_staged(const KParam
     int* tsm = reinterpret_cast<int*>(smem + p.off_tree);
 
     constexpr int TK = TREE % kTreeGlobal;  // walk kind without the slot placement
-    const int N = p.N;
     const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int hk = h / p.G;
     const int row0 = tile * p.rows;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
     const int nwarps = blockDim.x >> 5;
-    const int32_t* prow = p.parent + (size_t)b * N;
     // Everything that reads q, k, v, g, beta waits for the preceding kernel;
-    // with GDN_FLAG_EARLY_TREE the tree and the root's parent state are read
-    // before that (they were written before the preceding kernel started).
-    // Every node's raw k row, q row and v slice, and its g and beta, are
-    // copied to shared memory asynchronously (warp w copies nodes w,
-    // w + warps, ...); the tree work overlaps the copies unless it already ran
-    // before the wait.
+    // with GDN_FLAG_EARLY_TREE the tree (varlen offsets included) and the
+    // root's parent state are read before that (they were written before the
+    // preceding kernel started).  Every node's raw k row, q row and v slice,
+    // and its g and beta, are copied to shared memory asynchronously (warp w
+    // copies nodes w, w + warps, ...); the tree work overlaps the copies
+    // unless it already ran before the wait.
+    if (!p.early_tree)
+        pdl_wait_then_release();
+    Seq sq;
+    if (!seq_of(p, b, sq)) {
+        if (tid == 0)
+            report_status(p.status, GDN_ERR_BAD_TREE);
+        return;
+    }
+    const int N = sq.N;
+    const int32_t* prow = p.parent + sq.n0;
     const int per_node = p.raw_bytes / 16;  // 16-byte chunks per node
     constexpr int LR = LaneMap<DK, C, RL>::LR;
     auto stage = [&]() {
@@ -1089,7 +1118,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32) gdn_verify_staged(const KParam
         const QT* qg = static_cast<const QT*>(p.q);
         const QT* vg = static_cast<const QT*>(p.v);
         for (int n = warp; n < N; n += nwarps) {
-            const size_t node = (size_t)b * N + n;
+            const size_t node = (size_t)sq.n0 + n;
             const QT* krow = kg + (node * p.Hk + hk) * DK;
             const QT* qrow = qg + (node * p.Hk + hk) * DK;
             const QT* vrow = vg + (node * p.Hv + h) * p.dv + row0;
@@ -1112,16 +1141,14 @@ __global__ void __launch_bounds__(kMaxWarps * 32) gdn_verify_staged(const KParam
             }
         }
         for (int n = tid; n < N; n += blockDim.x) {
-            const size_t gi = ((size_t)b * N + n) * p.Hv + h;
+            const size_t gi = ((size_t)sq.n0 + n) * p.Hv + h;
             cp_async4(ab + n, p.g + gi);
             cp_async4(ab + N + n, p.beta + gi);
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
-    if (!p.early_tree) {
-        pdl_wait_then_release();
+    if (!p.early_tree)
         stage();
-    }
 
     // 1. the parent array (index order keeps it in shared memory; chain
     //    validation only checks it)
@@ -1167,16 +1194,16 @@ __global__ void __launch_bounds__(kMaxWarps * 32) gdn_verify_staged(const KParam
     }
     // 5. descriptors, then the walk
     if constexpr (TK == kTreeChain)
-        staged_finish<DK, C, RL, QT, ST, TREE>(S, p, NoTree{}, raw, ab, desc, slotbuf, sin_lane, b, h,
+        staged_finish<DK, C, RL, QT, ST, TREE>(S, p, sq, NoTree{}, raw, ab, desc, slotbuf, sin_lane, b, h,
                                                row0, L);
     else if constexpr (TK == kTreeIndex)
-        staged_finish<DK, C, RL, QT, ST, TREE>(S, p, IndexTree{tsm}, raw, ab, desc, slotbuf, sin_lane, b,
+        staged_finish<DK, C, RL, QT, ST, TREE>(S, p, sq, IndexTree{tsm}, raw, ab, desc, slotbuf, sin_lane, b,
                                                h, row0, L);
     else if constexpr (TK == kTreeWarp)
-        staged_finish<DK, C, RL, QT, ST, TREE>(S, p, MaskTree{tsm}, raw, ab, desc, slotbuf, sin_lane, b,
+        staged_finish<DK, C, RL, QT, ST, TREE>(S, p, sq, MaskTree{tsm}, raw, ab, desc, slotbuf, sin_lane, b,
                                                h, row0, L);
     else
-        staged_finish<DK, C, RL, QT, ST, TREE>(S, p, SmemTree{tv, N, warp}, raw, ab, desc, slotbuf,
+        staged_finish<DK, C, RL, QT, ST, TREE>(S, p, sq, SmemTree{tv, N, warp}, raw, ab, desc, slotbuf,
                                                sin_lane, b, h, row0, L);
 }
 
@@ -1190,7 +1217,7 @@ struct GlobalFetch {
     const QT* vg;
     const float* g;
     const float* beta;
-    size_t bN;  // b * N
+    size_t bN;  // the sequence's first node
     int Hk, Hv, dv, hk, h, row0;
     LaneMap<DK, C, RL> L;
     __device__ __forceinline__ void operator()(int y, float2 (&k2)[4 * C], float (&vr)[RL], float& a,
@@ -1282,9 +1309,6 @@ __global__ void __launch_bounds__((kMaxWarps + 1) * 32) gdn_verify_ring(const KP
     const uint32_t desc_off = (kChunk * p.raw_bytes + 15u) & ~15u;
     const uint32_t slot_bytes = desc_off + kChunk * (uint32_t)sizeof(PosDesc);
     float* slotbuf = reinterpret_cast<float*>(smem + p.off_slots);
-    const TreeView T(reinterpret_cast<int*>(smem + p.off_tree), p.N);
-
-    const int N = p.N;
     const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int hk = h / p.G;
     const int row0 = tile * p.rows;
@@ -1294,6 +1318,14 @@ __global__ void __launch_bounds__((kMaxWarps + 1) * 32) gdn_verify_ring(const KP
     const QT* vg = static_cast<const QT*>(p.v);
     if (!p.early_tree)
         pdl_wait_then_release();
+    Seq sq;
+    if (!seq_of(p, b, sq)) {
+        if (tid == 0)
+            report_status(p.status, GDN_ERR_BAD_TREE);
+        return;
+    }
+    const int N = sq.N;
+    const TreeView T(reinterpret_cast<int*>(smem + p.off_tree), N);
 
     if (tid == 0) {
         for (int i = 0; i < kRing; ++i) {
@@ -1307,7 +1339,7 @@ __global__ void __launch_bounds__((kMaxWarps + 1) * 32) gdn_verify_ring(const KP
         bool bad = false;
         if (INDEX || p.validate) {
             for (int n = tid; n < N; n += blockDim.x) {
-                const int pn = __ldg(p.parent + (size_t)b * N + n);
+                const int pn = __ldg(p.parent + (size_t)sq.n0 + n);
                 if (INDEX) {
                     T.par[n] = pn;
                     bad |= (n == 0) ? (pn != -1) : (pn < 0 || pn >= n);
@@ -1319,7 +1351,7 @@ __global__ void __launch_bounds__((kMaxWarps + 1) * 32) gdn_verify_ring(const KP
         ok = !__syncthreads_or(bad);
     } else {
         __syncthreads();
-        ok = build_walk(p.parent + (size_t)b * N, N, p.slots, T);
+        ok = build_walk(p.parent + (size_t)sq.n0, N, p.slots, T);
     }
     if (p.early_tree)
         pdl_wait_then_release();
@@ -1353,7 +1385,7 @@ __global__ void __launch_bounds__((kMaxWarps + 1) * 32) gdn_verify_ring(const KP
                     const int i = idx / per_pos, j = idx - i * per_pos;
                     const int pos = p0 + i;
                     const int n = (CHAIN || INDEX) ? pos : meta_node(T.meta[pos]);
-                    const size_t node = (size_t)b * N + n;
+                    const size_t node = (size_t)sq.n0 + n;
                     const QT* src;
                     if (j < QKCH)
                         src = kg + (node * p.Hk + hk) * DK + j * EPC;
@@ -1379,7 +1411,7 @@ __global__ void __launch_bounds__((kMaxWarps + 1) * 32) gdn_verify_ring(const KP
                 }
                 dn = meta_node(dm);
                 dpp = CHAIN ? dn - 1 : T.par[dn];
-                const size_t gi = ((size_t)b * N + dn) * p.Hv + h;
+                const size_t gi = ((size_t)sq.n0 + dn) * p.Hv + h;
                 da = gdn_gate(__ldg(p.g + gi));
                 dbe = __ldg(p.beta + gi);
             }
@@ -1431,15 +1463,15 @@ __global__ void __launch_bounds__((kMaxWarps + 1) * 32) gdn_verify_ring(const KP
         p.state_in + ((size_t)b * p.Hv + h) * p.dv * DK + (size_t)row0 * DK + L.tile_offset();
     StateT<C, RL> S;
     load_rows<DK, C, RL>(S, sin_lane);
-    const GlobalFetch<DK, C, RL, QT> gf{kg, vg, p.g, p.beta, (size_t)b * N, p.Hk, p.Hv, p.dv, hk, h, row0, L};
+    const GlobalFetch<DK, C, RL, QT> gf{kg, vg, p.g, p.beta, (size_t)sq.n0, p.Hk, p.Hv, p.dv, hk, h, row0, L};
     RingCtx<DK, C, RL, QT> ctx{full, empty, ring, p.raw_bytes, slot_bytes, desc_off, p.status, lane, gf};
     float* lane_slot = cta_slots<DK, TREE>(p, slotbuf) + 4 * threadIdx.x;
     if constexpr (CHAIN)
-        walk<DK, C, RL, QT, ST, TREE>(S, p, NoTree{}, lane_slot, sin_lane, b, h, row0, L, ctx);
+        walk<DK, C, RL, QT, ST, TREE>(S, p, sq, NoTree{}, lane_slot, sin_lane, b, h, row0, L, ctx);
     else if constexpr (INDEX)
-        walk<DK, C, RL, QT, ST, TREE>(S, p, IndexTree{T.par}, lane_slot, sin_lane, b, h, row0, L, ctx);
+        walk<DK, C, RL, QT, ST, TREE>(S, p, sq, IndexTree{T.par}, lane_slot, sin_lane, b, h, row0, L, ctx);
     else
-        walk<DK, C, RL, QT, ST, TREE>(S, p, SmemTree{T, N, warp}, lane_slot, sin_lane, b, h, row0, L, ctx);
+        walk<DK, C, RL, QT, ST, TREE>(S, p, sq, SmemTree{T, N, warp}, lane_slot, sin_lane, b, h, row0, L, ctx);
 }
 
 // ---------------------------------------------------------------------------

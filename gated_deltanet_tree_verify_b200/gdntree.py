@@ -81,6 +81,11 @@ def load_library() -> ctypes.CDLL:
     lib.gdn_tree_verify_static_ws.restype = ctypes.c_int
     lib.gdn_static_workspace_capacity.argtypes = []
     lib.gdn_static_workspace_capacity.restype = ctypes.c_size_t
+    lib.gdn_tree_verify_varlen.argtypes = [dp, vp, i32] + [vp] * 10 + [ctypes.c_size_t, vp]
+    lib.gdn_tree_verify_varlen.restype = ctypes.c_int
+    lib.gdn_tree_commit_varlen.argtypes = [dp, vp, i32, i32, ctypes.POINTER(vp), vp, vp, vp, i32,
+                                           ctypes.POINTER(vp), vp]
+    lib.gdn_tree_commit_varlen.restype = ctypes.c_int
     lib.gdn_tree_commit.argtypes = [dp, vp, vp, vp, vp, i32, vp, vp]
     lib.gdn_tree_commit.restype = ctypes.c_int
     lib.gdn_tree_commit_layers.argtypes = [dp, i32, ctypes.POINTER(vp), vp, vp, vp, i32,
@@ -233,4 +238,36 @@ def gdn_tree_commit_layers(desc: GdnTreeDesc, node_states, parent_idx, accept_pa
     rc = lib.gdn_tree_commit_layers(ctypes.byref(desc), n, ns, _ptr(parent_idx, "parent_idx"),
                                     _ptr(accept_path, "accept_path"), _ptr(accept_len, "accept_len"),
                                     int(max_path_len), so, _stream(stream))
+    return _check(rc, check)
+
+
+def gdn_tree_verify_varlen(desc: GdnTreeDesc, cu_nodes, total_nodes: int, q, k, v, g, beta, parent_idx, state_in,
+                           out, node_states, workspace=None, workspace_bytes: Optional[int] = None, stream=None,
+                           check: bool = True) -> int:
+    """Calls gdn_tree_verify_varlen (see include/gdntree.h): trees of
+    different sizes packed along the node dimension."""
+    lib = load_library()
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size() if isinstance(workspace, torch.Tensor) else 0
+    rc = lib.gdn_tree_verify_varlen(ctypes.byref(desc), _ptr(cu_nodes, "cu_nodes"), int(total_nodes),
+                                    _ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _ptr(g, "g"), _ptr(beta, "beta"),
+                                    _ptr(parent_idx, "parent_idx"), _ptr(state_in, "state_in"), _ptr(out, "out"),
+                                    _ptr(node_states, "node_states"), _ptr(workspace, "workspace"),
+                                    int(workspace_bytes), _stream(stream))
+    return _check(rc, check)
+
+
+def gdn_tree_commit_varlen(desc: GdnTreeDesc, cu_nodes, total_nodes: int, node_states, parent_idx, accept_path,
+                           accept_len, max_path_len: int, state_out, stream=None, check: bool = True) -> int:
+    """Calls gdn_tree_commit_varlen: ``node_states`` and ``state_out`` are
+    equal-length sequences of per-layer CUDA tensors (or int pointers)."""
+    lib = load_library()
+    if len(node_states) != len(state_out):
+        raise ValueError("node_states and state_out must have one entry per layer")
+    n = len(node_states)
+    ns = (ctypes.c_void_p * max(n, 1))(*[_ptr(t, "node_states") for t in node_states])
+    so = (ctypes.c_void_p * max(n, 1))(*[_ptr(t, "state_out") for t in state_out])
+    rc = lib.gdn_tree_commit_varlen(ctypes.byref(desc), _ptr(cu_nodes, "cu_nodes"), int(total_nodes), n, ns,
+                                    _ptr(parent_idx, "parent_idx"), _ptr(accept_path, "accept_path"),
+                                    _ptr(accept_len, "accept_len"), int(max_path_len), so, _stream(stream))
     return _check(rc, check)

@@ -169,6 +169,36 @@ gdn_status gdn_tree_verify_ws(const gdn_tree_desc* desc, const void* q, const vo
                               void* node_states, void* workspace, size_t workspace_bytes,
                               cudaStream_t stream);
 
+/*
+ * gdn_tree_verify_varlen -- gdn_tree_verify(_ws) for B trees of different
+ * sizes, packed along the node dimension.
+ *
+ *   desc->n_nodes  the most nodes any sequence has (N_max); desc->batch = B
+ *   cu_nodes       DEVICE [B + 1] int32: sequence b owns packed nodes
+ *                  cu_nodes[b] .. cu_nodes[b + 1] - 1, with cu_nodes[0] = 0,
+ *                  1 <= cu_nodes[b + 1] - cu_nodes[b] <= N_max and
+ *                  cu_nodes[B] = total_nodes (a sequence whose entries break
+ *                  this gets GDN_ERR_BAD_TREE through desc->status and
+ *                  nothing written)
+ *   total_nodes    T, B <= T <= B * N_max (host-checked)
+ *   q, k           [T][H_k][d_k];  v [T][H_v][d_v];  g, beta [T][H_v]
+ *   parent_idx     [T] int32, each sequence's parents as local indices
+ *                  (-1 for its root, 0 <= parent < n within the sequence)
+ *   out            [T][H_v][d_v]
+ *   node_states    [T][H_v][d_v][d_k] (PERSIST_LAST: [B][H_v][d_v][d_k])
+ *   state_in       [B][H_v][d_v][d_k], as for gdn_tree_verify
+ *   workspace      optional, as for gdn_tree_verify_ws (size from
+ *                  gdn_tree_verify_workspace_bytes with the same desc)
+ *
+ * Results for each sequence are bit-identical to gdn_tree_verify on that
+ * sequence alone.  With GDN_FLAG_EARLY_TREE, cu_nodes counts as tree data.
+ */
+gdn_status gdn_tree_verify_varlen(const gdn_tree_desc* desc, const int32_t* cu_nodes, int32_t total_nodes,
+                                  const void* q, const void* k, const void* v, const float* g,
+                                  const float* beta, const int32_t* parent_idx, const float* state_in,
+                                  float* out, void* node_states, void* workspace, size_t workspace_bytes,
+                                  cudaStream_t stream);
+
 /* Workspace bytes gdn_tree_verify_ws needs for a desc: B * H_v * d_v * d_k *
  * 4 * (stack slots, at most 4) for walks that keep branch states, 0 for
  * chains, f32 trees (their branch states are re-read from node_states) and
@@ -247,6 +277,18 @@ gdn_status gdn_tree_commit_layers(const gdn_tree_desc* desc, int32_t n_layers,
                                   const int32_t* accept_path, const int32_t* accept_len,
                                   int32_t max_path_len, float* const* state_out,
                                   cudaStream_t stream);
+
+/*
+ * gdn_tree_commit_varlen -- gdn_tree_commit_layers for the packed layout of
+ * gdn_tree_verify_varlen: node_states[l] as written there, parent_idx [T]
+ * local, accept_path [B][max_path_len] local node ids, the same cu_nodes and
+ * total_nodes.  A sequence with bad offsets gets GDN_ERR_BAD_TREE and its
+ * state_out is left untouched.
+ */
+gdn_status gdn_tree_commit_varlen(const gdn_tree_desc* desc, const int32_t* cu_nodes, int32_t total_nodes,
+                                  int32_t n_layers, const void* const* node_states, const int32_t* parent_idx,
+                                  const int32_t* accept_path, const int32_t* accept_len, int32_t max_path_len,
+                                  float* const* state_out, cudaStream_t stream);
 
 /* Largest N the tree (non-chain) path takes. */
 #define GDN_MAX_TREE_NODES 1024

@@ -204,3 +204,21 @@ def test_verify_ws_host_checks(lib):
     p = _ptrs()
     assert _verify_ws(d, p[8] + 64, need, p) == gdn.GDN_ERR_INVALID_ARG  # inside node_states
     assert _verify_ws(d, p[0], need, p) == gdn.GDN_ERR_INVALID_ARG       # on top of q
+
+
+def test_varlen_host_checks(lib):
+    d = _desc(batch=3)
+    q, k, v, g, beta, par, sin, out, ns = _ptrs(9)
+    cu = BASE + 30 * MB
+
+    def call(desc, cu_ptr, total):
+        return gdn.gdn_tree_verify_varlen(desc, cu_ptr, total, q, k, v, g, beta, par, sin, out, ns, None, 0,
+                                          stream=0, check=False)
+    assert call(d, None, 10) == gdn.GDN_ERR_INVALID_ARG          # no offsets
+    assert call(d, cu + 2, 10) == gdn.GDN_ERR_INVALID_ARG        # misaligned
+    assert call(d, cu, 2) == gdn.GDN_ERR_INVALID_ARG             # fewer nodes than sequences
+    assert call(d, cu, 3 * 23 + 1) == gdn.GDN_ERR_INVALID_ARG    # more than batch * n_nodes
+    assert call(_desc(batch=0), cu, 0) == gdn.GDN_OK
+    rc = gdn.gdn_tree_commit_varlen(d, None, 10, [ns], par, BASE + 31 * MB, BASE + 32 * MB, 4, [out],
+                                    stream=0, check=False)
+    assert rc == gdn.GDN_ERR_INVALID_ARG
