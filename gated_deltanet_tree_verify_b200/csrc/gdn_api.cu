@@ -51,7 +51,7 @@ gdn_status check_desc(const gdn_tree_desc* d, bool need_qkv)
         return fail(GDN_ERR_INVALID_ARG, "batch, n_nodes or head counts out of range%s");
     if (d->n_v_heads % d->n_k_heads != 0)
         return fail(GDN_ERR_INVALID_ARG, "n_v_heads is not a multiple of n_k_heads%s");
-    if ((d->flags & ~15u) != 0)
+    if ((d->flags & ~31u) != 0)
         return fail(GDN_ERR_INVALID_ARG, "unknown flag bits%s");
     const bool dk_ok = d->d_k == 32 || d->d_k == 64 || d->d_k == 128;
     const bool dv_ok = d->d_v == 32 || d->d_v == 64 || d->d_v == 128;
@@ -193,6 +193,28 @@ gdn_status verify_impl(const gdn_tree_desc* desc, const int32_t* cu, int32_t tot
     a.workspace = static_cast<float*>(workspace);
     a.cu_nodes = varlen ? cu : nullptr;
     a.total_nodes = varlen ? total : 0;
+    if (d.flags & GDN_FLAG_CHUNKED) {
+        if (varlen || workspace != nullptr || !gdn::chunked_supported(a))
+            return fail(GDN_ERR_UNSUPPORTED,
+                        "GDN_FLAG_CHUNKED needs CHAIN + PERSIST_LAST, bf16 q/k/v, d_k = 128, d_v %% 64 == 0%s");
+        const size_t B = d.batch, N = d.n_nodes, Hk = d.n_k_heads, Hv = d.n_v_heads, dk = d.d_k, dv = d.d_v;
+        const Range ins[] = {{q, B * N * Hk * dk * 2, "q"}, {k, B * N * Hk * dk * 2, "k"},
+                             {v, B * N * Hv * dv * 2, "v"}, {g, B * N * Hv * 4, "g"},
+                             {beta, B * N * Hv * 4, "beta"}, {state_in, B * Hv * dv * dk * 4, "state_in"}};
+        const Range outs[] = {{out, B * N * Hv * dv * 4, "out"}, {node_states, node_states_bytes(&d), "node_states"}};
+        if (overlap(outs[0], outs[1]))
+            return fail(GDN_ERR_INVALID_ARG, "out overlaps node_states%s");
+        for (const auto& o : outs)
+            for (const auto& i : ins)
+                if (overlap(o, i))
+                    return fail(GDN_ERR_INVALID_ARG, "an output overlaps input %s", i.name);
+        if (d.n_v_heads > 65535 || d.batch > 65535)
+            return fail(GDN_ERR_UNSUPPORTED, "batch or n_v_heads above the grid limit%s");
+        const cudaError_t e = gdn::launch_chunked(a, stream);
+        if (e != cudaSuccess)
+            return fail(GDN_ERR_CUDA, "verify launch failed: %s", cudaGetErrorString(e));
+        return GDN_OK;
+    }
     const gdn::VerifyGeom geom = gdn::verify_geometry(a, workspace != nullptr);
     if (geom.tiles <= 0 || geom.smem > 227 * 1024)
         return fail(GDN_ERR_UNSUPPORTED, "no launch geometry for this shape%s");

@@ -99,4 +99,9 @@ VerifyGeom verify_geometry(const VerifyArgs& a, bool use_workspace);
 cudaError_t launch_verify(const VerifyArgs& a, const VerifyGeom& geom, cudaStream_t stream);
 cudaError_t launch_commit(const CommitArgs& a, cudaStream_t stream);
 
+// Chains in chunks on the tensor cores (GDN_FLAG_CHUNKED): whether a call's
+// shapes are supported, and the launch.
+bool chunked_supported(const VerifyArgs& a);
+cudaError_t launch_chunked(const VerifyArgs& a, cudaStream_t stream);
+
 }  // namespace gdn

@@ -88,7 +88,14 @@ enum {
      * build the tree walk while the preceding kernel may still run, and wait
      * for it only before reading q, k, v, g, beta.  Without the flag every
      * global read waits for the preceding kernel to complete. */
-    GDN_FLAG_EARLY_TREE = 8
+    GDN_FLAG_EARLY_TREE = 8,
+    /* Chains only (with GDN_FLAG_CHAIN and GDN_FLAG_PERSIST_LAST, bf16 q/k/v,
+     * d_k = 128, d_v a multiple of 64, no varlen or workspace): run the chain
+     * in chunks of 64 tokens with tensor-core products (the chunked "WY" form
+     * of the delta rule), for long prefill-style chains.  Same results up to
+     * f32 rounding (products in split tf32), not bit-identical to the
+     * token-by-token path.  Unsupported shapes: GDN_ERR_UNSUPPORTED. */
+    GDN_FLAG_CHUNKED = 16
 };
 
 /* Problem description, shared by verify and commit. */

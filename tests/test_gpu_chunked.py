@@ -1,0 +1,87 @@
+"""GDN_FLAG_CHUNKED: chains in chunks of 64 tokens on the tensor cores.  The
+oracle (token by token, f64) fixes the answer; the chunked form must match it
+within the stated tolerances, for chain lengths around the chunk size, both
+state dtypes and gates that reset the state.  It is not bit-identical to the
+token-by-token path (different summation order), only close to it."""
+import numpy as np
+import pytest
+import torch
+
+import gated_deltanet_tree_verify_b200 as gdn
+import oracle
+from gdn_inputs import make_problem, make_workload
+from tests.gpu_util import assert_out_close, assert_states_close, rel_fro, run
+
+pytestmark = pytest.mark.gpu
+
+FLAGS = gdn.GDN_FLAG_CHAIN | gdn.GDN_FLAG_PERSIST_LAST
+
+
+def _chain(N, B=2, Hk=2, Hv=6, dv=128, seed=3, gate="softplus"):
+    prob = make_problem(batch=B, n_nodes=N, n_k_heads=Hk, n_v_heads=Hv, d_k=128, d_v=dv, tree="chain",
+                        seed=seed, qkv_dtype="bf16", gate=gate, accept="prefix")
+    prob.accept_path = torch.arange(N, dtype=torch.int32).repeat(B, 1).contiguous()
+    prob.accept_len = torch.full((B,), N, dtype=torch.int32)
+    return prob
+
+
+@pytest.mark.parametrize("N", [1, 5, 63, 64, 65, 100, 130, 257])
+@pytest.mark.parametrize("sd", ["f32", "f16"])
+def test_chunked_chain_matches_oracle(N, sd):
+    prob = _chain(N, gate="uniform_a" if N % 2 else "softplus")
+    res = run(prob, sd, flags=FLAGS | gdn.GDN_FLAG_CHUNKED)
+    assert res["status"] == 0
+    out, _, ex = oracle.verify_problem(prob, state_dtype=sd, want_exact=True, nthreads=8)
+    assert_out_close(res["out"], out)
+    assert_states_close(res["node_states"][:, 0], ex[:, -1], sd)
+    assert torch.equal(res["state_out"], res["node_states"][:, 0].float())
+    # close to the token-by-token kernel (not bitwise: different summation order)
+    ref = run(prob, sd, flags=FLAGS)
+    assert (res["out"] - ref["out"]).abs().max() <= 1e-4
+    r = rel_fro(res["node_states"][:, 0].double().numpy(), ref["node_states"][:, 0].double().numpy(),
+                axes=(-2, -1))
+    assert r.max() <= (1e-5 if sd == "f32" else 2e-3)
+
+
+def test_chunked_chain_reset_and_zero_beta():
+    prob = _chain(150)
+    prob.g[:, 70] = float("-inf")   # a = 0: the state restarts at token 70
+    prob.beta[:, 10:20] = 0.0       # no writes for 10 tokens
+    res = run(prob, "f32", flags=FLAGS | gdn.GDN_FLAG_CHUNKED)
+    assert res["status"] == 0
+    out, _, ex = oracle.verify_problem(prob, state_dtype="f32", want_exact=True, nthreads=8)
+    assert_out_close(res["out"], out)
+    assert_states_close(res["node_states"][:, 0], ex[:, -1], "f32")
+
+
+def test_chunked_long_chain4096_sampled():
+    prob = make_workload("long_chain4096", seed=4)
+    N = prob.n_nodes
+    prob.accept_path = torch.arange(N, dtype=torch.int32).repeat(prob.batch, 1).contiguous()
+    prob.accept_len = torch.full((prob.batch,), N, dtype=torch.int32)
+    res = run(prob, "f32", flags=FLAGS | gdn.GDN_FLAG_CHUNKED)
+    assert res["status"] == 0
+    rows = slice(40, 48)  # rows of S evolve independently given k
+    for b, h in [(0, 0), (3, 17), (7, 47)]:
+        hk = h // 3
+        out, st, ex = oracle.verify(prob.q[b:b + 1, :, hk:hk + 1], prob.k[b:b + 1, :, hk:hk + 1],
+                                    prob.v[b:b + 1, :, h:h + 1, rows], prob.g[b:b + 1, :, h:h + 1],
+                                    prob.beta[b:b + 1, :, h:h + 1], prob.parent[b:b + 1],
+                                    prob.state_in[b:b + 1, h:h + 1, rows], prob.scale, want_exact=True)
+        assert_out_close(res["out"][b:b + 1, :, h:h + 1, rows], out)
+        r = rel_fro(res["node_states"][b, 0, h, rows].double().numpy(), ex[0, -1, 0], axes=(-2, -1))
+        assert r <= 1e-3
+    assert np.isfinite(res["out"].numpy()).all()
+    assert torch.equal(res["state_out"], res["node_states"][:, 0])
+
+
+def test_chunked_is_refused_outside_its_shapes():
+    prob = _chain(70, dv=32)
+    d = {k: getattr(prob, k).cuda() for k in ("q", "k", "v", "g", "beta", "parent", "state_in")}
+    desc = gdn.make_desc(batch=2, n_nodes=70, n_k_heads=2, n_v_heads=6, d_k=128, d_v=32, scale=prob.scale,
+                         flags=FLAGS | gdn.GDN_FLAG_CHUNKED)
+    out = torch.empty(2, 70, 6, 32, device="cuda")
+    ns = torch.empty(2, 1, 6, 32, 128, device="cuda")
+    rc = gdn.gdn_tree_verify(desc, d["q"], d["k"], d["v"], d["g"], d["beta"], None, d["state_in"], out, ns,
+                             check=False)
+    assert rc == gdn.GDN_ERR_UNSUPPORTED
