@@ -636,6 +636,7 @@ def run_sweep(args):
     for sd, ws in (("f32", False), ("f16", False), ("f16", True)):
         points.append(dict(kind="varlen", budget=0, batch=8, state_dtype=sd, ws=ws))
     points.append(dict(kind="chain4096", budget=4095, batch=8, state_dtype="f32"))
+    points.append(dict(kind="chain4096", budget=4095, batch=8, state_dtype="f32", chunked=True))
     varlen_budgets = [8, 64, 22, 15, 32, 22, 48, 8]
     for pt in points:
         n = pt["budget"] + 1
@@ -647,6 +648,8 @@ def run_sweep(args):
             continue
         if pt["kind"] == "chain4096":
             flags = gdn.GDN_FLAG_CHAIN | gdn.GDN_FLAG_PERSIST_LAST
+            if pt.get("chunked"):
+                flags |= gdn.GDN_FLAG_CHUNKED
             t, R = _verify_point(batch=pt["batch"], n_nodes=n, tree="chain", state_dtype="f32", flags=flags,
                                  gate="uniform_a", reps=3, min_bytes=0)
             tokens = pt["batch"] * n
@@ -654,7 +657,8 @@ def run_sweep(args):
             flops = tokens * N_V_HEADS * D * D * 7.0  # dot S k, a S, u k^T, S q: 7 flops per element
             clock = args.sm_mhz * 1e6
             alu_peak = 148 * FP32_LANES_PER_SM * 2 * clock / 1e12
-            line = {"sweep": "chain4096_persist_last", "batch": pt["batch"], "tokens": n,
+            line = {"sweep": "chain4096_persist_last" + ("_chunked" if pt.get("chunked") else ""),
+                    "batch": pt["batch"], "tokens": n,
                     "state_dtype": "f32", "verify_ms": t * 1e3, "tokens_per_s": tokens / t,
                     "roofline": {"bound": "alu", "achieved": flops / t / 1e12, "unit": "TFLOP/s",
                                  "peak": alu_peak, "frac": flops / t / 1e12 / alu_peak,

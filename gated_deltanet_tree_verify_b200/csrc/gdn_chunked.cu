@@ -19,7 +19,7 @@
 //     P   = diag(beta) (V - diag(Gamma) K S_0^T)              [T x d_v]
 //     U   = (I + L)^-1 P,  L = diag(beta) (K K^T o R), strictly lower
 //     O   = scale (diag(Gamma) Q S_0^T + (Q K^T o R_incl) U)   [T x d_v]
-//     S_T = Gamma_{T-1} S_0 + U^T diag(r) K,  r_i = R[T-1][i]
+//     S_T = Gamma_{T-1} S_0 + (diag(r) U)^T K,  r_i = R[T-1][i]
 //
 // The products are tensor-core mma.sync (bf16 for K K^T and Q K^T, whose
 // operands are exact; tf32 otherwise).  f32 operands are split into two tf32
@@ -53,7 +53,7 @@ constexpr int TV = 64;           // d_v rows per CTA
 constexpr int kThreads = 256;    // 8 warps
 constexpr int KST = DK + 8;      // bf16 row stride of K, Q (272 bytes)
 constexpr int VST = TV + 8;      // bf16 row stride of the V tile
-constexpr int SST = DK + 4;      // f32 row stride of the state tile
+constexpr int SST = DK + 4;      // float2 row stride of the state tile: (value, tf32 remainder)
 constexpr int MST = T + 4;       // f32 row stride of T x T matrices and U
 
 struct Params {
@@ -77,9 +77,9 @@ constexpr int kOffK = 0;                              // K[2]
 constexpr int kOffQ = kOffK + 2 * kKQBytes;           // Q[2]
 constexpr int kOffV = kOffQ + 2 * kKQBytes;           // V[2]
 constexpr int kOffGB = kOffV + 2 * kVBytes;           // g[2][T], beta[2][T]
-constexpr int kOffS = kOffGB + 4 * T * 4;             // S [TV][SST] f32
-constexpr int kOffR = kOffS + TV * SST * 4;           // R [T][MST]
-constexpr int kOffL = kOffR + T * MST * 4;            // L, permuted [T][4][16] (row stride MST)
+constexpr int kOffS = kOffGB + 4 * T * 4;             // S [TV][SST] float2
+constexpr int kOffR = kOffS + TV * SST * 8;           // R [T][MST]
+constexpr int kOffL = kOffR + T * MST * 4;            // L [T][MST]
 constexpr int kOffM = kOffL + T * MST * 4;            // Q K^T o R_incl [T][MST]
 constexpr int kOffU = kOffM + T * MST * 4;            // P, then U [T][MST]
 constexpr int kOffA = kOffU + T * MST * 4;            // a [T], Gamma [T]
@@ -90,6 +90,12 @@ __device__ __forceinline__ uint32_t f2tf32(float x)
     uint32_t r;
     asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
     return r;
+}
+
+// The tf32 remainder of x: x - tf32(x), itself rounded to tf32.
+__device__ __forceinline__ float tf32_rem(float x)
+{
+    return __uint_as_float(f2tf32(__fsub_rn(x, __uint_as_float(f2tf32(x)))));
 }
 
 // x = hi + lo, both tf32 (lo is the rounding remainder, itself rounded).
@@ -184,7 +190,7 @@ __device__ void stage_chunk(const Params& p, unsigned char* smem, int buf, int c
 __global__ void __launch_bounds__(kThreads, 1) gdn_chain_chunked(const Params p)
 {
     extern __shared__ __align__(16) unsigned char smem[];
-    float* S = reinterpret_cast<float*>(smem + kOffS);
+    float2* S = reinterpret_cast<float2*>(smem + kOffS);
     float* Rm = reinterpret_cast<float*>(smem + kOffR);
     float* Lp = reinterpret_cast<float*>(smem + kOffL);
     float* Mq = reinterpret_cast<float*>(smem + kOffM);
@@ -206,7 +212,10 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_chain_chunked(const Params p)
         const float* src = p.state_in + (((size_t)b * p.Hv + h) * p.dv + row0) * DK;
         for (int i = tid; i < TV * DK / 4; i += kThreads) {
             const int r = i / (DK / 4), c4 = i % (DK / 4);
-            *reinterpret_cast<float4*>(S + r * SST + 4 * c4) = __ldg(reinterpret_cast<const float4*>(src) + i);
+            const float4 x = __ldg(reinterpret_cast<const float4*>(src) + i);
+            float4* d = reinterpret_cast<float4*>(S + r * SST + 4 * c4);
+            d[0] = make_float4(x.x, tf32_rem(x.x), x.y, tf32_rem(x.y));
+            d[1] = make_float4(x.z, tf32_rem(x.z), x.w, tf32_rem(x.w));
         }
     }
     stage_chunk(p, smem, 0, 0, b, h, hk, row0);
@@ -228,25 +237,48 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_chain_chunked(const Params p)
         const float* gch = reinterpret_cast<const float*>(smem + kOffGB) + buf * 2 * T;
         const float* bch = gch + T;
 
-        // 1. decays: a_t, Gamma_t = a_0 ... a_t, R[t][i] = a_{i+1} ... a_t
+        // 1. decays: a_t, Gamma_t = a_0 ... a_t, R[t][i] = a_{i+1} ... a_t for
+        //    i <= t, r_i = R[T-1][i].  Row t by 4 threads, thread s covering
+        //    i in [16 s, 16 s + 15]: a suffix product within its quarter
+        //    times the products of the later quarters up to t.
+        float* rvec = const_cast<float*>(gch);  // g is dead once a is known
         if (tid < T)
             Av[tid] = tid < Tc ? expf(gch[tid]) : 1.f;
         __syncthreads();
-        if (tid < T) {
-            const int t = tid;
-            float r = 1.f;
-            Rm[t * MST + t] = 1.f;
-            for (int i = t - 1; i >= 0; --i) {
-                r = __fmul_rn(r, Av[i + 1]);
-                Rm[t * MST + i] = r;
+        {
+            const int t = tid >> 2, q = tid & 3;
+            const int lo = 16 * q, hi = min(16 * q + 15, t);
+            float loc[16];
+            float run = 1.f;
+#pragma unroll
+            for (int m = 15; m >= 0; --m) {
+                // loc[m] = prod of a_j, j in (lo + m, hi]
+                loc[m] = run;
+                if (lo + m <= hi)
+                    run = __fmul_rn(run, Av[lo + m]);
             }
-            Gam[t] = __fmul_rn(r, Av[0]);
+            // run = prod of a_j, j in [lo, hi] (1 for a quarter past t)
+            float tail = __shfl_down_sync(0xffffffffu, run, 1);  // quarters q + 1 ..
+            const float t2 = __shfl_down_sync(0xffffffffu, tail, 1);
+            const float t3 = __shfl_down_sync(0xffffffffu, t2, 1);
+            tail = q == 3 ? 1.f : (q == 2 ? tail : (q == 1 ? __fmul_rn(tail, t2) : __fmul_rn(__fmul_rn(tail, t2), t3)));
+#pragma unroll
+            for (int m = 0; m < 16; ++m) {
+                const int i = lo + m;
+                if (i <= t) {
+                    const float r = __fmul_rn(loc[m], tail);
+                    Rm[t * MST + i] = r;
+                    if (t == T - 1)
+                        rvec[i] = r;
+                    if (i == 0)
+                        Gam[t] = __fmul_rn(r, Av[0]);
+                }
+            }
         }
         __syncthreads();
 
         // 2. K K^T and Q K^T (bf16, exact operands): this warp's 16 rows x 32
-        //    columns of each; then L = beta (K K^T o R) below the diagonal
-        //    (stored permuted: column i at [i % 4][i / 4] of its row) and
+        //    columns of each; then L = beta (K K^T o R) below the diagonal and
         //    M = Q K^T o R on and below it
         {
             const int cb = (warp >> 2) * 32;
@@ -277,8 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_chain_chunked(const Params p)
                     const int t = rb + g8 + (e >> 1) * 8;
                     const int i = cb + nt * 8 + 2 * t4 + (e & 1);
                     const float rr = i <= t ? Rm[t * MST + i] : 0.f;
-                    Lp[t * MST + (i & 3) * 16 + (i >> 2)] =
-                        i < t ? __fmul_rn(bch[t], __fmul_rn(ck[nt][e], rr)) : 0.f;
+                    Lp[t * MST + i] = i < t ? __fmul_rn(bch[t], __fmul_rn(ck[nt][e], rr)) : 0.f;
                     Mq[t * MST + i] = __fmul_rn(cq[nt][e], rr);
                 }
             }
@@ -298,9 +329,9 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_chain_chunked(const Params p)
 #pragma unroll
                 for (int nt = 0; nt < 4; ++nt) {
                     const int n = cb + nt * 8 + g8;  // state row (d_v index)
-                    uint32_t h0, l0, h1, l1;
-                    split(S[n * SST + ks + t4], h0, l0);
-                    split(S[n * SST + ks + t4 + 4], h1, l1);
+                    const float2 s0 = S[n * SST + ks + t4], s1 = S[n * SST + ks + t4 + 4];
+                    const uint32_t h0 = f2tf32(s0.x), l0 = __float_as_uint(s0.y);
+                    const uint32_t h1 = f2tf32(s1.x), l1 = __float_as_uint(s1.y);
                     mma_tf32(acc[nt], a0, a1, a2, a3, h0, h1);
                     mma_tf32(acc[nt], a0, a1, a2, a3, l0, l1);
                 }
@@ -318,32 +349,64 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_chain_chunked(const Params p)
         }
         __syncthreads();
 
-        // 4. (I + L) U = P by forward substitution: column col = tid / 4,
-        //    the 4 threads of a column split each dot product by j mod 4
+        // 4. (I + L) U = P in blocks of 16 rows.  (a) the inverses D_b of the
+        //    four unit lower triangular diagonal blocks, one column per
+        //    thread; (b) per block b: X = P_b - L_{b,<b} U_{<b}, then
+        //    U_b = D_b X, one row and 4 columns per thread.  D lives in this
+        //    chunk's V buffer (dead after step 3).
         {
-            const int col = tid >> 2, s = tid & 3;
-            float u[T / 4];
+            float* D = reinterpret_cast<float*>(smem + kOffV + buf * kVBytes);  // [4][16][16]
+            if (tid < T) {
+                const int blk = tid >> 4, j = tid & 15;
+                const float* Lb = Lp + (16 * blk) * MST + 16 * blk;
+                float d[16];
 #pragma unroll
-            for (int i = 0; i < T; ++i) {
-                float part = 0.f;
-                const float* lrow = Lp + i * MST + s * 16;  // L[i][4m + s], m = 0..15
+                for (int i = 0; i < 16; ++i) {
+                    float acc = 0.f;
 #pragma unroll
-                for (int m = 0; m < T / 4; ++m) {
-                    if (4 * m + s < i)
-                        part = __fmaf_rn(lrow[m], u[m], part);
+                    for (int k = 0; k < i; ++k)
+                        acc = __fmaf_rn(Lb[i * MST + k], k >= j ? d[k] : 0.f, acc);
+                    d[i] = i < j ? 0.f : (i == j ? 1.f : -acc);
+                    D[(blk * 16 + i) * 16 + j] = d[i];
                 }
-                part = __fadd_rn(part, __shfl_xor_sync(0xffffffffu, part, 1));
-                part = __fadd_rn(part, __shfl_xor_sync(0xffffffffu, part, 2));
-                const float ui = __fsub_rn(U[i * MST + col], part);
-                if ((i & 3) == s)
-                    u[i >> 2] = ui;
             }
-            __syncwarp();
+            __syncthreads();
+            const int r = tid >> 4, c0 = 4 * (tid & 15);  // a row of the block, 4 columns
+#pragma unroll 1
+            for (int blk = 0; blk < 4; ++blk) {
+                const int row = 16 * blk + r;
+                float4 x = *reinterpret_cast<const float4*>(U + row * MST + c0);
+                for (int k0 = 0; k0 < 16 * blk; k0 += 16) {
 #pragma unroll
-            for (int m = 0; m < T / 4; ++m)
-                U[(4 * m + s) * MST + col] = u[m];
+                    for (int kk = 0; kk < 16; ++kk) {
+                        const float l = Lp[row * MST + k0 + kk];
+                        const float4 u = *reinterpret_cast<const float4*>(U + (k0 + kk) * MST + c0);
+                        x.x = __fmaf_rn(-l, u.x, x.x);
+                        x.y = __fmaf_rn(-l, u.y, x.y);
+                        x.z = __fmaf_rn(-l, u.z, x.z);
+                        x.w = __fmaf_rn(-l, u.w, x.w);
+                    }
+                }
+                *reinterpret_cast<float4*>(U + row * MST + c0) = x;
+                __syncthreads();
+                float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+                const float* Dr = D + (blk * 16 + r) * 16;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    if (i <= r) {
+                        const float dd = Dr[i];
+                        const float4 xi = *reinterpret_cast<const float4*>(U + (16 * blk + i) * MST + c0);
+                        y.x = __fmaf_rn(dd, xi.x, y.x);
+                        y.y = __fmaf_rn(dd, xi.y, y.y);
+                        y.z = __fmaf_rn(dd, xi.z, y.z);
+                        y.w = __fmaf_rn(dd, xi.w, y.w);
+                    }
+                }
+                __syncthreads();
+                *reinterpret_cast<float4*>(U + row * MST + c0) = y;
+                __syncthreads();
+            }
         }
-        __syncthreads();
 
         // 5. O = scale (Gamma (Q S^T) + M U): 16 tokens x 32 rows per warp
         {
@@ -358,9 +421,9 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_chain_chunked(const Params p)
 #pragma unroll
                 for (int nt = 0; nt < 4; ++nt) {
                     const int n = cb + nt * 8 + g8;
-                    uint32_t h0, l0, h1, l1;
-                    split(S[n * SST + ks + t4], h0, l0);
-                    split(S[n * SST + ks + t4 + 4], h1, l1);
+                    const float2 s0 = S[n * SST + ks + t4], s1 = S[n * SST + ks + t4 + 4];
+                    const uint32_t h0 = f2tf32(s0.x), l0 = __float_as_uint(s0.y);
+                    const uint32_t h1 = f2tf32(s1.x), l1 = __float_as_uint(s1.y);
                     mma_tf32(qs[nt], a0, a1, a2, a3, h0, h1);
                     mma_tf32(qs[nt], a0, a1, a2, a3, l0, l1);
                 }
@@ -409,27 +472,25 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_chain_chunked(const Params p)
                 for (int e = 0; e < 4; ++e) {
                     const int m = rb + g8 + (e >> 1) * 8;
                     const int n = nb + nt * 8 + 2 * t4 + (e & 1);
-                    acc[nt][e] = __fmul_rn(gT, S[m * SST + n]);
+                    acc[nt][e] = __fmul_rn(gT, S[m * SST + n].x);
                 }
             }
 #pragma unroll 2
             for (int ks = 0; ks < T; ks += 8) {
-                // A[m][k] = U[k][m]
+                // A[m][k] = r_k U[k][m] (split); B = K, exact in tf32
+                const float r0 = rvec[ks + t4], r1 = rvec[ks + t4 + 4];
                 uint32_t ah[4], al[4];
-                split(U[(ks + t4) * MST + rb + g8], ah[0], al[0]);
-                split(U[(ks + t4) * MST + rb + g8 + 8], ah[1], al[1]);
-                split(U[(ks + t4 + 4) * MST + rb + g8], ah[2], al[2]);
-                split(U[(ks + t4 + 4) * MST + rb + g8 + 8], ah[3], al[3]);
-                const float r0 = Rm[(T - 1) * MST + ks + t4], r1 = Rm[(T - 1) * MST + ks + t4 + 4];
+                split(__fmul_rn(r0, U[(ks + t4) * MST + rb + g8]), ah[0], al[0]);
+                split(__fmul_rn(r0, U[(ks + t4) * MST + rb + g8 + 8]), ah[1], al[1]);
+                split(__fmul_rn(r1, U[(ks + t4 + 4) * MST + rb + g8]), ah[2], al[2]);
+                split(__fmul_rn(r1, U[(ks + t4 + 4) * MST + rb + g8 + 8]), ah[3], al[3]);
 #pragma unroll
                 for (int nt = 0; nt < 8; ++nt) {
                     const int n = nb + nt * 8 + g8;
-                    uint32_t h0, l0, h1, l1;
-                    split(__fmul_rn(r0, bf2f(K + (ks + t4) * KST + n)), h0, l0);
-                    split(__fmul_rn(r1, bf2f(K + (ks + t4 + 4) * KST + n)), h1, l1);
-                    mma_tf32(acc[nt], ah[0], ah[1], ah[2], ah[3], h0, h1);
-                    mma_tf32(acc[nt], ah[0], ah[1], ah[2], ah[3], l0, l1);
-                    mma_tf32(acc[nt], al[0], al[1], al[2], al[3], h0, h1);
+                    const uint32_t b0 = bf2tf(K + (ks + t4) * KST + n);
+                    const uint32_t b1 = bf2tf(K + (ks + t4 + 4) * KST + n);
+                    mma_tf32(acc[nt], ah[0], ah[1], ah[2], ah[3], b0, b1);
+                    mma_tf32(acc[nt], al[0], al[1], al[2], al[3], b0, b1);
                 }
             }
             __syncthreads();  // every warp is done reading S (steps 3, 5) and U
@@ -439,7 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_chain_chunked(const Params p)
                 for (int e = 0; e < 4; ++e) {
                     const int m = rb + g8 + (e >> 1) * 8;
                     const int n = nb + nt * 8 + 2 * t4 + (e & 1);
-                    S[m * SST + n] = acc[nt][e];
+                    S[m * SST + n] = make_float2(acc[nt][e], tf32_rem(acc[nt][e]));
                 }
             }
         }
@@ -450,7 +511,9 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_chain_chunked(const Params p)
     const size_t base = (((size_t)b * p.Hv + h) * p.dv + row0) * DK;
     for (int i = tid; i < TV * DK / 4; i += kThreads) {
         const int r = i / (DK / 4), c4 = i % (DK / 4);
-        const float4 x = *reinterpret_cast<const float4*>(S + r * SST + 4 * c4);
+        const float4 s01 = *reinterpret_cast<const float4*>(S + r * SST + 4 * c4);
+        const float4 s23 = *reinterpret_cast<const float4*>(S + r * SST + 4 * c4 + 2);
+        const float4 x = make_float4(s01.x, s01.z, s23.x, s23.z);
         if (p.state_f16) {
             const __half2 lo = __float22half2_rn(make_float2(x.x, x.y));
             const __half2 hi = __float22half2_rn(make_float2(x.z, x.w));
