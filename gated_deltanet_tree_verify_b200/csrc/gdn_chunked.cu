@@ -315,17 +315,23 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_chain_chunked(const Params p)
             }
         }
 
-        // 3. P = beta (V - Gamma (K S^T)): this warp's 16 tokens x 32 of the
-        //    64 rows; K exact in tf32, S split
+        // 3. P = beta (V - Gamma (K S^T)), and Q S^T for step 5 (kept in
+        //    registers): this warp's 16 tokens x 32 of the 64 rows; K and Q
+        //    exact in tf32, S split (the two products share its fragments)
+        float qs[4][4] = {};
         {
             const int cb = (warp >> 2) * 32;
             float acc[4][4] = {};
-#pragma unroll 4
+#pragma unroll 2
             for (int ks = 0; ks < DK; ks += 8) {
                 const uint32_t a0 = bf2tf(K + (rb + g8) * KST + ks + t4);
                 const uint32_t a1 = bf2tf(K + (rb + g8 + 8) * KST + ks + t4);
                 const uint32_t a2 = bf2tf(K + (rb + g8) * KST + ks + t4 + 4);
                 const uint32_t a3 = bf2tf(K + (rb + g8 + 8) * KST + ks + t4 + 4);
+                const uint32_t e0 = bf2tf(Q + (rb + g8) * KST + ks + t4);
+                const uint32_t e1 = bf2tf(Q + (rb + g8 + 8) * KST + ks + t4);
+                const uint32_t e2 = bf2tf(Q + (rb + g8) * KST + ks + t4 + 4);
+                const uint32_t e3 = bf2tf(Q + (rb + g8 + 8) * KST + ks + t4 + 4);
 #pragma unroll
                 for (int nt = 0; nt < 4; ++nt) {
                     const int n = cb + nt * 8 + g8;  // state row (d_v index)
@@ -334,6 +340,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_chain_chunked(const Params p)
                     const uint32_t h1 = f2tf32(s1.x), l1 = __float_as_uint(s1.y);
                     mma_tf32(acc[nt], a0, a1, a2, a3, h0, h1);
                     mma_tf32(acc[nt], a0, a1, a2, a3, l0, l1);
+                    mma_tf32(qs[nt], e0, e1, e2, e3, h0, h1);
+                    mma_tf32(qs[nt], e0, e1, e2, e3, l0, l1);
                 }
             }
 #pragma unroll
@@ -411,23 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_chain_chunked(const Params p)
         // 5. O = scale (Gamma (Q S^T) + M U): 16 tokens x 32 rows per warp
         {
             const int cb = (warp >> 2) * 32;
-            float qs[4][4] = {}, mu[4][4] = {};
-#pragma unroll 4
-            for (int ks = 0; ks < DK; ks += 8) {
-                const uint32_t a0 = bf2tf(Q + (rb + g8) * KST + ks + t4);
-                const uint32_t a1 = bf2tf(Q + (rb + g8 + 8) * KST + ks + t4);
-                const uint32_t a2 = bf2tf(Q + (rb + g8) * KST + ks + t4 + 4);
-                const uint32_t a3 = bf2tf(Q + (rb + g8 + 8) * KST + ks + t4 + 4);
-#pragma unroll
-                for (int nt = 0; nt < 4; ++nt) {
-                    const int n = cb + nt * 8 + g8;
-                    const float2 s0 = S[n * SST + ks + t4], s1 = S[n * SST + ks + t4 + 4];
-                    const uint32_t h0 = f2tf32(s0.x), l0 = __float_as_uint(s0.y);
-                    const uint32_t h1 = f2tf32(s1.x), l1 = __float_as_uint(s1.y);
-                    mma_tf32(qs[nt], a0, a1, a2, a3, h0, h1);
-                    mma_tf32(qs[nt], a0, a1, a2, a3, l0, l1);
-                }
-            }
+            float mu[4][4] = {};
 #pragma unroll 2
             for (int ks = 0; ks < T; ks += 8) {
                 uint32_t ah[4], al[4];
