@@ -97,8 +97,11 @@ VerifyGeom verify_geometry(const VerifyArgs& a, bool use_workspace)
             off_desc = off;
             off += (size_t)a.n_nodes * sizeof(PosDesc);
             off_ab = off;
-            off += align16((size_t)2 * a.n_nodes * 4);  // g (then a) | beta, by node
+            off += align16((size_t)3 * a.n_nodes * 4);  // g (then a) | beta | a', by node
         } else {
+            off_ab = off;  // 1 / |k| by node (GDN_FLAG_QK_L2NORM trees)
+            if ((a.flags & GDN_FLAG_QK_L2NORM) && !chain && !g.reload)
+                off += align16((size_t)a.n_nodes * 4);
             off_raw = off;
             off += (size_t)kRing * (align16(kChunk * raw_bytes) + kChunk * sizeof(PosDesc));
         }
@@ -161,6 +164,7 @@ cudaError_t launch_verify(const VerifyArgs& a, const VerifyGeom& geom, cudaStrea
     kp.persist_last = (a.flags & GDN_FLAG_PERSIST_LAST) ? 1 : 0;
     kp.validate = (a.flags & GDN_FLAG_VALIDATE) ? 1 : 0;
     kp.early_tree = (a.flags & GDN_FLAG_EARLY_TREE) ? 1 : 0;
+    kp.qk_norm = (a.flags & GDN_FLAG_QK_L2NORM) ? 1 : 0;
     kp.ws = geom.gslots ? a.workspace : nullptr;
     kp.cu = a.cu_nodes;
     kp.total = a.total_nodes;

@@ -111,6 +111,7 @@ struct KParams {
     float scale;
     int rows, warps, slots;
     int persist_last, validate, early_tree;
+    int qk_norm;         // GDN_FLAG_QK_L2NORM: k and q normalised per node inside the kernel
     float* ws;           // global stack slots (kTreeGlobal kinds): slots x rows x d_k per CTA
     const int32_t* cu;   // varlen: [B + 1] node offsets of the packed layout (N: the most per sequence)
     int total;           // varlen: nodes in the packed layout
@@ -141,8 +142,25 @@ __device__ __forceinline__ bool seq_of(const KParams& p, int b, Seq& q)
 // One walk position: its node and tree metadata, and the node's scalars.
 struct PosDesc {
     int4 i;    // node, metadata, recomputation start, parent
-    float4 f;  // a = exp(g), beta, k . q, unused
+    float4 f;  // a = exp(g), beta', k . q, a' (see node_scalars)
+    float4 x;  // output coefficient scale / |q| (read only with qk_norm), unused
 };
+
+// A node's scalars for the state step.  With q and k normalised inside the
+// kernel (qk_norm; rk = 1 / |k|, rq = 1 / |q|) the step runs on the raw
+// k, q: with S k^ = rk (S k) and u = beta (v - a S_p k^),
+//     u' = rk u = (beta rk) (v - (a rk) (S_p k)),   S_n = a S_p + u' k^T,
+//     o = scale S_n q^ = (scale rq) (a (S_p q) + u' (k . q)),
+// so beta' = beta rk, a' = a rk and the output coefficient scale rq.
+// Without it rk = rq = 1: beta' = beta, a' = a (bit for bit).
+__device__ __forceinline__ void node_scalars(float a, float beta, float rk, float& beta_p, float& a_p)
+{
+    beta_p = __fmul_rn(beta, rk);
+    a_p = __fmul_rn(a, rk);
+}
+
+// 1 / |x| from the sum of squares (epsilon 0: a zero vector gives inf).
+__device__ __forceinline__ float inv_norm(float ss) { return __fdiv_rn(1.f, __fsqrt_rn(ss)); }
 
 // ---------------------------------------------------------------------------
 // Lane geometry and per-node arithmetic
@@ -217,7 +235,7 @@ __device__ __forceinline__ float row_sum_first(const float (&cs)[C])
 template <int LR, int C, int RL, bool WITH_Q>
 __device__ __forceinline__ void gdn_step(StateT<C, RL>& S, const float2 (&k2)[4 * C],
                                          const float2 (&q2)[4 * C], const float (&vr)[RL], float a,
-                                         float beta, float (&pq)[RL], float (&uo)[RL])
+                                         float a_read, float beta, float (&pq)[RL], float (&uo)[RL])
 {
     float w[RL];
 #pragma unroll
@@ -246,7 +264,7 @@ __device__ __forceinline__ void gdn_step(StateT<C, RL>& S, const float2 (&k2)[4 
     const float2 a2 = make_float2(a, a);
 #pragma unroll
     for (int r = 0; r < RL; ++r) {
-        const float u = __fmul_rn(beta, __fsub_rn(vr[r], __fmul_rn(a, w[r])));
+        const float u = __fmul_rn(beta, __fsub_rn(vr[r], __fmul_rn(a_read, w[r])));
         uo[r] = u;
         const float2 u2 = make_float2(u, u);
 #pragma unroll
@@ -258,10 +276,10 @@ __device__ __forceinline__ void gdn_step(StateT<C, RL>& S, const float2 (&k2)[4 
 // State update only (recompute path): the same instructions on S.
 template <int LR, int C, int RL>
 __device__ __forceinline__ void gdn_update(StateT<C, RL>& S, const float2 (&k2)[4 * C],
-                                           const float (&vr)[RL], float a, float beta)
+                                           const float (&vr)[RL], float a, float a_read, float beta)
 {
     float pq[RL], uo[RL];
-    gdn_step<LR, C, RL, false>(S, k2, k2, vr, a, beta, pq, uo);
+    gdn_step<LR, C, RL, false>(S, k2, k2, vr, a, a_read, beta, pq, uo);
 }
 
 // Element e of the k (part 0) or q (part DK) row of a shared-memory record:
@@ -280,6 +298,22 @@ __device__ __forceinline__ float rec_elem(const float* rec, int part, int e)
 // k . q of one node's record, reduced by a group of 8 lanes (sub = lane % 8;
 // a warp handles four nodes at once; every lane of the warp must call it).
 // The same reduction wherever it is computed.
+template <int DK, int LR, typename RT>
+__device__ __forceinline__ float node_dot8(const RT* rec, int sub, int pa, int pb)
+{
+    float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+    for (int j = sub; j < DK; j += 16) {
+        acc0 = __fmaf_rn(rec_elem<DK, LR>(rec, pa, j), rec_elem<DK, LR>(rec, pb, j), acc0);
+        acc1 = __fmaf_rn(rec_elem<DK, LR>(rec, pa, j + 8), rec_elem<DK, LR>(rec, pb, j + 8), acc1);
+    }
+    float acc = __fadd_rn(acc0, acc1);
+#pragma unroll
+    for (int off = 4; off >= 1; off >>= 1)
+        acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, off));
+    return acc;
+}
+
 template <int DK, int LR, typename RT>
 __device__ __forceinline__ float node_kq8(const RT* rec, int sub)
 {
@@ -850,9 +884,9 @@ __device__ __forceinline__ void source_parent(StateT<C, RL>& S, int m, int pp, i
         tree.for_path(pp, start, [&](int y) {
             float2 k2[4 * C];
             float vr[RL];
-            float a, be;
-            fetch(y, k2, vr, a, be);
-            gdn_update<LR, C, RL>(S, k2, vr, a, be);
+            float a, ar, be;
+            fetch(y, k2, vr, a, ar, be);
+            gdn_update<LR, C, RL>(S, k2, vr, a, ar, be);
         });
     }
 }
@@ -937,12 +971,13 @@ __device__ __forceinline__ void walk(StateT<C, RL>& S, const KParams& p, const S
         widen_raw<C, RL>(R, k2, q2, vr);
         const float a = d.f.x;
         float pq[RL], u[RL];
-        gdn_step<LM::LR, C, RL, true>(S, k2, q2, vr, a, d.f.y, pq, u);
+        gdn_step<LM::LR, C, RL, true>(S, k2, q2, vr, a, d.f.w, d.f.y, pq, u);
         if (L.cl == 0) {
+            const float oc = p.qk_norm ? ctx.out_coef(pos) : p.scale;
             float* o = out_lane + (size_t)n * out_stride;
 #pragma unroll
             for (int r = 0; r < RL; ++r)
-                o[r * LM::RG] = __fmul_rn(p.scale, __fmaf_rn(u[r], d.f.z, __fmul_rn(a, pq[r])));
+                o[r * LM::RG] = __fmul_rn(oc, __fmaf_rn(u[r], d.f.z, __fmul_rn(a, pq[r])));
         }
         if (!p.persist_last || pos == N - 1)
             persist<DK, C, RL, ST>(S, ns_lane + (size_t)(p.persist_last ? 0 : n) * ns_stride);
@@ -982,11 +1017,12 @@ struct StagedFetch {
     int N;
     LaneMap<DK, C, RL> L;
     __device__ __forceinline__ void operator()(int y, float2 (&k2)[4 * C], float (&vr)[RL], float& a,
-                                               float& be) const
+                                               float& ar, float& be) const
     {
         load_k<DK, C, RL, RT>(recs + (size_t)y * rec_elems, L, k2, vr);
         a = ab[y];
         be = ab[N + y];
+        ar = ab[2 * N + y];
     }
 };
 
@@ -1003,6 +1039,7 @@ struct StagedCtx {
     // whether position pos's descriptor may be read before begin(pos)
     __device__ __forceinline__ bool ahead(int) const { return true; }
     __device__ __forceinline__ PosDesc desc(int pos) const { return desc_[pos]; }
+    __device__ __forceinline__ float out_coef(int pos) const { return desc_[pos].x.x; }
     __device__ __forceinline__ const RT* rec(int, int n) const { return recs + (size_t)n * rec_elems; }
     __device__ __forceinline__ StagedFetch<DK, C, RL, RT> fetcher() const
     {
@@ -1035,11 +1072,12 @@ __device__ __forceinline__ float* cta_slots(const KParams& p, float* slotbuf)
 }
 
 // Prologue pass of the staged kernel over walk positions, four per warp and
-// pass (8 lanes each): converts g to a = exp(g) in place (ab holds g | beta by
-// node) and writes each position's descriptor with k . q of its node.
+// pass (8 lanes each): turns ab (g | beta | -, by node) into a | beta' | a'
+// (node_scalars) and writes each position's descriptor with k . q of its
+// node (and, with qk_norm, the output coefficient).
 template <int DK, int LR, typename QT, class Tree>
 __device__ __forceinline__ void write_descs(const Tree& tree, const unsigned char* raw, uint32_t raw_bytes,
-                                            float* ab, PosDesc* desc, int N)
+                                            float* ab, PosDesc* desc, int N, int qk_norm, float scale)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
     const int sub = lane & 7;
@@ -1050,12 +1088,22 @@ __device__ __forceinline__ void write_descs(const Tree& tree, const unsigned cha
         const QT* rrec = reinterpret_cast<const QT*>(raw + (size_t)n * raw_bytes);
         const bool valid = p0 + (lane >> 3) < N;
         const float kq = node_kq8<DK, LR>(rrec, sub);
+        float rk = 1.f, rq = 1.f;
+        if (qk_norm) {
+            rk = inv_norm(node_dot8<DK, LR>(rrec, sub, 0, 0));
+            rq = inv_norm(node_dot8<DK, LR>(rrec, sub, DK, DK));
+        }
         if (sub == 0 && valid) {
             const float a = gdn_gate(ab[n]);
+            float bp, ap;
+            node_scalars(a, ab[N + n], rk, bp, ap);
             ab[n] = a;
+            ab[N + n] = bp;
+            ab[2 * N + n] = ap;
             PosDesc d;
             d.i = make_int4(n, m, tree.rstart(pos), tree.parent(n));
-            d.f = make_float4(a, ab[N + n], kq, 0.f);
+            d.f = make_float4(a, bp, kq, ap);
+            d.x = make_float4(__fmul_rn(scale, rq), 0.f, 0.f, 0.f);
             desc[pos] = d;
         }
     }
@@ -1068,7 +1116,7 @@ __device__ __forceinline__ void staged_finish(StateT<C, RL>& S, const KParams& p
                                               const LaneMap<DK, C, RL>& L)
 {
     constexpr int LR = LaneMap<DK, C, RL>::LR;
-    write_descs<DK, LR, QT>(tree, raw, p.raw_bytes, ab, desc, sq.N);
+    write_descs<DK, LR, QT>(tree, raw, p.raw_bytes, ab, desc, sq.N, p.qk_norm, p.scale);
     __syncthreads();
     const uint32_t rec_elems = p.raw_bytes / (uint32_t)sizeof(QT);
     StagedCtx<DK, C, RL, QT> ctx{reinterpret_cast<const QT*>(raw), desc, ab, rec_elems, sq.N, L};
@@ -1217,11 +1265,12 @@ struct GlobalFetch {
     const QT* vg;
     const float* g;
     const float* beta;
-    size_t bN;  // the sequence's first node
+    size_t bN;         // the sequence's first node
+    const float* rkn;  // qk_norm: 1 / |k| per node (written by the producer), else NULL
     int Hk, Hv, dv, hk, h, row0;
     LaneMap<DK, C, RL> L;
     __device__ __forceinline__ void operator()(int y, float2 (&k2)[4 * C], float (&vr)[RL], float& a,
-                                               float& be) const
+                                               float& ar, float& be) const
     {
         using LM = LaneMap<DK, C, RL>;
         const size_t node = bN + y;
@@ -1238,7 +1287,7 @@ struct GlobalFetch {
             vr[r] = Widen<QT>::load1(vg + (node * Hv + h) * dv + row0 + L.row + r * LM::RG);
         const size_t gi = node * Hv + h;
         a = gdn_gate(__ldg(g + gi));
-        be = __ldg(beta + gi);
+        node_scalars(a, __ldg(beta + gi), rkn != nullptr ? rkn[y] : 1.f, be, ar);
     }
 };
 
@@ -1284,6 +1333,10 @@ struct RingCtx {
     }
     // only within the chunk already waited for
     __device__ __forceinline__ bool ahead(int pos) const { return pos % kChunk != 0; }
+    __device__ __forceinline__ float out_coef(int pos) const
+    {
+        return reinterpret_cast<const PosDesc*>(slot(pos) + desc_off)[pos % kChunk].x.x;
+    }
     __device__ __forceinline__ const QT* rec(int pos, int) const
     {
         return reinterpret_cast<const QT*>(slot(pos) + (size_t)(pos % kChunk) * raw_bytes);
@@ -1326,6 +1379,8 @@ __global__ void __launch_bounds__((kMaxWarps + 1) * 32) gdn_verify_ring(const KP
     }
     const int N = sq.N;
     const TreeView T(reinterpret_cast<int*>(smem + p.off_tree), N);
+    // qk_norm on trees: 1 / |k| per node, for recomputations (chains never recompute)
+    float* rkn = (p.qk_norm && !CHAIN && !INDEX) ? reinterpret_cast<float*>(smem + p.off_ab) : nullptr;
 
     if (tid == 0) {
         for (int i = 0; i < kRing; ++i) {
@@ -1436,8 +1491,13 @@ __global__ void __launch_bounds__((kMaxWarps + 1) * 32) gdn_verify_ring(const KP
             for (int i0 = 0; i0 < cnt; i0 += 4) {
                 const int gi = i0 + (lane >> 3);
                 const int i = min(gi, cnt - 1);
-                const float kq =
-                    node_kq8<DK, LM::LR>(reinterpret_cast<const QT*>(base + (size_t)i * p.raw_bytes), lane & 7);
+                const QT* rrec = reinterpret_cast<const QT*>(base + (size_t)i * p.raw_bytes);
+                const float kq = node_kq8<DK, LM::LR>(rrec, lane & 7);
+                float rk = 1.f, rq = 1.f;
+                if (p.qk_norm) {
+                    rk = inv_norm(node_dot8<DK, LM::LR>(rrec, lane & 7, 0, 0));
+                    rq = inv_norm(node_dot8<DK, LM::LR>(rrec, lane & 7, DK, DK));
+                }
                 const int src_lane = i;
                 const int n = __shfl_sync(0xffffffffu, dn, src_lane);
                 const int m = __shfl_sync(0xffffffffu, dm, src_lane);
@@ -1446,10 +1506,15 @@ __global__ void __launch_bounds__((kMaxWarps + 1) * 32) gdn_verify_ring(const KP
                 const float a = __shfl_sync(0xffffffffu, da, src_lane);
                 const float be = __shfl_sync(0xffffffffu, dbe, src_lane);
                 if ((lane & 7) == 0 && gi < cnt) {
+                    float bp, ap;
+                    node_scalars(a, be, rk, bp, ap);
                     PosDesc d;
                     d.i = make_int4(n, m, rs, pp);
-                    d.f = make_float4(a, be, kq, 0.f);
+                    d.f = make_float4(a, bp, kq, ap);
+                    d.x = make_float4(__fmul_rn(p.scale, rq), 0.f, 0.f, 0.f);
                     sdesc[i] = d;
+                    if (rkn != nullptr)
+                        rkn[n] = rk;  // for recomputation of this node's subtree
                 }
             }
             mbar_arrive(&full[s]);
@@ -1463,7 +1528,7 @@ __global__ void __launch_bounds__((kMaxWarps + 1) * 32) gdn_verify_ring(const KP
         p.state_in + ((size_t)b * p.Hv + h) * p.dv * DK + (size_t)row0 * DK + L.tile_offset();
     StateT<C, RL> S;
     load_rows<DK, C, RL>(S, sin_lane);
-    const GlobalFetch<DK, C, RL, QT> gf{kg, vg, p.g, p.beta, (size_t)sq.n0, p.Hk, p.Hv, p.dv, hk, h, row0, L};
+    const GlobalFetch<DK, C, RL, QT> gf{kg, vg, p.g, p.beta, (size_t)sq.n0, rkn, p.Hk, p.Hv, p.dv, hk, h, row0, L};
     RingCtx<DK, C, RL, QT> ctx{full, empty, ring, p.raw_bytes, slot_bytes, desc_off, p.status, lane, gf};
     float* lane_slot = cta_slots<DK, TREE>(p, slotbuf) + 4 * threadIdx.x;
     if constexpr (CHAIN)

@@ -25,6 +25,7 @@ GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_BAD_TREE, GDN_ERR_BAD_
     GDN_ERR_CUDA, GDN_ERR_TIMEOUT = range(7)
 # flags
 GDN_FLAG_CHAIN, GDN_FLAG_PERSIST_LAST, GDN_FLAG_VALIDATE, GDN_FLAG_EARLY_TREE, GDN_FLAG_CHUNKED = 1, 2, 4, 8, 16
+GDN_FLAG_QK_L2NORM = 32
 GDN_MAX_TREE_NODES = 1024
 
 _TORCH_DTYPE = {GDN_F32: torch.float32, GDN_F16: torch.float16, GDN_BF16: torch.bfloat16}

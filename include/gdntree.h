@@ -95,7 +95,12 @@ enum {
      * of the delta rule), for long prefill-style chains.  Same results up to
      * f32 rounding (products in split tf32), not bit-identical to the
      * token-by-token path.  Unsupported shapes: GDN_ERR_UNSUPPORTED. */
-    GDN_FLAG_CHUNKED = 16
+    GDN_FLAG_CHUNKED = 16,
+    /* q and k are given raw; the kernel L2-normalises each (node, k-head)
+     * row, x / |x| with no epsilon (a zero row gives inf/NaN), as the
+     * workloads' input preparation does.  Folded into per-node scalars, so
+     * the node loop does the same work.  Not with GDN_FLAG_CHUNKED. */
+    GDN_FLAG_QK_L2NORM = 32
 };
 
 /* Problem description, shared by verify and commit. */

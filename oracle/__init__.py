@@ -52,6 +52,8 @@ def _load():
         lib.gdn_oracle_round.restype = c_double
         lib.gdn_oracle_round_array.argtypes = [c_int, dp, dp, c_i64]
         lib.gdn_oracle_round_array.restype = None
+        lib.gdn_oracle_l2norm_rows.argtypes = [dp, c_i64, c_int]
+        lib.gdn_oracle_l2norm_rows.restype = None
         lib.gdn_oracle_check_tree.argtypes = [c_int, ip]
         lib.gdn_oracle_check_tree.restype = c_int
         lib.gdn_oracle_check_path.argtypes = [c_int, ip, ip, c_int, c_int]
@@ -86,17 +88,28 @@ class OracleError(RuntimeError):
         self.code = code
 
 
+def l2norm_rows(x) -> np.ndarray:
+    """x / |x| over the last axis, in double (gdn_oracle_l2norm_rows)."""
+    y = _f64(x).copy()
+    _load().gdn_oracle_l2norm_rows(_dp(y), y.size // y.shape[-1], y.shape[-1])
+    return y
+
+
 def verify(q, k, v, g, beta, parent, state_in, scale: float, state_dtype: str = "f32",
-           want_exact: bool = False, nthreads: int = 1
+           want_exact: bool = False, nthreads: int = 1, qk_l2norm: bool = False
            ) -> Tuple[np.ndarray, np.ndarray, Optional[np.ndarray]]:
     """Run the tree recurrence.  Returns (out, persisted_states, exact_states).
 
     Shapes as in gdn_oracle.c.  ``persisted_states`` holds each node's state
     rounded to ``state_dtype`` (as float64 values); ``exact_states`` (only if
-    ``want_exact``) holds the unrounded float64 states.  Raises OracleError on a
-    bad tree or bad arguments.
+    ``want_exact``) holds the unrounded float64 states.  With ``qk_l2norm``
+    q and k are L2-normalised per (node, head) first (the preparation the
+    library's GDN_FLAG_QK_L2NORM fuses).  Raises OracleError on a bad tree or
+    bad arguments.
     """
     lib = _load()
+    if qk_l2norm:
+        q, k = l2norm_rows(q), l2norm_rows(k)
     q, k, v, g, beta, state_in = map(_f64, (q, k, v, g, beta, state_in))
     parent = _i32(parent)
     B, N, Hk, dk = q.shape
@@ -150,10 +163,12 @@ def check_path(parent_row, path_row, length: int) -> int:
     return _load().gdn_oracle_check_path(len(p), _ip(p), _ip(a), int(length), len(a))
 
 
-def verify_problem(prob, state_dtype: str = "f32", want_exact: bool = False, nthreads: int = 1):
+def verify_problem(prob, state_dtype: str = "f32", want_exact: bool = False, nthreads: int = 1,
+                   qk_l2norm: bool = False):
     """Convenience: run ``verify`` on a gdn_inputs.Problem."""
     return verify(prob.q, prob.k, prob.v, prob.g, prob.beta, prob.parent, prob.state_in,
-                  prob.scale, state_dtype=state_dtype, want_exact=want_exact, nthreads=nthreads)
+                  prob.scale, state_dtype=state_dtype, want_exact=want_exact, nthreads=nthreads,
+                  qk_l2norm=qk_l2norm)
 
 
 def verify_pair(prob, b: int, h: int, state_dtype: str = "f32", want_exact: bool = False):

@@ -72,6 +72,23 @@ void gdn_oracle_round_array(int state_dtype, const double* x, double* y, int64_t
 }
 
 /* parent[0] = -1 and 0 <= parent[n] < n for n >= 1. */
+/* L2 normalisation of n rows of length d, in place: x / sqrt(sum_j x_j^2),
+ * with no epsilon (a zero row becomes NaN).  This is the workloads' input
+ * preparation of q and k ("then L2-normalised per head", per node and
+ * head over d_k), which the library can fuse into its verify kernels. */
+void gdn_oracle_l2norm_rows(double* x, int64_t n, int d)
+{
+    for (int64_t r = 0; r < n; ++r) {
+        double* row = x + r * d;
+        double ss = 0.0;
+        for (int j = 0; j < d; ++j)
+            ss += row[j] * row[j];
+        const double nrm = sqrt(ss);
+        for (int j = 0; j < d; ++j)
+            row[j] = row[j] / nrm;
+    }
+}
+
 int gdn_oracle_check_tree(int n_nodes, const int32_t* parent)
 {
     if (n_nodes < 1 || parent[0] != -1)

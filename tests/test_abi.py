@@ -80,7 +80,8 @@ def test_verify_batch_zero_is_a_noop(lib):
     (dict(n_nodes=gdn.GDN_MAX_TREE_NODES + 1), gdn.GDN_ERR_UNSUPPORTED),
     (dict(qkv_dtype=gdn.GDN_F16), gdn.GDN_ERR_UNSUPPORTED),
     (dict(state_dtype=gdn.GDN_BF16), gdn.GDN_ERR_UNSUPPORTED),
-    (dict(flags=32), gdn.GDN_ERR_INVALID_ARG),
+    (dict(flags=64), gdn.GDN_ERR_INVALID_ARG),
+    (dict(flags=16 | 1 | 2 | 32), gdn.GDN_ERR_UNSUPPORTED),  # chunked + fused normalisation
     (dict(flags=16), gdn.GDN_ERR_UNSUPPORTED),      # chunked needs CHAIN + PERSIST_LAST
     (dict(flags=16 | 1 | 2, d_v=32), gdn.GDN_ERR_UNSUPPORTED),
     (dict(scale=float("nan")), gdn.GDN_ERR_INVALID_ARG),

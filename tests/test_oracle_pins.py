@@ -356,3 +356,49 @@ def test_hand_worked_example_d2():
         np.testing.assert_allclose(out[0, n, 0], np.array(O[n]) / r2, atol=1e-14)
     so = oracle.commit(st, par, np.array([[0, 1, 3]], np.int32), np.array([3], np.int32))
     np.testing.assert_allclose(so[0, 0], np.float32(np.array(S[3])), atol=0)
+
+
+# ----------------------------------------------------------------------------
+# q/k L2 normalisation (the workloads' input preparation, fused by the
+# library's GDN_FLAG_QK_L2NORM)
+# ----------------------------------------------------------------------------
+
+def test_l2norm_worked_example():
+    # 3-4-5 and 1-2-2-4 (norm 5) triangles, by hand
+    x = np.array([[3.0, 4.0, 0.0, 0.0], [1.0, 2.0, 2.0, 4.0]])
+    y = oracle.l2norm_rows(x)
+    np.testing.assert_array_equal(y[0], [0.6, 0.8, 0.0, 0.0])
+    np.testing.assert_allclose(y[1], [0.2, 0.4, 0.4, 0.8], rtol=0, atol=1e-15)
+
+
+def test_l2norm_invariants():
+    rng = np.random.default_rng(3)
+    x = rng.normal(size=(5, 7, 32))
+    y = oracle.l2norm_rows(x)
+    np.testing.assert_allclose(np.sqrt((y ** 2).sum(-1)), 1.0, rtol=0, atol=1e-14)
+    # direction kept: y is a positive multiple of x
+    ratio = y / x
+    np.testing.assert_allclose(ratio, np.broadcast_to(ratio[..., :1], ratio.shape), rtol=1e-12)
+    assert (ratio > 0).all()
+    # scale invariance and idempotence
+    np.testing.assert_allclose(oracle.l2norm_rows(3.5 * x), y, rtol=0, atol=1e-15)
+    np.testing.assert_allclose(oracle.l2norm_rows(y), y, rtol=0, atol=1e-15)
+    # epsilon 0: a zero row is NaN, not silently zero
+    z = oracle.l2norm_rows(np.zeros((1, 4)))
+    assert np.isnan(z).all()
+
+
+def test_verify_with_l2norm_equals_verify_on_normalised_inputs():
+    prob = make_problem(batch=1, n_nodes=6, n_k_heads=1, n_v_heads=2, d_k=8, d_v=4, tree="random", seed=5,
+                        qkv_dtype="f32")
+    rng = np.random.default_rng(9)
+    qr = prob.q.double().numpy() * rng.uniform(0.2, 5.0, size=prob.q.shape[:3] + (1,))
+    kr = prob.k.double().numpy() * rng.uniform(0.2, 5.0, size=prob.k.shape[:3] + (1,))
+    a = oracle.verify(qr, kr, prob.v, prob.g, prob.beta, prob.parent, prob.state_in, prob.scale,
+                      want_exact=True, qk_l2norm=True)
+    b = oracle.verify(oracle.l2norm_rows(qr), oracle.l2norm_rows(kr), prob.v, prob.g, prob.beta, prob.parent,
+                      prob.state_in, prob.scale, want_exact=True)
+    for x, y in zip(a, b):
+        np.testing.assert_array_equal(x, y)
+    # and the raw inputs were not unit (the normalisation did something)
+    assert abs(np.linalg.norm(kr[0, 0, 0]) - 1.0) > 1e-3
