@@ -88,6 +88,27 @@ def ddtree_like_tree(budget: int, gen: torch.Generator, top_k: int = 4,
     return np.asarray(parent, dtype=np.int32)
 
 
+def draft_logprobs(batch: int, max_depth: int, top_k: int, gen: torch.Generator,
+                   quantum: float = 0.0) -> np.ndarray:
+    """Synthetic drafter output for the tree builder: [batch][max_depth][top_k]
+    float32 log-probabilities, each row non-increasing (rank 0 best).
+
+    Per position: logits z ~ N(0, 2^2) for the top_k candidates and one more
+    entry r ~ N(0, 1) standing for the rest of the vocabulary; the row is
+    log_softmax([z, r]) restricted to the candidates, sorted descending.  With
+    quantum > 0 the values are rounded down to multiples of it, which makes
+    exact ties common.
+    """
+    z = torch.randn(batch, max_depth, top_k, generator=gen, dtype=torch.float64) * 2.0
+    r = torch.randn(batch, max_depth, 1, generator=gen, dtype=torch.float64)
+    lp = torch.log_softmax(torch.cat([z, r], dim=2), dim=2)[:, :, :top_k]
+    lp, _ = torch.sort(lp, dim=2, descending=True)
+    lp = lp.numpy()
+    if quantum > 0:
+        lp = np.floor(lp / quantum) * quantum
+    return np.ascontiguousarray(lp, dtype=np.float32)
+
+
 def tree_depths(parent: Sequence[int]) -> np.ndarray:
     d = np.zeros(len(parent), dtype=np.int32)
     for n in range(1, len(parent)):
