@@ -38,7 +38,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from gdn_inputs import make_problem  # noqa: E402
+from gdn_inputs import draft_logprobs, make_problem  # noqa: E402
 
 METRIC = "GDN tree-verify nodes/s and achieved HBM GB/s (% of B200 peak) at budget 22"
 UNIT = "tree-nodes/s"
@@ -618,6 +618,56 @@ def _varlen_point(*, budgets, state_dtype, workspace=False, reps=20, min_bytes=5
     return t, T * one + B * N_V_HEADS * D * D * 4, T
 
 
+def _build_point(*, batch, budget, max_depth=16, top_k=8, chain_seed=False, reps=50, seed=31):
+    """Mean time of one gdn_build_tree launch (graph-replayed back to back),
+    and the oracle's time per tree on this host for comparison."""
+    import gated_deltanet_tree_verify_b200 as gdn
+    from oracle import tree_build as tb
+    gen = torch.Generator().manual_seed(seed)
+    lp = draft_logprobs(batch, max_depth, top_k, gen)
+    lp_d = torch.from_numpy(lp).cuda()
+    N = budget + 1
+    par = torch.empty(batch, N, dtype=torch.int32, device="cuda")
+    dep = torch.empty_like(par)
+    rk = torch.empty_like(par)
+    sc = torch.empty(batch, N, device="cuda")
+    desc = gdn.make_build_desc(batch=batch, max_depth=max_depth, top_k=top_k, budget=budget,
+                               flags=gdn.GDN_BUILD_CHAIN_SEED if chain_seed else 0)
+
+    def run_all():
+        for _ in range(reps):
+            gdn.gdn_build_tree(desc, lp_d, par, node_depth=dep, node_rank=rk, node_score=sc)
+
+    run_all()
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=s):
+            run_all()
+    torch.cuda.current_stream().wait_stream(s)
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    t = e0.elapsed_time(e1) / 1e3 / reps
+    del graph
+    got = par.cpu().numpy()
+    want = tb.build_trees(lp, budget, chain_seed)[0]
+    t0 = time.perf_counter()
+    n_cpu = 0
+    while n_cpu < batch and time.perf_counter() - t0 < 2.0:
+        tb.build_tree(lp[n_cpu], budget, chain_seed)
+        n_cpu += 1
+    cpu_per_tree = (time.perf_counter() - t0) / max(1, n_cpu)
+    return t, bool((got == want).all()), cpu_per_tree
+
+
 def run_sweep(args):
     import gated_deltanet_tree_verify_b200 as gdn
     gdn.load_library()
@@ -637,8 +687,21 @@ def run_sweep(args):
         points.append(dict(kind="varlen", budget=0, batch=8, state_dtype=sd, ws=ws))
     points.append(dict(kind="chain4096", budget=4095, batch=8, state_dtype="f32"))
     points.append(dict(kind="chain4096", budget=4095, batch=8, state_dtype="f32", chunked=True))
+    for budget in (22, 64, 128, 1023):
+        for batch in (1, 8, 64):
+            points.append(dict(kind="build", budget=budget, batch=batch))
+    if args.sweep_kinds:
+        keep = set(args.sweep_kinds.split(","))
+        points = [pt for pt in points if pt["kind"] in keep]
     varlen_budgets = [8, 64, 22, 15, 32, 22, 48, 8]
     for pt in points:
+        if pt["kind"] == "build":
+            t, ok, cpu = _build_point(batch=pt["batch"], budget=pt["budget"])
+            print(json.dumps({"sweep": "build_tree", "budget": pt["budget"], "batch": pt["batch"],
+                              "max_depth": 16, "top_k": 8, "build_us": t * 1e6, "trees_per_s": pt["batch"] / t,
+                              "ns_per_pop": t * 1e9 / pt["budget"], "matches_oracle": ok,
+                              "oracle_us_per_tree": cpu * 1e6}), flush=True)
+            continue
         n = pt["budget"] + 1
         if pt["kind"] == "varlen":
             t, vb, T = _varlen_point(budgets=varlen_budgets, state_dtype=pt["state_dtype"], workspace=pt["ws"])
@@ -693,6 +756,9 @@ def main(argv=None):
     ap.add_argument("--sweep", action="store_true",
                     help="single-layer verify timings over budgets, batches, dtypes and the long chain "
                          "(one JSON line per point; not the benchmark line)")
+    ap.add_argument("--sweep-kinds", default="",
+                    help="comma-separated subset of the sweep's point kinds (tree, chain16, varlen, chain4096, "
+                         "build); default all")
     ap.add_argument("--sm-mhz", type=float, default=1965.0,
                     help="SM clock for the sweep's FP32 ALU roofline (default: the B200 maximum)")
     args = ap.parse_args(argv)

@@ -122,6 +122,7 @@ const char* gdn_status_str(gdn_status s)
         case GDN_ERR_BAD_PATH: return "GDN_ERR_BAD_PATH";
         case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
         case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT";
+        case GDN_ERR_BAD_INPUT: return "GDN_ERR_BAD_INPUT";
     }
     return "GDN_ERR_UNKNOWN";
 }
@@ -478,6 +479,93 @@ gdn_status gdn_tree_verify_static_ws(const gdn_tree_desc* desc, const void* q, c
         return st;
     return verify_impl(desc, nullptr, 0, q, k, v, g, beta, parent_idx, state_in, out, node_states, ws,
                        kStaticWorkspaceBytes, stream, false);
+}
+
+}  // extern "C"
+
+// ---- gdn_build_tree --------------------------------------------------------
+
+namespace {
+
+// K + K^2 + .. + K^D, saturated at 2^31.
+long long candidate_nodes(int D, int K)
+{
+    long long total = 0, layer = 1;
+    for (int d = 0; d < D; ++d) {
+        layer *= K;
+        total += layer;
+        if (total >= (1ll << 31))
+            return 1ll << 31;
+    }
+    return total;
+}
+
+}  // namespace
+
+extern "C" {
+
+gdn_status gdn_build_tree(const gdn_build_desc* desc, const float* logp, const int32_t* topk_ids,
+                          int32_t* parent_idx, int32_t* node_depth, int32_t* node_rank, int32_t* node_token,
+                          float* node_score, cudaStream_t stream)
+{
+    g_detail[0] = '\0';
+    if (desc == nullptr)
+        return fail(GDN_ERR_INVALID_ARG, "desc is NULL%s");
+    const gdn_build_desc& d = *desc;
+    if ((d.flags & ~3u) != 0)
+        return fail(GDN_ERR_INVALID_ARG, "unknown flag bits%s");
+    if (d.batch < 0 || d.max_depth < 1 || d.top_k < 1 || d.budget < 0)
+        return fail(GDN_ERR_INVALID_ARG, "batch, max_depth, top_k or budget out of range%s");
+    if (d.max_depth > 255 || d.top_k > 255 || d.max_depth * d.top_k > 4096)
+        return fail(GDN_ERR_UNSUPPORTED, "max_depth or top_k above 255, or max_depth * top_k above 4096%s");
+    if (d.budget > GDN_MAX_TREE_NODES - 1)
+        return fail(GDN_ERR_UNSUPPORTED, "budget above GDN_MAX_TREE_NODES - 1%s");
+    if (d.budget > candidate_nodes(d.max_depth, d.top_k))
+        return fail(GDN_ERR_INVALID_ARG, "budget exceeds the nodes the candidates span%s");
+    if (!logp || !parent_idx)
+        return fail(GDN_ERR_INVALID_ARG, "logp or parent_idx is NULL%s");
+    if (node_token && !topk_ids)
+        return fail(GDN_ERR_INVALID_ARG, "node_token needs topk_ids%s");
+    const struct { const void* p; const char* n; } al[] = {
+        {logp, "logp"}, {topk_ids, "topk_ids"}, {parent_idx, "parent_idx"}, {node_depth, "node_depth"},
+        {node_rank, "node_rank"}, {node_token, "node_token"}, {node_score, "node_score"}, {d.status, "status"}};
+    for (const auto& x : al)
+        if (x.p && !aligned(x.p, 4))
+            return fail(GDN_ERR_INVALID_ARG, "%s is misaligned", x.n);
+    if (d.batch == 0)
+        return GDN_OK;
+    const size_t B = d.batch, N = (size_t)d.budget + 1, cand = B * d.max_depth * d.top_k * 4;
+    const Range outs[] = {{parent_idx, B * N * 4, "parent_idx"}, {node_depth, B * N * 4, "node_depth"},
+                          {node_rank, B * N * 4, "node_rank"},   {node_token, B * N * 4, "node_token"},
+                          {node_score, B * N * 4, "node_score"}};
+    const Range ins[] = {{logp, cand, "logp"}, {topk_ids, node_token ? cand : 0, "topk_ids"}, {d.status, 4, "status"}};
+    for (size_t i = 0; i < sizeof(outs) / sizeof(outs[0]); ++i) {
+        for (const auto& x : ins)
+            if (overlap(outs[i], x))
+                return fail(GDN_ERR_INVALID_ARG, "an output overlaps input %s", x.name);
+        for (size_t j = i + 1; j < sizeof(outs) / sizeof(outs[0]); ++j)
+            if (overlap(outs[i], outs[j]))
+                return fail(GDN_ERR_INVALID_ARG, "outputs overlap (%s)", outs[j].name);
+    }
+
+    gdn::BuildArgs a{};
+    a.logp = logp;
+    a.topk_ids = node_token ? topk_ids : nullptr;
+    a.parent = parent_idx;
+    a.depth = node_depth;
+    a.rank = node_rank;
+    a.token = node_token;
+    a.score = node_score;
+    a.status = d.status;
+    a.batch = d.batch;
+    a.max_depth = d.max_depth;
+    a.top_k = d.top_k;
+    a.budget = d.budget;
+    a.flags = d.flags;
+    const cudaError_t e = gdn::launch_build_tree(a, stream);
+    if (e != cudaSuccess)
+        return fail(GDN_ERR_CUDA, "build_tree launch failed: %s", cudaGetErrorString(e));
+    return GDN_OK;
 }
 
 }  // extern "C"

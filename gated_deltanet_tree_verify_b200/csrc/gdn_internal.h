@@ -104,4 +104,20 @@ cudaError_t launch_commit(const CommitArgs& a, cudaStream_t stream);
 bool chunked_supported(const VerifyArgs& a);
 cudaError_t launch_chunked(const VerifyArgs& a, cudaStream_t stream);
 
+// Best-first draft-tree construction (gdn_build_tree), checked by the host.
+struct BuildArgs {
+    const float* logp;
+    const int32_t* topk_ids;
+    int32_t* parent;
+    int32_t* depth;
+    int32_t* rank;
+    int32_t* token;
+    float* score;
+    int32_t* status;
+    int batch, max_depth, top_k, budget;
+    uint32_t flags;
+};
+
+cudaError_t launch_build_tree(const BuildArgs& a, cudaStream_t stream);
+
 }  // namespace gdn

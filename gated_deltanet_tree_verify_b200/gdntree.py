@@ -22,11 +22,13 @@ HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "gdntree.h")
 GDN_F32, GDN_F16, GDN_BF16 = 0, 1, 2
 # gdn_status
 GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_BAD_TREE, GDN_ERR_BAD_PATH, \
-    GDN_ERR_CUDA, GDN_ERR_TIMEOUT = range(7)
+    GDN_ERR_CUDA, GDN_ERR_TIMEOUT, GDN_ERR_BAD_INPUT = range(8)
 # flags
 GDN_FLAG_CHAIN, GDN_FLAG_PERSIST_LAST, GDN_FLAG_VALIDATE, GDN_FLAG_EARLY_TREE, GDN_FLAG_CHUNKED = 1, 2, 4, 8, 16
 GDN_FLAG_QK_L2NORM = 32
 GDN_MAX_TREE_NODES = 1024
+# gdn_build_desc.flags
+GDN_BUILD_CHAIN_SEED, GDN_BUILD_VALIDATE = 1, 2
 
 _TORCH_DTYPE = {GDN_F32: torch.float32, GDN_F16: torch.float16, GDN_BF16: torch.bfloat16}
 _GDN_DTYPE = {torch.float32: GDN_F32, torch.float16: GDN_F16, torch.bfloat16: GDN_BF16}
@@ -43,6 +45,17 @@ class GdnTreeDesc(ctypes.Structure):
         ("scale", ctypes.c_float),
         ("qkv_dtype", ctypes.c_int32),
         ("state_dtype", ctypes.c_int32),
+        ("flags", ctypes.c_uint32),
+        ("status", ctypes.c_void_p),
+    ]
+
+
+class GdnBuildDesc(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32),
+        ("max_depth", ctypes.c_int32),
+        ("top_k", ctypes.c_int32),
+        ("budget", ctypes.c_int32),
         ("flags", ctypes.c_uint32),
         ("status", ctypes.c_void_p),
     ]
@@ -92,6 +105,8 @@ def load_library() -> ctypes.CDLL:
     lib.gdn_tree_commit_layers.argtypes = [dp, i32, ctypes.POINTER(vp), vp, vp, vp, i32,
                                            ctypes.POINTER(vp), vp]
     lib.gdn_tree_commit_layers.restype = ctypes.c_int
+    lib.gdn_build_tree.argtypes = [ctypes.POINTER(GdnBuildDesc)] + [vp] * 8
+    lib.gdn_build_tree.restype = ctypes.c_int
     lib.gdn_status_str.argtypes = [ctypes.c_int]
     lib.gdn_status_str.restype = ctypes.c_char_p
     lib.gdn_last_error_detail.argtypes = []
@@ -123,6 +138,14 @@ def make_desc(*, batch: int, n_nodes: int, n_k_heads: int, n_v_heads: int, d_k: 
     d.batch, d.n_nodes, d.n_k_heads, d.n_v_heads = batch, n_nodes, n_k_heads, n_v_heads
     d.d_k, d.d_v, d.scale = d_k, d_v, float(scale)
     d.qkv_dtype, d.state_dtype, d.flags = int(qkv_dtype), int(state_dtype), int(flags)
+    d.status = _ptr(status, "status") if status is not None else None
+    return d
+
+
+def make_build_desc(*, batch: int, max_depth: int, top_k: int, budget: int, flags: int = 0,
+                    status: Optional[torch.Tensor] = None) -> GdnBuildDesc:
+    d = GdnBuildDesc()
+    d.batch, d.max_depth, d.top_k, d.budget, d.flags = batch, max_depth, top_k, budget, int(flags)
     d.status = _ptr(status, "status") if status is not None else None
     return d
 
@@ -271,4 +294,15 @@ def gdn_tree_commit_varlen(desc: GdnTreeDesc, cu_nodes, total_nodes: int, node_s
     rc = lib.gdn_tree_commit_varlen(ctypes.byref(desc), _ptr(cu_nodes, "cu_nodes"), int(total_nodes), n, ns,
                                     _ptr(parent_idx, "parent_idx"), _ptr(accept_path, "accept_path"),
                                     _ptr(accept_len, "accept_len"), int(max_path_len), so, _stream(stream))
+    return _check(rc, check)
+
+
+def gdn_build_tree(desc: GdnBuildDesc, logp, parent_idx, topk_ids=None, node_depth=None, node_rank=None,
+                   node_token=None, node_score=None, stream=None, check: bool = True) -> int:
+    """Calls gdn_build_tree (see include/gdntree.h)."""
+    lib = load_library()
+    rc = lib.gdn_build_tree(ctypes.byref(desc), _ptr(logp, "logp"), _ptr(topk_ids, "topk_ids"),
+                            _ptr(parent_idx, "parent_idx"), _ptr(node_depth, "node_depth"),
+                            _ptr(node_rank, "node_rank"), _ptr(node_token, "node_token"),
+                            _ptr(node_score, "node_score"), _stream(stream))
     return _check(rc, check)

@@ -62,8 +62,10 @@ typedef enum {
     GDN_ERR_BAD_TREE = 3,     /* device-detected: parent[0] != -1 or parent[n] not in [0, n) */
     GDN_ERR_BAD_PATH = 4,     /* device-detected: accept path/length violates the tree */
     GDN_ERR_CUDA = 5,         /* a CUDA call failed; gdn_last_error_detail() says which */
-    GDN_ERR_TIMEOUT = 6       /* device-detected internal error: a bounded wait on an
+    GDN_ERR_TIMEOUT = 6,      /* device-detected internal error: a bounded wait on an
                                  on-chip barrier ran out and the kernel stopped early */
+    GDN_ERR_BAD_INPUT = 7     /* device-detected: input values break the call's contract
+                                 (gdn_build_tree with GDN_BUILD_VALIDATE) */
 } gdn_status;
 
 /* desc->flags bits. */
@@ -304,6 +306,65 @@ gdn_status gdn_tree_commit_varlen(const gdn_tree_desc* desc, const int32_t* cu_n
 
 /* Largest N the tree (non-chain) path takes. */
 #define GDN_MAX_TREE_NODES 1024
+
+/* gdn_build_desc.flags bits. */
+enum {
+    /* Take the greedy chain (rank 0 at every position, min(max_depth, budget)
+     * nodes) first, then fill the rest of the budget best-first (the chain
+     * pre-seed of build_ddtree, the GreenGames post, "From autoregressive to
+     * DDTree"). */
+    GDN_BUILD_CHAIN_SEED = 1,
+    /* Check on the device that every logp row is non-increasing and holds no
+     * NaN or +inf; a sequence that fails gets GDN_ERR_BAD_INPUT through
+     * status and none of its outputs are written. */
+    GDN_BUILD_VALIDATE = 2
+};
+
+/* Problem description of gdn_build_tree. */
+typedef struct gdn_build_desc {
+    int32_t batch;      /* B >= 0 sequences (0: the call does nothing) */
+    int32_t max_depth;  /* D, draft positions: 1..255 */
+    int32_t top_k;      /* K, candidates per position: 1..255; D * K <= 4096 */
+    int32_t budget;     /* drafts per tree, 0..GDN_MAX_TREE_NODES - 1 and at most
+                           the K + K^2 + .. + K^D nodes the candidates span;
+                           the tree has N = budget + 1 nodes */
+    uint32_t flags;     /* GDN_BUILD_* bits */
+    int32_t* status;    /* optional DEVICE int32, as gdn_tree_desc.status */
+} gdn_build_desc;
+
+/*
+ * gdn_build_tree -- best-first draft tree from the drafter's top-k candidates
+ * (build_ddtree, the GreenGames post, "From autoregressive to DDTree"; rank 0
+ * is each position's best candidate, "Key wins").
+ *
+ * A node is a sequence of ranks (r_1 .. r_d), d <= D; node 0 is the root
+ * (d = 0, score 0).  Its score is the float32 sum, accumulated from the root
+ * (score(child) = score(parent) + logp[d - 1][r_d], rounded to nearest), and
+ * the budget nodes taken are picked one at a time among the children of the
+ * nodes taken so far: highest score first, then lower depth, lower rank,
+ * lower parent index.  Each taken node gets the next index, so the output is
+ * a tree in the layout gdn_tree_verify reads (parent[0] = -1, parent[n] < n).
+ *
+ *   logp        [B][D][K] f32, each row non-increasing (rank 0 best), no NaN;
+ *               -inf allowed.  Read-only.
+ *   topk_ids    [B][D][K] int32 token ids of the candidates, or NULL
+ *   parent_idx  [B][N] int32 out
+ *   node_depth  [B][N] int32 out, d (0 for the root), or NULL
+ *   node_rank   [B][N] int32 out, r_d (0 for the root), or NULL
+ *   node_token  [B][N] int32 out, topk_ids[b][d - 1][r_d] (-1 for the root),
+ *               or NULL; needs topk_ids
+ *   node_score  [B][N] f32 out, the node's score, or NULL
+ *
+ * One warp per tree; all pointers 4-byte aligned device memory; outputs must
+ * not overlap each other or the inputs.  Errors: GDN_ERR_INVALID_ARG /
+ * GDN_ERR_UNSUPPORTED / GDN_ERR_CUDA from the host (nothing launched);
+ * GDN_ERR_BAD_INPUT through desc->status (GDN_BUILD_VALIDATE).  Rows that are
+ * not non-increasing without GDN_BUILD_VALIDATE give a valid tree that may
+ * differ from the rule above.
+ */
+gdn_status gdn_build_tree(const gdn_build_desc* desc, const float* logp, const int32_t* topk_ids,
+                          int32_t* parent_idx, int32_t* node_depth, int32_t* node_rank, int32_t* node_token,
+                          float* node_score, cudaStream_t stream);
 
 /* Bytes of node_states for a desc (B * N * H_v * d_v * d_k * element size, or
  * N replaced by 1 with GDN_FLAG_PERSIST_LAST); 0 for an invalid desc. */

@@ -26,7 +26,7 @@ def test_exports_every_declared_function(lib):
 def test_status_strings(lib):
     for code, name in [(0, "GDN_OK"), (1, "GDN_ERR_INVALID_ARG"), (2, "GDN_ERR_UNSUPPORTED"),
                        (3, "GDN_ERR_BAD_TREE"), (4, "GDN_ERR_BAD_PATH"), (5, "GDN_ERR_CUDA"),
-                       (6, "GDN_ERR_TIMEOUT")]:
+                       (6, "GDN_ERR_TIMEOUT"), (7, "GDN_ERR_BAD_INPUT")]:
         assert gdn.gdn_status_str(code) == name
     assert gdn.gdn_status_str(99) == "GDN_ERR_UNKNOWN"
 
@@ -225,3 +225,36 @@ def test_varlen_host_checks(lib):
     rc = gdn.gdn_tree_commit_varlen(d, None, 10, [ns], par, BASE + 31 * MB, BASE + 32 * MB, 4, [out],
                                     stream=0, check=False)
     assert rc == gdn.GDN_ERR_INVALID_ARG
+
+
+def test_build_desc_struct_layout():
+    # int32 x 4, uint32, padding, pointer
+    assert ctypes.sizeof(gdn.GdnBuildDesc) == 32
+    assert gdn.GdnBuildDesc.status.offset == 24
+
+
+def test_build_tree_host_checks(lib):
+    lp, ids, par, dep, rk, tok, sc = (BASE + i * MB for i in range(7))
+
+    def call(check_lp=lp, check_par=par, ids_=None, tok_=None, dep_=None, **kw):
+        base = dict(batch=2, max_depth=16, top_k=8, budget=22, flags=0)
+        base.update(kw)
+        d = gdn.make_build_desc(**base)
+        return gdn.gdn_build_tree(d, check_lp, check_par, topk_ids=ids_, node_depth=dep_, node_token=tok_,
+                                  stream=0, check=False)
+    assert call(batch=0) == gdn.GDN_OK
+    assert call(batch=0, budget=23, max_depth=2, top_k=2) == gdn.GDN_ERR_INVALID_ARG   # 2 + 4 = 6 candidates
+    assert call(batch=0, budget=6, max_depth=2, top_k=2) == gdn.GDN_OK
+    assert call(flags=4) == gdn.GDN_ERR_INVALID_ARG
+    assert call(max_depth=0) == gdn.GDN_ERR_INVALID_ARG
+    assert call(budget=-1) == gdn.GDN_ERR_INVALID_ARG
+    assert call(max_depth=256) == gdn.GDN_ERR_UNSUPPORTED
+    assert call(max_depth=128, top_k=64) == gdn.GDN_ERR_UNSUPPORTED              # D * K above 4096
+    assert call(budget=1024) == gdn.GDN_ERR_UNSUPPORTED
+    assert call(check_lp=None) == gdn.GDN_ERR_INVALID_ARG
+    assert call(check_par=None) == gdn.GDN_ERR_INVALID_ARG
+    assert call(tok_=tok) == gdn.GDN_ERR_INVALID_ARG                             # tokens need topk_ids
+    assert call(check_par=par + 2) == gdn.GDN_ERR_INVALID_ARG                     # misaligned
+    assert call(dep_=par + 4) == gdn.GDN_ERR_INVALID_ARG                          # outputs overlap
+    assert call(check_par=lp + 64) == gdn.GDN_ERR_INVALID_ARG                     # output inside logp
+    assert call(ids_=ids, tok_=ids + 4) == gdn.GDN_ERR_INVALID_ARG                # output inside topk_ids
