@@ -115,10 +115,12 @@ def hbm_peak():
 
 
 def kernel_source_digest():
+    """Digest of the sources the verify kernels are built from (the tree
+    builder, chunked chain and commit kernels live in files of their own)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gated_deltanet_tree_verify_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
+        if name.startswith("gdn_verify") or name in ("gdn_device.cuh", "gdn_internal.h"):
             with open(os.path.join(csrc, name), "rb") as f:
                 h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
@@ -190,6 +192,15 @@ class ClockSampler:
         self._stop.set()
         if self.ok:
             self._t.join()
+
+    def now(self):
+        """One SM clock reading (MHz), or None."""
+        if not self.ok:
+            return None
+        try:
+            return self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM)
+        except Exception:
+            return None
 
     def summary(self):
         if not self.ok or not self.samples:
@@ -694,50 +705,57 @@ def run_sweep(args):
         keep = set(args.sweep_kinds.split(","))
         points = [pt for pt in points if pt["kind"] in keep]
     varlen_budgets = [8, 64, 22, 15, 32, 22, 48, 8]
-    for pt in points:
-        if pt["kind"] == "build":
-            t, ok, cpu = _build_point(batch=pt["batch"], budget=pt["budget"])
-            print(json.dumps({"sweep": "build_tree", "budget": pt["budget"], "batch": pt["batch"],
-                              "max_depth": 16, "top_k": 8, "build_us": t * 1e6, "trees_per_s": pt["batch"] / t,
-                              "ns_per_pop": t * 1e9 / pt["budget"], "matches_oracle": ok,
-                              "oracle_us_per_tree": cpu * 1e6}), flush=True)
-            continue
-        n = pt["budget"] + 1
-        if pt["kind"] == "varlen":
-            t, vb, T = _varlen_point(budgets=varlen_budgets, state_dtype=pt["state_dtype"], workspace=pt["ws"])
-            print(json.dumps({"sweep": "varlen", "budgets": varlen_budgets, "state_dtype": pt["state_dtype"],
-                              "workspace": pt["ws"], "verify_us": t * 1e6, "node_layers_per_s": T / t,
-                              "gbps": vb / t / 1e9, "frac_of_hbm": vb / t / 1e9 / peak}), flush=True)
-            continue
-        if pt["kind"] == "chain4096":
-            flags = gdn.GDN_FLAG_CHAIN | gdn.GDN_FLAG_PERSIST_LAST
-            if pt.get("chunked"):
-                flags |= gdn.GDN_FLAG_CHUNKED
-            t, R = _verify_point(batch=pt["batch"], n_nodes=n, tree="chain", state_dtype="f32", flags=flags,
-                                 gate="uniform_a", reps=3, min_bytes=0)
-            tokens = pt["batch"] * n
-            io = tokens * (45444 - 4) + 2 * pt["batch"] * N_V_HEADS * D * D * 4
-            flops = tokens * N_V_HEADS * D * D * 7.0  # dot S k, a S, u k^T, S q: 7 flops per element
-            clock = args.sm_mhz * 1e6
-            alu_peak = 148 * FP32_LANES_PER_SM * 2 * clock / 1e12
-            line = {"sweep": "chain4096_persist_last" + ("_chunked" if pt.get("chunked") else ""),
-                    "batch": pt["batch"], "tokens": n,
-                    "state_dtype": "f32", "verify_ms": t * 1e3, "tokens_per_s": tokens / t,
-                    "roofline": {"bound": "alu", "achieved": flops / t / 1e12, "unit": "TFLOP/s",
-                                 "peak": alu_peak, "frac": flops / t / 1e12 / alu_peak,
-                                 "peak_source": f"148 SMs x 128 FP32 lanes x 2 x {args.sm_mhz:.0f} MHz"},
-                    "hbm_gbps": io / t / 1e9}
-        else:
-            tree = "ddtree" if pt["kind"] == "tree" else "chain"
-            flags = 0 if pt["kind"] == "tree" else gdn.GDN_FLAG_CHAIN
-            t, R = _verify_point(batch=pt["batch"], n_nodes=n, tree=tree, state_dtype=pt["state_dtype"],
-                                 flags=flags, workspace=pt.get("ws", False))
-            vb = verify_bytes(pt["batch"], n, pt["state_dtype"])
-            line = {"sweep": pt["kind"], "budget": pt["budget"], "batch": pt["batch"],
-                    "state_dtype": pt["state_dtype"], "workspace": pt.get("ws", False), "verify_us": t * 1e6,
-                    "node_layers_per_s": pt["batch"] * n / t, "gbps": vb / t / 1e9,
-                    "frac_of_hbm": vb / t / 1e9 / peak, "buffer_sets": R}
-        print(json.dumps(line), flush=True)
+    clocks = ClockSampler(0, period_s=0.01)
+    with clocks:
+        for pt in points:
+            _sweep_point(args, gdn, pt, peak, varlen_budgets, clocks)
+    print(json.dumps({"sweep": "clocks", **clocks.summary()}), flush=True)
+
+
+def _sweep_point(args, gdn, pt, peak, varlen_budgets, clocks):
+    """Times one sweep point and prints its JSON line (with the SM clock read
+    right after the timed region)."""
+    n = pt["budget"] + 1
+    if pt["kind"] == "build":
+        t, ok, cpu = _build_point(batch=pt["batch"], budget=pt["budget"])
+        line = {"sweep": "build_tree", "budget": pt["budget"], "batch": pt["batch"], "max_depth": 16, "top_k": 8,
+                "build_us": t * 1e6, "trees_per_s": pt["batch"] / t, "ns_per_pop": t * 1e9 / pt["budget"],
+                "matches_oracle": ok, "oracle_us_per_tree": cpu * 1e6}
+    elif pt["kind"] == "varlen":
+        t, vb, T = _varlen_point(budgets=varlen_budgets, state_dtype=pt["state_dtype"], workspace=pt["ws"])
+        line = {"sweep": "varlen", "budgets": varlen_budgets, "state_dtype": pt["state_dtype"],
+                "workspace": pt["ws"], "verify_us": t * 1e6, "node_layers_per_s": T / t,
+                "gbps": vb / t / 1e9, "frac_of_hbm": vb / t / 1e9 / peak}
+    elif pt["kind"] == "chain4096":
+        flags = gdn.GDN_FLAG_CHAIN | gdn.GDN_FLAG_PERSIST_LAST
+        if pt.get("chunked"):
+            flags |= gdn.GDN_FLAG_CHUNKED
+        t, R = _verify_point(batch=pt["batch"], n_nodes=n, tree="chain", state_dtype="f32", flags=flags,
+                             gate="uniform_a", reps=3, min_bytes=0)
+        tokens = pt["batch"] * n
+        io = tokens * (45444 - 4) + 2 * pt["batch"] * N_V_HEADS * D * D * 4
+        flops = tokens * N_V_HEADS * D * D * 7.0  # dot S k, a S, u k^T, S q: 7 flops per element
+        clock = args.sm_mhz * 1e6
+        alu_peak = 148 * FP32_LANES_PER_SM * 2 * clock / 1e12
+        line = {"sweep": "chain4096_persist_last" + ("_chunked" if pt.get("chunked") else ""),
+                "batch": pt["batch"], "tokens": n,
+                "state_dtype": "f32", "verify_ms": t * 1e3, "tokens_per_s": tokens / t,
+                "roofline": {"bound": "alu", "achieved": flops / t / 1e12, "unit": "TFLOP/s",
+                             "peak": alu_peak, "frac": flops / t / 1e12 / alu_peak,
+                             "peak_source": f"148 SMs x 128 FP32 lanes x 2 x {args.sm_mhz:.0f} MHz"},
+                "hbm_gbps": io / t / 1e9}
+    else:
+        tree = "ddtree" if pt["kind"] == "tree" else "chain"
+        flags = 0 if pt["kind"] == "tree" else gdn.GDN_FLAG_CHAIN
+        t, R = _verify_point(batch=pt["batch"], n_nodes=n, tree=tree, state_dtype=pt["state_dtype"],
+                             flags=flags, workspace=pt.get("ws", False))
+        vb = verify_bytes(pt["batch"], n, pt["state_dtype"])
+        line = {"sweep": pt["kind"], "budget": pt["budget"], "batch": pt["batch"],
+                "state_dtype": pt["state_dtype"], "workspace": pt.get("ws", False), "verify_us": t * 1e6,
+                "node_layers_per_s": pt["batch"] * n / t, "gbps": vb / t / 1e9,
+                "frac_of_hbm": vb / t / 1e9 / peak, "buffer_sets": R}
+    line["sm_mhz_after"] = clocks.now()
+    print(json.dumps(line), flush=True)
 
 
 def main(argv=None):

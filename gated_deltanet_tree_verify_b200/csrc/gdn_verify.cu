@@ -97,13 +97,15 @@ VerifyGeom verify_geometry(const VerifyArgs& a, bool use_workspace)
             off_desc = off;
             off += (size_t)a.n_nodes * sizeof(PosDesc);
             off_ab = off;
-            off += align16((size_t)3 * a.n_nodes * 4);  // g (then a) | beta | a', by node
+            // g (then a) | beta', by node; with q/k normalisation also a' and
+            // the output coefficient
+            off += align16((size_t)((a.flags & GDN_FLAG_QK_L2NORM) ? 4 : 2) * a.n_nodes * 4);
         } else {
             off_ab = off;  // 1 / |k| by node (GDN_FLAG_QK_L2NORM trees)
             if ((a.flags & GDN_FLAG_QK_L2NORM) && !chain && !g.reload)
                 off += align16((size_t)a.n_nodes * 4);
             off_raw = off;
-            off += (size_t)kRing * (align16(kChunk * raw_bytes) + kChunk * sizeof(PosDesc));
+            off += (size_t)kRing * (align16(kChunk * raw_bytes) + kChunk * (sizeof(PosDesc) + 4));
         }
         off_slots = off;
         off += align16(slot_bytes);

@@ -140,10 +140,12 @@ __device__ __forceinline__ bool seq_of(const KParams& p, int b, Seq& q)
 }
 
 // One walk position: its node and tree metadata, and the node's scalars.
+// With qk_norm, each position (ring) or node (staged) also has an output
+// coefficient scale / |q|, kept beside the descriptors so that they stay 32
+// bytes.
 struct PosDesc {
     int4 i;    // node, metadata, recomputation start, parent
     float4 f;  // a = exp(g), beta', k . q, a' (see node_scalars)
-    float4 x;  // output coefficient scale / |q| (read only with qk_norm), unused
 };
 
 // A node's scalars for the state step.  With q and k normalised inside the
@@ -299,6 +301,11 @@ __device__ __forceinline__ float rec_elem(const float* rec, int part, int e)
 // a warp handles four nodes at once; every lane of the warp must call it).
 // The same reduction wherever it is computed.
 template <int DK, int LR, typename RT>
+__device__ __forceinline__ float node_kq8(const RT* rec, int sub);
+
+// x . y of two rows of one node's record (part 0: k, part DK: q), reduced
+// by a group of 8 lanes like node_kq8.
+template <int DK, int LR, typename RT>
 __device__ __forceinline__ float node_dot8(const RT* rec, int sub, int pa, int pb)
 {
     float acc0 = 0.f, acc1 = 0.f;
@@ -312,6 +319,36 @@ __device__ __forceinline__ float node_dot8(const RT* rec, int sub, int pa, int p
     for (int off = 4; off >= 1; off >>= 1)
         acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, off));
     return acc;
+}
+
+// k . q, k . k and q . q of one node's record in one pass, each summed in
+// exactly node_kq8's order (so kq is bit-identical to it).  Not unrolled: it
+// runs in prologues only with GDN_FLAG_QK_L2NORM, and unrolled it would set
+// the register count of the whole kernel.
+template <int DK, int LR, typename RT>
+__device__ __forceinline__ void node_dots8(const RT* rec, int sub, float& kq, float& kk, float& qq)
+{
+    float q0 = 0.f, q1 = 0.f, k0 = 0.f, k1 = 0.f, s0 = 0.f, s1 = 0.f;
+#pragma unroll 1
+    for (int j = sub; j < DK; j += 16) {
+        const float ka = rec_elem<DK, LR>(rec, 0, j), qa = rec_elem<DK, LR>(rec, DK, j);
+        const float kb = rec_elem<DK, LR>(rec, 0, j + 8), qb = rec_elem<DK, LR>(rec, DK, j + 8);
+        q0 = __fmaf_rn(ka, qa, q0);
+        q1 = __fmaf_rn(kb, qb, q1);
+        k0 = __fmaf_rn(ka, ka, k0);
+        k1 = __fmaf_rn(kb, kb, k1);
+        s0 = __fmaf_rn(qa, qa, s0);
+        s1 = __fmaf_rn(qb, qb, s1);
+    }
+    kq = __fadd_rn(q0, q1);
+    kk = __fadd_rn(k0, k1);
+    qq = __fadd_rn(s0, s1);
+#pragma unroll
+    for (int off = 4; off >= 1; off >>= 1) {
+        kq = __fadd_rn(kq, __shfl_xor_sync(0xffffffffu, kq, off));
+        kk = __fadd_rn(kk, __shfl_xor_sync(0xffffffffu, kk, off));
+        qq = __fadd_rn(qq, __shfl_xor_sync(0xffffffffu, qq, off));
+    }
 }
 
 template <int DK, int LR, typename RT>
@@ -973,7 +1010,7 @@ __device__ __forceinline__ void walk(StateT<C, RL>& S, const KParams& p, const S
         float pq[RL], u[RL];
         gdn_step<LM::LR, C, RL, true>(S, k2, q2, vr, a, d.f.w, d.f.y, pq, u);
         if (L.cl == 0) {
-            const float oc = p.qk_norm ? ctx.out_coef(pos) : p.scale;
+            const float oc = p.qk_norm ? ctx.out_coef(pos, n) : p.scale;
             float* o = out_lane + (size_t)n * out_stride;
 #pragma unroll
             for (int r = 0; r < RL; ++r)
@@ -1012,9 +1049,10 @@ struct NoTree {
 template <int DK, int C, int RL, typename RT>
 struct StagedFetch {
     const RT* recs;
-    const float* ab;  // a | beta, by node
+    const float* ab;  // a | beta' (| a' | output coefficient with qk_norm), by node
     uint32_t rec_elems;
     int N;
+    int qk_norm;
     LaneMap<DK, C, RL> L;
     __device__ __forceinline__ void operator()(int y, float2 (&k2)[4 * C], float (&vr)[RL], float& a,
                                                float& ar, float& be) const
@@ -1022,7 +1060,7 @@ struct StagedFetch {
         load_k<DK, C, RL, RT>(recs + (size_t)y * rec_elems, L, k2, vr);
         a = ab[y];
         be = ab[N + y];
-        ar = ab[2 * N + y];
+        ar = qk_norm ? ab[2 * N + y] : a;
     }
 };
 
@@ -1033,17 +1071,18 @@ struct StagedCtx {
     const float* ab;
     uint32_t rec_elems;
     int N;
+    int qk_norm;
     LaneMap<DK, C, RL> L;
     __device__ __forceinline__ bool begin(int) { return true; }
     __device__ __forceinline__ void end(int) {}
     // whether position pos's descriptor may be read before begin(pos)
     __device__ __forceinline__ bool ahead(int) const { return true; }
     __device__ __forceinline__ PosDesc desc(int pos) const { return desc_[pos]; }
-    __device__ __forceinline__ float out_coef(int pos) const { return desc_[pos].x.x; }
+    __device__ __forceinline__ float out_coef(int, int n) const { return ab[3 * N + n]; }
     __device__ __forceinline__ const RT* rec(int, int n) const { return recs + (size_t)n * rec_elems; }
     __device__ __forceinline__ StagedFetch<DK, C, RL, RT> fetcher() const
     {
-        return StagedFetch<DK, C, RL, RT>{recs, ab, rec_elems, N, L};
+        return StagedFetch<DK, C, RL, RT>{recs, ab, rec_elems, N, qk_norm, L};
     }
 };
 
@@ -1072,9 +1111,9 @@ __device__ __forceinline__ float* cta_slots(const KParams& p, float* slotbuf)
 }
 
 // Prologue pass of the staged kernel over walk positions, four per warp and
-// pass (8 lanes each): turns ab (g | beta | -, by node) into a | beta' | a'
-// (node_scalars) and writes each position's descriptor with k . q of its
-// node (and, with qk_norm, the output coefficient).
+// pass (8 lanes each): turns ab (g | beta, by node) into a | beta'
+// (node_scalars; with qk_norm also a' and the output coefficient, by node)
+// and writes each position's descriptor with k . q of its node.
 template <int DK, int LR, typename QT, class Tree>
 __device__ __forceinline__ void write_descs(const Tree& tree, const unsigned char* raw, uint32_t raw_bytes,
                                             float* ab, PosDesc* desc, int N, int qk_norm, float scale)
@@ -1099,11 +1138,13 @@ __device__ __forceinline__ void write_descs(const Tree& tree, const unsigned cha
             node_scalars(a, ab[N + n], rk, bp, ap);
             ab[n] = a;
             ab[N + n] = bp;
-            ab[2 * N + n] = ap;
+            if (qk_norm) {
+                ab[2 * N + n] = ap;
+                ab[3 * N + n] = __fmul_rn(scale, rq);
+            }
             PosDesc d;
             d.i = make_int4(n, m, tree.rstart(pos), tree.parent(n));
             d.f = make_float4(a, bp, kq, ap);
-            d.x = make_float4(__fmul_rn(scale, rq), 0.f, 0.f, 0.f);
             desc[pos] = d;
         }
     }
@@ -1119,13 +1160,13 @@ __device__ __forceinline__ void staged_finish(StateT<C, RL>& S, const KParams& p
     write_descs<DK, LR, QT>(tree, raw, p.raw_bytes, ab, desc, sq.N, p.qk_norm, p.scale);
     __syncthreads();
     const uint32_t rec_elems = p.raw_bytes / (uint32_t)sizeof(QT);
-    StagedCtx<DK, C, RL, QT> ctx{reinterpret_cast<const QT*>(raw), desc, ab, rec_elems, sq.N, L};
+    StagedCtx<DK, C, RL, QT> ctx{reinterpret_cast<const QT*>(raw), desc, ab, rec_elems, sq.N, p.qk_norm, L};
     float* lane_slot = cta_slots<DK, TREE>(p, slotbuf) + 4 * threadIdx.x;
     walk<DK, C, RL, QT, ST, TREE>(S, p, sq, tree, lane_slot, sin_lane, b, h, row0, L, ctx);
 }
 
 template <int DK, int C, int RL, typename QT, typename ST, int TREE>
-__global__ void __launch_bounds__(kMaxWarps * 32) gdn_verify_staged(const KParams p)
+__device__ __forceinline__ void staged_body(const KParams& p)
 {
     constexpr int EPC = 16 / sizeof(QT);  // elements per 16-byte chunk
     constexpr int QKCH = DK / EPC;        // chunks per k (or q) row
@@ -1255,6 +1296,21 @@ __global__ void __launch_bounds__(kMaxWarps * 32) gdn_verify_staged(const KParam
                                                sin_lane, b, h, row0, L);
 }
 
+template <int DK, int C, int RL, typename QT, typename ST, int TREE>
+__global__ void __launch_bounds__(kMaxWarps * 32) gdn_verify_staged(const KParams p)
+{
+    staged_body<DK, C, RL, QT, ST, TREE>(p);
+}
+
+// Small trees walked from warp registers with one row per lane (small
+// grids), bf16 inputs: at most 80 registers, so that six CTAs fit on an SM
+// and the next layer's CTAs become resident while this layer's still run.
+template <int DK, int C, int RL, typename QT, typename ST, int TREE>
+__global__ void __launch_bounds__(kMaxWarps * 32, 6) gdn_verify_staged_dense(const KParams p)
+{
+    staged_body<DK, C, RL, QT, ST, TREE>(p);
+}
+
 // ---------------------------------------------------------------------------
 // Ring kernel: a producer warp streams chunks of walk positions
 // ---------------------------------------------------------------------------
@@ -1333,9 +1389,9 @@ struct RingCtx {
     }
     // only within the chunk already waited for
     __device__ __forceinline__ bool ahead(int pos) const { return pos % kChunk != 0; }
-    __device__ __forceinline__ float out_coef(int pos) const
+    __device__ __forceinline__ float out_coef(int pos, int) const
     {
-        return reinterpret_cast<const PosDesc*>(slot(pos) + desc_off)[pos % kChunk].x.x;
+        return reinterpret_cast<const float*>(slot(pos) + desc_off + kChunk * sizeof(PosDesc))[pos % kChunk];
     }
     __device__ __forceinline__ const QT* rec(int pos, int) const
     {
@@ -1360,7 +1416,7 @@ __global__ void __launch_bounds__((kMaxWarps + 1) * 32) gdn_verify_ring(const KP
     uint64_t* empty = full + kRing;
     unsigned char* ring = smem + p.off_raw;
     const uint32_t desc_off = (kChunk * p.raw_bytes + 15u) & ~15u;
-    const uint32_t slot_bytes = desc_off + kChunk * (uint32_t)sizeof(PosDesc);
+    const uint32_t slot_bytes = desc_off + kChunk * (uint32_t)(sizeof(PosDesc) + 4);
     float* slotbuf = reinterpret_cast<float*>(smem + p.off_slots);
     const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int hk = h / p.G;
@@ -1492,11 +1548,14 @@ __global__ void __launch_bounds__((kMaxWarps + 1) * 32) gdn_verify_ring(const KP
                 const int gi = i0 + (lane >> 3);
                 const int i = min(gi, cnt - 1);
                 const QT* rrec = reinterpret_cast<const QT*>(base + (size_t)i * p.raw_bytes);
-                const float kq = node_kq8<DK, LM::LR>(rrec, lane & 7);
-                float rk = 1.f, rq = 1.f;
+                float kq, rk = 1.f, rq = 1.f;
                 if (p.qk_norm) {
-                    rk = inv_norm(node_dot8<DK, LM::LR>(rrec, lane & 7, 0, 0));
-                    rq = inv_norm(node_dot8<DK, LM::LR>(rrec, lane & 7, DK, DK));
+                    float kk, qq;
+                    node_dots8<DK, LM::LR>(rrec, lane & 7, kq, kk, qq);
+                    rk = inv_norm(kk);
+                    rq = inv_norm(qq);
+                } else {
+                    kq = node_kq8<DK, LM::LR>(rrec, lane & 7);
                 }
                 const int src_lane = i;
                 const int n = __shfl_sync(0xffffffffu, dn, src_lane);
@@ -1511,8 +1570,8 @@ __global__ void __launch_bounds__((kMaxWarps + 1) * 32) gdn_verify_ring(const KP
                     PosDesc d;
                     d.i = make_int4(n, m, rs, pp);
                     d.f = make_float4(a, bp, kq, ap);
-                    d.x = make_float4(__fmul_rn(p.scale, rq), 0.f, 0.f, 0.f);
                     sdesc[i] = d;
+                    reinterpret_cast<float*>(sdesc + kChunk)[i] = __fmul_rn(p.scale, rq);
                     if (rkn != nullptr)
                         rkn[n] = rk;  // for recomputation of this node's subtree
                 }
@@ -1568,16 +1627,24 @@ cudaError_t grant_smem(size_t smem)
     return cudaSuccess;
 }
 
+template <auto KERNEL>
+cudaError_t launch_granted(const KParams& kp, dim3 grid, const VerifyGeom& geom, cudaStream_t stream)
+{
+    cudaError_t e = grant_smem<KERNEL>(geom.smem);
+    if (e != cudaSuccess)
+        return e;
+    return launch_pdl(KERNEL, grid, dim3(geom.warps * 32), geom.smem, stream, kp);
+}
+
 template <int DK, int C, int RL, typename QT, typename ST, int TREE>
 cudaError_t launch_staged(const KParams& kp, const VerifyArgs& a, const VerifyGeom& geom,
                           cudaStream_t stream)
 {
     dim3 grid(geom.tiles, a.n_v_heads, a.batch);
-    cudaError_t e = grant_smem<gdn_verify_staged<DK, C, RL, QT, ST, TREE>>(geom.smem);
-    if (e != cudaSuccess)
-        return e;
-    return launch_pdl(gdn_verify_staged<DK, C, RL, QT, ST, TREE>, grid, dim3(geom.warps * 32), geom.smem,
-                      stream, kp);
+    if constexpr (TREE == kTreeWarp && RL == 1 && sizeof(QT) == 2)
+        return launch_granted<gdn_verify_staged_dense<DK, C, RL, QT, ST, TREE>>(kp, grid, geom, stream);
+    else
+        return launch_granted<gdn_verify_staged<DK, C, RL, QT, ST, TREE>>(kp, grid, geom, stream);
 }
 
 template <int DK, int C, int RL, typename QT, typename ST, int TREE>
