@@ -30,6 +30,12 @@ size_t align16(size_t x) { return (x + 15) & ~size_t(15); }
 // lane (twice the warps, to hide the per-node dependency chain).
 constexpr long long kWarpsPerSmTarget = 16;
 constexpr long long kSms = 148;
+// Large grids (two rows per lane): shared-memory stack slots per CTA for
+// trees of <= 32, <= 96 and more nodes, and the warps per CTA of trees with
+// shared-memory slots above 32 nodes (the node records are staged once per
+// CTA, so wider CTAs spend less shared memory per row).
+constexpr int kLargeGridSlots[3] = {1, 2, 3};
+constexpr int kLargeTreeWarps = 8;
 
 template <int DK>
 cudaError_t launch_shapes(const verify::KParams& kp, const VerifyArgs& a, const VerifyGeom& g,
@@ -73,15 +79,18 @@ VerifyGeom verify_geometry(const VerifyArgs& a, bool use_workspace)
         while ((2 << k) <= a.n_nodes)
             ++k;
         g.gslots = use_workspace;
-        const int cap = g.gslots ? 4
-                                 : (a.n_nodes <= 32 ? (g.rows_per_lane == 2 ? 1 : 2) : (a.n_nodes <= 96 ? 3 : 4));
+        const int size_class = a.n_nodes <= 32 ? 0 : (a.n_nodes <= 96 ? 1 : 2);
+        const int cap = g.gslots ? 4 : (g.rows_per_lane == 2 ? kLargeGridSlots[size_class] : 2 + size_class);
         g.slots = k < 1 ? 1 : (k > cap ? cap : k);
     }
     const int rpw = rows_per_warp(g.chunks, g.rows_per_lane);
-    // Staged kernel first, else the ring kernel (which adds a producer warp).
-    for (int pass = 0; pass < 2; ++pass) {
-        const bool staged = pass == 0;
-        int warps = kMaxWarps;
+    // Staged kernel first (wide CTAs for large trees with shared-memory
+    // slots on large grids, then the usual width), else the ring kernel
+    // (which adds a producer warp).
+    const bool wide = !chain && !g.reload && !g.gslots && a.n_nodes > 32 && g.rows_per_lane == 2;
+    for (int pass = wide ? 0 : 1; pass < 3; ++pass) {
+        const bool staged = pass < 2;
+        int warps = pass == 0 ? kLargeTreeWarps : kSmallWarps;  // the ring kernel: kSmallWarps at most
         while (warps > 1 && a.d_v % (warps * rpw) != 0)
             --warps;
         const int rows = warps * rpw;

@@ -76,11 +76,12 @@
 namespace gdn {
 namespace verify {
 
-constexpr int kMaxWarps = 4;  // compute warps per CTA
+constexpr int kMaxWarps = 8;    // compute warps per CTA, at most
+constexpr int kSmallWarps = 4;  // compute warps per CTA, usually
 constexpr int kChunk = 8;     // walk positions per ring slot
 constexpr int kRing = 3;      // ring slots
 constexpr int kMaxDevices = 64;
-constexpr int kStagedMaxSmem = 100 * 1024;
+constexpr int kStagedMaxSmem = 112 * 1024;
 
 // Per-position walk metadata (tree mode), packed in one int32:
 //   bits 0..15 node id, 16..18 source of the parent state,
@@ -1297,7 +1298,15 @@ __device__ __forceinline__ void staged_body(const KParams& p)
 }
 
 template <int DK, int C, int RL, typename QT, typename ST, int TREE>
-__global__ void __launch_bounds__(kMaxWarps * 32) gdn_verify_staged(const KParams p)
+__global__ void __launch_bounds__(kSmallWarps * 32) gdn_verify_staged(const KParams p)
+{
+    staged_body<DK, C, RL, QT, ST, TREE>(p);
+}
+
+// Trees of more than 32 nodes with shared-memory slots on large grids:
+// kMaxWarps warps share one copy of the node records.
+template <int DK, int C, int RL, typename QT, typename ST, int TREE>
+__global__ void __launch_bounds__(kMaxWarps * 32) gdn_verify_staged_wide(const KParams p)
 {
     staged_body<DK, C, RL, QT, ST, TREE>(p);
 }
@@ -1306,7 +1315,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32) gdn_verify_staged(const KParam
 // grids), bf16 inputs: at most 80 registers, so that six CTAs fit on an SM
 // and the next layer's CTAs become resident while this layer's still run.
 template <int DK, int C, int RL, typename QT, typename ST, int TREE>
-__global__ void __launch_bounds__(kMaxWarps * 32, 6) gdn_verify_staged_dense(const KParams p)
+__global__ void __launch_bounds__(kSmallWarps * 32, 6) gdn_verify_staged_dense(const KParams p)
 {
     staged_body<DK, C, RL, QT, ST, TREE>(p);
 }
@@ -1401,14 +1410,14 @@ struct RingCtx {
 };
 
 template <int DK, int C, int RL, typename QT, typename ST, int TREE>
-__global__ void __launch_bounds__((kMaxWarps + 1) * 32) gdn_verify_ring(const KParams p)
+__global__ void __launch_bounds__((kSmallWarps + 1) * 32) gdn_verify_ring(const KParams p)
 {
     constexpr bool CHAIN = TREE == kTreeChain;
     constexpr bool INDEX = TREE == kTreeIndex;
     constexpr int EPC = 16 / sizeof(QT);  // elements per 16-byte chunk
     constexpr int QKCH = DK / EPC;        // chunks per k (or q) row
     using LM = LaneMap<DK, C, RL>;
-    constexpr int VCH_MAX = (kMaxWarps * LM::RPW + EPC - 1) / EPC;  // chunks per v slice, upper bound
+    constexpr int VCH_MAX = (kSmallWarps * LM::RPW + EPC - 1) / EPC;  // chunks per v slice, upper bound
     constexpr int MAXT = (kChunk * (2 * QKCH + VCH_MAX) + 31) / 32;
 
     extern __shared__ __align__(16) unsigned char smem[];
@@ -1643,8 +1652,13 @@ cudaError_t launch_staged(const KParams& kp, const VerifyArgs& a, const VerifyGe
     dim3 grid(geom.tiles, a.n_v_heads, a.batch);
     if constexpr (TREE == kTreeWarp && RL == 1 && sizeof(QT) == 2)
         return launch_granted<gdn_verify_staged_dense<DK, C, RL, QT, ST, TREE>>(kp, grid, geom, stream);
-    else
-        return launch_granted<gdn_verify_staged<DK, C, RL, QT, ST, TREE>>(kp, grid, geom, stream);
+    if constexpr (TREE == kTreeSmem && RL == 2) {
+        if (geom.warps > kSmallWarps)
+            return launch_granted<gdn_verify_staged_wide<DK, C, RL, QT, ST, TREE>>(kp, grid, geom, stream);
+    }
+    if (geom.warps > kSmallWarps)
+        return cudaErrorInvalidConfiguration;  // not reached: the geometry only widens the kinds above
+    return launch_granted<gdn_verify_staged<DK, C, RL, QT, ST, TREE>>(kp, grid, geom, stream);
 }
 
 template <int DK, int C, int RL, typename QT, typename ST, int TREE>
