@@ -128,8 +128,8 @@ VerifyGeom verify_geometry(const VerifyArgs& a, bool use_workspace)
             off += align16((size_t)a.n_nodes * 4);
         else if (warp_tree)
             off += kWarpTreeInts * 4;
-        else
-            off += (size_t)(kTreeArrays + warps) * a.n_nodes * 4;
+        else  // the arrays, then the walk's per-warp path scratch (also the mask builder's)
+            off += (size_t)(kTreeArrays + (warps > kMaskScratch ? warps : kMaskScratch)) * a.n_nodes * 4;
         if (staged && off > (size_t)kStagedMaxSmem)
             continue;
         g.staged = staged;

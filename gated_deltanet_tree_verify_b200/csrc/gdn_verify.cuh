@@ -705,6 +705,157 @@ static __device__ bool build_walk(const int32_t* prow, int N, int K, const TreeV
     return true;
 }
 
+// Trees of up to kMaskNodes nodes: the same walk as build_walk, built from
+// per-node bit masks in O(log depth) barrier rounds instead of O(depth)
+// serial chains.  Needs one thread per node and kMaskScratch ints per node
+// of scratch (T.path, which the walk only uses afterwards).
+constexpr int kMaskNodes = 128;
+constexpr int kMaskWords = kMaskNodes / 32;
+constexpr int kMaskScratch = 2 * kMaskWords;
+static __device__ bool build_walk_masked(const int32_t* prow, int N, int K, const TreeView& T)
+{
+    const int tid = threadIdx.x;
+    const bool own = tid < N;
+    unsigned* const anc = reinterpret_cast<unsigned*>(T.path);  // [N][4] ancestor-or-self masks
+    unsigned* const kids = anc + kMaskWords * N;                // [N][4] child masks
+    int pn = -1;
+    bool bad = false;
+    if (own) {
+        pn = __ldg(prow + tid);
+        T.par[tid] = pn;
+        bad = (tid == 0) ? (pn != -1) : (pn < 0 || pn >= tid);
+#pragma unroll
+        for (int w = 0; w < kMaskWords; ++w) {
+            kids[kMaskWords * tid + w] = 0u;
+            anc[kMaskWords * tid + w] = (w == (tid >> 5)) ? (1u << (tid & 31)) : 0u;
+        }
+        T.ord[tid] = pn;  // pointer-jumping target, until ord is written
+    }
+    if (__syncthreads_or(bad))
+        return false;
+    if (own && tid > 0)
+        atomicOr(&kids[kMaskWords * pn + (tid >> 5)], 1u << (tid & 31));
+    // ancestor masks: after round r, anc covers the 2^r nearest ancestors
+    unsigned m[kMaskWords];
+#pragma unroll
+    for (int w = 0; w < kMaskWords; ++w)
+        m[w] = own ? anc[kMaskWords * tid + w] : 0u;
+    int jump = pn;
+    while (__syncthreads_or(jump >= 0)) {
+        int nj = -1;
+        if (jump >= 0) {
+#pragma unroll
+            for (int w = 0; w < kMaskWords; ++w)
+                m[w] |= anc[kMaskWords * jump + w];
+            nj = T.ord[jump];
+        }
+        __syncthreads();
+        if (own) {
+#pragma unroll
+            for (int w = 0; w < kMaskWords; ++w)
+                anc[kMaskWords * tid + w] = m[w];
+            T.ord[tid] = nj;
+        }
+        jump = nj;
+    }
+    // subtree sizes (nodes whose masks hold this one) and child counts
+    int sz = 0;
+    if (own) {
+        const int w = tid >> 5;
+        const unsigned bit = 1u << (tid & 31);
+        for (int x = 0; x < N; ++x)
+            sz += (anc[kMaskWords * x + w] & bit) ? 1 : 0;
+        T.sz[tid] = sz;
+        int nch = 0;
+#pragma unroll
+        for (int w2 = 0; w2 < kMaskWords; ++w2)
+            nch += __popc(kids[kMaskWords * tid + w2]);
+        T.nch[tid] = nch;
+    }
+    __syncthreads();
+    // offset among the siblings (visited by increasing (subtree size,
+    // index)) and whether the node is its parent's last-visited child
+    if (own) {
+        int o = 0, is_last = 1;
+        if (tid > 0) {
+            o = 1;
+#pragma unroll
+            for (int w = 0; w < kMaskWords; ++w) {
+                unsigned bits = kids[kMaskWords * pn + w];
+                if (w == (tid >> 5))
+                    bits &= ~(1u << (tid & 31));
+                while (bits) {
+                    const int t = 32 * w + __ffs(bits) - 1;
+                    bits &= bits - 1;
+                    const int zt = T.sz[t];
+                    if (zt < sz || (zt == sz && t < tid))
+                        o += zt;
+                    else
+                        is_last = 0;
+                }
+            }
+        }
+        T.off[tid] = o;
+        T.last[tid] = is_last;
+    }
+    __syncthreads();
+    // preorder position and stack slot: sums of off and not-last over the
+    // root path
+    if (own) {
+        int pos = 0, l = 0;
+#pragma unroll
+        for (int w = 0; w < kMaskWords; ++w) {
+            unsigned bits = m[w];
+            while (bits) {
+                const int x = 32 * w + __ffs(bits) - 1;
+                bits &= bits - 1;
+                pos += T.off[x];
+                l += T.last[x] ? 0 : 1;
+            }
+        }
+        T.ord[pos] = tid;
+        T.lt[tid] = l;
+    }
+    __syncthreads();
+    if (own) {
+        const int pos = tid;
+        const int n = T.ord[pos];
+        const int pp = T.par[n];
+        int src, ld = 0, start = -1, save = 0;
+        if (pos == 0) {
+            src = kSrcRoot;
+        } else if (pp == T.ord[pos - 1]) {
+            src = kSrcCont;
+        } else if (T.lt[pp] < K) {
+            src = kSrcSlot;
+            ld = T.lt[pp];
+        } else {
+            src = kSrcRecompute;
+            // deepest saved ancestor of pp (strictly above it): the highest
+            // index among pp's ancestors that branches and sits in slot K - 1
+            for (int w = kMaskWords - 1; w >= 0 && start < 0; --w) {
+                unsigned bits = anc[kMaskWords * pp + w];
+                if (w == (pp >> 5))
+                    bits &= ~(1u << (pp & 31));
+                while (bits) {
+                    const int x = 32 * w + 31 - __clz(bits);
+                    bits &= ~(1u << (x & 31));
+                    if (T.nch[x] >= 2 && T.lt[x] == K - 1) {
+                        start = x;
+                        break;
+                    }
+                }
+            }
+        }
+        if (T.nch[n] >= 2 && T.lt[n] < K)
+            save = T.lt[n] + 1;
+        T.meta[pos] = n | (src << 16) | (save << 19) | (ld << 24);
+        T.rstart[pos] = start;
+    }
+    __syncthreads();
+    return true;
+}
+
 // Tree metadata held in shared memory (any N).
 struct SmemTree {
     TreeView T;
@@ -1268,7 +1419,8 @@ __device__ __forceinline__ void staged_body(const KParams& p)
         if (warp == 0 && !build_warp_walk(prow, N, p.slots, tsm))
             bad = true;
     } else if constexpr (TK == kTreeSmem) {
-        bad = !build_walk(prow, N, p.slots, tv);
+        bad = (N <= kMaskNodes && N <= (int)blockDim.x) ? !build_walk_masked(prow, N, p.slots, tv)
+                                                        : !build_walk(prow, N, p.slots, tv);
     }
     if (p.early_tree) {
         pdl_wait_then_release();
@@ -1471,7 +1623,8 @@ __global__ void __launch_bounds__((kSmallWarps + 1) * 32) gdn_verify_ring(const 
         ok = !__syncthreads_or(bad);
     } else {
         __syncthreads();
-        ok = build_walk(p.parent + (size_t)sq.n0, N, p.slots, T);
+        ok = (N <= kMaskNodes && N <= (int)blockDim.x) ? build_walk_masked(p.parent + (size_t)sq.n0, N, p.slots, T)
+                                                       : build_walk(p.parent + (size_t)sq.n0, N, p.slots, T);
     }
     if (p.early_tree)
         pdl_wait_then_release();
