@@ -144,6 +144,40 @@ def commit(states, parent, accept_path, accept_len) -> np.ndarray:
     return out
 
 
+def compact(rows, parent, accept_path, accept_len, cu_nodes=None):
+    """Accept-time compaction of per-node rows into path order.
+
+    After verification only the accepted root-to-leaf path's per-node data
+    is carried forward (the GreenGames post, "Key wins": the target features
+    are compacted after a sibling branch is accepted).  For each sequence b
+    whose path checks against its tree (as ``commit`` checks it):
+    dst[b][i] = rows[n0_b + path_b[i]] for i < len_b.
+
+    rows: [T, ...] per-node rows in the packed node layout (T = B * N, or
+    the varlen total with cu_nodes [B + 1] offsets); parent: [T] int32 local
+    indices.  Returns (dst [B, P, ...] with unwritten rows zero, written
+    [B, P] bool).  A bad path writes nothing for its sequence.
+    """
+    rows = np.asarray(rows)
+    parent, accept_path, accept_len = map(_i32, (parent, accept_path, accept_len))
+    B, P = accept_path.shape
+    if cu_nodes is None:
+        N = parent.shape[0] // B if B else 0
+        cu = np.arange(B + 1, dtype=np.int64) * N
+    else:
+        cu = np.asarray(cu_nodes, dtype=np.int64)
+    dst = np.zeros((B, P) + rows.shape[1:], dtype=rows.dtype)
+    written = np.zeros((B, P), dtype=bool)
+    for b in range(B):
+        n0, n1 = int(cu[b]), int(cu[b + 1])
+        if check_path(parent[n0:n1], accept_path[b], int(accept_len[b])) != OK:
+            continue
+        for i in range(int(accept_len[b])):
+            dst[b, i] = rows[n0 + int(accept_path[b, i])]
+            written[b, i] = True
+    return dst, written
+
+
 def round_to(state_dtype: str, x) -> np.ndarray:
     """Round float64 values to the persisted dtype and back (RNE)."""
     lib = _load()
