@@ -716,6 +716,45 @@ def _build_point(*, batch, budget, max_depth=16, top_k=8, chain_seed=False, reps
     return t, bool((got == want).all()), cpu_per_tree
 
 
+def _compact_point(*, batch, budget, row_bytes, reps=20, seed=41):
+    """Mean time of one gdn_tree_compact launch: the accepted paths' rows of
+    DDTree-style trees gathered into path order.  Returns (seconds, bytes
+    moved per launch: each accepted row read once and written once)."""
+    import gated_deltanet_tree_verify_b200 as gdn
+    n = budget + 1
+    prob = make_problem(batch=batch, n_nodes=n, n_k_heads=1, n_v_heads=1, d_k=32, d_v=32, tree="ddtree",
+                        seed=seed, qkv_dtype="f32", accept="leaf")
+    parent = prob.parent.cuda()
+    path, length = prob.accept_path.cuda(), prob.accept_len.cuda()
+    src = torch.empty(batch * n * row_bytes // 4, device="cuda")
+    dst = torch.empty(batch * path.shape[1] * row_bytes // 4, device="cuda")
+
+    def run_all():
+        for _ in range(reps):
+            gdn.gdn_tree_compact(src, parent, path, length, dst, batch=batch, n_nodes=n, row_bytes=row_bytes)
+
+    run_all()
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=s):
+            run_all()
+    torch.cuda.current_stream().wait_stream(s)
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    t = e0.elapsed_time(e1) / 1e3 / reps
+    del graph
+    return t, 2 * int(prob.accept_len.sum()) * row_bytes
+
+
 def run_sweep(args):
     import gated_deltanet_tree_verify_b200 as gdn
     gdn.load_library()
@@ -738,6 +777,9 @@ def run_sweep(args):
     for budget in (22, 64, 128, 1023):
         for batch in (1, 8, 64):
             points.append(dict(kind="build", budget=budget, batch=batch))
+    # compaction of the accepted paths' outputs (24 KB rows) and f16 states (1.5 MB rows)
+    for batch, row in ((1, 24576), (32, 24576), (8, 1572864), (32, 1572864)):
+        points.append(dict(kind="compact", budget=64, batch=batch, row_bytes=row))
     if args.sweep_kinds:
         keep = set(args.sweep_kinds.split(","))
         points = [pt for pt in points if pt["kind"] in keep]
@@ -758,6 +800,10 @@ def _sweep_point(args, gdn, pt, peak, varlen_budgets, clocks):
         line = {"sweep": "build_tree", "budget": pt["budget"], "batch": pt["batch"], "max_depth": 16, "top_k": 8,
                 "build_us": t * 1e6, "trees_per_s": pt["batch"] / t, "ns_per_pop": t * 1e9 / pt["budget"],
                 "matches_oracle": ok, "oracle_us_per_tree": cpu * 1e6}
+    elif pt["kind"] == "compact":
+        t, moved = _compact_point(batch=pt["batch"], budget=pt["budget"], row_bytes=pt["row_bytes"])
+        line = {"sweep": "compact", "budget": pt["budget"], "batch": pt["batch"], "row_bytes": pt["row_bytes"],
+                "compact_us": t * 1e6, "gbps": moved / t / 1e9, "frac_of_hbm": moved / t / 1e9 / peak}
     elif pt["kind"] == "varlen":
         t, vb, T = _varlen_point(budgets=varlen_budgets, state_dtype=pt["state_dtype"], workspace=pt["ws"])
         line = {"sweep": "varlen", "budgets": varlen_budgets, "state_dtype": pt["state_dtype"],
@@ -813,7 +859,7 @@ def main(argv=None):
                          "(one JSON line per point; not the benchmark line)")
     ap.add_argument("--sweep-kinds", default="",
                     help="comma-separated subset of the sweep's point kinds (tree, chain16, varlen, chain4096, "
-                         "build); default all")
+                         "build, compact); default all")
     ap.add_argument("--sm-mhz", type=float, default=1965.0,
                     help="SM clock for the sweep's FP32 ALU roofline (default: the B200 maximum)")
     args = ap.parse_args(argv)

@@ -569,3 +569,67 @@ gdn_status gdn_build_tree(const gdn_build_desc* desc, const float* logp, const i
 }
 
 }  // extern "C"
+
+// ---- gdn_tree_compact ------------------------------------------------------
+
+extern "C" {
+
+gdn_status gdn_tree_compact(int32_t batch, int32_t n_nodes, const int32_t* cu_nodes, int32_t total_nodes,
+                            size_t row_bytes, const void* src, const int32_t* parent_idx,
+                            const int32_t* accept_path, const int32_t* accept_len, int32_t max_path_len,
+                            void* dst, int32_t* status, cudaStream_t stream)
+{
+    g_detail[0] = '\0';
+    if (batch < 0 || n_nodes < 1 || max_path_len < 1)
+        return fail(GDN_ERR_INVALID_ARG, "batch, n_nodes or max_path_len out of range%s");
+    if (row_bytes == 0 || row_bytes % 16 != 0)
+        return fail(GDN_ERR_INVALID_ARG, "row_bytes is not a positive multiple of 16%s");
+    if (cu_nodes && (total_nodes < batch || (long long)total_nodes > (long long)batch * n_nodes))
+        return fail(GDN_ERR_INVALID_ARG, "total_nodes outside [batch, batch * n_nodes]%s");
+    if (!src || !dst || !parent_idx || !accept_path || !accept_len)
+        return fail(GDN_ERR_INVALID_ARG, "a required pointer is NULL%s");
+    if (!aligned(src, 16) || !aligned(dst, 16))
+        return fail(GDN_ERR_INVALID_ARG, "src or dst is not 16-byte aligned%s");
+    const struct { const void* p; const char* n; } al[] = {
+        {cu_nodes, "cu_nodes"}, {parent_idx, "parent_idx"}, {accept_path, "accept_path"},
+        {accept_len, "accept_len"}, {status, "status"}};
+    for (const auto& x : al)
+        if (x.p && !aligned(x.p, 4))
+            return fail(GDN_ERR_INVALID_ARG, "%s is misaligned", x.n);
+    if (batch == 0)
+        return GDN_OK;
+    if (batch > 65535)
+        return fail(GDN_ERR_UNSUPPORTED, "batch above the grid limit%s");
+    const size_t B = batch, T = cu_nodes ? (size_t)total_nodes : B * n_nodes;
+    const size_t pieces = (row_bytes + 65535) / 65536;
+    if (pieces > 65535)
+        return fail(GDN_ERR_UNSUPPORTED, "row_bytes above 4 GiB%s");
+    const Range out{dst, B * (size_t)max_path_len * row_bytes, "dst"};
+    const Range ins[] = {{src, T * row_bytes, "src"}, {parent_idx, T * 4, "parent_idx"},
+                         {accept_path, B * (size_t)max_path_len * 4, "accept_path"},
+                         {accept_len, B * 4, "accept_len"}, {cu_nodes, (B + 1) * 4, "cu_nodes"},
+                         {status, 4, "status"}};
+    for (const auto& x : ins)
+        if (overlap(out, x))
+            return fail(GDN_ERR_INVALID_ARG, "dst overlaps input %s", x.name);
+
+    gdn::CompactArgs a{};
+    a.src = src;
+    a.dst = dst;
+    a.parent = parent_idx;
+    a.accept_path = accept_path;
+    a.accept_len = accept_len;
+    a.cu_nodes = cu_nodes;
+    a.status = status;
+    a.batch = batch;
+    a.n_nodes = n_nodes;
+    a.total_nodes = cu_nodes ? total_nodes : batch * n_nodes;
+    a.max_path_len = max_path_len;
+    a.row_bytes = row_bytes;
+    const cudaError_t e = gdn::launch_compact(a, stream);
+    if (e != cudaSuccess)
+        return fail(GDN_ERR_CUDA, "compact launch failed: %s", cudaGetErrorString(e));
+    return GDN_OK;
+}
+
+}  // extern "C"

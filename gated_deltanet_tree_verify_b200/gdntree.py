@@ -107,6 +107,8 @@ def load_library() -> ctypes.CDLL:
     lib.gdn_tree_commit_layers.restype = ctypes.c_int
     lib.gdn_build_tree.argtypes = [ctypes.POINTER(GdnBuildDesc)] + [vp] * 8
     lib.gdn_build_tree.restype = ctypes.c_int
+    lib.gdn_tree_compact.argtypes = [i32, i32, vp, i32, ctypes.c_size_t, vp, vp, vp, vp, i32, vp, vp, vp]
+    lib.gdn_tree_compact.restype = ctypes.c_int
     lib.gdn_status_str.argtypes = [ctypes.c_int]
     lib.gdn_status_str.restype = ctypes.c_char_p
     lib.gdn_last_error_detail.argtypes = []
@@ -305,4 +307,22 @@ def gdn_build_tree(desc: GdnBuildDesc, logp, parent_idx, topk_ids=None, node_dep
                             _ptr(parent_idx, "parent_idx"), _ptr(node_depth, "node_depth"),
                             _ptr(node_rank, "node_rank"), _ptr(node_token, "node_token"),
                             _ptr(node_score, "node_score"), _stream(stream))
+    return _check(rc, check)
+
+
+def gdn_tree_compact(src, parent_idx, accept_path, accept_len, dst, *, batch: int, n_nodes: int,
+                     row_bytes: Optional[int] = None, max_path_len: Optional[int] = None, cu_nodes=None,
+                     total_nodes: int = 0, status=None, stream=None, check: bool = True) -> int:
+    """Calls gdn_tree_compact (see include/gdntree.h).  ``row_bytes``
+    defaults to dst's bytes per (sequence, path position), ``max_path_len``
+    to accept_path's second dimension."""
+    lib = load_library()
+    if row_bytes is None:
+        row_bytes = dst[0, 0].numel() * dst.element_size()
+    if max_path_len is None:
+        max_path_len = accept_path.shape[1]
+    rc = lib.gdn_tree_compact(int(batch), int(n_nodes), _ptr(cu_nodes, "cu_nodes"), int(total_nodes),
+                              int(row_bytes), _ptr(src, "src"), _ptr(parent_idx, "parent_idx"),
+                              _ptr(accept_path, "accept_path"), _ptr(accept_len, "accept_len"),
+                              int(max_path_len), _ptr(dst, "dst"), _ptr(status, "status"), _stream(stream))
     return _check(rc, check)

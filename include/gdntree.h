@@ -304,6 +304,37 @@ gdn_status gdn_tree_commit_varlen(const gdn_tree_desc* desc, const int32_t* cu_n
                                   const int32_t* accept_path, const int32_t* accept_len, int32_t max_path_len,
                                   float* const* state_out, cudaStream_t stream);
 
+/*
+ * gdn_tree_compact -- accept-time compaction: carry only the accepted path's
+ * per-node rows forward, in path order (the target-feature compaction after
+ * a sibling accept, the GreenGames post, "Key wins").  For every sequence b
+ * whose path checks against its tree (path[0] = 0, parent[path[i]] =
+ * path[i-1], 1 <= accept_len[b] <= min(max_path_len, N_b)):
+ *
+ *     dst[b][i] = src[n0_b + accept_path[b][i]]      for i < accept_len[b]
+ *
+ *   src          [T][row_bytes] per-node rows (outputs, features, states...;
+ *                the bytes are copied as they are), T = B * n_nodes, or the
+ *                packed varlen total.  Read-only.
+ *   cu_nodes     NULL (every sequence has n_nodes nodes), or [B + 1] device
+ *                int32 offsets as for gdn_tree_verify_varlen (n_nodes is then
+ *                the most per sequence, total_nodes = cu_nodes[B])
+ *   parent_idx   [T] int32, each sequence's parents as local indices
+ *   accept_path  [B][max_path_len] int32, accept_len [B] int32
+ *   dst          [B][max_path_len][row_bytes]; rows at i >= accept_len[b]
+ *                are left untouched
+ *   status       optional device int32: GDN_ERR_BAD_PATH (or
+ *                GDN_ERR_BAD_TREE for bad offsets); that sequence's dst rows
+ *                are left untouched
+ * row_bytes a positive multiple of 16; src and dst 16-byte aligned, the int32
+ * arrays 4-byte aligned; dst must not overlap any input.  Errors:
+ * GDN_ERR_INVALID_ARG / GDN_ERR_UNSUPPORTED / GDN_ERR_CUDA from the host.
+ */
+gdn_status gdn_tree_compact(int32_t batch, int32_t n_nodes, const int32_t* cu_nodes, int32_t total_nodes,
+                            size_t row_bytes, const void* src, const int32_t* parent_idx,
+                            const int32_t* accept_path, const int32_t* accept_len, int32_t max_path_len,
+                            void* dst, int32_t* status, cudaStream_t stream);
+
 /* Largest N the tree (non-chain) path takes. */
 #define GDN_MAX_TREE_NODES 1024
 

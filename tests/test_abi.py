@@ -258,3 +258,27 @@ def test_build_tree_host_checks(lib):
     assert call(dep_=par + 4) == gdn.GDN_ERR_INVALID_ARG                          # outputs overlap
     assert call(check_par=lp + 64) == gdn.GDN_ERR_INVALID_ARG                     # output inside logp
     assert call(ids_=ids, tok_=ids + 4) == gdn.GDN_ERR_INVALID_ARG                # output inside topk_ids
+
+
+def test_compact_host_checks(lib):
+    src, par, path, ln, dst, cu = (BASE + i * MB for i in range(6))
+
+    def call(**kw):
+        base = dict(batch=2, n_nodes=23, row_bytes=24576, max_path_len=17)
+        args = dict(src=src, par=par, path=path, ln=ln, dst=dst)
+        for k in list(kw):
+            if k in args:
+                args[k] = kw.pop(k)
+        base.update(kw)
+        return gdn.gdn_tree_compact(args["src"], args["par"], args["path"], args["ln"], args["dst"], stream=0,
+                                    check=False, **base)
+    assert call(batch=0) == gdn.GDN_OK
+    assert call(batch=-1) == gdn.GDN_ERR_INVALID_ARG
+    assert call(row_bytes=24) == gdn.GDN_ERR_INVALID_ARG          # not a multiple of 16
+    assert call(max_path_len=0) == gdn.GDN_ERR_INVALID_ARG
+    assert call(src=None) == gdn.GDN_ERR_INVALID_ARG
+    assert call(dst=dst + 8) == gdn.GDN_ERR_INVALID_ARG          # misaligned
+    assert call(ln=ln + 2) == gdn.GDN_ERR_INVALID_ARG
+    assert call(dst=src + 4096) == gdn.GDN_ERR_INVALID_ARG       # overlaps src
+    assert call(cu_nodes=cu, total_nodes=1) == gdn.GDN_ERR_INVALID_ARG  # fewer nodes than sequences
+    assert call(cu_nodes=cu, total_nodes=47) == gdn.GDN_ERR_INVALID_ARG  # above batch * n_nodes
