@@ -58,7 +58,7 @@ typedef enum {
 typedef enum {
     GDN_OK = 0,
     GDN_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned or overlapping buffers */
-    GDN_ERR_UNSUPPORTED = 2,  /* a shape or dtype this build has no kernel for */
+    GDN_ERR_UNSUPPORTED = 2,  /* a shape or dtype the library has no kernel for */
     GDN_ERR_BAD_TREE = 3,     /* device-detected: parent[0] != -1 or parent[n] not in [0, n) */
     GDN_ERR_BAD_PATH = 4,     /* device-detected: accept path/length violates the tree */
     GDN_ERR_CUDA = 5,         /* a CUDA call failed; gdn_last_error_detail() says which */

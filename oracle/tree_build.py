@@ -8,7 +8,7 @@ decoding (the GreenGames post, "From autoregressive to DDTree": the tree is
 built by ``build_ddtree`` from the drafter's per-position top-k candidates,
 optionally pre-seeded with the greedy chain; "Key wins": candidates are
 ordered best first, rank 0 at the root side).  The pages give no formula;
-the reading (also stated in the design doc) is:
+the reading taken here is:
 
 * ``logp[d][r]`` is the log-probability of the rank-r candidate at draft
   position d + 1 (r = 0 the best, each row non-increasing).
