@@ -10,6 +10,7 @@
 
 #include <cuda_runtime.h>
 
+#include "gdn_compact.h"
 #include "gdn_internal.h"
 #include "gdntree.h"
 

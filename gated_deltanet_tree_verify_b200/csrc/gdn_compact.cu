@@ -15,6 +15,7 @@
 
 #include <cuda_runtime.h>
 
+#include "gdn_compact.h"
 #include "gdn_device.cuh"
 #include "gdn_internal.h"
 

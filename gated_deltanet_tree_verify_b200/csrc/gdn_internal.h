@@ -120,19 +120,4 @@ struct BuildArgs {
 
 cudaError_t launch_build_tree(const BuildArgs& a, cudaStream_t stream);
 
-// Accept-time compaction (gdn_tree_compact), checked by the host.
-struct CompactArgs {
-    const void* src;
-    void* dst;
-    const int32_t* parent;
-    const int32_t* accept_path;
-    const int32_t* accept_len;
-    const int32_t* cu_nodes;  // NULL: n_nodes per sequence
-    int32_t* status;
-    int batch, n_nodes, total_nodes, max_path_len;
-    size_t row_bytes;
-};
-
-cudaError_t launch_compact(const CompactArgs& a, cudaStream_t stream);
-
 }  // namespace gdn
