@@ -1358,7 +1358,25 @@ __device__ __forceinline__ void staged_body(const KParams& p)
         const QT* kg = static_cast<const QT*>(p.k);
         const QT* qg = static_cast<const QT*>(p.q);
         const QT* vg = static_cast<const QT*>(p.v);
-        for (int n = warp; n < N; n += nwarps) {
+        if constexpr (sizeof(QT) == 2) {
+            // k and q rows: 2 QKCH chunks per node over all threads (a warp
+            // per node at d_k = 128), then the v slices
+            constexpr int KQ = 2 * QKCH;
+            for (int idx = tid; idx < N * KQ; idx += blockDim.x) {
+                const int n = idx / KQ, c = idx % KQ;
+                const size_t node = (size_t)sq.n0 + n;
+                const QT* src = (c < QKCH ? kg : qg) + (node * p.Hk + hk) * DK + (c % QKCH) * EPC;
+                cp_async16(raw + (size_t)n * p.raw_bytes + 16 * c, src);
+            }
+            const int vch = per_node - KQ;  // rows / 8
+            for (int idx = tid; idx < N * vch; idx += blockDim.x) {
+                const int n = idx / vch, c = idx - n * vch;
+                const size_t node = (size_t)sq.n0 + n;
+                cp_async16(raw + (size_t)n * p.raw_bytes + 16 * (KQ + c),
+                           vg + (node * p.Hv + h) * p.dv + row0 + c * EPC);
+            }
+        }
+        for (int n = warp; n < N && sizeof(QT) == 4; n += nwarps) {
             const size_t node = (size_t)sq.n0 + n;
             const QT* krow = kg + (node * p.Hk + hk) * DK;
             const QT* qrow = qg + (node * p.Hk + hk) * DK;
