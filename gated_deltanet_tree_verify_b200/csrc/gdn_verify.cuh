@@ -304,11 +304,57 @@ __device__ __forceinline__ float rec_elem(const float* rec, int part, int e)
 template <int DK, int LR, typename RT>
 __device__ __forceinline__ float node_kq8(const RT* rec, int sub);
 
+// bf16 records: lane sub of the group takes the DK / 8 consecutive elements
+// [DK / 8 * sub, DK / 8 * (sub + 1)) of a row, in 16-byte loads (8-byte at
+// DK = 32), widened to pairs.
+template <int DK>
+__device__ __forceinline__ void row_part8(const __nv_bfloat16* rec, int part, int sub, float2 (&x)[DK / 16])
+{
+    constexpr int E = DK / 8;
+    const __nv_bfloat16* base = rec + part + E * sub;
+    if constexpr (E >= 8) {
+#pragma unroll
+        for (int c = 0; c < E / 8; ++c) {
+            float2 y[4];
+            Widen<__nv_bfloat16>::lds8(base + 8 * c, y);
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+                x[4 * c + t] = y[t];
+        }
+    } else {
+        const uint2 u = *reinterpret_cast<const uint2*>(base);
+        x[0] = bf16x2_to_float2(u.x);
+        x[1] = bf16x2_to_float2(u.y);
+    }
+}
+
+// x . y over a group of 8 lanes holding row_part8 pieces: the lane's pairs
+// in order with packed FMAs, its two halves, then the xor butterfly.
+template <int NP>
+__device__ __forceinline__ float group_dot8(const float2 (&x)[NP], const float2 (&y)[NP])
+{
+    float2 acc = __fmul2_rn(x[0], y[0]);
+#pragma unroll
+    for (int t = 1; t < NP; ++t)
+        acc = __ffma2_rn(x[t], y[t], acc);
+    float s = __fadd_rn(acc.x, acc.y);
+#pragma unroll
+    for (int off = 4; off >= 1; off >>= 1)
+        s = __fadd_rn(s, __shfl_xor_sync(0xffffffffu, s, off));
+    return s;
+}
+
 // x . y of two rows of one node's record (part 0: k, part DK: q), reduced
 // by a group of 8 lanes like node_kq8.
 template <int DK, int LR, typename RT>
 __device__ __forceinline__ float node_dot8(const RT* rec, int sub, int pa, int pb)
 {
+    if constexpr (sizeof(RT) == 2) {
+        float2 x[DK / 16], y[DK / 16];
+        row_part8<DK>(rec, pa, sub, x);
+        row_part8<DK>(rec, pb, sub, y);
+        return group_dot8(x, y);
+    }
     float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
     for (int j = sub; j < DK; j += 16) {
@@ -329,6 +375,15 @@ __device__ __forceinline__ float node_dot8(const RT* rec, int sub, int pa, int p
 template <int DK, int LR, typename RT>
 __device__ __forceinline__ void node_dots8(const RT* rec, int sub, float& kq, float& kk, float& qq)
 {
+    if constexpr (sizeof(RT) == 2) {
+        float2 x[DK / 16], y[DK / 16];
+        row_part8<DK>(rec, 0, sub, x);
+        row_part8<DK>(rec, DK, sub, y);
+        kq = group_dot8(x, y);
+        kk = group_dot8(x, x);
+        qq = group_dot8(y, y);
+        return;
+    }
     float q0 = 0.f, q1 = 0.f, k0 = 0.f, k1 = 0.f, s0 = 0.f, s1 = 0.f;
 #pragma unroll 1
     for (int j = sub; j < DK; j += 16) {
@@ -355,6 +410,8 @@ __device__ __forceinline__ void node_dots8(const RT* rec, int sub, float& kq, fl
 template <int DK, int LR, typename RT>
 __device__ __forceinline__ float node_kq8(const RT* rec, int sub)
 {
+    if constexpr (sizeof(RT) == 2)
+        return node_dot8<DK, LR>(rec, sub, 0, DK);
     float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
     for (int j = sub; j < DK; j += 16) {
