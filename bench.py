@@ -546,10 +546,12 @@ FP32_LANES_PER_SM = 128  # FP32 CUDA-core lanes per SM (B200); 148 SMs
 
 
 def _verify_point(*, batch, n_nodes, tree, state_dtype, flags=0, gate="softplus", reps=20,
-                  min_bytes=512 << 20, seed=11, workspace=False):
+                  min_bytes=512 << 20, seed=11, workspace=False, planned=False):
     """Mean time of one verify launch, over graph replays of R launches on R
     distinct buffer sets (R sized so the sets together exceed min_bytes).
-    With ``workspace``, through gdn_tree_verify_ws (one workspace per set)."""
+    With ``workspace``, through gdn_tree_verify_ws (one workspace per set);
+    with ``planned``, through gdn_tree_verify_planned with each set's plan
+    built beforehand (a step builds it once for all its layers)."""
     import gated_deltanet_tree_verify_b200 as gdn
     persist_last = bool(flags & gdn.GDN_FLAG_PERSIST_LAST)
     tdt = torch.float32 if state_dtype == "f32" else torch.float16
@@ -573,10 +575,18 @@ def _verify_point(*, batch, n_nodes, tree, state_dtype, flags=0, gate="softplus"
     ws_bytes = gdn.gdn_tree_verify_workspace_bytes(desc) if workspace else 0
     for _, d in sets:
         d["ws"] = torch.empty(max(ws_bytes, 16) // 4, device="cuda") if ws_bytes else None
+    plan_bytes = gdn.gdn_tree_plan_bytes(desc) if planned else 0
+    for _, d in sets:
+        d["plan"] = torch.empty(max(plan_bytes, 16) // 4, dtype=torch.int32, device="cuda") if planned else None
+        if planned:
+            gdn.gdn_tree_plan(desc, d["parent"], d["plan"], plan_bytes)
 
     def run_all():
         for _, d in sets:
-            if d["ws"] is not None:
+            if d["plan"] is not None:
+                gdn.gdn_tree_verify_planned(desc, d["plan"], d["q"], d["k"], d["v"], d["g"], d["beta"],
+                                            d["parent"], d["state_in"], d["out"], d["ns"], plan_bytes=plan_bytes)
+            elif d["ws"] is not None:
                 gdn.gdn_tree_verify_ws(desc, d["q"], d["k"], d["v"], d["g"], d["beta"], d["parent"],
                                        d["state_in"], d["out"], d["ns"], d["ws"], ws_bytes)
             else:
@@ -767,6 +777,7 @@ def run_sweep(args):
                 points.append(dict(kind="tree", budget=budget, batch=batch, state_dtype=sd))
                 if sd == "f16":
                     points.append(dict(kind="tree", budget=budget, batch=batch, state_dtype=sd, ws=True))
+                    points.append(dict(kind="tree", budget=budget, batch=batch, state_dtype=sd, planned=True))
     for sd in ("f32", "f16"):
         points.append(dict(kind="chain16", budget=15, batch=1, state_dtype=sd))
     # varlen: 8 trees of budgets 8..64 in one launch
@@ -831,10 +842,11 @@ def _sweep_point(args, gdn, pt, peak, varlen_budgets, clocks):
         tree = "ddtree" if pt["kind"] == "tree" else "chain"
         flags = 0 if pt["kind"] == "tree" else gdn.GDN_FLAG_CHAIN
         t, R = _verify_point(batch=pt["batch"], n_nodes=n, tree=tree, state_dtype=pt["state_dtype"],
-                             flags=flags, workspace=pt.get("ws", False))
+                             flags=flags, workspace=pt.get("ws", False), planned=pt.get("planned", False))
         vb = verify_bytes(pt["batch"], n, pt["state_dtype"])
         line = {"sweep": pt["kind"], "budget": pt["budget"], "batch": pt["batch"],
-                "state_dtype": pt["state_dtype"], "workspace": pt.get("ws", False), "verify_us": t * 1e6,
+                "state_dtype": pt["state_dtype"], "workspace": pt.get("ws", False),
+                "planned": pt.get("planned", False), "verify_us": t * 1e6,
                 "node_layers_per_s": pt["batch"] * n / t, "gbps": vb / t / 1e9,
                 "frac_of_hbm": vb / t / 1e9 / peak, "buffer_sets": R}
     line["sm_mhz_after"] = clocks.now()

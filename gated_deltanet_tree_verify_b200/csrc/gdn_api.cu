@@ -160,7 +160,8 @@ gdn::VerifyArgs verify_args(const gdn_tree_desc& d)
 gdn_status verify_impl(const gdn_tree_desc* desc, const int32_t* cu, int32_t total, const void* q,
                        const void* k, const void* v, const float* g, const float* beta,
                        const int32_t* parent_idx, const float* state_in, float* out, void* node_states,
-                       void* workspace, size_t workspace_bytes, cudaStream_t stream, bool varlen)
+                       void* workspace, size_t workspace_bytes, cudaStream_t stream, bool varlen,
+                       const void* plan = nullptr, size_t plan_bytes = 0)
 {
     g_detail[0] = '\0';
     gdn_status st = check_desc(desc, true);
@@ -220,6 +221,16 @@ gdn_status verify_impl(const gdn_tree_desc* desc, const int32_t* cu, int32_t tot
     const gdn::VerifyGeom geom = gdn::verify_geometry(a, workspace != nullptr);
     if (geom.tiles <= 0 || geom.smem > 227 * 1024)
         return fail(GDN_ERR_UNSUPPORTED, "no launch geometry for this shape%s");
+    size_t plan_need = 0;
+    if (plan != nullptr) {
+        const gdn::PlanGeom pg = gdn::plan_geometry(a);
+        if (pg.needed) {
+            plan_need = (size_t)d.batch * pg.stride * 4;
+            if (!aligned(plan, 16) || plan_bytes < plan_need)
+                return fail(GDN_ERR_INVALID_ARG, "plan misaligned or smaller than gdn_tree_plan_bytes()%s");
+            a.plan = static_cast<const int32_t*>(plan);
+        }
+    }
     if (d.n_v_heads > 65535 || d.batch > 65535)
         return fail(GDN_ERR_UNSUPPORTED, "batch or n_v_heads above the grid limit%s");
     if (geom.gslots && workspace_bytes < geom.ws_bytes)
@@ -232,7 +243,8 @@ gdn_status verify_impl(const gdn_tree_desc* desc, const int32_t* cu, int32_t tot
                          {v, T * Hv * dv * es, "v"},     {g, T * Hv * 4, "g"},
                          {beta, T * Hv * 4, "beta"},     {parent_idx, T * 4, "parent_idx"},
                          {state_in, B * Hv * dv * dk * 4, "state_in"},
-                         {d.status, 4, "status"},       {a.cu_nodes, (B + 1) * 4, "cu_nodes"}};
+                         {d.status, 4, "status"},       {a.cu_nodes, (B + 1) * 4, "cu_nodes"},
+                         {a.plan, plan_need, "plan"}};
     const Range outs[] = {{out, T * Hv * dv * 4, "out"},
                           {node_states, node_states_bytes_v(d, a.cu_nodes, total), "node_states"},
                           {geom.gslots ? workspace : nullptr, geom.ws_bytes, "workspace"}};
@@ -631,6 +643,67 @@ gdn_status gdn_tree_compact(int32_t batch, int32_t n_nodes, const int32_t* cu_no
     if (e != cudaSuccess)
         return fail(GDN_ERR_CUDA, "compact launch failed: %s", cudaGetErrorString(e));
     return GDN_OK;
+}
+
+}  // extern "C"
+
+// ---- tree plans ----------------------------------------------------------
+
+extern "C" {
+
+size_t gdn_tree_plan_bytes(const gdn_tree_desc* desc)
+{
+    if (check_desc(desc, true) != GDN_OK || (desc->flags & GDN_FLAG_CHUNKED))
+        return 0;
+    const gdn::PlanGeom pg = gdn::plan_geometry(verify_args(*desc));
+    return pg.needed ? (size_t)desc->batch * pg.stride * 4 : 0;
+}
+
+gdn_status gdn_tree_plan(const gdn_tree_desc* desc, const int32_t* parent_idx, void* plan, size_t plan_bytes,
+                         cudaStream_t stream)
+{
+    g_detail[0] = '\0';
+    gdn_status st = check_desc(desc, true);
+    if (st != GDN_OK)
+        return st;
+    const gdn_tree_desc& d = *desc;
+    if (d.flags & GDN_FLAG_CHUNKED)
+        return fail(GDN_ERR_UNSUPPORTED, "chunked chains have no tree plan%s");
+    const gdn::VerifyArgs a0 = verify_args(d);
+    const gdn::PlanGeom pg = gdn::plan_geometry(a0);
+    if (!pg.needed || d.batch == 0)
+        return GDN_OK;  // this walk kind builds nothing: the plan is not read
+    const size_t need = (size_t)d.batch * pg.stride * 4;
+    if (!parent_idx || !plan)
+        return fail(GDN_ERR_INVALID_ARG, "parent_idx or plan is NULL%s");
+    if (!aligned(parent_idx, 4) || !aligned(plan, 16) || (d.status && !aligned(d.status, 4)))
+        return fail(GDN_ERR_INVALID_ARG, "a pointer is misaligned%s");
+    if (plan_bytes < need)
+        return fail(GDN_ERR_INVALID_ARG, "plan smaller than gdn_tree_plan_bytes()%s");
+    const Range pr{plan, need, "plan"};
+    if (overlap(pr, Range{parent_idx, (size_t)d.batch * d.n_nodes * 4, "parent_idx"}) ||
+        overlap(pr, Range{d.status, 4, "status"}))
+        return fail(GDN_ERR_INVALID_ARG, "plan overlaps an input%s");
+    if (d.batch > (1 << 30))
+        return fail(GDN_ERR_UNSUPPORTED, "batch above the grid limit%s");
+    gdn::VerifyArgs a = a0;
+    a.parent = parent_idx;
+    a.status = d.status;
+    const cudaError_t e = gdn::launch_plan(a, pg, static_cast<int32_t*>(plan), stream);
+    if (e != cudaSuccess)
+        return fail(GDN_ERR_CUDA, "plan launch failed: %s", cudaGetErrorString(e));
+    return GDN_OK;
+}
+
+gdn_status gdn_tree_verify_planned(const gdn_tree_desc* desc, const void* plan, size_t plan_bytes, const void* q,
+                                   const void* k, const void* v, const float* g, const float* beta,
+                                   const int32_t* parent_idx, const float* state_in, float* out,
+                                   void* node_states, cudaStream_t stream)
+{
+    if (desc && (desc->flags & GDN_FLAG_CHUNKED))
+        return fail(GDN_ERR_UNSUPPORTED, "chunked chains have no tree plan%s");
+    return verify_impl(desc, nullptr, 0, q, k, v, g, beta, parent_idx, state_in, out, node_states, nullptr, 0,
+                       stream, false, plan, plan_bytes);
 }
 
 }  // extern "C"

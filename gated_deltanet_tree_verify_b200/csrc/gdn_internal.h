@@ -51,7 +51,19 @@ struct VerifyArgs {
     float* workspace;  // optional: stack slots in global memory
     const int32_t* cu_nodes;  // optional (varlen): [batch + 1] node offsets; n_nodes = the most per sequence
     int total_nodes;          // varlen: cu_nodes[batch]
+    const int32_t* plan;      // optional: walks from gdn_tree_plan
 };
+
+// Layout of a tree plan (gdn_tree_plan) for a verify call's geometry: whether
+// the call's walk kind uses one (trees walked with stack slots), the int32
+// per sequence, and the signature each sequence's header carries.
+struct PlanGeom {
+    bool needed;
+    bool warp_kind;  // MaskTree (<= 32 nodes, staged) else TreeView arrays
+    int slots, n_nodes, stride, sig;
+};
+PlanGeom plan_geometry(const VerifyArgs& a);
+cudaError_t launch_plan(const VerifyArgs& a, const PlanGeom& pg, int32_t* plan, cudaStream_t stream);
 
 // Layers one commit launch covers (more are split over several launches).
 constexpr int kMaxCommitLayers = 64;

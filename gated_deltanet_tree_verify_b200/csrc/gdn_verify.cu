@@ -185,12 +185,96 @@ cudaError_t launch_verify(const VerifyArgs& a, const VerifyGeom& geom, cudaStrea
     kp.off_ab = geom.off_ab;
     kp.off_slots = geom.off_slots;
     kp.off_tree = geom.off_tree;
+    if (a.plan != nullptr) {
+        const PlanGeom pg = plan_geometry(a);
+        if (pg.needed) {
+            kp.plan = a.plan;
+            kp.plan_stride = pg.stride;
+            kp.plan_sig = pg.sig;
+        }
+    }
     switch (a.d_k) {
         case 32: return launch_shapes<32>(kp, a, geom, stream);
         case 64: return launch_shapes<64>(kp, a, geom, stream);
         case 128: return launch_shapes<128>(kp, a, geom, stream);
         default: return cudaErrorInvalidValue;
     }
+}
+
+// ---------------------------------------------------------------------------
+// Tree plans: the walk of each sequence built once, for every layer of a step
+// ---------------------------------------------------------------------------
+
+PlanGeom plan_geometry(const VerifyArgs& a)
+{
+    PlanGeom pg{};
+    const VerifyGeom g = verify_geometry(a, false);
+    const bool chain = (a.flags & GDN_FLAG_CHAIN) != 0;
+    pg.needed = !chain && !g.reload && g.tiles > 0;
+    pg.warp_kind = g.warp_tree;
+    pg.slots = g.slots;
+    pg.n_nodes = a.n_nodes;
+    pg.stride = verify::kPlanHeader + (pg.warp_kind ? 128 : ((4 * a.n_nodes + 3) & ~3));
+    pg.sig = 0x6D000000 | ((pg.warp_kind ? 1 : 2) << 20) | ((pg.slots & 15) << 16) | (a.n_nodes & 0xffff);
+    return pg;
+}
+
+namespace verify {
+namespace {
+
+constexpr int kPlanThreads = 256;
+
+// One CTA per sequence: the walk exactly as the staged kernels build it.
+__global__ void __launch_bounds__(kPlanThreads)
+    gdn_plan_kernel(const int32_t* parent, int N, int K, int warp_kind, int sig, int32_t* plan, int stride,
+                    int32_t* status)
+{
+    extern __shared__ __align__(16) unsigned char smem[];
+    int* tsm = reinterpret_cast<int*>(smem);
+    pdl_wait_then_release();
+    const int b = blockIdx.x, tid = threadIdx.x;
+    const int32_t* prow = parent + (size_t)b * N;
+    bool ok;
+    if (warp_kind) {
+        bool w_ok = true;
+        if (tid < 32)
+            w_ok = build_warp_walk(prow, N, K, tsm);
+        ok = !__syncthreads_or(!w_ok);
+    } else {
+        const TreeView tv(tsm, N);
+        ok = (N <= kMaskNodes && N <= (int)blockDim.x) ? build_walk_masked(prow, N, K, tv)
+                                                        : build_walk(prow, N, K, tv);
+    }
+    int32_t* pl = plan + (size_t)b * stride;
+    const int cnt = warp_kind ? 128 : 4 * N;
+    if (ok)
+        for (int i = tid; i < cnt; i += blockDim.x)
+            pl[kPlanHeader + i] = tsm[i];
+    if (tid == 0) {
+        pl[0] = sig;
+        pl[1] = ok ? 1 : 0;
+        pl[2] = N;
+        pl[3] = 0;
+        if (!ok)
+            report_status(status, GDN_ERR_BAD_TREE);
+    }
+}
+
+}  // namespace
+}  // namespace verify
+
+cudaError_t launch_plan(const VerifyArgs& a, const PlanGeom& pg, int32_t* plan, cudaStream_t stream)
+{
+    const size_t smem = pg.warp_kind ? (size_t)kWarpTreeInts * 4
+                                     : (size_t)(kTreeArrays + kMaskScratch) * a.n_nodes * 4;
+    if (smem > 48 * 1024) {
+        const cudaError_t e = cudaFuncSetAttribute(verify::gdn_plan_kernel,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess)
+            return e;
+    }
+    return launch_pdl(verify::gdn_plan_kernel, dim3(a.batch), dim3(verify::kPlanThreads), smem, stream, a.parent,
+                      a.n_nodes, pg.slots, pg.warp_kind ? 1 : 0, pg.sig, plan, pg.stride, a.status);
 }
 
 }  // namespace gdn

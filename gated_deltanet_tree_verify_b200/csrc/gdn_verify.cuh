@@ -118,7 +118,15 @@ struct KParams {
     int total;           // varlen: nodes in the packed layout
     uint32_t raw_bytes;  // one node's record (k row | q row | v slice) in bytes
     uint32_t off_raw, off_desc, off_ab, off_slots, off_tree;
+    const int32_t* plan;  // optional: walks built by gdn_tree_plan (see kPlanHeader), else NULL
+    int plan_stride;      // int32 per sequence in the plan
+    int plan_sig;         // the signature the plan must carry
 };
+
+// A tree plan holds, per sequence, a header [signature, ok, N, 0] and then
+// the walk as the staged kernels keep it in shared memory: for trees of <= 32
+// nodes MaskTree's 128 ints, else TreeView's par | ord | meta | rstart.
+constexpr int kPlanHeader = 4;
 
 // The nodes of sequence b: n0 .. n0 + N - 1 of the node dimension (N = p.N
 // and n0 = b N, or from the varlen offsets).
@@ -1490,7 +1498,23 @@ __device__ __forceinline__ void staged_body(const KParams& p)
     // 3. the walk: warp 0 builds it for trees of <= 32 nodes; all threads for
     //    larger trees
     const TreeView tv(tsm, N);
-    if constexpr (TK == kTreeWarp) {
+    if ((TK == kTreeWarp || TK == kTreeSmem) && p.plan != nullptr) {
+        // the walk was built once for all layers: copy it (written before
+        // the preceding kernel started when the tree is read early)
+        const int32_t* pl = p.plan + (size_t)b * p.plan_stride;
+        const int cnt = TK == kTreeWarp ? 128 : 4 * N;
+        for (int i = 4 * tid; i < cnt; i += 4 * blockDim.x)
+            cp_async16(tsm + i, pl + kPlanHeader + i);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        const int sig = __ldg(pl), ok = __ldg(pl + 1), pn = __ldg(pl + 2);
+        if (sig != p.plan_sig || pn != N) {
+            bad = true;
+            if (tid == 0)
+                report_status(p.status, GDN_ERR_BAD_INPUT);
+        } else if (ok != 1) {
+            bad = true;
+        }
+    } else if constexpr (TK == kTreeWarp) {
         if (warp == 0 && !build_warp_walk(prow, N, p.slots, tsm))
             bad = true;
     } else if constexpr (TK == kTreeSmem) {
@@ -1696,6 +1720,22 @@ __global__ void __launch_bounds__((kSmallWarps + 1) * 32) gdn_verify_ring(const 
             }
         }
         ok = !__syncthreads_or(bad);
+    } else if (p.plan != nullptr) {
+        // the walk from the plan (see the staged kernel)
+        const int32_t* pl = p.plan + (size_t)b * p.plan_stride;
+        for (int i = 4 * tid; i < 4 * N; i += 4 * blockDim.x)
+            cp_async16(T.par + i, pl + kPlanHeader + i);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        const int sig = __ldg(pl), pok = __ldg(pl + 1), pn = __ldg(pl + 2);
+        if (sig != p.plan_sig || pn != N) {
+            if (tid == 0)
+                report_status(p.status, GDN_ERR_BAD_INPUT);
+            ok = false;
+        } else {
+            ok = pok == 1;
+        }
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        __syncthreads();
     } else {
         __syncthreads();
         ok = (N <= kMaskNodes && N <= (int)blockDim.x) ? build_walk_masked(p.parent + (size_t)sq.n0, N, p.slots, T)

@@ -109,6 +109,12 @@ def load_library() -> ctypes.CDLL:
     lib.gdn_build_tree.restype = ctypes.c_int
     lib.gdn_tree_compact.argtypes = [i32, i32, vp, i32, ctypes.c_size_t, vp, vp, vp, vp, i32, vp, vp, vp]
     lib.gdn_tree_compact.restype = ctypes.c_int
+    lib.gdn_tree_plan_bytes.argtypes = [dp]
+    lib.gdn_tree_plan_bytes.restype = ctypes.c_size_t
+    lib.gdn_tree_plan.argtypes = [dp, vp, vp, ctypes.c_size_t, vp]
+    lib.gdn_tree_plan.restype = ctypes.c_int
+    lib.gdn_tree_verify_planned.argtypes = [dp, vp, ctypes.c_size_t] + [vp] * 10
+    lib.gdn_tree_verify_planned.restype = ctypes.c_int
     lib.gdn_status_str.argtypes = [ctypes.c_int]
     lib.gdn_status_str.restype = ctypes.c_char_p
     lib.gdn_last_error_detail.argtypes = []
@@ -325,4 +331,32 @@ def gdn_tree_compact(src, parent_idx, accept_path, accept_len, dst, *, batch: in
                               int(row_bytes), _ptr(src, "src"), _ptr(parent_idx, "parent_idx"),
                               _ptr(accept_path, "accept_path"), _ptr(accept_len, "accept_len"),
                               int(max_path_len), _ptr(dst, "dst"), _ptr(status, "status"), _stream(stream))
+    return _check(rc, check)
+
+
+def gdn_tree_plan_bytes(desc: GdnTreeDesc) -> int:
+    return int(load_library().gdn_tree_plan_bytes(ctypes.byref(desc)))
+
+
+def _nbytes(t, given):
+    if given is not None:
+        return int(given)
+    return t.numel() * t.element_size() if isinstance(t, torch.Tensor) else 0
+
+
+def gdn_tree_plan(desc: GdnTreeDesc, parent_idx, plan, plan_bytes: Optional[int] = None, stream=None,
+                  check: bool = True) -> int:
+    """Calls gdn_tree_plan (see include/gdntree.h)."""
+    rc = load_library().gdn_tree_plan(ctypes.byref(desc), _ptr(parent_idx, "parent_idx"), _ptr(plan, "plan"),
+                                      _nbytes(plan, plan_bytes), _stream(stream))
+    return _check(rc, check)
+
+
+def gdn_tree_verify_planned(desc: GdnTreeDesc, plan, q, k, v, g, beta, parent_idx, state_in, out, node_states,
+                            plan_bytes: Optional[int] = None, stream=None, check: bool = True) -> int:
+    """Calls gdn_tree_verify_planned (see include/gdntree.h)."""
+    rc = load_library().gdn_tree_verify_planned(
+        ctypes.byref(desc), _ptr(plan, "plan"), _nbytes(plan, plan_bytes), _ptr(q, "q"), _ptr(k, "k"),
+        _ptr(v, "v"), _ptr(g, "g"), _ptr(beta, "beta"), _ptr(parent_idx, "parent_idx"),
+        _ptr(state_in, "state_in"), _ptr(out, "out"), _ptr(node_states, "node_states"), _stream(stream))
     return _check(rc, check)

@@ -335,6 +335,40 @@ gdn_status gdn_tree_compact(int32_t batch, int32_t n_nodes, const int32_t* cu_no
                             const int32_t* accept_path, const int32_t* accept_len, int32_t max_path_len,
                             void* dst, int32_t* status, cudaStream_t stream);
 
+/*
+ * Tree plans.  Every layer of a model verifies the same tree, and the walk
+ * the kernels take through it (a depth-first order, which nodes keep their
+ * state for later siblings, which re-derive it) depends only on the tree and
+ * the launch shape.  gdn_tree_plan builds it once per step (one CTA per
+ * sequence) into a caller-owned device buffer; gdn_tree_verify_planned then
+ * copies it instead of building it in every CTA of every layer.  A
+ * data-layout convenience of this library: the source pages describe no
+ * counterpart.
+ *
+ * gdn_tree_plan_bytes(desc): bytes of the plan for desc (the same desc as
+ *   the verify calls; B sequences x a stride that depends on N and the walk
+ *   kind), or 0 when the call's walk builds nothing (chains, and f32 trees,
+ *   which re-read branch parents in index order): the plan is then not
+ *   needed and not read.
+ * gdn_tree_plan(desc, parent_idx, plan, plan_bytes, stream): parent_idx as
+ *   for gdn_tree_verify; plan 16-byte aligned, plan_bytes >= the above.  A
+ *   malformed tree gets GDN_ERR_BAD_TREE through desc->status and is marked
+ *   so in the plan (the planned verify then writes nothing for it).
+ * gdn_tree_verify_planned(desc, plan, plan_bytes, ...): gdn_tree_verify's
+ *   arguments and results, with the walks taken from the plan, which must
+ *   come from gdn_tree_plan with the same desc, parent_idx and batch (a plan
+ *   built for another shape is reported as GDN_ERR_BAD_INPUT through
+ *   desc->status and nothing is written).  Bit-identical to gdn_tree_verify.
+ *   Not with GDN_FLAG_CHUNKED or varlen layouts.
+ */
+size_t gdn_tree_plan_bytes(const gdn_tree_desc* desc);
+gdn_status gdn_tree_plan(const gdn_tree_desc* desc, const int32_t* parent_idx, void* plan, size_t plan_bytes,
+                         cudaStream_t stream);
+gdn_status gdn_tree_verify_planned(const gdn_tree_desc* desc, const void* plan, size_t plan_bytes, const void* q,
+                                   const void* k, const void* v, const float* g, const float* beta,
+                                   const int32_t* parent_idx, const float* state_in, float* out,
+                                   void* node_states, cudaStream_t stream);
+
 /* Largest N the tree (non-chain) path takes. */
 #define GDN_MAX_TREE_NODES 1024
 

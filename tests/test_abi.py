@@ -282,3 +282,23 @@ def test_compact_host_checks(lib):
     assert call(dst=src + 4096) == gdn.GDN_ERR_INVALID_ARG       # overlaps src
     assert call(cu_nodes=cu, total_nodes=1) == gdn.GDN_ERR_INVALID_ARG  # fewer nodes than sequences
     assert call(cu_nodes=cu, total_nodes=47) == gdn.GDN_ERR_INVALID_ARG  # above batch * n_nodes
+
+
+def test_plan_bytes_and_host_checks(lib):
+    f16 = _desc(state_dtype=gdn.GDN_F16, batch=8, n_nodes=65)
+    need = gdn.gdn_tree_plan_bytes(f16)
+    assert need > 0 and need % 16 == 0
+    assert gdn.gdn_tree_plan_bytes(_desc(batch=8, n_nodes=65)) == 0            # f32 trees re-read parents
+    assert gdn.gdn_tree_plan_bytes(_desc(flags=gdn.GDN_FLAG_CHAIN, state_dtype=gdn.GDN_F16)) == 0
+    assert gdn.gdn_tree_plan_bytes(_desc(d_k=48)) == 0
+    par, plan = BASE, BASE + 4 * MB
+    assert gdn.gdn_tree_plan(f16, par, plan, need - 16, stream=0, check=False) == gdn.GDN_ERR_INVALID_ARG
+    assert gdn.gdn_tree_plan(f16, par, plan + 8, need, stream=0, check=False) == gdn.GDN_ERR_INVALID_ARG
+    assert gdn.gdn_tree_plan(f16, None, plan, need, stream=0, check=False) == gdn.GDN_ERR_INVALID_ARG
+    assert gdn.gdn_tree_plan(f16, par, par, need, stream=0, check=False) == gdn.GDN_ERR_INVALID_ARG  # overlap
+    # nothing to build: fine with no buffer at all
+    assert gdn.gdn_tree_plan(_desc(batch=8, n_nodes=65), par, None, 0, stream=0, check=False) == gdn.GDN_OK
+    q, k, v, g, beta, p_, sin, out, ns = _ptrs(9)
+    rc = gdn.gdn_tree_verify_planned(f16, plan, q, k, v, g, beta, p_, sin, out, ns, plan_bytes=need - 16,
+                                     stream=0, check=False)
+    assert rc == gdn.GDN_ERR_INVALID_ARG
