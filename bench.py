@@ -253,13 +253,25 @@ class Stack:
                                        n_v_heads=N_V_HEADS, d_k=D, d_v=D, scale=self.scale,
                                        qkv_dtype=gdn.GDN_BF16, state_dtype=sd,
                                        flags=gdn.GDN_FLAG_EARLY_TREE)
+        # Trees walked with stack slots (f16 states): the walk is planned once
+        # per step and read by all layers.
+        self.plan_bytes = gdn.gdn_tree_plan_bytes(self.desc)
+        self.plan = (torch.empty(self.plan_bytes // 4, dtype=torch.int32, device=device)
+                     if self.plan_bytes else None)
 
     def verify_all(self, stream=None):
         g = self.gdn
+        if self.plan is not None:
+            g.gdn_tree_plan(self.desc, self.parent, self.plan, self.plan_bytes, stream=stream)
         for layer, d in enumerate(self.dev):
-            g.gdn_tree_verify(self.desc if layer == 0 else self.desc_next, d["q"], d["k"], d["v"],
-                              d["g"], d["beta"], self.parent, d["state"], d["out"], d["ns"],
-                              stream=stream)
+            desc = self.desc if layer == 0 else self.desc_next
+            if self.plan is not None:
+                g.gdn_tree_verify_planned(desc, self.plan, d["q"], d["k"], d["v"], d["g"], d["beta"],
+                                          self.parent, d["state"], d["out"], d["ns"], plan_bytes=self.plan_bytes,
+                                          stream=stream)
+            else:
+                g.gdn_tree_verify(desc, d["q"], d["k"], d["v"], d["g"], d["beta"], self.parent, d["state"],
+                                  d["out"], d["ns"], stream=stream)
 
     def commit_all(self, stream=None):
         # one launch commits the accepted path on every layer
@@ -268,7 +280,7 @@ class Stack:
                                         [d["state"] for d in self.dev], stream=stream)
 
     def launches_per_step(self):
-        return self.layers + (self.layers + 63) // 64
+        return self.layers + (self.layers + 63) // 64 + (1 if self.plan is not None else 0)
 
 
 def stage(msg):
@@ -432,10 +444,18 @@ def run_e2e(stack, args, ws, device, stream):
                 in_ev[l].record(copy_s)
         stream.wait_stream(back_s)  # the previous step's outputs have been read
         stream.wait_event(tree_ev)
+        if stack.plan is not None:
+            gdn.gdn_tree_plan(stack.desc, stack.parent, stack.plan, stack.plan_bytes, stream=stream)
         for l, (d, v) in enumerate(zip(stack.dev, dev_views)):
             stream.wait_event(in_ev[l])
-            gdn.gdn_tree_verify(stack.desc if l == 0 else stack.desc_next, v["q"], v["k"], v["v"], v["g"],
-                                v["beta"], stack.parent, d["state"], d["out"], d["ns"], stream=stream)
+            desc = stack.desc if l == 0 else stack.desc_next
+            if stack.plan is not None:
+                gdn.gdn_tree_verify_planned(desc, stack.plan, v["q"], v["k"], v["v"], v["g"], v["beta"],
+                                            stack.parent, d["state"], d["out"], d["ns"],
+                                            plan_bytes=stack.plan_bytes, stream=stream)
+            else:
+                gdn.gdn_tree_verify(desc, v["q"], v["k"], v["v"], v["g"], v["beta"], stack.parent, d["state"],
+                                    d["out"], d["ns"], stream=stream)
             out_ev[l].record(stream)
         stack.commit_all(stream=stream)
         with torch.cuda.stream(back_s):

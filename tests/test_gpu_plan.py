@@ -31,12 +31,10 @@ def _outputs(B, N, Hv, tdt, fill=float("nan")):
 
 
 @pytest.mark.parametrize("B,N,sd,Hv", [
-    (1, 23, "f16", 12),     # small grid, tree of <= 32 nodes (warp-built walk, capped kernel)
     (32, 23, "f16", 48),    # large grid, warp-built walk, one stack slot
     (8, 65, "f16", 48),     # large grid, 8-warp CTAs, mask-built walk
-    (1, 65, "f16", 12),     # small grid, mask-built walk
-    (2, 200, "f16", 12),    # serial walk builder (> 128 nodes)
-    (1, 129, "f16", 48),    # ring kernel: builds its own walk, plan not read
+    (16, 200, "f16", 48),   # serial walk builder (> 128 nodes)
+    (8, 129, "f16", 48),    # ring kernel reading the plan
 ])
 def test_planned_equals_unplanned(B, N, sd, Hv):
     prob, d, tdt, desc, status = _setup(B, N, sd, seed=N + B, Hk=Hv // 3, Hv=Hv)
@@ -57,6 +55,20 @@ def test_planned_equals_unplanned(B, N, sd, Hv):
                        s2.view(torch.int16) if tdt == torch.float16 else s2.view(torch.int32))
 
 
+@pytest.mark.parametrize("B,N", [(1, 23), (2, 65)])
+def test_small_grids_need_no_plan(B, N):
+    # one row per lane: the walk is built while the previous layer runs
+    prob, d, tdt, desc, status = _setup(B, N, "f16", seed=5)
+    assert gdn.gdn_tree_plan_bytes(desc) == 0
+    o1, s1 = _outputs(B, N, 12, tdt)
+    o2, s2 = _outputs(B, N, 12, tdt)
+    gdn.gdn_tree_verify(desc, d["q"], d["k"], d["v"], d["g"], d["beta"], d["parent"], d["state_in"], o1, s1)
+    gdn.gdn_tree_verify_planned(desc, None, d["q"], d["k"], d["v"], d["g"], d["beta"], d["parent"],
+                                d["state_in"], o2, s2, plan_bytes=0)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(s1.view(torch.int16), s2.view(torch.int16))
+
+
 def test_plan_not_needed_for_f32_trees():
     prob, d, tdt, desc, status = _setup(2, 23, "f32", seed=3)
     assert gdn.gdn_tree_plan_bytes(desc) == 0
@@ -71,7 +83,7 @@ def test_plan_not_needed_for_f32_trees():
 
 @pytest.mark.parametrize("N", [23, 65])
 def test_plan_of_a_malformed_tree(N):
-    prob, d, tdt, desc, status = _setup(3, N, "f16", seed=7)
+    prob, d, tdt, desc, status = _setup(8, N, "f16", seed=7, Hk=16, Hv=48)
     par = d["parent"].clone()
     par[1, N - 1] = N - 1                     # sequence 1: a node that is its own parent
     plan = torch.empty(gdn.gdn_tree_plan_bytes(desc) // 4, dtype=torch.int32, device="cuda")
@@ -79,27 +91,27 @@ def test_plan_of_a_malformed_tree(N):
     torch.cuda.synchronize()
     assert int(status.item()) == gdn.GDN_ERR_BAD_TREE
     status.zero_()
-    o, s = _outputs(3, N, 12, tdt)
+    o, s = _outputs(8, N, 48, tdt)
     gdn.gdn_tree_verify_planned(desc, plan, d["q"], d["k"], d["v"], d["g"], d["beta"], par, d["state_in"], o, s)
-    o_ref, s_ref = _outputs(3, N, 12, tdt)
+    o_ref, s_ref = _outputs(8, N, 48, tdt)
     gdn.gdn_tree_verify(desc, d["q"], d["k"], d["v"], d["g"], d["beta"], par, d["state_in"], o_ref, s_ref)
     torch.cuda.synchronize()
     assert int(status.item()) == gdn.GDN_ERR_BAD_TREE
     assert torch.isnan(o[1]).all()            # nothing written for the bad sequence
-    for b in (0, 2):
+    for b in (0, 2, 7):
         assert torch.equal(o[b], o_ref[b])
 
 
 def test_plan_for_another_shape_is_rejected():
-    # a plan built at batch 32 (one stack slot) read by a batch-1 call (two
-    # slots): same size per sequence, other walk -> GDN_ERR_BAD_INPUT
-    _, d32, tdt, desc32, _ = _setup(32, 23, "f16", seed=9, Hk=16, Hv=48)
-    plan = torch.empty(gdn.gdn_tree_plan_bytes(desc32) // 4, dtype=torch.int32, device="cuda")
-    gdn.gdn_tree_plan(desc32, d32["parent"], plan)
-    prob, d, tdt, desc1, status = _setup(1, 23, "f16", seed=9, Hk=16, Hv=48)
-    assert gdn.gdn_tree_plan_bytes(desc1) <= plan.numel() * 4
-    o, s = _outputs(1, 23, 48, tdt)
-    gdn.gdn_tree_verify_planned(desc1, plan, d["q"], d["k"], d["v"], d["g"], d["beta"], d["parent"],
+    # a plan built for 65-node trees read by a 64-node call: the plan is
+    # large enough, its walks are not for these trees -> GDN_ERR_BAD_INPUT
+    _, d65, tdt, desc65, _ = _setup(8, 65, "f16", seed=9, Hk=16, Hv=48)
+    plan = torch.empty(gdn.gdn_tree_plan_bytes(desc65) // 4, dtype=torch.int32, device="cuda")
+    gdn.gdn_tree_plan(desc65, d65["parent"], plan)
+    prob, d, tdt, desc64, status = _setup(8, 64, "f16", seed=9, Hk=16, Hv=48)
+    assert 0 < gdn.gdn_tree_plan_bytes(desc64) <= plan.numel() * 4
+    o, s = _outputs(8, 64, 48, tdt)
+    gdn.gdn_tree_verify_planned(desc64, plan, d["q"], d["k"], d["v"], d["g"], d["beta"], d["parent"],
                                 d["state_in"], o, s)
     torch.cuda.synchronize()
     assert int(status.item()) == gdn.GDN_ERR_BAD_INPUT
