@@ -199,7 +199,7 @@ def make_problem(*, batch: int, n_nodes: int, n_k_heads: int, n_v_heads: int,
                  d_k: int, d_v: int, tree: str, seed: int, qkv_dtype: str = "bf16",
                  gate: str = "softplus", scale: Optional[float] = None,
                  accept: str = "leaf", top_k: int = 4, max_depth: int = 16,
-                 parents: Optional[np.ndarray] = None) -> Problem:
+                 parents: Optional[np.ndarray] = None, raw_gates: bool = False) -> Problem:
     """Draw one seeded problem.
 
     tree: "chain" | "random" | "ddtree" | "given" (then ``parents`` [B][N]).
@@ -207,6 +207,8 @@ def make_problem(*, batch: int, n_nodes: int, n_k_heads: int, n_v_heads: int,
       generator seeded with seed + b; the remaining tensors come from one
       generator seeded with ``seed`` (drawn after the trees).
     gate: "softplus" -> g = -softplus(N(0,1)); "uniform_a" -> g = ln U(0.5, 1).
+    raw_gates (with gate "softplus"): g and beta hold the N(0,1) draws
+      themselves, untransformed (the same draws as without it).
     accept: "leaf" -> root to a uniformly chosen leaf; "prefix" -> root to a
       uniformly chosen node on the chain (chains); "node" -> root to a
       uniformly chosen node; "root" -> the root alone (no tree walk, so it
@@ -233,14 +235,20 @@ def make_problem(*, batch: int, n_nodes: int, n_k_heads: int, n_v_heads: int,
     q = _l2n(torch.randn(batch, n_nodes, n_k_heads, d_k, generator=gen)).to(dt)
     k = _l2n(torch.randn(batch, n_nodes, n_k_heads, d_k, generator=gen)).to(dt)
     v = torch.randn(batch, n_nodes, n_v_heads, d_v, generator=gen).to(dt)
+    if raw_gates and gate != "softplus":
+        raise ValueError("raw_gates needs gate='softplus'")
     if gate == "softplus":
-        g = -torch.nn.functional.softplus(torch.randn(batch, n_nodes, n_v_heads, generator=gen))
+        g = torch.randn(batch, n_nodes, n_v_heads, generator=gen)
+        if not raw_gates:
+            g = -torch.nn.functional.softplus(g)
     elif gate == "uniform_a":
         a = 0.5 + 0.5 * torch.rand(batch, n_nodes, n_v_heads, generator=gen)
         g = torch.log(a)
     else:
         raise ValueError(gate)
-    beta = torch.sigmoid(torch.randn(batch, n_nodes, n_v_heads, generator=gen))
+    beta = torch.randn(batch, n_nodes, n_v_heads, generator=gen)
+    if not raw_gates:
+        beta = torch.sigmoid(beta)
     state_in = 0.1 * torch.randn(batch, n_v_heads, d_v, d_k, generator=gen)
     paths = []
     for b in range(batch):

@@ -54,6 +54,8 @@ def _load():
         lib.gdn_oracle_round_array.restype = None
         lib.gdn_oracle_l2norm_rows.argtypes = [dp, c_i64, c_int]
         lib.gdn_oracle_l2norm_rows.restype = None
+        lib.gdn_oracle_gates.argtypes = [dp, dp, dp, dp, c_i64]
+        lib.gdn_oracle_gates.restype = None
         lib.gdn_oracle_check_tree.argtypes = [c_int, ip]
         lib.gdn_oracle_check_tree.restype = c_int
         lib.gdn_oracle_check_path.argtypes = [c_int, ip, ip, c_int, c_int]
@@ -95,21 +97,35 @@ def l2norm_rows(x) -> np.ndarray:
     return y
 
 
+def gates(x, y) -> Tuple[np.ndarray, np.ndarray]:
+    """(g, beta) = (-softplus(x), sigmoid(y)) elementwise, in double
+    (gdn_oracle_gates)."""
+    x, y = _f64(x), _f64(y)
+    assert x.shape == y.shape
+    g, beta = np.empty_like(x), np.empty_like(y)
+    _load().gdn_oracle_gates(_dp(x), _dp(y), _dp(g), _dp(beta), x.size)
+    return g, beta
+
+
 def verify(q, k, v, g, beta, parent, state_in, scale: float, state_dtype: str = "f32",
-           want_exact: bool = False, nthreads: int = 1, qk_l2norm: bool = False
-           ) -> Tuple[np.ndarray, np.ndarray, Optional[np.ndarray]]:
+           want_exact: bool = False, nthreads: int = 1, qk_l2norm: bool = False,
+           raw_gates: bool = False) -> Tuple[np.ndarray, np.ndarray, Optional[np.ndarray]]:
     """Run the tree recurrence.  Returns (out, persisted_states, exact_states).
 
     Shapes as in gdn_oracle.c.  ``persisted_states`` holds each node's state
     rounded to ``state_dtype`` (as float64 values); ``exact_states`` (only if
     ``want_exact``) holds the unrounded float64 states.  With ``qk_l2norm``
     q and k are L2-normalised per (node, head) first (the preparation the
-    library's GDN_FLAG_QK_L2NORM fuses).  Raises OracleError on a bad tree or
-    bad arguments.
+    library's GDN_FLAG_QK_L2NORM fuses).  With ``raw_gates`` g and beta hold
+    the pre-activations x and y, and the recurrence runs on g = -softplus(x),
+    beta = sigmoid(y) (``gates``; the library's GDN_FLAG_GATES).  Raises
+    OracleError on a bad tree or bad arguments.
     """
     lib = _load()
     if qk_l2norm:
         q, k = l2norm_rows(q), l2norm_rows(k)
+    if raw_gates:
+        g, beta = gates(g, beta)
     q, k, v, g, beta, state_in = map(_f64, (q, k, v, g, beta, state_in))
     parent = _i32(parent)
     B, N, Hk, dk = q.shape
@@ -198,11 +214,11 @@ def check_path(parent_row, path_row, length: int) -> int:
 
 
 def verify_problem(prob, state_dtype: str = "f32", want_exact: bool = False, nthreads: int = 1,
-                   qk_l2norm: bool = False):
+                   qk_l2norm: bool = False, raw_gates: bool = False):
     """Convenience: run ``verify`` on a gdn_inputs.Problem."""
     return verify(prob.q, prob.k, prob.v, prob.g, prob.beta, prob.parent, prob.state_in,
                   prob.scale, state_dtype=state_dtype, want_exact=want_exact, nthreads=nthreads,
-                  qk_l2norm=qk_l2norm)
+                  qk_l2norm=qk_l2norm, raw_gates=raw_gates)
 
 
 def verify_pair(prob, b: int, h: int, state_dtype: str = "f32", want_exact: bool = False):

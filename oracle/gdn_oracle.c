@@ -30,7 +30,9 @@
  *
  * Pins: every function here is checked by tests against closed forms and
  * invariants (identity, reset, delta-rule write, linearity, GQA grouping,
- * path composition, a hand-worked example), never against itself.
+ * path composition, a hand-worked example; for the gate maps, their values
+ * at ln 3 and 0, the softplus and sigmoid symmetries and the limits), never
+ * against itself.
  *
  * Layouts, row-major with the last index contiguous:
  *   q, k        [B][N][H_k][d_k]
@@ -86,6 +88,27 @@ void gdn_oracle_l2norm_rows(double* x, int64_t n, int d)
         const double nrm = sqrt(ss);
         for (int j = 0; j < d; ++j)
             row[j] = row[j] / nrm;
+    }
+}
+
+/* The gate maps of the workloads' input recipe, in double: from raw
+ * pre-activations x and y, the decay's log g = -softplus(x) = -log(1 + e^x)
+ * and the write strength beta = sigmoid(y) = 1 / (1 + e^-y) (the library's
+ * GDN_FLAG_GATES applies them inside its verify kernels).  softplus is taken
+ * as max(x, 0) + log1p(e^-|x|) and sigmoid through e^-|y|, forms that
+ * neither overflow nor cancel: x = +inf gives g = -inf (a = 0, a reset),
+ * x = -inf gives g = 0 (a = 1); y = +-inf gives beta = 1 or 0; NaN stays NaN. */
+void gdn_oracle_gates(const double* x, const double* y, double* g, double* beta, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i) {
+        const double xi = x[i], yi = y[i];
+        g[i] = isnan(xi) ? xi : -(fmax(xi, 0.0) + log1p(exp(-fabs(xi))));
+        if (isnan(yi))
+            beta[i] = yi;
+        else if (yi >= 0.0)
+            beta[i] = 1.0 / (1.0 + exp(-yi));
+        else
+            beta[i] = exp(yi) / (1.0 + exp(yi));
     }
 }
 
