@@ -52,7 +52,7 @@ gdn_status check_desc(const gdn_tree_desc* d, bool need_qkv)
         return fail(GDN_ERR_INVALID_ARG, "batch, n_nodes or head counts out of range%s");
     if (d->n_v_heads % d->n_k_heads != 0)
         return fail(GDN_ERR_INVALID_ARG, "n_v_heads is not a multiple of n_k_heads%s");
-    if ((d->flags & ~63u) != 0)
+    if ((d->flags & ~127u) != 0)
         return fail(GDN_ERR_INVALID_ARG, "unknown flag bits%s");
     const bool dk_ok = d->d_k == 32 || d->d_k == 64 || d->d_k == 128;
     const bool dv_ok = d->d_v == 32 || d->d_v == 64 || d->d_v == 128;
@@ -197,7 +197,8 @@ gdn_status verify_impl(const gdn_tree_desc* desc, const int32_t* cu, int32_t tot
     a.cu_nodes = varlen ? cu : nullptr;
     a.total_nodes = varlen ? total : 0;
     if (d.flags & GDN_FLAG_CHUNKED) {
-        if (varlen || workspace != nullptr || (d.flags & GDN_FLAG_QK_L2NORM) || !gdn::chunked_supported(a))
+        if (varlen || workspace != nullptr || (d.flags & (GDN_FLAG_QK_L2NORM | GDN_FLAG_GATES)) ||
+            !gdn::chunked_supported(a))
             return fail(GDN_ERR_UNSUPPORTED,
                         "GDN_FLAG_CHUNKED needs CHAIN + PERSIST_LAST, bf16 q/k/v, d_k = 128, d_v %% 64 == 0%s");
         const size_t B = d.batch, N = d.n_nodes, Hk = d.n_k_heads, Hv = d.n_v_heads, dk = d.d_k, dv = d.d_v;

@@ -176,6 +176,7 @@ cudaError_t launch_verify(const VerifyArgs& a, const VerifyGeom& geom, cudaStrea
     kp.validate = (a.flags & GDN_FLAG_VALIDATE) ? 1 : 0;
     kp.early_tree = (a.flags & GDN_FLAG_EARLY_TREE) ? 1 : 0;
     kp.qk_norm = (a.flags & GDN_FLAG_QK_L2NORM) ? 1 : 0;
+    kp.gates = (a.flags & GDN_FLAG_GATES) ? 1 : 0;
     kp.ws = geom.gslots ? a.workspace : nullptr;
     kp.cu = a.cu_nodes;
     kp.total = a.total_nodes;

@@ -93,9 +93,24 @@ __device__ __forceinline__ int meta_src(int m) { return (m >> 16) & 7; }
 __device__ __forceinline__ int meta_save(int m) { return ((m >> 19) & 31) - 1; }
 __device__ __forceinline__ int meta_load(int m) { return (m >> 24) & 31; }
 
-// The decay gate a = exp(g), compiled once so that every caller gets
-// identical bits.
-static __device__ __noinline__ float gdn_gate(float g) { return expf(g); }
+// A node's decay a and write strength beta from its g and beta inputs,
+// compiled once so that every caller gets identical bits: a = exp(g).  With
+// raw gates (GDN_FLAG_GATES) g and beta hold x and y with g = -softplus(x)
+// and beta = sigmoid(y), so a = exp(-softplus(x)) = 1 / (1 + e^x) and
+// beta = 1 / (1 + e^-y) (x = +inf gives a = 0, a reset).
+static __device__ __noinline__ float2 gdn_gates(float g, float beta, int raw)
+{
+    if (raw)
+        return make_float2(__fdiv_rn(1.f, __fadd_rn(1.f, expf(g))), __fdiv_rn(1.f, __fadd_rn(1.f, expf(-beta))));
+    return make_float2(expf(g), beta);
+}
+
+__device__ __forceinline__ void gate_scalars(float g, float beta, int raw, float& a, float& be)
+{
+    const float2 r = gdn_gates(g, beta, raw);
+    a = r.x;
+    be = r.y;
+}
 
 struct KParams {
     const void* q;
@@ -113,6 +128,7 @@ struct KParams {
     int rows, warps, slots;
     int persist_last, validate, early_tree;
     int qk_norm;         // GDN_FLAG_QK_L2NORM: k and q normalised per node inside the kernel
+    int gates;           // GDN_FLAG_GATES: g and beta are raw (gate_scalars)
     float* ws;           // global stack slots (kTreeGlobal kinds): slots x rows x d_k per CTA
     const int32_t* cu;   // varlen: [B + 1] node offsets of the packed layout (N: the most per sequence)
     int total;           // varlen: nodes in the packed layout
@@ -1333,7 +1349,8 @@ __device__ __forceinline__ float* cta_slots(const KParams& p, float* slotbuf)
 // and writes each position's descriptor with k . q of its node.
 template <int DK, int LR, typename QT, class Tree>
 __device__ __forceinline__ void write_descs(const Tree& tree, const unsigned char* raw, uint32_t raw_bytes,
-                                            float* ab, PosDesc* desc, int N, int qk_norm, float scale)
+                                            float* ab, PosDesc* desc, int N, int qk_norm, int gates,
+                                            float scale)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
     const int sub = lane & 7;
@@ -1350,9 +1367,9 @@ __device__ __forceinline__ void write_descs(const Tree& tree, const unsigned cha
             rq = inv_norm(node_dot8<DK, LR>(rrec, sub, DK, DK));
         }
         if (sub == 0 && valid) {
-            const float a = gdn_gate(ab[n]);
-            float bp, ap;
-            node_scalars(a, ab[N + n], rk, bp, ap);
+            float a, be, bp, ap;
+            gate_scalars(ab[n], ab[N + n], gates, a, be);
+            node_scalars(a, be, rk, bp, ap);
             ab[n] = a;
             ab[N + n] = bp;
             if (qk_norm) {
@@ -1374,7 +1391,7 @@ __device__ __forceinline__ void staged_finish(StateT<C, RL>& S, const KParams& p
                                               const LaneMap<DK, C, RL>& L)
 {
     constexpr int LR = LaneMap<DK, C, RL>::LR;
-    write_descs<DK, LR, QT>(tree, raw, p.raw_bytes, ab, desc, sq.N, p.qk_norm, p.scale);
+    write_descs<DK, LR, QT>(tree, raw, p.raw_bytes, ab, desc, sq.N, p.qk_norm, p.gates, p.scale);
     __syncthreads();
     const uint32_t rec_elems = p.raw_bytes / (uint32_t)sizeof(QT);
     StagedCtx<DK, C, RL, QT> ctx{reinterpret_cast<const QT*>(raw), desc, ab, rec_elems, sq.N, p.qk_norm, L};
@@ -1585,6 +1602,7 @@ struct GlobalFetch {
     const float* rkn;  // qk_norm: 1 / |k| per node (written by the producer), else NULL
     int Hk, Hv, dv, hk, h, row0;
     LaneMap<DK, C, RL> L;
+    int gates;
     __device__ __forceinline__ void operator()(int y, float2 (&k2)[4 * C], float (&vr)[RL], float& a,
                                                float& ar, float& be) const
     {
@@ -1602,8 +1620,9 @@ struct GlobalFetch {
         for (int r = 0; r < RL; ++r)
             vr[r] = Widen<QT>::load1(vg + (node * Hv + h) * dv + row0 + L.row + r * LM::RG);
         const size_t gi = node * Hv + h;
-        a = gdn_gate(__ldg(g + gi));
-        node_scalars(a, __ldg(beta + gi), rkn != nullptr ? rkn[y] : 1.f, be, ar);
+        float bt;
+        gate_scalars(__ldg(g + gi), __ldg(beta + gi), gates, a, bt);
+        node_scalars(a, bt, rkn != nullptr ? rkn[y] : 1.f, be, ar);
     }
 };
 
@@ -1786,7 +1805,7 @@ __global__ void __launch_bounds__((kSmallWarps + 1) * 32) gdn_verify_ring(const 
             }
             // lane i < cnt: position p0 + i's node, metadata and scalars
             int dn = 0, dm = 0, drs = -1, dpp = -1;
-            float da = 0.f, dbe = 0.f;
+            float da = 0.f, dbe = 0.f;  // g and beta here; a and beta once the records are stored
             if (lane < cnt) {
                 const int pos = p0 + lane;
                 if constexpr (CHAIN) {
@@ -1800,7 +1819,7 @@ __global__ void __launch_bounds__((kSmallWarps + 1) * 32) gdn_verify_ring(const 
                 dn = meta_node(dm);
                 dpp = CHAIN ? dn - 1 : T.par[dn];
                 const size_t gi = ((size_t)sq.n0 + dn) * p.Hv + h;
-                da = gdn_gate(__ldg(p.g + gi));
+                da = __ldg(p.g + gi);
                 dbe = __ldg(p.beta + gi);
             }
 #pragma unroll
@@ -1820,6 +1839,9 @@ __global__ void __launch_bounds__((kSmallWarps + 1) * 32) gdn_verify_ring(const 
                     *reinterpret_cast<uint4*>(base + (size_t)i * p.raw_bytes + off) = regs[t];
                 }
             }
+            // (the gate call comes after the record registers are dead)
+            if (lane < cnt)
+                gate_scalars(da, dbe, p.gates, da, dbe);
             __syncwarp();
             for (int i0 = 0; i0 < cnt; i0 += 4) {
                 const int gi = i0 + (lane >> 3);
@@ -1864,7 +1886,8 @@ __global__ void __launch_bounds__((kSmallWarps + 1) * 32) gdn_verify_ring(const 
         p.state_in + ((size_t)b * p.Hv + h) * p.dv * DK + (size_t)row0 * DK + L.tile_offset();
     StateT<C, RL> S;
     load_rows<DK, C, RL>(S, sin_lane);
-    const GlobalFetch<DK, C, RL, QT> gf{kg, vg, p.g, p.beta, (size_t)sq.n0, rkn, p.Hk, p.Hv, p.dv, hk, h, row0, L};
+    const GlobalFetch<DK, C, RL, QT> gf{kg, vg, p.g, p.beta, (size_t)sq.n0, rkn, p.Hk, p.Hv, p.dv, hk, h, row0, L,
+                                        p.gates};
     RingCtx<DK, C, RL, QT> ctx{full, empty, ring, p.raw_bytes, slot_bytes, desc_off, p.status, lane, gf};
     float* lane_slot = cta_slots<DK, TREE>(p, slotbuf) + 4 * threadIdx.x;
     if constexpr (CHAIN)

@@ -26,6 +26,7 @@ GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_BAD_TREE, GDN_ERR_BAD_
 # flags
 GDN_FLAG_CHAIN, GDN_FLAG_PERSIST_LAST, GDN_FLAG_VALIDATE, GDN_FLAG_EARLY_TREE, GDN_FLAG_CHUNKED = 1, 2, 4, 8, 16
 GDN_FLAG_QK_L2NORM = 32
+GDN_FLAG_GATES = 64
 GDN_MAX_TREE_NODES = 1024
 # gdn_build_desc.flags
 GDN_BUILD_CHAIN_SEED, GDN_BUILD_VALIDATE = 1, 2

@@ -102,7 +102,13 @@ enum {
      * row, x / |x| with no epsilon (a zero row gives inf/NaN), as the
      * workloads' input preparation does.  Folded into per-node scalars, so
      * the node loop does the same work.  Not with GDN_FLAG_CHUNKED. */
-    GDN_FLAG_QK_L2NORM = 32
+    GDN_FLAG_QK_L2NORM = 32,
+    /* g and beta are given raw: they hold the pre-activations x and y of the
+     * gates g = -softplus(x) = -log(1 + e^x) and beta = sigmoid(y), the
+     * workloads' gate recipe, and the kernels apply both (as
+     * a = exp(g) = 1 / (1 + e^x) and beta = 1 / (1 + e^-y), in f32, once per
+     * node).  x = +inf gives a = 0 (a reset).  Not with GDN_FLAG_CHUNKED. */
+    GDN_FLAG_GATES = 64
 };
 
 /* Problem description, shared by verify and commit. */

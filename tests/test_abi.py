@@ -80,14 +80,22 @@ def test_verify_batch_zero_is_a_noop(lib):
     (dict(n_nodes=gdn.GDN_MAX_TREE_NODES + 1), gdn.GDN_ERR_UNSUPPORTED),
     (dict(qkv_dtype=gdn.GDN_F16), gdn.GDN_ERR_UNSUPPORTED),
     (dict(state_dtype=gdn.GDN_BF16), gdn.GDN_ERR_UNSUPPORTED),
-    (dict(flags=64), gdn.GDN_ERR_INVALID_ARG),
+    (dict(flags=128), gdn.GDN_ERR_INVALID_ARG),     # no such flag
     (dict(flags=16 | 1 | 2 | 32), gdn.GDN_ERR_UNSUPPORTED),  # chunked + fused normalisation
+    (dict(flags=16 | 1 | 2 | 64), gdn.GDN_ERR_UNSUPPORTED),  # chunked + fused gates
     (dict(flags=16), gdn.GDN_ERR_UNSUPPORTED),      # chunked needs CHAIN + PERSIST_LAST
     (dict(flags=16 | 1 | 2, d_v=32), gdn.GDN_ERR_UNSUPPORTED),
     (dict(scale=float("nan")), gdn.GDN_ERR_INVALID_ARG),
 ])
 def test_verify_rejects_bad_desc(lib, kw, code):
     assert _verify(_desc(**kw)) == code
+
+
+def test_fused_gates_flag_passes_the_host_checks(lib):
+    assert gdn.GDN_FLAG_GATES == 64
+    for f in (gdn.GDN_FLAG_GATES, gdn.GDN_FLAG_GATES | gdn.GDN_FLAG_QK_L2NORM,
+              gdn.GDN_FLAG_GATES | gdn.GDN_FLAG_CHAIN | gdn.GDN_FLAG_PERSIST_LAST):
+        assert _verify(_desc(batch=0, flags=f)) == gdn.GDN_OK
 
 
 def test_verify_rejects_null_desc(lib):
