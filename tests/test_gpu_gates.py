@@ -115,3 +115,19 @@ def test_gates_flag_changes_results():
     a = run(prob, "f32", flags=GATES)
     b = run(prob, "f32")
     assert (a["out"] - b["out"]).abs().max() > 1e-3
+
+
+@pytest.mark.parametrize("sd", ["f32", "f16"])
+def test_gates_varlen(sd):
+    # packed trees of different sizes: each sequence against the oracle alone
+    from tests.test_gpu_varlen import _run_varlen
+    sizes, trees = [1, 9, 23, 40], ["chain", "random", "ddtree", "ddtree"]
+    seqs = [_problem(batch=1, n_nodes=n, n_k_heads=4, n_v_heads=12, d_k=128, d_v=128, tree=t, seed=90 + i)
+            for i, (n, t) in enumerate(zip(sizes, trees))]
+    vr = _run_varlen(seqs, sd, flags=GATES, commit=False)
+    assert vr["status"] == 0
+    for i, s in enumerate(seqs):
+        a, b = int(vr["cu"][i]), int(vr["cu"][i + 1])
+        out, _, ex = oracle.verify_problem(s, state_dtype=sd, want_exact=True, nthreads=8, raw_gates=True)
+        assert_out_close(vr["out"][a:b][None], out)
+        assert_states_close(vr["node_states"][a:b][None], ex, sd)
