@@ -138,6 +138,8 @@ typedef struct gdn_tree_desc {
  *   q, k        [B][N][H_k][d_k]    qkv_dtype (bf16 or f32), read-only
  *   v           [B][N][H_v][d_v]    qkv_dtype, read-only
  *   g, beta     [B][N][H_v]         f32, read-only; a_n = exp(g_n), g = -inf resets
+ *                                   (with GDN_FLAG_GATES the raw x, y of
+ *                                   g = -softplus(x), beta = sigmoid(y))
  *   parent_idx  [B][N]              int32, parent[b][0] = -1 and
  *                                   0 <= parent[b][n] < n; may be NULL only
  *                                   with GDN_FLAG_CHAIN and without VALIDATE
