@@ -253,8 +253,9 @@ class Stack:
                                        n_v_heads=N_V_HEADS, d_k=D, d_v=D, scale=self.scale,
                                        qkv_dtype=gdn.GDN_BF16, state_dtype=sd,
                                        flags=gdn.GDN_FLAG_EARLY_TREE)
-        # Trees walked with stack slots (f16 states): the walk is planned once
-        # per step and read by all layers.
+        # Trees walked with stack slots on large grids (f16 states, f32 trees
+        # above 32 nodes): the walk is planned once per step and read by all
+        # layers.
         self.plan_bytes = gdn.gdn_tree_plan_bytes(self.desc)
         self.plan = (torch.empty(self.plan_bytes // 4, dtype=torch.int32, device=device)
                      if self.plan_bytes else None)
@@ -808,6 +809,7 @@ def run_sweep(args):
                 points.append(dict(kind="tree", budget=budget, batch=batch, state_dtype=sd))
                 if sd == "f16":
                     points.append(dict(kind="tree", budget=budget, batch=batch, state_dtype=sd, ws=True))
+                if sd == "f16" or budget >= 32:
                     points.append(dict(kind="tree", budget=budget, batch=batch, state_dtype=sd, planned=True))
     for sd in ("f32", "f16"):
         points.append(dict(kind="chain16", budget=15, batch=1, state_dtype=sd))

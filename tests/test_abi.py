@@ -192,8 +192,12 @@ def test_verify_workspace_bytes(lib):
     assert gdn.gdn_tree_verify_workspace_bytes(_desc(state_dtype=gdn.GDN_F16, n_nodes=3)) == 48 * 128 * 128 * 4
     assert gdn.gdn_tree_verify_workspace_bytes(_desc(state_dtype=gdn.GDN_F16, batch=3, n_nodes=129)) == \
         3 * 48 * 128 * 128 * 4 * 4
-    # f32 trees re-read branch states from node_states; chains keep none
+    # f32 trees re-read branch states from node_states, except trees above 32
+    # nodes on large grids (two rows per lane), which keep slots; chains keep none
     assert gdn.gdn_tree_verify_workspace_bytes(_desc()) == 0
+    assert gdn.gdn_tree_verify_workspace_bytes(_desc(batch=8, n_nodes=32)) == 0
+    assert gdn.gdn_tree_verify_workspace_bytes(_desc(batch=1, n_nodes=65)) == 0
+    assert gdn.gdn_tree_verify_workspace_bytes(_desc(batch=8, n_nodes=65)) == 8 * 48 * 128 * 128 * 4 * 4
     assert gdn.gdn_tree_verify_workspace_bytes(_desc(state_dtype=gdn.GDN_F16, flags=gdn.GDN_FLAG_CHAIN)) == 0
     assert gdn.gdn_tree_verify_workspace_bytes(_desc(flags=gdn.GDN_FLAG_PERSIST_LAST)) > 0
     assert gdn.gdn_tree_verify_workspace_bytes(_desc(d_k=48)) == 0
@@ -296,7 +300,8 @@ def test_plan_bytes_and_host_checks(lib):
     f16 = _desc(state_dtype=gdn.GDN_F16, batch=8, n_nodes=65)
     need = gdn.gdn_tree_plan_bytes(f16)
     assert need > 0 and need % 16 == 0
-    assert gdn.gdn_tree_plan_bytes(_desc(batch=8, n_nodes=65)) == 0            # f32 trees re-read parents
+    assert gdn.gdn_tree_plan_bytes(_desc(batch=8, n_nodes=23)) == 0            # f32 trees re-read parents
+    assert gdn.gdn_tree_plan_bytes(_desc(batch=8, n_nodes=65)) > 0             # ... except large ones on large grids
     assert gdn.gdn_tree_plan_bytes(_desc(flags=gdn.GDN_FLAG_CHAIN, state_dtype=gdn.GDN_F16)) == 0
     assert gdn.gdn_tree_plan_bytes(_desc(d_k=48)) == 0
     par, plan = BASE, BASE + 4 * MB
@@ -305,7 +310,7 @@ def test_plan_bytes_and_host_checks(lib):
     assert gdn.gdn_tree_plan(f16, None, plan, need, stream=0, check=False) == gdn.GDN_ERR_INVALID_ARG
     assert gdn.gdn_tree_plan(f16, par, par, need, stream=0, check=False) == gdn.GDN_ERR_INVALID_ARG  # overlap
     # nothing to build: fine with no buffer at all
-    assert gdn.gdn_tree_plan(_desc(batch=8, n_nodes=65), par, None, 0, stream=0, check=False) == gdn.GDN_OK
+    assert gdn.gdn_tree_plan(_desc(batch=8, n_nodes=23), par, None, 0, stream=0, check=False) == gdn.GDN_OK
     q, k, v, g, beta, p_, sin, out, ns = _ptrs(9)
     rc = gdn.gdn_tree_verify_planned(f16, plan, q, k, v, g, beta, p_, sin, out, ns, plan_bytes=need - 16,
                                      stream=0, check=False)
