@@ -70,10 +70,11 @@ VerifyGeom verify_geometry(const VerifyArgs& a, bool use_workspace)
     // branch's parent state from node_states and walk in index order.  On
     // large grids, trees above 32 nodes walk depth first with shared-memory
     // slots instead (measured 4-13 % faster at batch 8 and 32, budgets 32 to
-    // 128); at one row per lane re-reading is faster at most budgets.  Both
-    // give identical bits.
+    // 128); at one row per lane re-reading is faster at most budgets, and so
+    // it is for packed trees of mixed sizes, whose shared memory is sized
+    // for the largest.  Both give identical bits.
     g.reload = !chain && a.state_dtype == GDN_F32 && !persist_last &&
-               !(g.rows_per_lane == 2 && a.n_nodes > 32);
+               !(g.rows_per_lane == 2 && a.n_nodes > 32 && a.cu_nodes == nullptr);
     if (chain || g.reload) {
         g.slots = 0;
     } else {

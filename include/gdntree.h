@@ -169,8 +169,8 @@ gdn_status gdn_tree_verify(const gdn_tree_desc* desc, const void* q, const void*
  *
  * A tree walk keeps the f32 states of branching nodes until their later
  * children run: with state_dtype f16, with GDN_FLAG_PERSIST_LAST, and with
- * f32 trees above 32 nodes on large grids (elsewhere an f32 walk re-reads
- * parent states from node_states and needs no workspace).  Without a
+ * f32 trees above 32 nodes on large grids, not packed (elsewhere an f32 walk
+ * re-reads parent states from node_states and needs no workspace).  Without a
  * workspace they live in shared memory, which caps the resident CTAs per SM
  * for trees above ~32 nodes; with one they live in global memory (mostly
  * L2), each loaded one node ahead of its use.  Results are bit-identical
