@@ -357,8 +357,9 @@ gdn_status gdn_tree_compact(int32_t batch, int32_t n_nodes, const int32_t* cu_no
  *
  * gdn_tree_plan_bytes(desc): bytes of the plan for desc (the same desc as
  *   the verify calls; B sequences x a stride that depends on N and the walk
- *   kind), or 0 when the call does not read one: chains and f32 trees (which
- *   re-read branch parents in index order) build no walk, and small grids
+ *   kind), or 0 when the call does not read one: chains and f32 trees of
+ *   at most 32 nodes (which re-read branch parents in index order, as f32
+ *   trees do on small grids) build no walk, and small grids
  *   (batch x heads too small for two rows per lane) build it while the
  *   previous layer still runs (GDN_FLAG_EARLY_TREE), where it costs nothing.
  * gdn_tree_plan(desc, parent_idx, plan, plan_bytes, stream): parent_idx as
