@@ -12,6 +12,7 @@ import subprocess
 import pytest
 
 import oracle
+from tests import test_oracle_gates as gate_pins
 from tests import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "gdn_oracle.c")
@@ -42,6 +43,13 @@ MUTANTS = {
                           "accept_path[(size_t)b * max_path_len + (accept_len[b] > 1 ? accept_len[b] - 2 : 0)]"),
     "path_link_unchecked": ("if (parent[path[i]] != path[i - 1])", "if (0)"),
     "tree_order_unchecked": ("if (parent[n] < 0 || parent[n] >= n)", "if (parent[n] < 0 || parent[n] >= n_nodes)"),
+    # the gate maps g = -softplus(x), beta = sigmoid(y)
+    "softplus_sign": ("g[i] = isnan(xi) ? xi : -(fmax(xi, 0.0) + log1p(exp(-fabs(xi))));",
+                      "g[i] = isnan(xi) ? xi : (fmax(xi, 0.0) + log1p(exp(-fabs(xi))));"),
+    "softplus_max_term_dropped": ("-(fmax(xi, 0.0) + log1p(exp(-fabs(xi))))", "-(log1p(exp(-fabs(xi))))"),
+    "sigmoid_sign_positive_branch": ("beta[i] = 1.0 / (1.0 + exp(-yi));", "beta[i] = 1.0 / (1.0 + exp(yi));"),
+    "sigmoid_negative_branch_flipped": ("beta[i] = exp(yi) / (1.0 + exp(yi));", "beta[i] = 1.0 / (1.0 + exp(yi));"),
+    "gate_inputs_swapped": ("const double xi = x[i], yi = y[i];", "const double xi = y[i], yi = x[i];"),
 }
 
 PINS = [
@@ -62,6 +70,10 @@ PINS = [
     pins.test_bad_trees_rejected,
     pins.test_bad_paths_rejected,
     pins.test_hand_worked_example_d2,
+    gate_pins.test_gate_values_at_closed_forms,
+    gate_pins.test_gate_symmetries,
+    gate_pins.test_gate_limits,
+    gate_pins.test_verify_raw_gates_wiring,
 ]
 
 
@@ -84,7 +96,7 @@ def test_pins_catch_mutant(name, tmp_path, monkeypatch):
     real = oracle._load()
     mut = ctypes.CDLL(lib_path)
     for fn in ("gdn_oracle_verify", "gdn_oracle_commit", "gdn_oracle_round", "gdn_oracle_round_array",
-               "gdn_oracle_check_tree", "gdn_oracle_check_path"):
+               "gdn_oracle_check_tree", "gdn_oracle_check_path", "gdn_oracle_gates", "gdn_oracle_l2norm_rows"):
         getattr(mut, fn).argtypes = getattr(real, fn).argtypes
         getattr(mut, fn).restype = getattr(real, fn).restype
     monkeypatch.setattr(oracle, "_lib", mut)
