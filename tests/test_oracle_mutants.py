@@ -43,6 +43,9 @@ MUTANTS = {
                           "accept_path[(size_t)b * max_path_len + (accept_len[b] > 1 ? accept_len[b] - 2 : 0)]"),
     "path_link_unchecked": ("if (parent[path[i]] != path[i - 1])", "if (0)"),
     "tree_order_unchecked": ("if (parent[n] < 0 || parent[n] >= n)", "if (parent[n] < 0 || parent[n] >= n_nodes)"),
+    # the q/k L2 normalisation
+    "l2norm_without_sqrt": ("const double nrm = sqrt(ss);", "const double nrm = ss;"),
+    "l2norm_sums_magnitudes": ("ss += row[j] * row[j];", "ss += fabs(row[j]);"),
     # the gate maps g = -softplus(x), beta = sigmoid(y)
     "softplus_sign": ("g[i] = isnan(xi) ? xi : -(fmax(xi, 0.0) + log1p(exp(-fabs(xi))));",
                       "g[i] = isnan(xi) ? xi : (fmax(xi, 0.0) + log1p(exp(-fabs(xi))));"),
@@ -70,6 +73,8 @@ PINS = [
     pins.test_bad_trees_rejected,
     pins.test_bad_paths_rejected,
     pins.test_hand_worked_example_d2,
+    pins.test_l2norm_worked_example,
+    pins.test_l2norm_invariants,
     gate_pins.test_gate_values_at_closed_forms,
     gate_pins.test_gate_symmetries,
     gate_pins.test_gate_limits,
