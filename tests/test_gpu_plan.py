@@ -1,7 +1,6 @@
 """gdn_tree_plan + gdn_tree_verify_planned: bit-identical to gdn_tree_verify
 (which the parity tests hold to the oracle) for every walk kind that builds
 a walk, with malformed trees and mismatched plans reported."""
-import numpy as np
 import pytest
 import torch
 
