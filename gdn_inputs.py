@@ -20,7 +20,9 @@ no epsilon; v ~ N(0,1); g = -softplus(N(0,1)) (or g = ln U(0.5, 1) for the long
 chain); beta = sigmoid(N(0,1)); state_in ~ N(0, 0.1^2).  q/k/v are then rounded
 to the requested input dtype (bf16 or f32); the rounded values are what both
 sides see.  Draw order from one ``torch.Generator``: tree, q, k, v, g, beta,
-state_in, accept path.
+state_in, accept path.  With ``raw_gates`` the g and beta draws are returned
+as drawn (the N(0,1) pre-activations), for callers that apply the gate maps
+themselves.
 """
 from __future__ import annotations
 
