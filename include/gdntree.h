@@ -225,8 +225,11 @@ gdn_status gdn_tree_verify_varlen(const gdn_tree_desc* desc, const int32_t* cu_n
 
 /* Workspace bytes gdn_tree_verify_ws needs for a desc: B * H_v * d_v * d_k *
  * 4 * (stack slots, at most 4) for walks that keep branch states, 0 for
- * chains, f32 trees (their branch states are re-read from node_states) and
- * invalid descs.  Independent of the buffers' addresses. */
+ * chains, f32 trees whose walk re-reads branch states from node_states (32
+ * nodes or fewer, or small grids) and invalid descs.  Computed from the desc
+ * alone, so for packed trees (whose f32 walks always re-read) it can ask for
+ * a workspace the call then leaves unused.  Independent of the buffers'
+ * addresses. */
 size_t gdn_tree_verify_workspace_bytes(const gdn_tree_desc* desc);
 
 /*
