@@ -16,8 +16,9 @@
  * GreenGames post, "TL;DR" and "Why the experiment exists"; applied per tree
  * node as in the DDTree row of the dflash-caddtree-integrations README, "What's
  * in here").  The root takes S_p = state_in.  Every node's state is persisted
- * from inside the verify kernel (the persist-write kernel of the GreenGames
- * post, "Key wins") in fp32 or f16 (its "f16 intermediate cache"), so that the
+ * from inside the verify kernel (the GreenGames post, "Key wins": the kernel
+ * that computes a state also writes it) in fp32 or f16 (the post's f16 cache
+ * of intermediate states), so that the
  * accepted root-to-leaf path is committed by a copy, without re-running it.
  *
  * Conventions shared by every entry point:

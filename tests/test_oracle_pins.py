@@ -3,8 +3,9 @@
 None of these re-types the oracle's formula.  Each checks a property that the
 gated delta rule (Gated DeltaNet recurrence; named as ggml_gated_delta_net in
 the GreenGames post, "TL;DR") and the tree/commit contract (DDTree row of the
-dflash-caddtree-integrations README, "What's in here": W=1 byte-identical,
-branch-state invariants; GreenGames "Key wins": persist-write, f16 cache) fix,
+dflash-caddtree-integrations README, "What's in here": a width-1 tree equals
+the chain exactly, branch states are kept consistent; GreenGames "Key wins":
+states written by the kernel that computes them, in f16 or f32) fix,
 chosen so that a dropped term, a wrong sign or index, or a transposed operand
 fails at least one of them.
 """
