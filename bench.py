@@ -37,12 +37,14 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from gdn_inputs import draft_logprobs, make_problem  # noqa: E402
+from gdn_inputs import (ddtree_like_tree, draft_logprobs, make_device_inputs, make_problem,  # noqa: E402
+                        root_path)
 
 METRIC = "GDN tree-verify nodes/s and achieved HBM GB/s (% of B200 peak) at budget 22"
 UNIT = "tree-nodes/s"
 N_K_HEADS, N_V_HEADS, D = 16, 48, 128
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0  # the B200 HBM3e figure the target is stated against (context beside the measured peak)
 
 
 # ----------------------------------------------------------------------------
@@ -283,6 +285,20 @@ class Stack:
         return self.layers + (self.layers + 63) // 64 + (1 if self.plan is not None else 0)
 
 
+def workload_config(args, ws):
+    """The workload's config keys, shared by both arms of the benchmark."""
+    n_nodes = args.budget + 1
+    step_bytes = (verify_bytes(args.batch, n_nodes, args.state_dtype) + commit_bytes(args.batch, args.state_dtype)) \
+        * args.layers
+    return {"workload": f"ddtree_budget{args.budget}_{args.layers}layers_b{args.batch}",
+            "batch_per_rank": args.batch, "global_batch": args.batch * ws, "budget": args.budget,
+            "n_nodes": n_nodes, "layers": args.layers, "n_k_heads": N_K_HEADS, "n_v_heads": N_V_HEADS,
+            "d_k": D, "d_v": D, "qkv": "bf16", "state_dtype": args.state_dtype,
+            "parallelism": f"replicas{ws}",
+            "l2": "inputs larger than L2: each step touches %.2f GB of distinct per-layer buffers"
+                  % (step_bytes / 1e9)}
+
+
 def stage(msg):
     print(f"[bench] {time.strftime('%H:%M:%S')} {msg}", file=sys.stderr, flush=True)
 
@@ -332,14 +348,21 @@ def run_ours(args, ws, rank, local):
     torch.cuda.synchronize()
     stage("timed region")
     sampler = ClockSampler(local)
+    nvtx = torch.cuda.nvtx
     with sampler:
+        nvtx.range_push("timed steps")
         for i in range(K):
             ev[i][0].record(stream)
+            nvtx.range_push("verify x%d" % args.layers)
             gv.replay()
+            nvtx.range_pop()
             ev[i][1].record(stream)
+            nvtx.range_push("commit x%d" % args.layers)
             gc.replay()
+            nvtx.range_pop()
             ev[i][2].record(stream)
         torch.cuda.synchronize()
+        nvtx.range_pop()
     barrier(ws)
     verify_ms = sum(e[0].elapsed_time(e[1]) for e in ev)
     commit_ms = sum(e[1].elapsed_time(e[2]) for e in ev)
@@ -361,20 +384,16 @@ def run_ours(args, ws, rank, local):
     # step's inputs go host->device from pinned memory, the 48 layers' outputs
     # come back device->host; the recurrent state stays resident on the GPU.
     stage("end-to-end leg")
+    torch.cuda.nvtx.range_push("end-to-end leg")
     e2e = run_e2e(stack, args, ws, device, stream)
+    torch.cuda.nvtx.range_pop()
 
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": K, "warmup": args.warmup,
         "ms_per_step": max_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic",
-        "config": {"workload": f"ddtree_budget{args.budget}_{args.layers}layers_b{args.batch}",
-                   "batch_per_rank": args.batch, "global_batch": args.batch * ws,
-                   "budget": args.budget, "n_nodes": stack.n_nodes, "layers": args.layers,
-                   "n_k_heads": N_K_HEADS, "n_v_heads": N_V_HEADS, "d_k": D, "d_v": D, "qkv": "bf16",
-                   "state_dtype": args.state_dtype, "parallelism": f"replicas{ws}",
-                   "l2": "inputs larger than L2: each step touches %.2f GB of distinct per-layer buffers"
-                         % ((vb + cb) * args.layers / 1e9),
-                   "timing": "CUDA graphs of 48 verify launches + 1 all-layer commit launch, CUDA events per step"},
+        "config": workload_config(args, ws),
+        "timing": "CUDA graphs of 48 verify launches + 1 all-layer commit launch, CUDA events per step",
         "node_layers_per_s": value * args.layers,
         "verify_gbps": achieved,
         "commit_gbps": cb / avg_commit_s / 1e9,
@@ -383,11 +402,19 @@ def run_ours(args, ws, rank, local):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "kernel": "gdn_verify_kernel", "peak_source": f"{peak_kind} copy bandwidth",
-                     "algorithmic_bytes_per_launch": vb},
+                     "algorithmic_bytes_per_launch": vb,
+                     "frac_of_nominal": achieved / NOMINAL_HBM_GBS,
+                     "nominal_peak": NOMINAL_HBM_GBS},
         "e2e": e2e,
         "gpu_launches": stack.launches_per_step() * K,
         "clocks": sampler.summary(),
     }
+    if not args.no_target:
+        # every rank runs the same points (replicas); rank 0 reports its own
+        stage("target points")
+        torch.cuda.nvtx.range_push("target points")
+        result["target"] = run_target(args, device, stream, local)
+        torch.cuda.nvtx.range_pop()
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         stage("cpu baseline (oracle)")
         result["cpu_baseline"] = cpu_baseline(args, stack)
@@ -396,6 +423,139 @@ def run_ours(args, ws, rank, local):
         gc.reset()
         dist.destroy_process_group()
     return result if rank == 0 else None
+
+
+# Points of the batched-tree target (>= 70 % of the HBM roofline at budget
+# >= 22 with batch >= 8, for f32 and f16 persisted states): (budget, batch,
+# persisted state dtype).
+TARGET_POINTS = ((22, 8, "f32"), (22, 8, "f16"), (32, 8, "f16"), (64, 8, "f16"), (128, 8, "f16"),
+                 (64, 32, "f16"), (128, 32, "f16"))
+TARGET_SET_BYTES = 24 << 30  # device memory for one point's distinct layer buffers
+
+
+def _target_point(budget, batch, state_dtype, *, layers, device, stream, local, seed, min_timed_s=0.25):
+    """One target point: the step's 48 verify launches in one CUDA graph (the
+    tree planned once per step, as in the headline step), each launch on its
+    own layer buffers; layers cycle through as many distinct buffer sets as
+    fit in TARGET_SET_BYTES (every set is several times the L2), then one
+    all-layer commit launch over the distinct sets.  Timed with CUDA events
+    over graph replays, with the SM clock sampled meanwhile."""
+    import gated_deltanet_tree_verify_b200 as gdn
+    n = budget + 1
+    tdt = torch.float32 if state_dtype == "f32" else torch.float16
+    sd = gdn.GDN_F32 if state_dtype == "f32" else gdn.GDN_F16
+    vb = verify_bytes(batch, n, state_dtype)
+    cb = commit_bytes(batch, state_dtype)
+    per_set = vb + 2 * batch * N_V_HEADS * D * D * 4
+    n_sets = max(2, min(layers, TARGET_SET_BYTES // per_set))
+    parent = np.stack([ddtree_like_tree(budget, torch.Generator().manual_seed(seed + b)) for b in range(batch)])
+    sets = []
+    for l in range(n_sets):
+        d = make_device_inputs(parent=parent, n_k_heads=N_K_HEADS, n_v_heads=N_V_HEADS, d_k=D, d_v=D,
+                               seed=seed * 1000 + l, device=device)
+        d["out"] = torch.empty(batch, n, N_V_HEADS, D, device=device)
+        d["ns"] = torch.empty(batch, n, N_V_HEADS, D, D, device=device, dtype=tdt)
+        sets.append(d)
+    par = sets[0]["parent"]
+    scale = D ** -0.5
+    desc = gdn.make_desc(batch=batch, n_nodes=n, n_k_heads=N_K_HEADS, n_v_heads=N_V_HEADS, d_k=D, d_v=D,
+                         scale=scale, qkv_dtype=gdn.GDN_BF16, state_dtype=sd)
+    desc_next = gdn.make_desc(batch=batch, n_nodes=n, n_k_heads=N_K_HEADS, n_v_heads=N_V_HEADS, d_k=D, d_v=D,
+                              scale=scale, qkv_dtype=gdn.GDN_BF16, state_dtype=sd, flags=gdn.GDN_FLAG_EARLY_TREE)
+    plan_bytes = gdn.gdn_tree_plan_bytes(desc)
+    plan = torch.empty(max(plan_bytes, 16) // 4, dtype=torch.int32, device=device) if plan_bytes else None
+    # accept the path to the last node taken (a leaf of a best-first tree)
+    paths = [root_path(parent[b], n - 1) for b in range(batch)]
+    max_len = max(len(pt) for pt in paths)
+    path = torch.tensor([pt + [-1] * (max_len - len(pt)) for pt in paths], dtype=torch.int32, device=device)
+    plen = torch.tensor([len(pt) for pt in paths], dtype=torch.int32, device=device)
+
+    def verify_step():
+        if plan is not None:
+            gdn.gdn_tree_plan(desc, par, plan, plan_bytes)
+        for l in range(layers):
+            d = sets[l % n_sets]
+            dd = desc if l == 0 else desc_next
+            if plan is not None:
+                gdn.gdn_tree_verify_planned(dd, plan, d["q"], d["k"], d["v"], d["g"], d["beta"], par,
+                                            d["state_in"], d["out"], d["ns"], plan_bytes=plan_bytes)
+            else:
+                gdn.gdn_tree_verify(dd, d["q"], d["k"], d["v"], d["g"], d["beta"], par, d["state_in"],
+                                    d["out"], d["ns"])
+
+    # the commit writes a separate state_out per set (the headline commits in
+    # place; here the inputs must stay for the next replay)
+    outs = [torch.empty(batch, N_V_HEADS, D, D, device=device) for _ in range(n_sets)]
+
+    def commit_step():
+        gdn.gdn_tree_commit_layers(desc, [d["ns"] for d in sets], par, path, plen, max_len, outs)
+
+    side = torch.cuda.Stream(device)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        verify_step()
+        commit_step()
+    stream.wait_stream(side)
+    torch.cuda.synchronize()
+    gv, gc = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gv):
+        verify_step()
+    with torch.cuda.graph(gc):
+        commit_step()
+    for _ in range(3):
+        gv.replay()
+        gc.replay()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    gv.replay()
+    torch.cuda.synchronize()
+    reps = max(3, min(200, int(min_timed_s / max(time.perf_counter() - t0, 1e-6))))
+    e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    sampler = ClockSampler(local, period_s=0.01)
+    with sampler:
+        e[0].record(stream)
+        for _ in range(reps):
+            gv.replay()
+        e[1].record(stream)
+        for _ in range(reps):
+            gc.replay()
+        e[2].record(stream)
+        torch.cuda.synchronize()
+    verify_s = e[0].elapsed_time(e[1]) / 1e3 / (reps * layers)
+    commit_s = e[1].elapsed_time(e[2]) / 1e3 / (reps * n_sets)
+    peak, peak_kind = hbm_peak()
+    achieved = vb / verify_s / 1e9
+    step_gbps = (vb + cb) / (verify_s + commit_s) / 1e9
+    point = {"budget": budget, "batch": batch, "n_nodes": n, "state_dtype": state_dtype, "layers": layers,
+             "distinct_layer_buffers": n_sets, "planned": plan is not None,
+             "verify_us_per_launch": verify_s * 1e6, "commit_us_per_layer": commit_s * 1e6,
+             "algorithmic_bytes_per_launch": vb, "achieved_gbps": achieved, "peak_gbps": peak,
+             "frac": achieved / peak, "frac_of_nominal": achieved / NOMINAL_HBM_GBS,
+             "step_frac": step_gbps / peak, "node_layers_per_s": batch * n / verify_s,
+             "reps": reps, "clocks": sampler.summary()}
+    del gv, gc
+    sets.clear()
+    outs.clear()
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return point
+
+
+def run_target(args, device, stream, local):
+    """The batched-tree target points (TARGET_POINTS), each a 48-layer step
+    of verify launches timed on its own; see _target_point."""
+    peak, peak_kind = hbm_peak()
+    points = []
+    for budget, batch, sd in TARGET_POINTS:
+        torch.cuda.nvtx.range_push(f"target budget {budget} batch {batch} {sd}")
+        points.append(_target_point(budget, batch, sd, layers=args.layers, device=device, stream=stream,
+                                    local=local, seed=args.seed + 101 * budget + batch))
+        torch.cuda.nvtx.range_pop()
+    return {"bar": 0.70, "bound": "hbm", "peak": peak, "peak_source": f"{peak_kind} copy bandwidth",
+            "nominal_peak": NOMINAL_HBM_GBS, "points": points,
+            "met": all(pt["frac"] >= 0.70 for pt in points),
+            "timing": "per point: CUDA graph of 48 verify launches (+ tree plan) replayed back to back, CUDA "
+                      "events around the replays; distinct buffer sets per layer, each larger than L2"}
 
 
 def run_e2e(stack, args, ws, device, stream):
@@ -520,49 +680,73 @@ def cpu_baseline(args, stack, budget_s=12.0):
 
 
 def run_reference(args, ws, rank):
-    """The oracle as the reference arm, on this host's cores.  Each step is
-    one layer's verify of the same workload: all 48 v-heads over every core
-    when K + W such steps end within a few minutes, else a bounded slice of
-    v-heads on one thread.  Scaled to tree-nodes/s through 48 layers."""
+    """The oracle as the reference arm, on this host's cores, on the same
+    workload and config as the CUDA arm.  A step is one whole 48-layer step
+    (every layer with its own inputs, all 48 v-heads over every core) when
+    K + W such steps end within about 150 s; otherwise each step is a bounded
+    sample of it (the same number of layers every step, or a slice of v-heads
+    of one layer on one thread), timed as it ran, and the throughput is
+    scaled to the whole step from the sampled fraction.  ``steps`` and
+    ``ms_per_step`` are always what was timed."""
     if rank != 0:
         return None
     import oracle
     oracle._load()
     nthreads = os.cpu_count() or 1
-    prob = make_problem(batch=args.batch, n_nodes=args.budget + 1, n_k_heads=N_K_HEADS, n_v_heads=N_V_HEADS,
-                        d_k=D, d_v=D, tree="ddtree", seed=args.seed, qkv_dtype="bf16", accept="leaf")
+    n_nodes = args.budget + 1
+    first = make_problem(batch=args.batch, n_nodes=n_nodes, n_k_heads=N_K_HEADS, n_v_heads=N_V_HEADS, d_k=D,
+                         d_v=D, tree="ddtree", seed=args.seed, qkv_dtype="bf16", accept="leaf")
+    probs = [first] + [make_problem(batch=args.batch, n_nodes=n_nodes, n_k_heads=N_K_HEADS, n_v_heads=N_V_HEADS,
+                                    d_k=D, d_v=D, tree="given", parents=first.parent.numpy(),
+                                    seed=args.seed * 1000 + layer, qkv_dtype="bf16", accept="root")
+                       for layer in range(1, args.layers)]
     total = args.steps + args.warmup
     budget_s = 150.0
-    t_layer = _oracle_layer_seconds(prob, nthreads, args.state_dtype)  # also pages the oracle in
-    if total * t_layer <= budget_s:
-        for _ in range(args.warmup):
-            _oracle_layer_seconds(prob, nthreads, args.state_dtype)
-        spent = sum(_oracle_layer_seconds(prob, nthreads, args.state_dtype) for _ in range(args.steps))
-        step_s = spent / args.steps * args.layers
-        cores = nthreads
-        sample = (f"one of {args.layers} layers per step, all 48 v-heads (batch {args.batch}, "
-                  f"{args.budget + 1} nodes) over {nthreads} threads, scaled to the full step")
+    t_layer = _oracle_layer_seconds(first, nthreads, args.state_dtype)  # also pages the oracle in
+    t_layer = min(t_layer, _oracle_layer_seconds(first, nthreads, args.state_dtype))
+    if total * t_layer * args.layers <= budget_s:
+        layers_per_step, heads, cores = args.layers, None, nthreads
+        fraction = 1.0
+        sample = (f"whole steps: all {args.layers} layers (own inputs per layer), all 48 v-heads, batch "
+                  f"{args.batch}, {n_nodes} nodes, over {nthreads} threads")
+    elif total * t_layer <= budget_s:
+        layers_per_step = max(1, min(args.layers, int(budget_s / (total * t_layer))))
+        heads, cores = None, nthreads
+        fraction = layers_per_step / args.layers
+        sample = (f"{layers_per_step} of {args.layers} layers per step (all 48 v-heads, batch {args.batch}, "
+                  f"{n_nodes} nodes) over {nthreads} threads; throughput scaled to the whole step")
     else:
-        t_head = _oracle_layer_seconds(prob, 1, args.state_dtype, heads=[0])
-        heads_per_step = max(1, min(N_V_HEADS, int(budget_s / max(total * t_head, 1e-6))))
-        for i in range(args.warmup):
-            _oracle_layer_seconds(prob, 1, args.state_dtype, heads=[i % N_V_HEADS])
-        spent = 0.0
-        for i in range(args.steps):
-            heads = [(i * heads_per_step + j) % N_V_HEADS for j in range(heads_per_step)]
-            spent += _oracle_layer_seconds(prob, 1, args.state_dtype, heads=heads)
-        step_s = spent / (args.steps * heads_per_step) * N_V_HEADS * args.layers
-        cores = 1
-        sample = (f"{heads_per_step} of 48 v-heads of one of {args.layers} layers per step "
-                  f"(batch {args.batch}, {args.budget + 1} nodes), single thread, scaled to the full step")
-    value = args.batch * (args.budget + 1) / step_s
+        t_head = _oracle_layer_seconds(first, 1, args.state_dtype, heads=[0])
+        n_heads = max(1, min(N_V_HEADS, int(budget_s / max(total * t_head, 1e-6))))
+        layers_per_step, heads, cores = 1, n_heads, 1
+        fraction = n_heads / (N_V_HEADS * args.layers)
+        sample = (f"{n_heads} of 48 v-heads of one of {args.layers} layers per step (batch {args.batch}, "
+                  f"{n_nodes} nodes), single thread; throughput scaled to the whole step")
+
+    def one_step(i):
+        t = 0.0
+        for j in range(layers_per_step):
+            prob = probs[(i * layers_per_step + j) % args.layers]
+            if heads is None:
+                t += _oracle_layer_seconds(prob, nthreads, args.state_dtype)
+            else:
+                t += _oracle_layer_seconds(prob, 1, args.state_dtype,
+                                           heads=[(i * heads + h) % N_V_HEADS for h in range(heads)])
+        return t
+
+    for i in range(args.warmup):
+        one_step(i)
+    spent = sum(one_step(args.warmup + i) for i in range(args.steps))
+    ms_per_step = spent / args.steps * 1e3
+    full_step_s = spent / args.steps / fraction
+    value = args.batch * n_nodes / full_step_s
     return {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-        "config": {"workload": f"ddtree_budget{args.budget}_{args.layers}layers_b{args.batch}",
-                   "batch_per_rank": args.batch, "budget": args.budget, "layers": args.layers,
-                   "state_dtype": args.state_dtype, "parallelism": "cpu"},
+        "config": workload_config(args, ws),
+        "timing": "host wall clock (perf_counter) around each oracle call",
+        "sample_fraction_of_step": fraction, "ms_per_full_step": full_step_s * 1e3,
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -898,6 +1082,8 @@ def main(argv=None):
     ap.add_argument("--seed", type=int, default=2)
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-target", action="store_true",
+                    help="skip the batched-tree target points (budget 22-128, batch 8 and 32, f32 and f16)")
     ap.add_argument("--sweep", action="store_true",
                     help="single-layer verify timings over budgets, batches, dtypes and the long chain "
                          "(one JSON line per point; not the benchmark line)")

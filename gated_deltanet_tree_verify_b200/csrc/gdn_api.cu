@@ -2,11 +2,11 @@
 // checks, then one kernel launch on the caller's stream.  See include/gdntree.h
 // for the contract of each call.
 
-#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include <cuda_runtime.h>
 
@@ -444,8 +444,54 @@ constexpr int kMaxStaticDevices = 64;
 // One buffer per device context, shared by every call in the process.
 __device__ __align__(256) unsigned char g_static_ws[kStaticWorkspaceBytes];
 
-// Device address of g_static_ws per device, looked up on first use there.
-std::atomic<void*> g_static_ws_addr[kMaxStaticDevices];
+// The device address of g_static_ws belongs to the context the module was
+// loaded in: a cudaDeviceReset, or another context made current through the
+// driver API, gives a new context with its own copy of the array.  So the
+// address is cached per device together with the unique id of the context it
+// was looked up in (cuCtxGetId ids are never reused within a process), and
+// looked up again whenever the current context differs.  The two driver
+// calls are resolved once through the runtime, so the library does not link
+// libcuda itself; without them the address is looked up on every call.
+using CtxGetCurrentFn = int (*)(void**);
+using CtxGetIdFn = int (*)(void*, unsigned long long*);
+
+struct StaticWsCache {
+    unsigned long long ctx_id;
+    void* addr;
+};
+
+std::mutex g_static_ws_lock;
+StaticWsCache g_static_ws_cache[kMaxStaticDevices];
+std::once_flag g_ctx_fn_once;
+CtxGetCurrentFn g_ctx_get_current = nullptr;
+CtxGetIdFn g_ctx_get_id = nullptr;
+
+void resolve_ctx_fns()
+{
+    void* a = nullptr;
+    void* b = nullptr;
+    cudaDriverEntryPointQueryResult qa = cudaDriverEntryPointSymbolNotFound, qb = qa;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) == cudaSuccess &&
+        cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) == cudaSuccess &&
+        qa == cudaDriverEntryPointSuccess && qb == cudaDriverEntryPointSuccess && a && b) {
+        g_ctx_get_current = reinterpret_cast<CtxGetCurrentFn>(a);
+        g_ctx_get_id = reinterpret_cast<CtxGetIdFn>(b);
+    }
+    cudaGetLastError();  // a failed lookup leaves no sticky error behind
+}
+
+// Id of the context current on this thread; false when there is none yet or
+// the driver calls are unavailable.
+bool current_ctx_id(unsigned long long* id)
+{
+    std::call_once(g_ctx_fn_once, resolve_ctx_fns);
+    if (g_ctx_get_current == nullptr)
+        return false;
+    void* ctx = nullptr;
+    if (g_ctx_get_current(&ctx) != 0 || ctx == nullptr)
+        return false;
+    return g_ctx_get_id(ctx, id) == 0;
+}
 
 gdn_status static_ws_address(void** out)
 {
@@ -455,12 +501,22 @@ gdn_status static_ws_address(void** out)
         return fail(GDN_ERR_CUDA, "cudaGetDevice failed: %s", cudaGetErrorString(e));
     if (dev < 0 || dev >= kMaxStaticDevices)
         return fail(GDN_ERR_UNSUPPORTED, "device ordinal above the static workspace table%s");
-    void* p = g_static_ws_addr[dev].load(std::memory_order_acquire);
-    if (p == nullptr) {
-        e = cudaGetSymbolAddress(&p, g_static_ws);
-        if (e != cudaSuccess)
-            return fail(GDN_ERR_CUDA, "cudaGetSymbolAddress failed: %s", cudaGetErrorString(e));
-        g_static_ws_addr[dev].store(p, std::memory_order_release);
+    unsigned long long id = 0;
+    const bool have_id = current_ctx_id(&id);
+    std::lock_guard<std::mutex> guard(g_static_ws_lock);
+    StaticWsCache& c = g_static_ws_cache[dev];
+    if (have_id && c.addr != nullptr && c.ctx_id == id) {
+        *out = c.addr;
+        return GDN_OK;
+    }
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_ws);
+    if (e != cudaSuccess)
+        return fail(GDN_ERR_CUDA, "cudaGetSymbolAddress failed: %s", cudaGetErrorString(e));
+    // the lookup above made the runtime's context current if none was
+    if (have_id || current_ctx_id(&id)) {
+        c.ctx_id = id;
+        c.addr = p;
     }
     *out = p;
     return GDN_OK;

@@ -12,8 +12,9 @@
 // Each CTA copies 4096 elements of one (layer, sequence).  Its threads load
 // the path's last node id and start loading their part of that node's state
 // right away (from a clamped, always in-bounds address), while warp 0 checks
-// the whole path against the tree (path[0] = 0, parent[path[i]] = path[i-1]);
-// the stores happen only for a valid path.
+// the tree (parent[0] = -1, 0 <= parent[n] < n) and the whole path against it
+// (path[0] = 0, parent[path[i]] = path[i-1]); the stores happen only for a
+// valid tree and path.
 
 #include <cstdint>
 
@@ -104,7 +105,17 @@ __global__ void __launch_bounds__(kCommitThreads) gdn_commit_kernel(const CParam
     }
 
     if (tid < 32) {
-        bool ok = len_ok;
+        // the tree itself: parent[0] = -1 and 0 <= parent[n] < n (a path can
+        // only be checked against a well-formed tree)
+        bool tree_ok = seq_ok;
+        if (tree_ok && p.parent) {
+            for (int n = tid; n < N; n += 32) {
+                const int pn = __ldg(p.parent + (size_t)n0 + n);
+                tree_ok &= (n == 0) ? (pn == -1) : (pn >= 0 && pn < n);
+            }
+        }
+        tree_ok = __all_sync(0xffffffffu, tree_ok);
+        bool ok = len_ok && tree_ok;
         if (ok) {
             for (int i = tid; i < len; i += 32) {
                 const int xi = __ldg(path + i);
@@ -122,12 +133,12 @@ __global__ void __launch_bounds__(kCommitThreads) gdn_commit_kernel(const CParam
         if (ok && p.persist_last && __ldg(path + len - 1) != N - 1)
             ok = false;
         if (tid == 0)
-            s_ok = ok ? 1 : 0;
+            s_ok = ok ? 1 : (tree_ok ? 0 : -1);
     }
     __syncthreads();
-    if (!s_ok) {
+    if (s_ok != 1) {
         if (blockIdx.x == 0 && layer == 0 && tid == 0)
-            report_status(p.status, seq_ok ? GDN_ERR_BAD_PATH : GDN_ERR_BAD_TREE);
+            report_status(p.status, s_ok == 0 ? GDN_ERR_BAD_PATH : GDN_ERR_BAD_TREE);
         return;
     }
     float* dst = p.state_out[layer] + (size_t)b * p.per_seq;

@@ -277,6 +277,35 @@ def make_problem(*, batch: int, n_nodes: int, n_k_heads: int, n_v_heads: int,
                    scale=(1.0 / math.sqrt(d_k)) if scale is None else float(scale))
 
 
+def make_device_inputs(*, parent: np.ndarray, n_k_heads: int, n_v_heads: int, d_k: int, d_v: int,
+                       seed: int, device, qkv_dtype: str = "bf16") -> dict:
+    """One layer's q, k, v, g, beta and state_in for the trees in ``parent``
+    ([B][N] int32), drawn on ``device`` with a seeded device generator.
+
+    The value recipe is make_problem's (q, k ~ N(0,1) L2-normalised over d_k,
+    v ~ N(0,1), g = -softplus(N(0,1)), beta = sigmoid(N(0,1)), state_in ~
+    N(0, 0.1^2), q/k/v rounded to the input dtype); only the generator
+    differs, so large timing workloads need not be drawn on the host.
+    Returns device tensors keyed q, k, v, g, beta, state_in, parent.
+    """
+    par = torch.from_numpy(np.ascontiguousarray(parent, dtype=np.int32))
+    B, N = par.shape
+    gen = torch.Generator(device=device).manual_seed(seed)
+    dt = _DTYPES[qkv_dtype]
+
+    def randn(*shape):
+        return torch.randn(*shape, generator=gen, device=device)
+
+    q = _l2n(randn(B, N, n_k_heads, d_k)).to(dt)
+    k = _l2n(randn(B, N, n_k_heads, d_k)).to(dt)
+    v = randn(B, N, n_v_heads, d_v).to(dt)
+    g = -torch.nn.functional.softplus(randn(B, N, n_v_heads))
+    beta = torch.sigmoid(randn(B, N, n_v_heads))
+    state_in = 0.1 * randn(B, n_v_heads, d_v, d_k)
+    return dict(q=q.contiguous(), k=k.contiguous(), v=v.contiguous(), g=g.contiguous(),
+                beta=beta.contiguous(), state_in=state_in.contiguous(), parent=par.to(device))
+
+
 # The five workloads.  Sizes are per layer; ``layers`` is how many GDN layers a
 # step stacks (each layer with its own buffers).
 WORKLOADS = {

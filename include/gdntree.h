@@ -250,6 +250,15 @@ size_t gdn_tree_verify_workspace_bytes(const gdn_tree_desc* desc);
  * Calls on one device must be ordered (one stream, or events between
  * streams); two calls in flight at once on different streams or host
  * threads overwrite each other's branch states and give wrong results.
+ *
+ * Memory: every CUDA context that loads the library holds the buffer's
+ * 32 MiB on its device until the context ends, whether or not this entry
+ * point is ever called.  The buffer's address belongs to the context: the
+ * library looks it up with cudaGetSymbolAddress the first time it runs in a
+ * context (identified by its driver context id), and again after the current
+ * context changes (a cudaDeviceReset, or another context made current through
+ * the driver API).  Make the first call on each device before capturing it
+ * into a CUDA graph.
  */
 gdn_status gdn_tree_verify_static_ws(const gdn_tree_desc* desc, const void* q, const void* k,
                                      const void* v, const float* g, const float* beta,
@@ -276,8 +285,11 @@ size_t gdn_static_workspace_capacity(void);
  *                verify call (commit reads only node_states), but must not
  *                overlap node_states.
  *
- * Errors: host-side as for verify; GDN_ERR_BAD_PATH (or GDN_ERR_BAD_TREE)
- * through desc->status, and state_out[b] is then left untouched.
+ * Errors: host-side as for verify.  Through desc->status: GDN_ERR_BAD_TREE
+ * when sequence b's parent_idx is not a tree (parent[0] = -1 and
+ * 0 <= parent[n] < n for every node, checked before the path), else
+ * GDN_ERR_BAD_PATH when its path breaks the rules above; state_out[b] is then
+ * left untouched.
  */
 gdn_status gdn_tree_commit(const gdn_tree_desc* desc, const void* node_states,
                            const int32_t* parent_idx, const int32_t* accept_path,
