@@ -75,6 +75,17 @@ def test_chunked_long_chain4096_sampled():
     assert torch.equal(res["state_out"], res["node_states"][:, 0])
 
 
+def test_chunked_long_chain4096_rows_of_every_tile():
+    from tests.test_gpu_parity import CHAIN_PAIRS, CHAIN_ROWS, _chain_rows_parity
+    prob = make_workload("long_chain4096", seed=4)
+    N = prob.n_nodes
+    prob.accept_path = torch.arange(N, dtype=torch.int32).repeat(prob.batch, 1).contiguous()
+    prob.accept_len = torch.full((prob.batch,), N, dtype=torch.int32)
+    res = run(prob, "f32", flags=FLAGS | gdn.GDN_FLAG_CHUNKED)
+    assert res["status"] == 0
+    _chain_rows_parity(prob, res, CHAIN_PAIRS, CHAIN_ROWS)
+
+
 def test_chunked_is_refused_outside_its_shapes():
     prob = _chain(70, dv=32)
     d = {k: getattr(prob, k).cuda() for k in ("q", "k", "v", "g", "beta", "parent", "state_in")}
