@@ -21,6 +21,9 @@ struct VerifyGeom {
     bool warp_tree;       // staged tree walked from warp registers (N <= 32)
     bool reload;          // branch parents re-read from f32 node_states (no stack)
     bool gslots;          // stack slots in the caller's workspace (global memory)
+    bool tslots;          // stack slots in tensor memory (the wide kernel)
+    int tmem_cols;        // tslots: tensor-memory columns allocated per CTA
+    int tmem_slot_cols;   // tslots: columns from one slot to the next
     size_t ws_bytes;      // workspace the launch needs (gslots), else 0
     int chunks;           // lane shape: chunks of 8 state columns per lane and row (1 or 2)
     int rows_per_lane;    // lane shape: rows per lane (1 or 2)

@@ -36,6 +36,9 @@ constexpr long long kSms = 148;
 // CTA, so wider CTAs spend less shared memory per row).
 constexpr int kLargeGridSlots[3] = {1, 2, 3};
 constexpr int kLargeTreeWarps = 8;
+// Stack slots the wide kernel keeps in tensor memory (4 x 64 columns: two
+// CTAs per SM fill its 512).
+constexpr int kMaxTmemSlots = 4;
 
 template <int DK>
 cudaError_t launch_shapes(const verify::KParams& kp, const VerifyArgs& a, const VerifyGeom& g,
@@ -75,6 +78,7 @@ VerifyGeom verify_geometry(const VerifyArgs& a, bool use_workspace)
     // for the largest.  Both give identical bits.
     g.reload = !chain && a.state_dtype == GDN_F32 && !persist_last &&
                !(g.rows_per_lane == 2 && a.n_nodes > 32 && a.cu_nodes == nullptr);
+    int tmem_slots = 0;
     if (chain || g.reload) {
         g.slots = 0;
     } else {
@@ -87,9 +91,16 @@ VerifyGeom verify_geometry(const VerifyArgs& a, bool use_workspace)
         while ((2 << k) <= a.n_nodes)
             ++k;
         g.gslots = use_workspace;
+        // The wide kernel (two rows per lane, trees above 32 nodes, fixed
+        // node counts) keeps its slots in tensor memory, which the kernels
+        // do not otherwise use: up to kMaxTmemSlots of them, none in shared
+        // memory.
+        g.tslots = !chain && !g.reload && !g.gslots && a.n_nodes > 32 && g.rows_per_lane == 2 &&
+                   a.cu_nodes == nullptr;
         const int size_class = a.n_nodes <= 32 ? 0 : (a.n_nodes <= 96 ? 1 : 2);
         const int cap = g.gslots ? 4 : (g.rows_per_lane == 2 ? kLargeGridSlots[size_class] : 2 + size_class);
         g.slots = k < 1 ? 1 : (k > cap ? cap : k);
+        tmem_slots = k < 1 ? 1 : (k > kMaxTmemSlots ? kMaxTmemSlots : k);
     }
     const int rpw = rows_per_warp(g.chunks, g.rows_per_lane);
     // Staged kernel first (wide CTAs for large trees with shared-memory
@@ -105,7 +116,11 @@ VerifyGeom verify_geometry(const VerifyArgs& a, bool use_workspace)
         if (a.d_v % rows != 0 || (rows * es) % 16 != 0)
             continue;
         const size_t raw_bytes = (size_t)(2 * a.d_k + rows) * es;
-        const size_t slot_bytes = g.gslots ? 0 : (size_t)g.slots * rows * a.d_k * 4;
+        // tensor-memory slots need the full 8 warps (a lane's 32 floats are
+        // one 32-column store); otherwise shared-memory slots as usual
+        const bool tmem = g.tslots && pass == 0 && warps == kLargeTreeWarps && rows * a.d_k == 32 * 32 * warps;
+        const int slots = tmem ? tmem_slots : g.slots;
+        const size_t slot_bytes = (g.gslots || tmem) ? 0 : (size_t)slots * rows * a.d_k * 4;
         size_t off = 64;  // mbarriers
         size_t off_raw = 0, off_desc = 0, off_ab = 0, off_slots = 0;
         if (staged) {
@@ -153,6 +168,17 @@ VerifyGeom verify_geometry(const VerifyArgs& a, bool use_workspace)
         g.off_tree = (uint32_t)off_tree;
         g.smem = off;
         g.ws_bytes = g.gslots ? (size_t)a.batch * a.n_v_heads * a.d_v * a.d_k * g.slots * 4 : 0;
+        g.slots = slots;
+        g.tslots = tmem;
+        if (tmem) {
+            // a lane's slot is 32 columns; the warps that share a lane
+            // quarter sit side by side
+            g.tmem_slot_cols = 32 * ((warps + 3) / 4);
+            int cols = 32;
+            while (cols < g.slots * g.tmem_slot_cols)
+                cols *= 2;
+            g.tmem_cols = cols;
+        }
         break;
     }
     return g;
@@ -186,6 +212,8 @@ cudaError_t launch_verify(const VerifyArgs& a, const VerifyGeom& geom, cudaStrea
     kp.qk_norm = (a.flags & GDN_FLAG_QK_L2NORM) ? 1 : 0;
     kp.gates = (a.flags & GDN_FLAG_GATES) ? 1 : 0;
     kp.ws = geom.gslots ? a.workspace : nullptr;
+    kp.tmem_cols = geom.tmem_cols;
+    kp.tmem_slot_cols = geom.tmem_slot_cols;
     kp.cu = a.cu_nodes;
     kp.total = a.total_nodes;
     kp.raw_bytes = geom.raw_bytes;

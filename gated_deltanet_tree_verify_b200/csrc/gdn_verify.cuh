@@ -130,6 +130,8 @@ struct KParams {
     int qk_norm;         // GDN_FLAG_QK_L2NORM: k and q normalised per node inside the kernel
     int gates;           // GDN_FLAG_GATES: g and beta are raw (gate_scalars)
     float* ws;           // global stack slots (kTreeGlobal kinds): slots x rows x d_k per CTA
+    int tmem_cols;       // tensor-memory stack slots (kTreeTmem kinds): columns allocated per CTA
+    int tmem_slot_cols;  // ... and columns from one slot to the next
     const int32_t* cu;   // varlen: [B + 1] node offsets of the packed layout (N: the most per sequence)
     int total;           // varlen: nodes in the packed layout
     uint32_t raw_bytes;  // one node's record (k row | q row | v slice) in bytes
@@ -545,6 +547,39 @@ __device__ __forceinline__ void load_slot(StateT<C, RL>& S, const float* lane_sl
             S.s[r][2 * j] = make_float2(x.x, x.y);
             S.s[r][2 * j + 1] = make_float2(x.z, x.w);
         }
+    }
+}
+
+// Stack slots in tensor memory: a lane's 8 C RL floats are the 32-bit
+// columns taddr .. taddr + 8 C RL - 1 of its TMEM lane (one warp-wide store
+// or load of 32 columns).
+template <int C, int RL>
+__device__ __forceinline__ void tmem_save_slot(const StateT<C, RL>& S, uint32_t taddr)
+{
+    static_assert(8 * C * RL == 32, "tensor-memory slots hold 32 floats per lane");
+    uint32_t r[32];
+#pragma unroll
+    for (int i = 0; i < RL; ++i) {
+#pragma unroll
+        for (int t = 0; t < 4 * C; ++t) {
+            r[(i * 4 * C + t) * 2] = __float_as_uint(S.s[i][t].x);
+            r[(i * 4 * C + t) * 2 + 1] = __float_as_uint(S.s[i][t].y);
+        }
+    }
+    tmem_st32(taddr, r);
+}
+
+template <int C, int RL>
+__device__ __forceinline__ void tmem_load_slot(StateT<C, RL>& S, uint32_t taddr)
+{
+    static_assert(8 * C * RL == 32, "tensor-memory slots hold 32 floats per lane");
+    uint32_t r[32];
+    tmem_ld32(taddr, r);
+#pragma unroll
+    for (int i = 0; i < RL; ++i) {
+#pragma unroll
+        for (int t = 0; t < 4 * C; ++t)
+            S.s[i][t] = make_float2(__uint_as_float(r[(i * 4 * C + t) * 2]), __uint_as_float(r[(i * 4 * C + t) * 2 + 1]));
     }
 }
 
@@ -1137,18 +1172,18 @@ static __device__ bool build_warp_walk(const int32_t* prow, int N, int K, int* w
 // position whose metadata says the state is not already in registers: a
 // stack slot, or recomputation from the deepest saved ancestor (start; -1:
 // from state_in).  fetch(y, k2, vr, a, beta) supplies node y's inputs.
-template <int DK, int C, int RL, class Tree, class Fetch>
+template <int DK, int C, int RL, class Tree, class SlotLoad, class Fetch>
 __device__ __forceinline__ void source_parent(StateT<C, RL>& S, int m, int pp, int start, const KParams& p,
-                                              const Tree& tree, const float* lane_slot, int slot_floats,
-                                              int stride, const float* sin_lane, Fetch fetch)
+                                              const Tree& tree, SlotLoad slot_load, const float* sin_lane,
+                                              Fetch fetch)
 {
     constexpr int LR = LaneMap<DK, C, RL>::LR;
     const int src = meta_src(m);
     if (src == kSrcSlot) {
-        load_slot<C, RL>(S, lane_slot + (size_t)meta_load(m) * slot_floats, stride);
+        slot_load(S, meta_load(m));
     } else if (src == kSrcRecompute) {
         if (start >= 0)
-            load_slot<C, RL>(S, lane_slot + (size_t)(p.slots - 1) * slot_floats, stride);
+            slot_load(S, p.slots - 1);
         else
             load_rows<DK, C, RL>(S, sin_lane);
         tree.for_path(pp, start, [&](int y) {
@@ -1161,10 +1196,12 @@ __device__ __forceinline__ void source_parent(StateT<C, RL>& S, int m, int pp, i
     }
 }
 
-// Walk kinds.  kTreeGlobal added to kTreeWarp or kTreeSmem: the stack slots
-// live in a caller workspace in global memory (L2) instead of shared memory,
-// and a slot the next position needs is loaded one node ahead.
-enum : int { kTreeChain = 0, kTreeWarp = 1, kTreeSmem = 2, kTreeIndex = 3, kTreeGlobal = 4 };
+// Walk kinds (bits 0-1) and where a walk's stack slots live (bits 2-3).
+// kTreeGlobal added to kTreeWarp or kTreeSmem: the stack slots live in a
+// caller workspace in global memory (L2) instead of shared memory, and a
+// slot the next position needs is loaded one node ahead.  kTreeTmem added to
+// kTreeSmem: they live in the CTA's tensor memory (the wide kernel only).
+enum : int { kTreeChain = 0, kTreeWarp = 1, kTreeSmem = 2, kTreeIndex = 3, kTreeGlobal = 4, kTreeTmem = 8 };
 
 // The walk over positions [0, N): per position, find the parent state,
 // update, write the output and persist.  The context supplies each
@@ -1173,13 +1210,14 @@ enum : int { kTreeChain = 0, kTreeWarp = 1, kTreeSmem = 2, kTreeIndex = 3, kTree
 // when everything is staged).
 template <int DK, int C, int RL, typename RT, typename ST, int TREE, class Tree, class Ctx>
 __device__ __forceinline__ void walk(StateT<C, RL>& S, const KParams& p, const Seq& sq, const Tree& tree,
-                                     float* lane_slot, const float* sin_lane, int b, int h, int row0,
-                                     const LaneMap<DK, C, RL>& L, Ctx& ctx)
+                                     float* lane_slot, uint32_t tslot, const float* sin_lane, int b, int h,
+                                     int row0, const LaneMap<DK, C, RL>& L, Ctx& ctx)
 {
     using LM = LaneMap<DK, C, RL>;
     constexpr bool CHAIN = TREE == kTreeChain;
     constexpr bool INDEX = TREE == kTreeIndex;
-    constexpr bool GSLOT = TREE >= kTreeGlobal;
+    constexpr bool GSLOT = (TREE & kTreeGlobal) != 0;
+    constexpr bool TSLOT = (TREE & kTreeTmem) != 0;
     const int N = sq.N;
     const size_t ns_stride = (size_t)p.Hv * p.dv * DK;  // elements between nodes' states
     ST* const ns_lane = static_cast<ST*>(p.node_states) + (size_t)(p.persist_last ? b : sq.n0) * ns_stride +
@@ -1188,6 +1226,12 @@ __device__ __forceinline__ void walk(StateT<C, RL>& S, const KParams& p, const S
     float* const out_lane = p.out + (size_t)sq.n0 * out_stride + (size_t)h * p.dv + row0 + L.row;
     const int slot_floats = p.rows * DK;
     const int stride = p.warps * 32 * 4;
+    auto slot_load = [&](StateT<C, RL>& X, int s) {
+        if constexpr (TSLOT)
+            tmem_load_slot<C, RL>(X, tslot + (uint32_t)(s * p.tmem_slot_cols));
+        else
+            load_slot<C, RL>(X, lane_slot + (size_t)s * slot_floats, stride);
+    };
     // Index order and workspace slots: the next position's parent state,
     // loaded one node ahead.  (Asking for it in L1 instead, with prefetch
     // hints and a load where it is needed, saves ~40 registers but was
@@ -1220,8 +1264,7 @@ __device__ __forceinline__ void walk(StateT<C, RL>& S, const KParams& p, const S
             if (GSLOT && have_next)
                 S = Sn;  // this position's slot, loaded at the previous one
             else if (src != kSrcCont && src != kSrcRoot)
-                source_parent<DK, C, RL>(S, d.i.y, d.i.w, d.i.z, p, tree, lane_slot, slot_floats, stride,
-                                         sin_lane, ctx.fetcher());
+                source_parent<DK, C, RL>(S, d.i.y, d.i.w, d.i.z, p, tree, slot_load, sin_lane, ctx.fetcher());
             if constexpr (GSLOT) {
                 // the next position's slot.  A node whose successor in the
                 // walk reloads a slot is a leaf, so this position saves
@@ -1253,8 +1296,12 @@ __device__ __forceinline__ void walk(StateT<C, RL>& S, const KParams& p, const S
             persist<DK, C, RL, ST>(S, ns_lane + (size_t)(p.persist_last ? 0 : n) * ns_stride);
         if constexpr (!CHAIN && !INDEX) {
             const int save = meta_save(d.i.y);
-            if (save >= 0)
-                save_slot<C, RL>(S, lane_slot + (size_t)save * slot_floats, stride);
+            if (save >= 0) {
+                if constexpr (TSLOT)
+                    tmem_save_slot<C, RL>(S, tslot + (uint32_t)(save * p.tmem_slot_cols));
+                else
+                    save_slot<C, RL>(S, lane_slot + (size_t)save * slot_floats, stride);
+            }
         }
         if constexpr (INDEX) {
             if (have_next)
@@ -1335,7 +1382,7 @@ __device__ __forceinline__ void cp_async4(void* dst_smem, const void* src_gmem)
 template <int DK, int TREE>
 __device__ __forceinline__ float* cta_slots(const KParams& p, float* slotbuf)
 {
-    if constexpr (TREE >= kTreeGlobal) {
+    if constexpr ((TREE & kTreeGlobal) != 0) {
         const size_t cta = ((size_t)blockIdx.z * p.Hv + blockIdx.y) * gridDim.x + blockIdx.x;
         return p.ws + cta * (size_t)p.slots * p.rows * DK;
     } else {
@@ -1387,7 +1434,7 @@ __device__ __forceinline__ void write_descs(const Tree& tree, const unsigned cha
 template <int DK, int C, int RL, typename QT, typename ST, int TREE, class Tree>
 __device__ __forceinline__ void staged_finish(StateT<C, RL>& S, const KParams& p, const Seq& sq, const Tree& tree,
                                               const unsigned char* raw, float* ab, PosDesc* desc, float* slotbuf,
-                                              const float* sin_lane, int b, int h, int row0,
+                                              uint32_t tbase, const float* sin_lane, int b, int h, int row0,
                                               const LaneMap<DK, C, RL>& L)
 {
     constexpr int LR = LaneMap<DK, C, RL>::LR;
@@ -1396,11 +1443,15 @@ __device__ __forceinline__ void staged_finish(StateT<C, RL>& S, const KParams& p
     const uint32_t rec_elems = p.raw_bytes / (uint32_t)sizeof(QT);
     StagedCtx<DK, C, RL, QT> ctx{reinterpret_cast<const QT*>(raw), desc, ab, rec_elems, sq.N, p.qk_norm, L};
     float* lane_slot = cta_slots<DK, TREE>(p, slotbuf) + 4 * threadIdx.x;
-    walk<DK, C, RL, QT, ST, TREE>(S, p, sq, tree, lane_slot, sin_lane, b, h, row0, L, ctx);
+    // tensor-memory slots: warp w's lanes are TMEM lanes 32 (w mod 4) ..; the
+    // warps that share a lane quarter use columns 32 apart
+    const int warp = threadIdx.x >> 5;
+    const uint32_t tslot = tbase + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(32 * (warp >> 2));
+    walk<DK, C, RL, QT, ST, TREE>(S, p, sq, tree, lane_slot, tslot, sin_lane, b, h, row0, L, ctx);
 }
 
 template <int DK, int C, int RL, typename QT, typename ST, int TREE>
-__device__ __forceinline__ void staged_body(const KParams& p)
+__device__ __forceinline__ void staged_body(const KParams& p, uint32_t tbase)
 {
     constexpr int EPC = 16 / sizeof(QT);  // elements per 16-byte chunk
     constexpr int QKCH = DK / EPC;        // chunks per k (or q) row
@@ -1411,7 +1462,7 @@ __device__ __forceinline__ void staged_body(const KParams& p)
     float* slotbuf = reinterpret_cast<float*>(smem + p.off_slots);
     int* tsm = reinterpret_cast<int*>(smem + p.off_tree);
 
-    constexpr int TK = TREE % kTreeGlobal;  // walk kind without the slot placement
+    constexpr int TK = TREE & 3;  // walk kind without the slot placement
     const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int hk = h / p.G;
     const int row0 = tile * p.rows;
@@ -1552,31 +1603,52 @@ __device__ __forceinline__ void staged_body(const KParams& p)
     }
     // 5. descriptors, then the walk
     if constexpr (TK == kTreeChain)
-        staged_finish<DK, C, RL, QT, ST, TREE>(S, p, sq, NoTree{}, raw, ab, desc, slotbuf, sin_lane, b, h,
+        staged_finish<DK, C, RL, QT, ST, TREE>(S, p, sq, NoTree{}, raw, ab, desc, slotbuf, tbase, sin_lane, b, h,
                                                row0, L);
     else if constexpr (TK == kTreeIndex)
-        staged_finish<DK, C, RL, QT, ST, TREE>(S, p, sq, IndexTree{tsm}, raw, ab, desc, slotbuf, sin_lane, b,
+        staged_finish<DK, C, RL, QT, ST, TREE>(S, p, sq, IndexTree{tsm}, raw, ab, desc, slotbuf, tbase, sin_lane, b,
                                                h, row0, L);
     else if constexpr (TK == kTreeWarp)
-        staged_finish<DK, C, RL, QT, ST, TREE>(S, p, sq, MaskTree{tsm}, raw, ab, desc, slotbuf, sin_lane, b,
+        staged_finish<DK, C, RL, QT, ST, TREE>(S, p, sq, MaskTree{tsm}, raw, ab, desc, slotbuf, tbase, sin_lane, b,
                                                h, row0, L);
     else
-        staged_finish<DK, C, RL, QT, ST, TREE>(S, p, sq, SmemTree{tv, N, warp}, raw, ab, desc, slotbuf,
+        staged_finish<DK, C, RL, QT, ST, TREE>(S, p, sq, SmemTree{tv, N, warp}, raw, ab, desc, slotbuf, tbase,
                                                sin_lane, b, h, row0, L);
 }
 
 template <int DK, int C, int RL, typename QT, typename ST, int TREE>
 __global__ void __launch_bounds__(kSmallWarps * 32) gdn_verify_staged(const KParams p)
 {
-    staged_body<DK, C, RL, QT, ST, TREE>(p);
+    staged_body<DK, C, RL, QT, ST, TREE>(p, 0u);
 }
 
 // Trees of more than 32 nodes with shared-memory slots on large grids:
 // kMaxWarps warps share one copy of the node records.
+// With kTreeTmem the stack slots live in tensor memory: warp 0 allocates
+// p.tmem_cols columns before anything else and frees them after every path
+// through the body (its early exits are CTA-wide, so all threads get back
+// here).
 template <int DK, int C, int RL, typename QT, typename ST, int TREE>
 __global__ void __launch_bounds__(kMaxWarps * 32) gdn_verify_staged_wide(const KParams p)
 {
-    staged_body<DK, C, RL, QT, ST, TREE>(p);
+    if constexpr ((TREE & kTreeTmem) != 0) {
+        __shared__ uint32_t tbase;
+        if (threadIdx.x < 32)
+            tmem_alloc(&tbase, (uint32_t)p.tmem_cols);
+        tmem_fence_before_sync();
+        __syncthreads();
+        tmem_fence_after_sync();
+        staged_body<DK, C, RL, QT, ST, TREE>(p, tbase);
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");  // this thread's slot stores are done
+        tmem_fence_before_sync();
+        __syncthreads();
+        if (threadIdx.x < 32) {
+            tmem_fence_after_sync();
+            tmem_free(tbase, (uint32_t)p.tmem_cols);
+        }
+    } else {
+        staged_body<DK, C, RL, QT, ST, TREE>(p, 0u);
+    }
 }
 
 // Small trees walked from warp registers with one row per lane (small
@@ -1585,7 +1657,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32) gdn_verify_staged_wide(const K
 template <int DK, int C, int RL, typename QT, typename ST, int TREE>
 __global__ void __launch_bounds__(kSmallWarps * 32, 6) gdn_verify_staged_dense(const KParams p)
 {
-    staged_body<DK, C, RL, QT, ST, TREE>(p);
+    staged_body<DK, C, RL, QT, ST, TREE>(p, 0u);
 }
 
 // ---------------------------------------------------------------------------
@@ -1891,11 +1963,11 @@ __global__ void __launch_bounds__((kSmallWarps + 1) * 32) gdn_verify_ring(const 
     RingCtx<DK, C, RL, QT> ctx{full, empty, ring, p.raw_bytes, slot_bytes, desc_off, p.status, lane, gf};
     float* lane_slot = cta_slots<DK, TREE>(p, slotbuf) + 4 * threadIdx.x;
     if constexpr (CHAIN)
-        walk<DK, C, RL, QT, ST, TREE>(S, p, sq, NoTree{}, lane_slot, sin_lane, b, h, row0, L, ctx);
+        walk<DK, C, RL, QT, ST, TREE>(S, p, sq, NoTree{}, lane_slot, 0u, sin_lane, b, h, row0, L, ctx);
     else if constexpr (INDEX)
-        walk<DK, C, RL, QT, ST, TREE>(S, p, sq, IndexTree{T.par}, lane_slot, sin_lane, b, h, row0, L, ctx);
+        walk<DK, C, RL, QT, ST, TREE>(S, p, sq, IndexTree{T.par}, lane_slot, 0u, sin_lane, b, h, row0, L, ctx);
     else
-        walk<DK, C, RL, QT, ST, TREE>(S, p, sq, SmemTree{T, N, warp}, lane_slot, sin_lane, b, h, row0, L, ctx);
+        walk<DK, C, RL, QT, ST, TREE>(S, p, sq, SmemTree{T, N, warp}, lane_slot, 0u, sin_lane, b, h, row0, L, ctx);
 }
 
 // ---------------------------------------------------------------------------
@@ -1943,10 +2015,12 @@ cudaError_t launch_staged(const KParams& kp, const VerifyArgs& a, const VerifyGe
     dim3 grid(geom.tiles, a.n_v_heads, a.batch);
     if constexpr (TREE == kTreeWarp && RL == 1 && sizeof(QT) == 2)
         return launch_granted<gdn_verify_staged_dense<DK, C, RL, QT, ST, TREE>>(kp, grid, geom, stream);
-    if constexpr (TREE == kTreeSmem && RL == 2) {
+    if constexpr ((TREE == kTreeSmem || TREE == kTreeSmem + kTreeTmem) && RL == 2) {
         if (geom.warps > kSmallWarps)
             return launch_granted<gdn_verify_staged_wide<DK, C, RL, QT, ST, TREE>>(kp, grid, geom, stream);
     }
+    if constexpr ((TREE & kTreeTmem) != 0)
+        return cudaErrorInvalidConfiguration;  // not reached: tensor-memory slots only with the wide kernel
     if (geom.warps > kSmallWarps)
         return cudaErrorInvalidConfiguration;  // not reached: the geometry only widens the kinds above
     return launch_granted<gdn_verify_staged<DK, C, RL, QT, ST, TREE>>(kp, grid, geom, stream);
@@ -1976,6 +2050,10 @@ cudaError_t launch_one(const KParams& kp, const VerifyArgs& a, const VerifyGeom&
         if (geom.warp_tree)
             return geom.gslots ? launch_staged<DK, C, RL, QT, ST, kTreeWarp + kTreeGlobal>(kp, a, geom, stream)
                                : launch_staged<DK, C, RL, QT, ST, kTreeWarp>(kp, a, geom, stream);
+        if constexpr (RL == 2 && C * RL * 8 == 32) {
+            if (geom.tslots)
+                return launch_staged<DK, C, RL, QT, ST, kTreeSmem + kTreeTmem>(kp, a, geom, stream);
+        }
         return geom.gslots ? launch_staged<DK, C, RL, QT, ST, kTreeSmem + kTreeGlobal>(kp, a, geom, stream)
                            : launch_staged<DK, C, RL, QT, ST, kTreeSmem>(kp, a, geom, stream);
     }
