@@ -96,7 +96,7 @@ VerifyGeom verify_geometry(const VerifyArgs& a, bool use_workspace)
         // do not otherwise use: up to kMaxTmemSlots of them, none in shared
         // memory.
         g.tslots = !chain && !g.reload && !g.gslots && a.n_nodes > 32 && g.rows_per_lane == 2 &&
-                   a.cu_nodes == nullptr;
+                   a.cu_nodes == nullptr && !persist_last && !(a.flags & GDN_FLAG_QK_L2NORM);
         const int size_class = a.n_nodes <= 32 ? 0 : (a.n_nodes <= 96 ? 1 : 2);
         const int cap = g.gslots ? 4 : (g.rows_per_lane == 2 ? kLargeGridSlots[size_class] : 2 + size_class);
         g.slots = k < 1 ? 1 : (k > cap ? cap : k);

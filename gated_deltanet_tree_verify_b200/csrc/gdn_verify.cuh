@@ -1218,9 +1218,14 @@ __device__ __forceinline__ void walk(StateT<C, RL>& S, const KParams& p, const S
     constexpr bool INDEX = TREE == kTreeIndex;
     constexpr bool GSLOT = (TREE & kTreeGlobal) != 0;
     constexpr bool TSLOT = (TREE & kTreeTmem) != 0;
+    // tensor-memory walks are never launched with last-only persistence or
+    // in-kernel q/k normalisation (the host geometry), so for them both are
+    // compile-time off and the node loop carries neither test
+    const bool persist_last = !TSLOT && p.persist_last;
+    const bool qk_norm = !TSLOT && p.qk_norm;
     const int N = sq.N;
     const size_t ns_stride = (size_t)p.Hv * p.dv * DK;  // elements between nodes' states
-    ST* const ns_lane = static_cast<ST*>(p.node_states) + (size_t)(p.persist_last ? b : sq.n0) * ns_stride +
+    ST* const ns_lane = static_cast<ST*>(p.node_states) + (size_t)(persist_last ? b : sq.n0) * ns_stride +
                         (size_t)h * p.dv * DK + (size_t)row0 * DK + L.tile_offset();
     const size_t out_stride = (size_t)p.Hv * p.dv;
     float* const out_lane = p.out + (size_t)sq.n0 * out_stride + (size_t)h * p.dv + row0 + L.row;
@@ -1286,14 +1291,14 @@ __device__ __forceinline__ void walk(StateT<C, RL>& S, const KParams& p, const S
         float pq[RL], u[RL];
         gdn_step<LM::LR, C, RL, true>(S, k2, q2, vr, a, d.f.w, d.f.y, pq, u);
         if (L.cl == 0) {
-            const float oc = p.qk_norm ? ctx.out_coef(pos, n) : p.scale;
+            const float oc = qk_norm ? ctx.out_coef(pos, n) : p.scale;
             float* o = out_lane + (size_t)n * out_stride;
 #pragma unroll
             for (int r = 0; r < RL; ++r)
                 o[r * LM::RG] = __fmul_rn(oc, __fmaf_rn(u[r], d.f.z, __fmul_rn(a, pq[r])));
         }
-        if (!p.persist_last || pos == N - 1)
-            persist<DK, C, RL, ST>(S, ns_lane + (size_t)(p.persist_last ? 0 : n) * ns_stride);
+        if (!persist_last || pos == N - 1)
+            persist<DK, C, RL, ST>(S, ns_lane + (size_t)(persist_last ? 0 : n) * ns_stride);
         if constexpr (!CHAIN && !INDEX) {
             const int save = meta_save(d.i.y);
             if (save >= 0) {
