@@ -39,6 +39,10 @@ constexpr int kLargeTreeWarps = 8;
 // Stack slots the wide kernel keeps in tensor memory (4 x 64 columns: two
 // CTAs per SM fill its 512).
 constexpr int kMaxTmemSlots = 4;
+// Smallest tree that the wide kernel walks with tensor-memory slots; smaller
+// trees stay on 4-warp CTAs (the wide kernel with tensor-memory slots measured
+// 3-13 % slower for budgets 8-22 at batch 8, equal at batch 32).
+constexpr int kTmemMinNodes = 33;
 
 template <int DK>
 cudaError_t launch_shapes(const verify::KParams& kp, const VerifyArgs& a, const VerifyGeom& g,
@@ -91,12 +95,11 @@ VerifyGeom verify_geometry(const VerifyArgs& a, bool use_workspace)
         while ((2 << k) <= a.n_nodes)
             ++k;
         g.gslots = use_workspace;
-        // The wide kernel (two rows per lane, trees above 32 nodes, fixed
-        // node counts) keeps its slots in tensor memory, which the kernels
-        // do not otherwise use: up to kMaxTmemSlots of them, none in shared
-        // memory.
-        g.tslots = !chain && !g.reload && !g.gslots && a.n_nodes > 32 && g.rows_per_lane == 2 &&
-                   a.cu_nodes == nullptr && !persist_last && !(a.flags & GDN_FLAG_QK_L2NORM);
+        // The wide kernel (two rows per lane, trees above 32 nodes) keeps
+        // its slots in tensor memory, which the kernels do not otherwise
+        // use: up to kMaxTmemSlots of them, none in shared memory.
+        g.tslots = !chain && !g.reload && !g.gslots && a.n_nodes >= kTmemMinNodes && g.rows_per_lane == 2 &&
+                   !persist_last && !(a.flags & GDN_FLAG_QK_L2NORM);
         const int size_class = a.n_nodes <= 32 ? 0 : (a.n_nodes <= 96 ? 1 : 2);
         const int cap = g.gslots ? 4 : (g.rows_per_lane == 2 ? kLargeGridSlots[size_class] : 2 + size_class);
         g.slots = k < 1 ? 1 : (k > cap ? cap : k);
@@ -106,7 +109,7 @@ VerifyGeom verify_geometry(const VerifyArgs& a, bool use_workspace)
     // Staged kernel first (wide CTAs for large trees with shared-memory
     // slots on large grids, then the usual width), else the ring kernel
     // (which adds a producer warp).
-    const bool wide = !chain && !g.reload && !g.gslots && a.n_nodes > 32 && g.rows_per_lane == 2;
+    const bool wide = !chain && !g.reload && !g.gslots && g.rows_per_lane == 2 && (a.n_nodes > 32 || g.tslots);
     for (int pass = wide ? 0 : 1; pass < 3; ++pass) {
         const bool staged = pass < 2;
         int warps = pass == 0 ? kLargeTreeWarps : kSmallWarps;  // the ring kernel: kSmallWarps at most

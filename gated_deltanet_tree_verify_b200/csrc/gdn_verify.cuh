@@ -2020,7 +2020,7 @@ cudaError_t launch_staged(const KParams& kp, const VerifyArgs& a, const VerifyGe
     dim3 grid(geom.tiles, a.n_v_heads, a.batch);
     if constexpr (TREE == kTreeWarp && RL == 1 && sizeof(QT) == 2)
         return launch_granted<gdn_verify_staged_dense<DK, C, RL, QT, ST, TREE>>(kp, grid, geom, stream);
-    if constexpr ((TREE == kTreeSmem || TREE == kTreeSmem + kTreeTmem) && RL == 2) {
+    if constexpr ((TREE == kTreeSmem || TREE == kTreeSmem + kTreeTmem || TREE == kTreeWarp + kTreeTmem) && RL == 2) {
         if (geom.warps > kSmallWarps)
             return launch_granted<gdn_verify_staged_wide<DK, C, RL, QT, ST, TREE>>(kp, grid, geom, stream);
     }
@@ -2052,9 +2052,14 @@ cudaError_t launch_one(const KParams& kp, const VerifyArgs& a, const VerifyGeom&
             return launch_staged<DK, C, RL, QT, ST, kTreeChain>(kp, a, geom, stream);
         if (geom.reload)
             return launch_staged<DK, C, RL, QT, ST, kTreeIndex>(kp, a, geom, stream);
-        if (geom.warp_tree)
+        if (geom.warp_tree) {
+            if constexpr (RL == 2 && C * RL * 8 == 32) {
+                if (geom.tslots)
+                    return launch_staged<DK, C, RL, QT, ST, kTreeWarp + kTreeTmem>(kp, a, geom, stream);
+            }
             return geom.gslots ? launch_staged<DK, C, RL, QT, ST, kTreeWarp + kTreeGlobal>(kp, a, geom, stream)
                                : launch_staged<DK, C, RL, QT, ST, kTreeWarp>(kp, a, geom, stream);
+        }
         if constexpr (RL == 2 && C * RL * 8 == 32) {
             if (geom.tslots)
                 return launch_staged<DK, C, RL, QT, ST, kTreeSmem + kTreeTmem>(kp, a, geom, stream);

@@ -89,6 +89,29 @@ def test_varlen_equals_each_sequence_alone(sd, workspace):
     assert_states_close(vr["node_states"][a:b][None], ex, sd)
 
 
+@pytest.mark.parametrize("sd", ["f32", "f16"])
+def test_varlen_48_heads_equals_each_sequence_alone(sd):
+    # Eight packed trees on 48 v-heads: the grid of the batched workloads,
+    # where f16 trees above 32 nodes take the wide kernel (stack slots in
+    # tensor memory).  Bit-identical to each sequence alone (a small grid,
+    # another lane shape), and sampled (sequence, head) pairs against the oracle.
+    sizes = [9, 65, 23, 16, 33, 23, 49, 9]
+    seqs = _seqs(sizes, ["ddtree"] * 8, Hk=16, Hv=48, seed=70)
+    vr = _run_varlen(seqs, sd)
+    assert vr["status"] == 0
+    for i, s in enumerate(seqs):
+        a, b = int(vr["cu"][i]), int(vr["cu"][i + 1])
+        ref = run(s, sd)
+        assert torch.equal(vr["out"][a:b], ref["out"][0]), i
+        assert torch.equal(vr["node_states"][a:b], ref["node_states"][0]), i
+        assert torch.equal(vr["state_out"][i], ref["state_out"][0]), i
+    for i, h in [(1, 0), (6, 47), (4, 20)]:
+        a, b = int(vr["cu"][i]), int(vr["cu"][i + 1])
+        out, _, ex = oracle.verify_pair(seqs[i], 0, h, state_dtype=sd, want_exact=True)
+        assert_out_close(vr["out"][a:b, h:h + 1][None], out)
+        assert_states_close(vr["node_states"][a:b, h:h + 1][None], ex, sd)
+
+
 def test_varlen_chains_with_persist_last():
     sizes = [5, 64, 17]
     seqs = _seqs(sizes, ["chain"] * 3)
