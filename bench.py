@@ -564,7 +564,10 @@ def run_e2e(stack, args, ws, device, stream):
     tree to the device, runs the 48 verify launches and the commit, and reads
     every layer's output back.  Layer l + 1's inputs are copied on a copy
     stream while layer l runs, and layer l's output is read back on a third
-    stream as soon as it is written; steps do not overlap each other."""
+    stream as soon as it is written; steps do not overlap each other.  The
+    step is captured once as a CUDA graph (the library's calls are stream
+    operations, so they capture) and replayed per step; every replay copies
+    the inputs up and the outputs down again."""
     gdn = stack.gdn
     K = max(3, min(args.steps, args.e2e_steps))
     keys = ("q", "k", "v", "g", "beta")
@@ -592,8 +595,10 @@ def run_e2e(stack, args, ws, device, stream):
     out_ev = [torch.cuda.Event() for _ in range(L)]
     tree_ev = torch.cuda.Event()
 
-    def step():
-        copy_s.wait_stream(stream)  # the previous step's launches are done with the inputs
+    def step(cs, eager):
+        """One step on compute stream cs: inputs up on copy_s, launches on cs,
+        each layer's output down on back_s once it is written."""
+        copy_s.wait_stream(cs)  # the previous step's launches are done with the inputs
         with torch.cuda.stream(copy_s):
             stack.parent.copy_(host_tree["parent"], non_blocking=True)
             stack.accept_path.copy_(host_tree["ap"], non_blocking=True)
@@ -602,47 +607,74 @@ def run_e2e(stack, args, ws, device, stream):
             for l, (hbuf, dbuf) in enumerate(host):
                 dbuf.copy_(hbuf, non_blocking=True)
                 in_ev[l].record(copy_s)
-        stream.wait_stream(back_s)  # the previous step's outputs have been read
-        stream.wait_event(tree_ev)
+        if eager:
+            cs.wait_stream(back_s)  # the previous step's outputs have been read
+        cs.wait_event(tree_ev)
         if stack.plan is not None:
-            gdn.gdn_tree_plan(stack.desc, stack.parent, stack.plan, stack.plan_bytes, stream=stream)
+            gdn.gdn_tree_plan(stack.desc, stack.parent, stack.plan, stack.plan_bytes, stream=cs)
         for l, (d, v) in enumerate(zip(stack.dev, dev_views)):
-            stream.wait_event(in_ev[l])
+            cs.wait_event(in_ev[l])
             desc = stack.desc if l == 0 else stack.desc_next
             if stack.plan is not None:
                 gdn.gdn_tree_verify_planned(desc, stack.plan, v["q"], v["k"], v["v"], v["g"], v["beta"],
                                             stack.parent, d["state"], d["out"], d["ns"],
-                                            plan_bytes=stack.plan_bytes, stream=stream)
+                                            plan_bytes=stack.plan_bytes, stream=cs)
             else:
                 gdn.gdn_tree_verify(desc, v["q"], v["k"], v["v"], v["g"], v["beta"], stack.parent, d["state"],
-                                    d["out"], d["ns"], stream=stream)
-            out_ev[l].record(stream)
-        stack.commit_all(stream=stream)
+                                    d["out"], d["ns"], stream=cs)
+            out_ev[l].record(cs)
+        stack.commit_all(stream=cs)
         with torch.cuda.stream(back_s):
             for l, (o, d) in enumerate(zip(outs, stack.dev)):
                 back_s.wait_event(out_ev[l])
                 o.copy_(d["out"], non_blocking=True)
-        stream.wait_stream(back_s)
+        cs.wait_stream(back_s)
 
     with torch.cuda.stream(stream):
         for _ in range(max(3, args.warmup // 4)):
-            step()
+            step(stream, True)
         torch.cuda.synchronize()
+    # The step as one CUDA graph (its copies are real memcpy nodes, done
+    # again on every replay), as a serving loop would run it; eager calls
+    # if the capture is refused.
+    graph, mode = None, "eager"
+    try:
+        cap = torch.cuda.Stream(device)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=cap):
+            step(cap, False)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                graph.replay()
+        torch.cuda.synchronize()
+        mode = "graph"
+    except Exception as e:  # pragma: no cover - depends on the torch build
+        stage(f"end-to-end graph capture refused ({type(e).__name__}: {e}); eager calls")
+        graph = None
+        torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
         barrier(ws)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(K):
-            step()
+            if graph is not None:
+                graph.replay()
+            else:
+                step(stream, True)
         e1.record(stream)
         torch.cuda.synchronize()
     barrier(ws)
     ms = e0.elapsed_time(e1)
     max_ms, units, value = aggregate(ms, args.batch * stack.n_nodes * K, ws, device)
+    if graph is not None:
+        del graph
+    api = ("gdn_tree_plan + gdn_tree_verify(_planned) x 48 + gdn_tree_commit_layers with pinned host buffers: "
+           "one packed input copy per layer on a copy stream and one output read per layer on a third stream, "
+           "overlapped with the launches within a step; ")
+    api += ("the step captured once as a CUDA graph and replayed per step (copies included)" if mode == "graph"
+            else "eager ctypes calls")
     return {"value": value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "steps": K, "ms_per_step": max_ms / K,
-            "api": "gdn_tree_verify x 48 + gdn_tree_commit_layers (eager ctypes calls); pinned host buffers, "
-                   "one packed input copy per layer on a copy stream and one output read per layer on a "
-                   "third stream, overlapped with the launches within a step"}
+            "steps": K, "ms_per_step": max_ms / K, "mode": mode, "api": api}
 
 
 # ----------------------------------------------------------------------------
