@@ -46,13 +46,18 @@
 //
 // One CTA per (sequence, v-head, 128 rows of d_v), 9 warps: warps 0-3 own
 // the state rows (one row per thread: the elementwise steps between the
-// products), warps 4-7 stage inputs and prepare each chunk's S-independent
-// operands one chunk ahead, warp 8 issues the MMAs.  Hand-offs are
-// mbarriers; every wait is bounded and a timeout is reported as a status.
+// products), warps 4-7 prepare each chunk's S-independent operands one chunk
+// ahead, warp 8 issues the MMAs.  k, q and v arrive by TMA (tensor maps over
+// this GPU's q, k and v; one thread issues the copies, an mbarrier counts
+// the bytes), and each chunk's outputs leave as one TMA store of a 64-token
+// x 128-row tile staged in shared memory.  Hand-offs are mbarriers; every
+// wait is bounded and a timeout is reported as a status.
 
 #include <atomic>
 #include <cstdint>
+#include <mutex>
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -77,7 +82,8 @@ constexpr uint32_t kColAS = 128;  // S in 3 bf16 parts, 64 columns each (A of X^
 constexpr uint32_t kColAP = 128;  //   after that product: P^T in 3 parts of 32 columns
 constexpr uint32_t kColU = 224;   //   and U^T, f32 [d_v x T]
 constexpr uint32_t kColAUr = 128; //   after that: U^T diag(r) in 3 parts (A of the update)
-constexpr uint32_t kColAU = 224;  //   and U^T in 2 parts (A of U^T M^T)
+constexpr uint32_t kColAU0 = 288;  //   and U^T in 2 parts (A of U^T M^T): part 0 in the
+constexpr uint32_t kColAU1 = 224;  //   spare columns, part 1 over the first half of U^T
 constexpr uint32_t kColX = 320;   // X^T, f32 [d_v x T]; later U^T M^T
 constexpr uint32_t kColY = 384;   // Y^T, f32 [d_v x T]
 constexpr uint32_t kColKQ = 448;  // [K; Q] K^T, f32 [2T x T] (lanes = K rows, then Q rows)
@@ -91,12 +97,14 @@ constexpr int kTTBytes = T * T * 2;       // one bf16 part of a 64 x 64 operand
 constexpr int kKTBytes = DK * T * 2;      // K^T, 128 rows x 64 tokens
 constexpr int LST = T + 1;                // f32 row stride of L and M
 constexpr int AST = T + 4;                // f32 row stride of the inverse (16-byte rows)
+constexpr int kOutBytes = T * TM * 4;     // one chunk's outputs, f32 [t][row]
 constexpr int kOffKQ = 0;                          // [2]
-constexpr int kOffV = kOffKQ + 2 * kKQBytes;       // [2]
-constexpr int kOffAb = kOffV + 2 * kVBytes;        // [3 parts]
+constexpr int kOffV = kOffKQ + 2 * kKQBytes;
+constexpr int kOffAb = kOffV + kVBytes;            // [3 parts]
 constexpr int kOffM = kOffAb + 3 * kTTBytes;       // [2 parts]
 constexpr int kOffKT = kOffM + 2 * kTTBytes;
-constexpr int kOffL = kOffKT + kKTBytes;           // L, f32 [T][LST]
+constexpr int kOffOut = kOffKT + kKTBytes;
+constexpr int kOffL = kOffOut + kOutBytes;         // L, f32 [T][LST]
 constexpr int kOffMf = kOffL + T * LST * 4;        // M, f32 [T][LST]
 constexpr int kOffAi = kOffMf + T * LST * 4;       // (I + L)^-1, f32 [T][AST]
 constexpr int kOffGB = kOffAi + T * AST * 4;       // [2][g | beta], f32
@@ -104,10 +112,11 @@ constexpr int kOffDec = kOffGB + 2 * 2 * T * 4;    // [3][Gamma | r], f32
 constexpr int kOffA = kOffDec + 3 * 2 * T * 4;     // a = exp(g), f32 [T]
 constexpr int kOffBar = kOffA + T * 4;             // mbarriers, tmem base, abort flag
 constexpr int kSmem = kOffBar + 256;
+static_assert(kSmem <= 227 * 1024, "shared memory");
 
 // mbarriers (index into the array at kOffBar)
 enum Bar {
-    kKqFull0 = 0,  // chunk inputs staged in buffer 0 / 1 (128 preparation threads)
+    kKqFull0 = 0,  // k, q of a chunk landed in buffer 0 / 1 (TMA bytes)
     kKqFull1 = 1,
     kKqMma = 2,    // [K; Q] K^T done (MMA commit)
     kKqFree = 3,   // [K; Q] K^T read out (128)
@@ -121,7 +130,8 @@ enum Bar {
     kMktReady = 13,// M parts and K^T written (128)
     kCdDone = 14,  // update and U^T M^T done (commit)
     kFin = 15,     // all MMAs retired (commit)
-    kNumBars = 16
+    kVFull = 16,   // v of a chunk landed (TMA bytes)
+    kNumBars = 17
 };
 
 struct Params {
@@ -252,6 +262,20 @@ struct Sync {
     __device__ __forceinline__ void arrive(int b) const { mbar_arrive(bar + b); }
 };
 
+// Whether the phase with the given parity has completed, without waiting.
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity)
+{
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
 // Named barrier over the 128 preparation threads.
 __device__ __forceinline__ void prep_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
@@ -271,14 +295,23 @@ __device__ __forceinline__ bool prep_all(bool ok)
     return r != 0;
 }
 
-// Whether ok holds for the whole warp (tensor-memory accesses are warp-wide).
-__device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xffffffffu, ok); }
-
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src)
+// Named barrier over the 128 row threads, and the same with a vote.
+__device__ __forceinline__ void row_sync() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
+
+__device__ __forceinline__ bool row_all(bool ok)
 {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, 2, 128, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(ok ? 1u : 0u)
+        : "memory");
+    return r != 0;
 }
 
 __device__ __forceinline__ void cp_async4(uint32_t dst, const void* src)
@@ -286,132 +319,178 @@ __device__ __forceinline__ void cp_async4(uint32_t dst, const void* src)
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
 }
 
+// ---- TMA -------------------------------------------------------------------------------------
+
+// The barrier's current phase also waits for `bytes` bytes of TMA data.
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+// Box of a 4-d tensor map at (x, y, z, w) into shared memory (no multicast);
+// completion counted in bytes on bar.  Elements outside the tensor read 0.
+__device__ __forceinline__ void tma_load(uint32_t dst, const CUtensorMap* tm, int x, int y, int z, int w,
+                                         uint64_t* bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], "
+        "[%6];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_addr(bar))
+        : "memory");
+}
+
+// Shared memory to the box of a 4-d tensor map at (x, y, z, w); elements
+// outside the tensor are not written.
+__device__ __forceinline__ void tma_store(const CUtensorMap* tm, uint32_t src, int x, int y, int z, int w)
+{
+    asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(tm)),
+                 "r"(src), "r"(x), "r"(y), "r"(z), "r"(w)
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+struct Maps {
+    CUtensorMap k, q, v, out;  // 4-d: (d, head, token, sequence)
+};
+
 // ---- preparation warps ---------------------------------------------------------------
 
-// Stage chunk c's k and q rows (canonical layout, K rows 0..63 then Q rows),
-// the CTA's 128-row slice of v ([t][row]), g and beta.  Tokens past the
-// chain's end and rows past d_v are zero (k = q = v = 0, beta = 0, g = 0:
-// they leave the state unchanged; their outputs are not written).
-__device__ void stage_chunk(const Params& p, unsigned char* smem, int buf, int c, int b, int h, int hk, int row0,
-                            int ptid)
+// Chunk c's k and q rows into buffer buf in the canonical layout (K rows
+// 0..63, then Q rows): one copy per 8-column piece, 64 tokens each.  Tokens
+// past the chain's end read 0.  One thread.
+__device__ __forceinline__ void load_kq(const Maps& mp, unsigned char* smem, uint64_t* bar, int buf, int c, int b,
+                                        int hk)
 {
-    const int t0 = c * T;
     const uint32_t kq = smem_addr(smem + kOffKQ + buf * kKQBytes);
-    const uint32_t vb = smem_addr(smem + kOffV + buf * kVBytes);
-    for (int i = ptid; i < 2 * T * (DK / 8); i += 128) {
-        const int which = i / (T * (DK / 8));
-        const int t = (i / (DK / 8)) % T, pc = i % (DK / 8);
-        const int n = which * T + t;
-        const uint32_t dst = kq + pc * (2 * T * 16) + (n >> 3) * 128 + (n & 7) * 16;
-        if (t0 + t < p.N) {
-            const size_t node = (size_t)b * p.N + t0 + t;
-            cp_async16(dst, (which == 0 ? p.k : p.q) + (node * p.Hk + hk) * DK + pc * 8);
-        } else {
-            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
-        }
+    mbar_expect_tx(bar, kKQBytes);
+#pragma unroll 1
+    for (int pc = 0; pc < DK / 8; ++pc) {
+        tma_load(kq + pc * (2 * T * 16), &mp.k, 8 * pc, hk, c * T, b, bar);
+        tma_load(kq + pc * (2 * T * 16) + T * 16, &mp.q, 8 * pc, hk, c * T, b, bar);
     }
-    for (int i = ptid; i < T * (TM / 8); i += 128) {
-        const int t = i / (TM / 8), pc = i % (TM / 8);
-        const uint32_t dst = vb + t * (TM * 2) + pc * 16;
-        if (t0 + t < p.N && row0 + pc * 8 < p.dv) {
-            const size_t node = (size_t)b * p.N + t0 + t;
-            cp_async16(dst, p.v + (node * p.Hv + h) * p.dv + row0 + pc * 8);
-        } else {
-            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
-        }
-    }
-    {
-        const int t = ptid & (T - 1), which = ptid >> 6;  // 0: g, 1: beta
-        const uint32_t dst = smem_addr(smem + kOffGB) + (buf * 2 * T + which * T + t) * 4;
-        if (t0 + t < p.N) {
-            const size_t gi = ((size_t)b * p.N + t0 + t) * p.Hv + h;
-            cp_async4(dst, (which == 0 ? p.g : p.beta) + gi);
-        } else {
-            asm volatile("st.shared.u32 [%0], %1;" ::"r"(dst), "r"(0u) : "memory");
-        }
+}
+
+// Chunk c's 128-row slice of v, [t][row]; rows past d_v and tokens past the
+// end read 0.  One thread.
+__device__ __forceinline__ void load_v(const Maps& mp, unsigned char* smem, uint64_t* bar, int c, int b, int h,
+                                       int row0)
+{
+    mbar_expect_tx(bar, kVBytes);
+    tma_load(smem_addr(smem + kOffV), &mp.v, row0, h, c * T, b, bar);
+}
+
+// g and beta of chunk c into buffer buf (0 past the end: a = 1, beta = 0);
+// one element per thread.
+__device__ __forceinline__ void load_gb(const Params& p, unsigned char* smem, int buf, int c, int b, int h, int ptid)
+{
+    const int t = ptid & (T - 1), which = ptid >> 6;  // 0: g, 1: beta
+    const uint32_t dst = smem_addr(smem + kOffGB) + (buf * 2 * T + which * T + t) * 4;
+    if (c * T + t < p.N) {
+        const size_t gi = ((size_t)b * p.N + c * T + t) * p.Hv + h;
+        cp_async4(dst, (which == 0 ? p.g : p.beta) + gi);
+    } else {
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(dst), "r"(0u) : "memory");
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
 }
 
+// Rows 16 I .. 16 I + 15 of block column J of (I + L)^-1 (columns c0 .. c0 +
+// NC - 1 for this lane, row i = lane % 16) for I = J + 1 .. 3, from the
+// diagonal blocks' inverses already in Ai: X = -L_(I, J..I-1) Ai_(J..I-1, J),
+// then Ai_(I, J) = Ai_(I, I) X.  One warp; the rows it reads are its own.
+template <int NC>
+__device__ __forceinline__ void block_column(const float* L, float* Ai, int J, int c0, int lane)
+{
+    const int i = lane & 15;
+#pragma unroll 1
+    for (int I = J + 1; I < 4; ++I) {
+        const int R0 = 16 * I;
+        float x[NC];
+#pragma unroll
+        for (int e = 0; e < NC; ++e)
+            x[e] = 0.f;
+        const float* Lr = L + (R0 + i) * LST;
+#pragma unroll 4
+        for (int k = 16 * J; k < R0; ++k) {
+            const float l = Lr[k];
+#pragma unroll
+            for (int e = 0; e < NC; e += 4) {
+                const float4 a = *reinterpret_cast<const float4*>(Ai + k * AST + c0 + e);
+                x[e] = __fmaf_rn(-l, a.x, x[e]);
+                x[e + 1] = __fmaf_rn(-l, a.y, x[e + 1]);
+                x[e + 2] = __fmaf_rn(-l, a.z, x[e + 2]);
+                x[e + 3] = __fmaf_rn(-l, a.w, x[e + 3]);
+            }
+        }
+        float* dst = Ai + (R0 + i) * AST + c0;
+#pragma unroll
+        for (int e = 0; e < NC; e += 4)
+            *reinterpret_cast<float4*>(dst + e) = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
+        __syncwarp();
+        float y[NC];
+#pragma unroll
+        for (int e = 0; e < NC; ++e)
+            y[e] = 0.f;
+        const float* Dr = Ai + (R0 + i) * AST + R0;  // row i of the block's inverse
+#pragma unroll 4
+        for (int i2 = 0; i2 < 16; ++i2) {
+            const float dd = i2 <= i ? Dr[i2] : 0.f;
+#pragma unroll
+            for (int e = 0; e < NC; e += 4) {
+                const float4 a = *reinterpret_cast<const float4*>(Ai + (R0 + i2) * AST + c0 + e);
+                y[e] = __fmaf_rn(dd, a.x, y[e]);
+                y[e + 1] = __fmaf_rn(dd, a.y, y[e + 1]);
+                y[e + 2] = __fmaf_rn(dd, a.z, y[e + 2]);
+                y[e + 3] = __fmaf_rn(dd, a.w, y[e + 3]);
+            }
+        }
+        __syncwarp();
+#pragma unroll
+        for (int e = 0; e < NC; e += 4)
+            *reinterpret_cast<float4*>(dst + e) = make_float4(y[e], y[e + 1], y[e + 2], y[e + 3]);
+        __syncwarp();
+    }
+}
+
 // (I + L)^-1 for the unit lower triangular I + L (L strictly lower, f32
-// [T][LST]) into Ai (f32 [T][AST], whose entries above the diagonal stay 0):
-// the four 16 x 16 diagonal blocks by forward substitution, one column per
-// thread; then block rows 1..3, X = -L_(I, <I) Ai_(<I, <I) and
-// Ai_(I, <I) = Ai_(I,I) X, 8 columns of one row per thread.
+// [T][LST]) into Ai (f32 [T][AST], whose entries above the diagonal stay 0).
+// Warp w inverts diagonal block w (one column per lane); then the block
+// columns, each by its own warp (block column 0 split over warps 0 and 1),
+// with no barrier between warps until the end.
 __device__ void invert_unit_lower(const float* L, float* Ai, int ptid)
 {
-    if (ptid < T) {
-        const int blk = ptid >> 4, j = ptid & 15;
-        const float* Lb = L + (16 * blk) * LST + 16 * blk;
+    const int pw = ptid >> 5, lane = ptid & 31;
+    if (lane < 16) {
+        const float* __restrict__ Lb = L + (16 * pw) * LST + 16 * pw;
+        const int j = lane;
         float d[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             float acc = 0.f;
 #pragma unroll
             for (int k = 0; k < i; ++k)
-                acc = __fmaf_rn(Lb[i * LST + k], k >= j ? d[k] : 0.f, acc);
+                acc = __fmaf_rn(Lb[i * LST + k], d[k], acc);  // d[k] = 0 for k < j
             d[i] = i < j ? 0.f : (i == j ? 1.f : -acc);
-            Ai[(16 * blk + i) * AST + 16 * blk + j] = d[i];
         }
+        float* Ac = Ai + (16 * pw) * AST + 16 * pw + j;
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            Ac[i * AST] = d[i];
     }
     prep_sync();
-#pragma unroll 1
-    for (int I = 1; I < 4; ++I) {
-        const int R0 = 16 * I;
-        const int i = ptid & 15, c0 = 8 * (ptid >> 4);  // row of the block row, first of 8 columns
-        const bool act = c0 < R0;
-        float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        if (act) {
-            const float* Lr = L + (R0 + i) * LST;
-            for (int k = c0; k < R0; ++k) {  // Ai[k][c] = 0 for k < c
-                const float l = Lr[k];
-                const float4 a0 = *reinterpret_cast<const float4*>(Ai + k * AST + c0);
-                const float4 a1 = *reinterpret_cast<const float4*>(Ai + k * AST + c0 + 4);
-                x[0] = __fmaf_rn(-l, a0.x, x[0]);
-                x[1] = __fmaf_rn(-l, a0.y, x[1]);
-                x[2] = __fmaf_rn(-l, a0.z, x[2]);
-                x[3] = __fmaf_rn(-l, a0.w, x[3]);
-                x[4] = __fmaf_rn(-l, a1.x, x[4]);
-                x[5] = __fmaf_rn(-l, a1.y, x[5]);
-                x[6] = __fmaf_rn(-l, a1.z, x[6]);
-                x[7] = __fmaf_rn(-l, a1.w, x[7]);
-            }
-            float* dst = Ai + (R0 + i) * AST + c0;  // X in the block's own place
-            *reinterpret_cast<float4*>(dst) = make_float4(x[0], x[1], x[2], x[3]);
-            *reinterpret_cast<float4*>(dst + 4) = make_float4(x[4], x[5], x[6], x[7]);
-        }
-        prep_sync();
-        if (act) {
-            float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            const float* Dr = Ai + (R0 + i) * AST + R0;  // the block's inverse, row i
-            for (int i2 = 0; i2 <= i; ++i2) {
-                const float dd = Dr[i2];
-                const float4 a0 = *reinterpret_cast<const float4*>(Ai + (R0 + i2) * AST + c0);
-                const float4 a1 = *reinterpret_cast<const float4*>(Ai + (R0 + i2) * AST + c0 + 4);
-                y[0] = __fmaf_rn(dd, a0.x, y[0]);
-                y[1] = __fmaf_rn(dd, a0.y, y[1]);
-                y[2] = __fmaf_rn(dd, a0.z, y[2]);
-                y[3] = __fmaf_rn(dd, a0.w, y[3]);
-                y[4] = __fmaf_rn(dd, a1.x, y[4]);
-                y[5] = __fmaf_rn(dd, a1.y, y[5]);
-                y[6] = __fmaf_rn(dd, a1.z, y[6]);
-                y[7] = __fmaf_rn(dd, a1.w, y[7]);
-            }
-            x[0] = y[0], x[1] = y[1], x[2] = y[2], x[3] = y[3];
-            x[4] = y[4], x[5] = y[5], x[6] = y[6], x[7] = y[7];
-        }
-        prep_sync();
-        if (act) {
-            float* dst = Ai + (R0 + i) * AST + c0;
-            *reinterpret_cast<float4*>(dst) = make_float4(x[0], x[1], x[2], x[3]);
-            *reinterpret_cast<float4*>(dst + 4) = make_float4(x[4], x[5], x[6], x[7]);
-        }
-        prep_sync();
-    }
+    if (pw < 2)
+        block_column<4>(L, Ai, 0, 8 * pw + 4 * (lane >> 4), lane);
+    else
+        block_column<8>(L, Ai, pw - 1, 16 * (pw - 1) + 8 * (lane >> 4), lane);
+    prep_sync();
 }
 
-__device__ void prep_role(const Params& p, unsigned char* smem, const Sync& sy, uint32_t tbase, int b, int h,
-                          int hk, int row0, int n_chunks)
+// kq_loads[j]: k/q loads this thread issued into buffer j (thread 0 only).
+__device__ void prep_role(const Params& p, const Maps& mp, unsigned char* smem, const Sync& sy, uint32_t tbase,
+                          int b, int h, int hk, int n_chunks, int (&kq_loads)[2])
 {
     const int ptid = threadIdx.x - kPrep0;
     const int pw = ptid >> 5;                  // lane quarter of tensor memory
@@ -424,76 +503,108 @@ __device__ void prep_role(const Params& p, unsigned char* smem, const Sync& sy, 
 
     for (int i = ptid; i < T * AST; i += 128)
         Ai[i] = 0.f;
-    stage_chunk(p, smem, 0, 0, b, h, hk, row0, ptid);
+    if (ptid == 0) {
+        load_kq(mp, smem, sy.bar + kKqFull0, 0, 0, b, hk);
+        ++kq_loads[0];
+        if (n_chunks > 1) {
+            load_kq(mp, smem, sy.bar + kKqFull1, 1, 1, b, hk);
+            ++kq_loads[1];
+        }
+    }
+    load_gb(p, smem, 0, 0, b, h, ptid);
     if (n_chunks > 1)
-        stage_chunk(p, smem, 1, 1, b, h, hk, row0, ptid);
+        load_gb(p, smem, 1, 1, b, h, ptid);
 
     for (int c = 0; c < n_chunks; ++c) {
         const int buf = c & 1, slot = c % 3;
         const float* gb = reinterpret_cast<const float*>(smem + kOffGB) + buf * 2 * T;
         float* Gam = reinterpret_cast<float*>(smem + kOffDec) + slot * 2 * T;
         float* rv = Gam + T;
-        // 1. this chunk's inputs have landed
+        // 1. this chunk's g and beta; decays a = exp(g), then Gamma_t =
+        //    a_0 ... a_t and r_t = a_{t+1} ... a_{T-1} by thread t of the K rows
         if (c == 0 && n_chunks > 1)
             asm volatile("cp.async.wait_group 1;" ::: "memory");
         else
             asm volatile("cp.async.wait_group 0;" ::: "memory");
-        fence_proxy_async();
-        sy.arrive(kKqFull0 + buf);
         prep_sync();
         if (ptid < T)
             av[ptid] = expf(gb[ptid]);
         prep_sync();
-        // 2. read this thread's row of [K; Q] K^T; the row's decays
-        //    R[t][i] = a_{i+1} ... a_t come from a running product over i
-        //    from t down to 0, which ends at Gamma_t
+        if (!qrow) {
+            float gm = 1.f, rr = 1.f;
+#pragma unroll
+            for (int e = 0; e < T / 4; ++e) {
+                const float4 a4 = reinterpret_cast<const float4*>(av)[e];
+                const float a[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+                for (int f = 0; f < 4; ++f) {
+                    if (4 * e + f <= t)
+                        gm = __fmul_rn(gm, a[f]);
+                    else
+                        rr = __fmul_rn(rr, a[f]);
+                }
+            }
+            Gam[t] = gm;
+            rv[t] = rr;
+        }
+        sy.arrive(kDec0 + slot);
+        // 2. this thread's row of [K; Q] K^T times the row's decays
+        //    R[t][i] = a_{i+1} ... a_t, a running product over i from t down
+        //    to 0: L (K rows) and M (Q rows)
         if (!prep_all(sy.wait(kKqMma, c & 1)))
             return;
         tmem_fence_after_sync();
-        uint32_t d[64];
         {
-            uint32_t (&d0)[32] = *reinterpret_cast<uint32_t(*)[32]>(d);
-            uint32_t (&d1)[32] = *reinterpret_cast<uint32_t(*)[32]>(d + 32);
+            const float bt = gb[T + t];
+            float* rowp = (qrow ? Mf : L) + t * LST;
             const uint32_t ta = tbase + ((uint32_t)(32 * pw) << 16) + kColKQ;
-            tmem_ld32(ta, d0);
-            tmem_ld32(ta + 32, d1);
+            float run = 1.f;
+#pragma unroll 1
+            for (int hs = 1; hs >= 0; --hs) {
+                uint32_t d[32];
+                float a[32];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float4 x = reinterpret_cast<const float4*>(av + 32 * hs)[e];
+                    a[4 * e] = x.x, a[4 * e + 1] = x.y, a[4 * e + 2] = x.z, a[4 * e + 3] = x.w;
+                }
+                tmem_ld32(ta + 32 * hs, d);
+                float val[32];
+#pragma unroll
+                for (int e = 31; e >= 0; --e) {
+                    const int i = 32 * hs + e;
+                    const float kk = __uint_as_float(d[e]);
+                    if (qrow)
+                        val[e] = i <= t ? __fmul_rn(kk, run) : 0.f;
+                    else
+                        val[e] = i < t ? __fmul_rn(bt, __fmul_rn(kk, run)) : 0.f;
+                    if (i <= t)
+                        run = __fmul_rn(run, a[e]);
+                }
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    rowp[32 * hs + e] = val[e];
+            }
         }
         tmem_fence_before_sync();
         sy.arrive(kKqFree);
-        {
-            const float bt = gb[T + t];
-            float* row = (qrow ? Mf : L) + t * LST;
-            float run = 1.f;
-#pragma unroll
-            for (int i = T - 1; i >= 0; --i) {
-                const float kk = __uint_as_float(d[i]);
-                float val;
-                if (qrow)
-                    val = i <= t ? __fmul_rn(kk, run) : 0.f;
-                else
-                    val = i < t ? __fmul_rn(bt, __fmul_rn(kk, run)) : 0.f;
-                row[i] = val;
-                if (!qrow && t == T - 1)
-                    rv[i] = run;
-                if (i <= t)
-                    run = __fmul_rn(run, av[i]);
-            }
-            if (!qrow)
-                Gam[t] = run;
-        }
-        sy.arrive(kDec0 + slot);
         prep_sync();
         // 3. Ai = (I + L)^-1
         invert_unit_lower(L, Ai, ptid);
-        // 4. Ab = Ai diag(beta) in 3 bf16 parts, once the previous chunk's
-        //    U^T product is done with them; then stage chunk c + 1 into the
-        //    buffer the previous chunk has left
+        // 4. once the previous chunk's U^T product is done with Ab (and with
+        //    the buffers of chunk c - 1): chunk c + 1's k, q, g and beta start
+        //    loading; Ab = Ai diag(beta) in 3 bf16 parts
         if (c > 0) {
             if (!prep_all(sy.wait(kUDone, (c - 1) & 1)))
                 return;
+            if (ptid == 0 && c + 1 < n_chunks) {
+                load_kq(mp, smem, sy.bar + kKqFull0 + ((c + 1) & 1), (c + 1) & 1, c + 1, b, hk);
+                ++kq_loads[(c + 1) & 1];
+            }
             if (c + 1 < n_chunks)
-                stage_chunk(p, smem, (c + 1) & 1, c + 1, b, h, hk, row0, ptid);
+                load_gb(p, smem, (c + 1) & 1, c + 1, b, h, ptid);
         }
+#pragma unroll 1
         for (int it = ptid; it < T * (T / 8); it += 128) {
             const int tt = it & (T - 1), pc = it >> 6;
             const float4 a0 = *reinterpret_cast<const float4*>(Ai + tt * AST + 8 * pc);
@@ -520,9 +631,10 @@ __device__ void prep_role(const Params& p, unsigned char* smem, const Sync& sy, 
         fence_proxy_async();
         sy.arrive(kAbReady);
         // 5. M in 2 bf16 parts and K^T, once the previous chunk's update and
-        //    U^T M^T products are done with them
-        if (c > 0 && !prep_all(sy.wait(kCdDone, (c - 1) & 1)))
+        //    U^T M^T products are done with them (and this chunk's k is in)
+        if (!prep_all((c == 0 || sy.wait(kCdDone, (c - 1) & 1)) && sy.wait(kKqFull0 + buf, (c >> 1) & 1)))
             return;
+#pragma unroll 1
         for (int it = ptid; it < T * (T / 8); it += 128) {
             const int tt = it & (T - 1), pc = it >> 6;
             const float* mr = Mf + tt * LST + 8 * pc;
@@ -597,53 +709,59 @@ __device__ void mma_role(unsigned char* smem, const Sync& sy, uint32_t tbase, in
             return;
         tmem_fence_after_sync();
 #pragma unroll
-        for (int part = 0; part < 3; ++part)
-#pragma unroll
-            for (int ks = 0; ks < DK / 16; ++ks)
-                mma_ts(tbase + kColX, tbase + kColAS + 64 * part + 8 * ks, kdesc(kq + ks * 2 * kKQLbo, kKQLbo),
-                       idesc_bf16(2 * T), (part | ks) != 0 ? 1u : 0u);
+        for (int q = 0; q < 3 * (DK / 16); ++q) {
+            const int part = q >> 3, ks = q & 7;
+            mma_ts(tbase + kColX, tbase + kColAS + 64 * part + 8 * ks, kdesc(kq + ks * 2 * kKQLbo, kKQLbo),
+                   idesc_bf16(2 * T), q != 0 ? 1u : 0u);
+        }
         mma_commit(sy.bar + kXyDone);
-        // the next chunk's [K; Q] K^T
-        if (c + 1 < n_chunks) {
-            if (!sy.wait(kKqFull0 + ((c + 1) & 1), ((c + 1) >> 1) & 1) || !sy.wait(kKqFree, c & 1))
+        // the next chunk's [K; Q] K^T and this chunk's U^T = P^T Ab^T, in
+        // the order their operands become ready; U^T from the part products
+        // (P, Ab) of weight at least 2^-16
+        bool kq_done = c + 1 >= n_chunks, u_done = false;
+        const long long t0 = clock64();
+        while (!(kq_done && u_done)) {
+            if (*sy.abort || clock64() - t0 > (1ll << 31)) {
+                *sy.abort = 1;
+                report_status(sy.status, kStatusTimeout);
                 return;
-            tmem_fence_after_sync();
-            kq_product(c + 1);
-        }
-        // U^T = P^T Ab^T: part products (P, Ab) with at most 2^-16 weight
-        if (!sy.wait(kApReady, c & 1) || !sy.wait(kAbReady, c & 1))
-            return;
-        tmem_fence_after_sync();
-        {
-            const int pp[6] = {0, 0, 1, 0, 1, 2}, pa[6] = {0, 1, 0, 2, 1, 0};
+            }
+            if (!kq_done && mbar_test(sy.bar + kKqFull0 + ((c + 1) & 1), ((c + 1) >> 1) & 1) &&
+                mbar_test(sy.bar + kKqFree, c & 1)) {
+                tmem_fence_after_sync();
+                kq_product(c + 1);
+                kq_done = true;
+            }
+            if (!u_done && mbar_test(sy.bar + kApReady, c & 1) && mbar_test(sy.bar + kAbReady, c & 1)) {
+                tmem_fence_after_sync();
 #pragma unroll
-            for (int q = 0; q < 6; ++q)
-#pragma unroll
-                for (int ks = 0; ks < T / 16; ++ks)
-                    mma_ts(tbase + kColU, tbase + kColAP + 32 * pp[q] + 8 * ks,
-                           kdesc(ab + pa[q] * kTTBytes + ks * 2 * kTTLbo, kTTLbo), idesc_bf16(T),
-                           (q | ks) != 0 ? 1u : 0u);
+                for (int q = 0; q < 6 * (T / 16); ++q) {
+                    const int pr = q >> 2, ks = q & 3;
+                    const int pp = pr == 2 ? 1 : (pr == 4 ? 1 : (pr == 5 ? 2 : 0));  // (0,0) (0,1) (1,0) (0,2) (1,1) (2,0)
+                    const int pa = pr == 1 ? 1 : (pr == 3 ? 2 : (pr == 4 ? 1 : 0));
+                    mma_ts(tbase + kColU, tbase + kColAP + 32 * pp + 8 * ks,
+                           kdesc(ab + pa * kTTBytes + ks * 2 * kTTLbo, kTTLbo), idesc_bf16(T), q != 0 ? 1u : 0u);
+                }
+                mma_commit(sy.bar + kUDone);
+                u_done = true;
+            }
         }
-        mma_commit(sy.bar + kUDone);
         // S += (U^T diag(r)) K and U^T M^T
         if (!sy.wait(kAuReady, c & 1) || !sy.wait(kMktReady, c & 1))
             return;
         tmem_fence_after_sync();
 #pragma unroll
-        for (int part = 0; part < 3; ++part)
+        for (int q = 0; q < 3 * (T / 16); ++q) {
+            const int part = q >> 2, ks = q & 3;
+            mma_ts(tbase + kColS, tbase + kColAUr + 32 * part + 8 * ks, kdesc(kt + ks * 2 * kKTLbo, kKTLbo),
+                   idesc_bf16(DK), 1u);
+        }
 #pragma unroll
-            for (int ks = 0; ks < T / 16; ++ks)
-                mma_ts(tbase + kColS, tbase + kColAUr + 32 * part + 8 * ks, kdesc(kt + ks * 2 * kKTLbo, kKTLbo),
-                       idesc_bf16(DK), 1u);
-        {
-            const int pu[3] = {0, 0, 1}, pm[3] = {0, 1, 0};
-#pragma unroll
-            for (int q = 0; q < 3; ++q)
-#pragma unroll
-                for (int ks = 0; ks < T / 16; ++ks)
-                    mma_ts(tbase + kColX, tbase + kColAU + 32 * pu[q] + 8 * ks,
-                           kdesc(mm + pm[q] * kTTBytes + ks * 2 * kTTLbo, kTTLbo), idesc_bf16(T),
-                           (q | ks) != 0 ? 1u : 0u);
+        for (int q = 0; q < 3 * (T / 16); ++q) {
+            const int pr = q >> 2, ks = q & 3;  // (U, M) parts: (0,0) (0,1) (1,0)
+            const uint32_t au = pr == 2 ? kColAU1 : kColAU0;
+            mma_ts(tbase + kColX, tbase + au + 8 * ks, kdesc(mm + (pr == 1 ? kTTBytes : 0) + ks * 2 * kTTLbo, kTTLbo),
+                   idesc_bf16(T), q != 0 ? 1u : 0u);
         }
         mma_commit(sy.bar + kCdDone);
     }
@@ -651,54 +769,69 @@ __device__ void mma_role(unsigned char* smem, const Sync& sy, uint32_t tbase, in
 
 // ---- row warps ----------------------------------------------------------------------------------
 
-// This thread's row of the previous chunk's outputs: scale (Gamma_t Y^T + U^T M^T).
-__device__ __forceinline__ void write_outputs(const Params& p, uint32_t trow, const float* Gam, int b, int h,
-                                              int row, int t0)
+// The previous chunk's outputs, scale (Gamma_t Y^T + U^T M^T): each thread
+// writes its row of the [t][row] tile in shared memory, then one thread
+// stores the tile with TMA (after the previous store has read it).
+__device__ __forceinline__ void write_outputs(const Params& p, const Maps& mp, unsigned char* smem, uint32_t trow,
+                                              const float* Gam, int b, int h, int row0, int t0)
 {
-    const int Tc = min(T, p.N - t0);
-#pragma unroll
+    const int m = threadIdx.x;
+    float* tile = reinterpret_cast<float*>(smem + kOffOut) + m;
+    if (m == 0)
+        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+    row_sync();
+#pragma unroll 1
     for (int hs = 0; hs < 2; ++hs) {
         uint32_t y[32], o[32];
+        float gm[32];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float4 x = reinterpret_cast<const float4*>(Gam + 32 * hs)[e];
+            gm[4 * e] = x.x, gm[4 * e + 1] = x.y, gm[4 * e + 2] = x.z, gm[4 * e + 3] = x.w;
+        }
         tmem_ld32(trow + kColY + 32 * hs, y);
         tmem_ld32(trow + kColX + 32 * hs, o);
-        if (row < p.dv) {
-            float* dst = p.out + ((size_t)b * p.N + t0) * p.Hv * p.dv + (size_t)h * p.dv + row;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int tt = 32 * hs + i;
-                if (tt < Tc)
-                    dst[(size_t)tt * p.Hv * p.dv] =
-                        __fmul_rn(p.scale, __fmaf_rn(Gam[tt], __uint_as_float(y[i]), __uint_as_float(o[i])));
-            }
-        }
+        for (int i = 0; i < 32; ++i)
+            tile[(32 * hs + i) * TM] =
+                __fmul_rn(p.scale, __fmaf_rn(gm[i], __uint_as_float(y[i]), __uint_as_float(o[i])));
     }
+    fence_proxy_async();
+    row_sync();
+    if (m == 0)
+        tma_store(&mp.out, smem_addr(smem + kOffOut), row0, h, t0, b);
 }
 
-__device__ void row_role(const Params& p, unsigned char* smem, const Sync& sy, uint32_t tbase, int b, int h,
-                         int row0, int n_chunks)
+// v_loads: v loads this thread issued (thread 0 issues them all).
+__device__ void row_role(const Params& p, const Maps& mp, unsigned char* smem, const Sync& sy, uint32_t tbase, int b,
+                         int h, int row0, int n_chunks, int& v_loads)
 {
     const int tid = threadIdx.x, warp = tid >> 5;
     const int m = tid;              // state row within the tile (lane quarter = warp)
     const int row = row0 + m;       // row of d_v
     const uint32_t trow = tbase + ((uint32_t)(32 * warp) << 16);
     const float* decs = reinterpret_cast<const float*>(smem + kOffDec);
+    if (tid == 0) {
+        load_v(mp, smem, sy.bar + kVFull, 0, b, h, row0);
+        ++v_loads;
+    }
 
     for (int c = 0; c < n_chunks; ++c) {
         const int slot = c % 3;
         const float* Gam = decs + slot * 2 * T;
         const float* rv = Gam + T;
-        if (!warp_all(sy.wait(kDec0 + slot, (c / 3) & 1)))
+        if (!row_all(sy.wait(kDec0 + slot, (c / 3) & 1)))
             return;
         const float gT = Gam[T - 1];
         // 0. the previous chunk's outputs; S into 3 bf16 parts (A of X^T | Y^T),
         //    and Gamma_{T-1} S back as the update's accumulator
         if (c > 0) {
-            if (!warp_all(sy.wait(kCdDone, (c - 1) & 1)))
+            if (!row_all(sy.wait(kCdDone, (c - 1) & 1)))
                 return;
             tmem_fence_after_sync();
-            write_outputs(p, trow, decs + ((c - 1) % 3) * 2 * T, b, h, row, (c - 1) * T);
+            write_outputs(p, mp, smem, trow, decs + ((c - 1) % 3) * 2 * T, b, h, row0, (c - 1) * T);
         }
-#pragma unroll
+#pragma unroll 1
         for (int s = 0; s < 4; ++s) {
             uint32_t x[32];
             if (c == 0) {
@@ -738,26 +871,30 @@ __device__ void row_role(const Params& p, unsigned char* smem, const Sync& sy, u
         sy.arrive(kAsReady);
 
         // 1. P^T = V^T - X^T diag(Gamma) into 3 bf16 parts (A of U^T)
-        if (!warp_all(sy.wait(kXyDone, c & 1) && sy.wait(kKqFull0 + (c & 1), (c >> 1) & 1)))
+        if (!row_all(sy.wait(kXyDone, c & 1) && sy.wait(kVFull, c & 1)))
             return;
         tmem_fence_after_sync();
         {
-            const unsigned short* V =
-                reinterpret_cast<const unsigned short*>(smem + kOffV + (c & 1) * kVBytes) + m;
-#pragma unroll
+            const unsigned short* V = reinterpret_cast<const unsigned short*>(smem + kOffV) + m;
+#pragma unroll 1
             for (int hs = 0; hs < 2; ++hs) {
                 uint32_t x[32];
+                float gm[32], vv[32];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float4 g4 = reinterpret_cast<const float4*>(Gam + 32 * hs)[e];
+                    gm[4 * e] = g4.x, gm[4 * e + 1] = g4.y, gm[4 * e + 2] = g4.z, gm[4 * e + 3] = g4.w;
+                }
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    vv[e] = __uint_as_float((uint32_t)V[(32 * hs + e) * TM] << 16);
                 tmem_ld32(trow + kColX + 32 * hs, x);
                 uint32_t p1[16], p2[16], p3[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int tt = 32 * hs + 2 * e;
-                    const float v0 = __uint_as_float((uint32_t)V[tt * TM] << 16);
-                    const float v1 = __uint_as_float((uint32_t)V[(tt + 1) * TM] << 16);
-                    split3(__fsub_rn(v0, __fmul_rn(Gam[tt], __uint_as_float(x[2 * e]))),
-                           __fsub_rn(v1, __fmul_rn(Gam[tt + 1], __uint_as_float(x[2 * e + 1]))), p1[e], p2[e],
-                           p3[e]);
-                }
+                for (int e = 0; e < 16; ++e)
+                    split3(__fsub_rn(vv[2 * e], __fmul_rn(gm[2 * e], __uint_as_float(x[2 * e]))),
+                           __fsub_rn(vv[2 * e + 1], __fmul_rn(gm[2 * e + 1], __uint_as_float(x[2 * e + 1]))), p1[e],
+                           p2[e], p3[e]);
                 tmem_st16(trow + kColAP + 16 * hs, p1);
                 tmem_st16(trow + kColAP + 32 + 16 * hs, p2);
                 tmem_st16(trow + kColAP + 64 + 16 * hs, p3);
@@ -767,38 +904,39 @@ __device__ void row_role(const Params& p, unsigned char* smem, const Sync& sy, u
         tmem_fence_before_sync();
         sy.arrive(kApReady);
 
-        // 2. U^T diag(r) in 3 parts (A of the update), U^T in 2 (A of U^T M^T)
-        if (!warp_all(sy.wait(kUDone, c & 1)))
+        // 2. U^T diag(r) in 3 parts (A of the update), U^T in 2 (A of U^T M^T);
+        //    each half of U^T is read before anything is written over it.
+        //    Every row thread is done with this chunk's v: the next one loads.
+        if (!row_all(sy.wait(kUDone, c & 1)))
             return;
+        if (tid == 0 && c + 1 < n_chunks) {
+            load_v(mp, smem, sy.bar + kVFull, c + 1, b, h, row0);
+            ++v_loads;
+        }
         tmem_fence_after_sync();
-        {
-            uint32_t u[64];
-            {
-                uint32_t (&u0)[32] = *reinterpret_cast<uint32_t(*)[32]>(u);
-                uint32_t (&u1)[32] = *reinterpret_cast<uint32_t(*)[32]>(u + 32);
-                tmem_ld32(trow + kColU, u0);
-                tmem_ld32(trow + kColU + 32, u1);
+#pragma unroll 1
+        for (int hs = 0; hs < 2; ++hs) {
+            uint32_t u[32];
+            float rr[32];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float4 r4 = reinterpret_cast<const float4*>(rv + 32 * hs)[e];
+                rr[4 * e] = r4.x, rr[4 * e + 1] = r4.y, rr[4 * e + 2] = r4.z, rr[4 * e + 3] = r4.w;
             }
+            tmem_ld32(trow + kColU + 32 * hs, u);
+            uint32_t p1[16], p2[16], p3[16];
 #pragma unroll
-            for (int hs = 0; hs < 2; ++hs) {
-                uint32_t p1[16], p2[16], p3[16];
+            for (int e = 0; e < 16; ++e)
+                split3(__fmul_rn(rr[2 * e], __uint_as_float(u[2 * e])), __fmul_rn(rr[2 * e + 1], __uint_as_float(u[2 * e + 1])),
+                       p1[e], p2[e], p3[e]);
+            tmem_st16(trow + kColAUr + 16 * hs, p1);
+            tmem_st16(trow + kColAUr + 32 + 16 * hs, p2);
+            tmem_st16(trow + kColAUr + 64 + 16 * hs, p3);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int tt = 32 * hs + 2 * e;
-                    split3(__fmul_rn(rv[tt], __uint_as_float(u[tt])), __fmul_rn(rv[tt + 1], __uint_as_float(u[tt + 1])),
-                           p1[e], p2[e], p3[e]);
-                }
-                tmem_st16(trow + kColAUr + 16 * hs, p1);
-                tmem_st16(trow + kColAUr + 32 + 16 * hs, p2);
-                tmem_st16(trow + kColAUr + 64 + 16 * hs, p3);
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int tt = 32 * hs + 2 * e;
-                    split2(__uint_as_float(u[tt]), __uint_as_float(u[tt + 1]), p1[e], p2[e]);
-                }
-                tmem_st16(trow + kColAU + 16 * hs, p1);
-                tmem_st16(trow + kColAU + 32 + 16 * hs, p2);
-            }
+            for (int e = 0; e < 16; ++e)
+                split2(__uint_as_float(u[2 * e]), __uint_as_float(u[2 * e + 1]), p1[e], p2[e]);
+            tmem_st16(trow + kColAU0 + 16 * hs, p1);
+            tmem_st16(trow + kColAU1 + 16 * hs, p2);
         }
         tmem_wait_st();
         tmem_fence_before_sync();
@@ -806,12 +944,12 @@ __device__ void row_role(const Params& p, unsigned char* smem, const Sync& sy, u
     }
 
     // the last chunk's outputs and the last state -> node_states[b][0][h][row][:]
-    if (!warp_all(sy.wait(kCdDone, (n_chunks - 1) & 1)))
+    if (!row_all(sy.wait(kCdDone, (n_chunks - 1) & 1)))
         return;
     tmem_fence_after_sync();
-    write_outputs(p, trow, decs + ((n_chunks - 1) % 3) * 2 * T, b, h, row, (n_chunks - 1) * T);
+    write_outputs(p, mp, smem, trow, decs + ((n_chunks - 1) % 3) * 2 * T, b, h, row0, (n_chunks - 1) * T);
     const size_t base = (((size_t)b * p.Hv + h) * p.dv + row) * DK;
-#pragma unroll
+#pragma unroll 1
     for (int s = 0; s < 4; ++s) {
         uint32_t x[32];
         tmem_ld32(trow + kColS + 32 * s, x);
@@ -840,7 +978,16 @@ __device__ void row_role(const Params& p, unsigned char* smem, const Sync& sy, u
     }
 }
 
-__global__ void __launch_bounds__(kThreads, 1) gdn_chain_chunked(const Params p)
+// Bounded wait, ignoring the abort flag, for a phase of TMA data this thread
+// asked for: the copy must land before the CTA's shared memory goes away.
+__device__ __forceinline__ void drain(uint64_t* bar, uint32_t parity)
+{
+    const long long t0 = clock64();
+    while (!mbar_try_wait_suspend(bar, parity, 20000u) && clock64() - t0 < (1ll << 31)) {
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) gdn_chain_chunked(const Params p, const __grid_constant__ Maps mp)
 {
     extern __shared__ __align__(1024) unsigned char smem[];
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
@@ -856,7 +1003,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_chain_chunked(const Params p)
     // allocates all 512 columns
     pdl_wait_then_release();
     if (threadIdx.x == 0) {
-        const uint32_t counts[kNumBars] = {128, 128, 1, 128, 128, 128, 128, 128, 1, 128, 128, 1, 128, 128, 1, 1};
+        const uint32_t counts[kNumBars] = {1, 1, 1, 128, 128, 128, 128, 128, 1, 128, 128, 1, 128, 128, 1, 1, 1};
         for (int i = 0; i < kNumBars; ++i)
             mbar_init(bars + i, counts[i]);
         *abort_flag = 0;
@@ -864,17 +1011,36 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_chain_chunked(const Params p)
     }
     if (warp == 0)
         tmem_alloc(tslot, kTmemCols);
+    if (threadIdx.x == 32) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&mp.k)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&mp.q)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&mp.v)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&mp.out)) : "memory");
+    }
     tmem_fence_before_sync();
     __syncthreads();
     tmem_fence_after_sync();
     const uint32_t tbase = *tslot;
     const Sync sy{bars, abort_flag, p.status};
 
+    // Each TMA load is waited for by the thread that issued it before the CTA
+    // can leave (a barrier has at most one phase outstanding: a buffer is
+    // reloaded only after its previous load was used).
     if (warp < 4) {
-        row_role(p, smem, sy, tbase, b, h, row0, n_chunks);
+        int v_loads = 0;
+        row_role(p, mp, smem, sy, tbase, b, h, row0, n_chunks, v_loads);
+        if (threadIdx.x == 0) {
+            if (v_loads > 0)
+                drain(bars + kVFull, (uint32_t)(v_loads - 1) & 1);
+            asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+        }
     } else if (warp < 8) {
-        prep_role(p, smem, sy, tbase, b, h, hk, row0, n_chunks);
+        int kq_loads[2] = {0, 0};
+        prep_role(p, mp, smem, sy, tbase, b, h, hk, n_chunks, kq_loads);
         asm volatile("cp.async.wait_all;" ::: "memory");
+        for (int j = 0; j < 2; ++j)
+            if (kq_loads[j] > 0)
+                drain(bars + kKqFull0 + j, (uint32_t)(kq_loads[j] - 1) & 1);
     } else if ((threadIdx.x & 31) == 0) {
         mma_role(smem, sy, tbase, n_chunks);
         // every MMA issued has retired before the tensor memory is freed
@@ -900,6 +1066,43 @@ bool chunked_supported(const VerifyArgs& a)
            (a.flags & GDN_FLAG_CHAIN) && (a.flags & GDN_FLAG_PERSIST_LAST) && a.cu_nodes == nullptr;
 }
 
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled_fn()
+{
+    static std::once_flag once;
+    static EncodeTiledFn fn = nullptr;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess && f)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+        cudaGetLastError();  // a failed lookup leaves no sticky error behind
+    });
+    return fn;
+}
+
+// A 4-d map (d, head, token, sequence) over a [batch][N][heads][d] tensor,
+// boxes of (box_d, 1, 64, 1); elements outside read as zero.
+bool encode_map(EncodeTiledFn fn, CUtensorMap* m, const void* base, CUtensorMapDataType type, size_t esize,
+                uint64_t d, uint64_t heads, uint64_t N, uint64_t batch, uint32_t box_d)
+{
+    const cuuint64_t dims[4] = {d, heads, N, batch};
+    const cuuint64_t strides[3] = {d * esize, heads * d * esize, N * heads * d * esize};
+    const cuuint32_t box[4] = {box_d, 1, (cuuint32_t)chunked::T, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(m, type, 4, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
 cudaError_t launch_chunked(const VerifyArgs& a, cudaStream_t stream)
 {
     using namespace chunked;
@@ -920,6 +1123,16 @@ cudaError_t launch_chunked(const VerifyArgs& a, cudaStream_t stream)
     p.G = a.n_v_heads / a.n_k_heads;
     p.scale = a.scale;
     p.state_f16 = a.state_dtype == GDN_F16 ? 1 : 0;
+    const EncodeTiledFn fn = encode_tiled_fn();
+    if (fn == nullptr)
+        return cudaErrorNotSupported;
+    Maps mp;
+    const uint64_t N = a.n_nodes, B = a.batch;
+    if (!encode_map(fn, &mp.k, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, a.n_k_heads, N, B, 8) ||
+        !encode_map(fn, &mp.q, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, a.n_k_heads, N, B, 8) ||
+        !encode_map(fn, &mp.v, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.d_v, a.n_v_heads, N, B, TM) ||
+        !encode_map(fn, &mp.out, a.out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.d_v, a.n_v_heads, N, B, TM))
+        return cudaErrorInvalidValue;
     // opt in to kSmem bytes of dynamic shared memory, once per device
     static std::atomic<int> granted[64];
     int dev = 0;
@@ -934,7 +1147,7 @@ cudaError_t launch_chunked(const VerifyArgs& a, cudaStream_t stream)
             granted[dev].store(1);
     }
     dim3 grid((a.d_v + TM - 1) / TM, a.n_v_heads, a.batch);
-    return launch_pdl(gdn_chain_chunked, grid, dim3(kThreads), (size_t)kSmem, stream, p);
+    return launch_pdl(gdn_chain_chunked, grid, dim3(kThreads), (size_t)kSmem, stream, p, mp);
 }
 
 }  // namespace gdn
