@@ -72,7 +72,7 @@ namespace {
 constexpr int T = 64;           // tokens per chunk
 constexpr int DK = 128;         // d_k
 constexpr int TM = 128;         // state rows (d_v) per CTA: the MMAs' M
-constexpr int kThreads = 288;   // warps 0-3 rows, 4-7 preparation, 8 MMA issue
+constexpr int kThreads = 320;   // warps 0-3 rows, 4-7 preparation, 8 MMA issue, 9 k/q loads
 constexpr int kPrep0 = 128;     // first preparation thread
 
 // Tensor-memory columns (128 lanes x 512 columns of 32 bits, all of it).
@@ -119,7 +119,7 @@ enum Bar {
     kKqFull0 = 0,  // k, q of a chunk landed in buffer 0 / 1 (TMA bytes)
     kKqFull1 = 1,
     kKqMma = 2,    // [K; Q] K^T done (MMA commit)
-    kKqFree = 3,   // [K; Q] K^T read out (128)
+    kDkqFree = 3,  // [K; Q] K^T read out (128)
     kDec0 = 4,     // decays of a chunk written, slots 0..2 (128)
     kAsReady = 7,  // state parts written, previous outputs read (128 row threads)
     kXyDone = 8,   // X^T | Y^T done (commit)
@@ -131,7 +131,9 @@ enum Bar {
     kCdDone = 14,  // update and U^T M^T done (commit)
     kFin = 15,     // all MMAs retired (commit)
     kVFull = 16,   // v of a chunk landed (TMA bytes)
-    kNumBars = 17
+    kKqBuf0 = 17,  // k/q buffer 0 / 1 no longer read: the chunk's MMAs (commit) and K^T (128)
+    kKqBuf1 = 18,
+    kNumBars = 19
 };
 
 struct Params {
@@ -488,9 +490,8 @@ __device__ void invert_unit_lower(const float* L, float* Ai, int ptid)
     prep_sync();
 }
 
-// kq_loads[j]: k/q loads this thread issued into buffer j (thread 0 only).
-__device__ void prep_role(const Params& p, const Maps& mp, unsigned char* smem, const Sync& sy, uint32_t tbase,
-                          int b, int h, int hk, int n_chunks, int (&kq_loads)[2])
+__device__ void prep_role(const Params& p, unsigned char* smem, const Sync& sy, uint32_t tbase, int b, int h,
+                          int n_chunks)
 {
     const int ptid = threadIdx.x - kPrep0;
     const int pw = ptid >> 5;                  // lane quarter of tensor memory
@@ -503,14 +504,6 @@ __device__ void prep_role(const Params& p, const Maps& mp, unsigned char* smem, 
 
     for (int i = ptid; i < T * AST; i += 128)
         Ai[i] = 0.f;
-    if (ptid == 0) {
-        load_kq(mp, smem, sy.bar + kKqFull0, 0, 0, b, hk);
-        ++kq_loads[0];
-        if (n_chunks > 1) {
-            load_kq(mp, smem, sy.bar + kKqFull1, 1, 1, b, hk);
-            ++kq_loads[1];
-        }
-    }
     load_gb(p, smem, 0, 0, b, h, ptid);
     if (n_chunks > 1)
         load_gb(p, smem, 1, 1, b, h, ptid);
@@ -587,20 +580,15 @@ __device__ void prep_role(const Params& p, const Maps& mp, unsigned char* smem, 
             }
         }
         tmem_fence_before_sync();
-        sy.arrive(kKqFree);
+        sy.arrive(kDkqFree);
         prep_sync();
         // 3. Ai = (I + L)^-1
         invert_unit_lower(L, Ai, ptid);
-        // 4. once the previous chunk's U^T product is done with Ab (and with
-        //    the buffers of chunk c - 1): chunk c + 1's k, q, g and beta start
-        //    loading; Ab = Ai diag(beta) in 3 bf16 parts
+        // 4. once the previous chunk's U^T product is done with Ab: chunk
+        //    c + 1's g and beta start loading; Ab = Ai diag(beta) in 3 bf16 parts
         if (c > 0) {
             if (!prep_all(sy.wait(kUDone, (c - 1) & 1)))
                 return;
-            if (ptid == 0 && c + 1 < n_chunks) {
-                load_kq(mp, smem, sy.bar + kKqFull0 + ((c + 1) & 1), (c + 1) & 1, c + 1, b, hk);
-                ++kq_loads[(c + 1) & 1];
-            }
             if (c + 1 < n_chunks)
                 load_gb(p, smem, (c + 1) & 1, c + 1, b, h, ptid);
         }
@@ -674,6 +662,26 @@ __device__ void prep_role(const Params& p, const Maps& mp, unsigned char* smem, 
         }
         fence_proxy_async();
         sy.arrive(kMktReady);
+        sy.arrive(kKqBuf0 + buf);
+    }
+}
+
+// ---- k/q loads ---------------------------------------------------------------------------
+
+// One thread: chunks 0 and 1, then chunk c + 2 into buffer c % 2 once chunk
+// c's MMAs and K^T are done with it.  kq_loads[j]: loads issued into buffer j.
+__device__ void load_role(const Maps& mp, unsigned char* smem, const Sync& sy, int b, int hk, int n_chunks,
+                          int (&kq_loads)[2])
+{
+    for (int c = 0; c < n_chunks && c < 2; ++c) {
+        load_kq(mp, smem, sy.bar + kKqFull0 + c, c, c, b, hk);
+        ++kq_loads[c];
+    }
+    for (int c = 0; c + 2 < n_chunks; ++c) {
+        if (!sy.wait(kKqBuf0 + (c & 1), (c >> 1) & 1))
+            return;
+        load_kq(mp, smem, sy.bar + kKqFull0 + (c & 1), c & 1, c + 2, b, hk);
+        ++kq_loads[c & 1];
     }
 }
 
@@ -715,6 +723,7 @@ __device__ void mma_role(unsigned char* smem, const Sync& sy, uint32_t tbase, in
                    idesc_bf16(2 * T), q != 0 ? 1u : 0u);
         }
         mma_commit(sy.bar + kXyDone);
+        mma_commit(sy.bar + kKqBuf0 + (c & 1));  // with [K; Q] K^T of c, issued before
         // the next chunk's [K; Q] K^T and this chunk's U^T = P^T Ab^T, in
         // the order their operands become ready; U^T from the part products
         // (P, Ab) of weight at least 2^-16
@@ -727,7 +736,7 @@ __device__ void mma_role(unsigned char* smem, const Sync& sy, uint32_t tbase, in
                 return;
             }
             if (!kq_done && mbar_test(sy.bar + kKqFull0 + ((c + 1) & 1), ((c + 1) >> 1) & 1) &&
-                mbar_test(sy.bar + kKqFree, c & 1)) {
+                mbar_test(sy.bar + kDkqFree, c & 1)) {
                 tmem_fence_after_sync();
                 kq_product(c + 1);
                 kq_done = true;
@@ -1003,7 +1012,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_chain_chunked(const Params p,
     // allocates all 512 columns
     pdl_wait_then_release();
     if (threadIdx.x == 0) {
-        const uint32_t counts[kNumBars] = {1, 1, 1, 128, 128, 128, 128, 128, 1, 128, 128, 1, 128, 128, 1, 1, 1};
+        const uint32_t counts[kNumBars] = {1, 1, 1, 128, 128, 128, 128, 128, 1, 128, 128, 1, 128, 128, 1, 1, 1, 129, 129};
         for (int i = 0; i < kNumBars; ++i)
             mbar_init(bars + i, counts[i]);
         *abort_flag = 0;
@@ -1035,12 +1044,17 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_chain_chunked(const Params p,
             asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
         }
     } else if (warp < 8) {
-        int kq_loads[2] = {0, 0};
-        prep_role(p, mp, smem, sy, tbase, b, h, hk, n_chunks, kq_loads);
+        prep_role(p, smem, sy, tbase, b, h, n_chunks);
         asm volatile("cp.async.wait_all;" ::: "memory");
-        for (int j = 0; j < 2; ++j)
-            if (kq_loads[j] > 0)
-                drain(bars + kKqFull0 + j, (uint32_t)(kq_loads[j] - 1) & 1);
+    } else if (warp == 9) {
+        if ((threadIdx.x & 31) == 0) {
+            int kq_loads[2] = {0, 0};
+            load_role(mp, smem, sy, b, hk, n_chunks, kq_loads);
+            if (kq_loads[0] > 0)
+                drain(bars + kKqFull0, (uint32_t)(kq_loads[0] - 1) & 1);
+            if (kq_loads[1] > 0)
+                drain(bars + kKqFull1, (uint32_t)(kq_loads[1] - 1) & 1);
+        }
     } else if ((threadIdx.x & 31) == 0) {
         mma_role(smem, sy, tbase, n_chunks);
         // every MMA issued has retired before the tensor memory is freed
