@@ -44,10 +44,11 @@
 // Rounding differs from the token-by-token path (different summation
 // order), so this is an opt-in mode, not the chain fast path.
 //
-// One CTA per (sequence, v-head, 128 rows of d_v), 9 warps: warps 0-3 own
-// the state rows (one row per thread: the elementwise steps between the
-// products), warps 4-7 prepare each chunk's S-independent operands one chunk
-// ahead, warp 8 issues the MMAs.  k, q and v arrive by TMA (tensor maps over
+// One CTA per (sequence, v-head, 128 rows of d_v), 14 warps: warps 0-7 own
+// the state rows (two threads per row, in warps w and w + 4, each with half
+// of the columns of the elementwise steps between the products), warps 8-11
+// prepare each chunk's S-independent operands one chunk ahead, warp 12
+// issues the MMAs, warp 13 the k/q loads.  k, q and v arrive by TMA (tensor maps over
 // this GPU's q, k and v; one thread issues the copies, an mbarrier counts
 // the bytes), and each chunk's outputs leave as one TMA store of a 64-token
 // x 128-row tile staged in shared memory.  Hand-offs are mbarriers; every
@@ -72,8 +73,9 @@ namespace {
 constexpr int T = 64;           // tokens per chunk
 constexpr int DK = 128;         // d_k
 constexpr int TM = 128;         // state rows (d_v) per CTA: the MMAs' M
-constexpr int kThreads = 320;   // warps 0-3 rows, 4-7 preparation, 8 MMA issue, 9 k/q loads
-constexpr int kPrep0 = 128;     // first preparation thread
+constexpr int kThreads = 448;   // warps 0-7 rows, 8-11 preparation, 12 MMA issue, 13 k/q loads
+constexpr int kRows = 256;      // row threads: two per state row, each with half of every step
+constexpr int kPrep0 = 256;     // first preparation thread
 
 // Tensor-memory columns (128 lanes x 512 columns of 32 bits, all of it).
 constexpr uint32_t kTmemCols = 512;
@@ -121,12 +123,12 @@ enum Bar {
     kKqMma = 2,    // [K; Q] K^T done (MMA commit)
     kDkqFree = 3,  // [K; Q] K^T read out (128)
     kDec0 = 4,     // decays of a chunk written, slots 0..2 (128)
-    kAsReady = 7,  // state parts written, previous outputs read (128 row threads)
+    kAsReady = 7,  // state parts written, previous outputs read (256 row threads)
     kXyDone = 8,   // X^T | Y^T done (commit)
-    kApReady = 9,  // P^T parts written (128)
+    kApReady = 9,  // P^T parts written (256)
     kAbReady = 10, // Ab parts written (128)
     kUDone = 11,   // U^T done (commit)
-    kAuReady = 12, // U^T parts written (128)
+    kAuReady = 12, // U^T parts written (256)
     kMktReady = 13,// M parts and K^T written (128)
     kCdDone = 14,  // update and U^T M^T done (commit)
     kFin = 15,     // all MMAs retired (commit)
@@ -299,8 +301,8 @@ __device__ __forceinline__ bool prep_all(bool ok)
 
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-// Named barrier over the 128 row threads, and the same with a vote.
-__device__ __forceinline__ void row_sync() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
+// Named barrier over the 256 row threads, and the same with a vote.
+__device__ __forceinline__ void row_sync() { asm volatile("bar.sync 2, 256;" ::: "memory"); }
 
 __device__ __forceinline__ bool row_all(bool ok)
 {
@@ -308,7 +310,7 @@ __device__ __forceinline__ bool row_all(bool ok)
     asm volatile(
         "{\n\t.reg .pred p, q;\n\t"
         "setp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.and.pred q, 2, 128, p;\n\t"
+        "bar.red.and.pred q, 2, 256, p;\n\t"
         "selp.u32 %0, 1, 0, q;\n\t}"
         : "=r"(r)
         : "r"(ok ? 1u : 0u)
@@ -399,14 +401,16 @@ __device__ __forceinline__ void load_gb(const Params& p, unsigned char* smem, in
     asm volatile("cp.async.commit_group;" ::: "memory");
 }
 
-// Rows 16 I .. 16 I + 15 of block column J of (I + L)^-1 (columns c0 .. c0 +
-// NC - 1 for this lane, row i = lane % 16) for I = J + 1 .. 3, from the
-// diagonal blocks' inverses already in Ai: X = -L_(I, J..I-1) Ai_(J..I-1, J),
-// then Ai_(I, J) = Ai_(I, I) X.  One warp; the rows it reads are its own.
+// Rows 16 I .. 16 I + 15 of block column J of (I + L)^-1, columns c0 ..
+// c0 + NC - 1, for I = J + 1 .. 3, from the diagonal blocks' inverses already
+// in Ai: X = -L_(I, J..I-1) Ai_(J..I-1, J), then Ai_(I, J) = Ai_(I, I) X.  One
+// warp: lane = row i (lane % 16) and a parity kh (lane / 16); each sum runs
+// over the terms of its parity and the two halves meet with one shuffle.  The
+// rows the warp reads are its own.
 template <int NC>
 __device__ __forceinline__ void block_column(const float* L, float* Ai, int J, int c0, int lane)
 {
-    const int i = lane & 15;
+    const int i = lane & 15, kh = lane >> 4;
 #pragma unroll 1
     for (int I = J + 1; I < 4; ++I) {
         const int R0 = 16 * I;
@@ -416,21 +420,26 @@ __device__ __forceinline__ void block_column(const float* L, float* Ai, int J, i
             x[e] = 0.f;
         const float* Lr = L + (R0 + i) * LST;
 #pragma unroll 4
-        for (int k = 16 * J; k < R0; ++k) {
+        for (int k = 16 * J + kh; k < R0; k += 2) {
             const float l = Lr[k];
 #pragma unroll
             for (int e = 0; e < NC; e += 4) {
                 const float4 a = *reinterpret_cast<const float4*>(Ai + k * AST + c0 + e);
-                x[e] = __fmaf_rn(-l, a.x, x[e]);
-                x[e + 1] = __fmaf_rn(-l, a.y, x[e + 1]);
-                x[e + 2] = __fmaf_rn(-l, a.z, x[e + 2]);
-                x[e + 3] = __fmaf_rn(-l, a.w, x[e + 3]);
+                x[e] = __fmaf_rn(l, a.x, x[e]);
+                x[e + 1] = __fmaf_rn(l, a.y, x[e + 1]);
+                x[e + 2] = __fmaf_rn(l, a.z, x[e + 2]);
+                x[e + 3] = __fmaf_rn(l, a.w, x[e + 3]);
             }
         }
-        float* dst = Ai + (R0 + i) * AST + c0;
 #pragma unroll
-        for (int e = 0; e < NC; e += 4)
-            *reinterpret_cast<float4*>(dst + e) = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
+        for (int e = 0; e < NC; ++e)
+            x[e] = -__fadd_rn(x[e], __shfl_xor_sync(0xffffffffu, x[e], 16));
+        float* dst = Ai + (R0 + i) * AST + c0;
+        if (kh == 0) {
+#pragma unroll
+            for (int e = 0; e < NC; e += 4)
+                *reinterpret_cast<float4*>(dst + e) = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
+        }
         __syncwarp();
         float y[NC];
 #pragma unroll
@@ -438,7 +447,7 @@ __device__ __forceinline__ void block_column(const float* L, float* Ai, int J, i
             y[e] = 0.f;
         const float* Dr = Ai + (R0 + i) * AST + R0;  // row i of the block's inverse
 #pragma unroll 4
-        for (int i2 = 0; i2 < 16; ++i2) {
+        for (int i2 = kh; i2 < 16; i2 += 2) {
             const float dd = i2 <= i ? Dr[i2] : 0.f;
 #pragma unroll
             for (int e = 0; e < NC; e += 4) {
@@ -449,10 +458,15 @@ __device__ __forceinline__ void block_column(const float* L, float* Ai, int J, i
                 y[e + 3] = __fmaf_rn(dd, a.w, y[e + 3]);
             }
         }
-        __syncwarp();
 #pragma unroll
-        for (int e = 0; e < NC; e += 4)
-            *reinterpret_cast<float4*>(dst + e) = make_float4(y[e], y[e + 1], y[e + 2], y[e + 3]);
+        for (int e = 0; e < NC; ++e)
+            y[e] = __fadd_rn(y[e], __shfl_xor_sync(0xffffffffu, y[e], 16));
+        __syncwarp();
+        if (kh == 0) {
+#pragma unroll
+            for (int e = 0; e < NC; e += 4)
+                *reinterpret_cast<float4*>(dst + e) = make_float4(y[e], y[e + 1], y[e + 2], y[e + 3]);
+        }
         __syncwarp();
     }
 }
@@ -471,11 +485,15 @@ __device__ void invert_unit_lower(const float* L, float* Ai, int ptid)
         float d[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-            float acc = 0.f;
+            float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-            for (int k = 0; k < i; ++k)
-                acc = __fmaf_rn(Lb[i * LST + k], d[k], acc);  // d[k] = 0 for k < j
-            d[i] = i < j ? 0.f : (i == j ? 1.f : -acc);
+            for (int k = 0; k + 1 < i; k += 2) {  // d[k] = 0 for k < j
+                acc0 = __fmaf_rn(Lb[i * LST + k], d[k], acc0);
+                acc1 = __fmaf_rn(Lb[i * LST + k + 1], d[k + 1], acc1);
+            }
+            if (i & 1)
+                acc0 = __fmaf_rn(Lb[i * LST + i - 1], d[i - 1], acc0);
+            d[i] = i < j ? 0.f : (i == j ? 1.f : -__fadd_rn(acc0, acc1));
         }
         float* Ac = Ai + (16 * pw) * AST + 16 * pw + j;
 #pragma unroll
@@ -484,9 +502,9 @@ __device__ void invert_unit_lower(const float* L, float* Ai, int ptid)
     }
     prep_sync();
     if (pw < 2)
-        block_column<4>(L, Ai, 0, 8 * pw + 4 * (lane >> 4), lane);
+        block_column<8>(L, Ai, 0, 8 * pw, lane);
     else
-        block_column<8>(L, Ai, pw - 1, 16 * (pw - 1) + 8 * (lane >> 4), lane);
+        block_column<16>(L, Ai, pw - 1, 16 * (pw - 1), lane);
     prep_sync();
 }
 
@@ -730,6 +748,7 @@ __device__ void mma_role(unsigned char* smem, const Sync& sy, uint32_t tbase, in
         bool kq_done = c + 1 >= n_chunks, u_done = false;
         const long long t0 = clock64();
         while (!(kq_done && u_done)) {
+            __nanosleep(32);  // leave the issue slots to the warps being waited for
             if (*sy.abort || clock64() - t0 > (1ll << 31)) {
                 *sy.abort = 1;
                 report_status(sy.status, kStatusTimeout);
@@ -784,13 +803,12 @@ __device__ void mma_role(unsigned char* smem, const Sync& sy, uint32_t tbase, in
 __device__ __forceinline__ void write_outputs(const Params& p, const Maps& mp, unsigned char* smem, uint32_t trow,
                                               const float* Gam, int b, int h, int row0, int t0)
 {
-    const int m = threadIdx.x;
+    const int m = threadIdx.x & (TM - 1), hs = threadIdx.x >> 7;  // row; half of the tokens
     float* tile = reinterpret_cast<float*>(smem + kOffOut) + m;
-    if (m == 0)
+    if (threadIdx.x == 0)
         asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
     row_sync();
-#pragma unroll 1
-    for (int hs = 0; hs < 2; ++hs) {
+    {
         uint32_t y[32], o[32];
         float gm[32];
 #pragma unroll
@@ -807,7 +825,7 @@ __device__ __forceinline__ void write_outputs(const Params& p, const Maps& mp, u
     }
     fence_proxy_async();
     row_sync();
-    if (m == 0)
+    if (threadIdx.x == 0)
         tma_store(&mp.out, smem_addr(smem + kOffOut), row0, h, t0, b);
 }
 
@@ -816,9 +834,10 @@ __device__ void row_role(const Params& p, const Maps& mp, unsigned char* smem, c
                          int h, int row0, int n_chunks, int& v_loads)
 {
     const int tid = threadIdx.x, warp = tid >> 5;
-    const int m = tid;              // state row within the tile (lane quarter = warp)
+    const int m = tid & (TM - 1);   // state row within the tile (lane quarter = warp % 4)
+    const int half = tid >> 7;      // which half of each step's columns
     const int row = row0 + m;       // row of d_v
-    const uint32_t trow = tbase + ((uint32_t)(32 * warp) << 16);
+    const uint32_t trow = tbase + ((uint32_t)(32 * (warp & 3)) << 16);
     const float* decs = reinterpret_cast<const float*>(smem + kOffDec);
     if (tid == 0) {
         load_v(mp, smem, sy.bar + kVFull, 0, b, h, row0);
@@ -841,7 +860,7 @@ __device__ void row_role(const Params& p, const Maps& mp, unsigned char* smem, c
             write_outputs(p, mp, smem, trow, decs + ((c - 1) % 3) * 2 * T, b, h, row0, (c - 1) * T);
         }
 #pragma unroll 1
-        for (int s = 0; s < 4; ++s) {
+        for (int s = 2 * half; s < 2 * half + 2; ++s) {
             uint32_t x[32];
             if (c == 0) {
                 if (row < p.dv) {
@@ -885,8 +904,8 @@ __device__ void row_role(const Params& p, const Maps& mp, unsigned char* smem, c
         tmem_fence_after_sync();
         {
             const unsigned short* V = reinterpret_cast<const unsigned short*>(smem + kOffV) + m;
-#pragma unroll 1
-            for (int hs = 0; hs < 2; ++hs) {
+            {
+                const int hs = half;
                 uint32_t x[32];
                 float gm[32], vv[32];
 #pragma unroll
@@ -923,8 +942,8 @@ __device__ void row_role(const Params& p, const Maps& mp, unsigned char* smem, c
             ++v_loads;
         }
         tmem_fence_after_sync();
-#pragma unroll 1
-        for (int hs = 0; hs < 2; ++hs) {
+        {
+            const int hs = half;
             uint32_t u[32];
             float rr[32];
 #pragma unroll
@@ -945,6 +964,10 @@ __device__ void row_role(const Params& p, const Maps& mp, unsigned char* smem, c
             for (int e = 0; e < 16; ++e)
                 split2(__uint_as_float(u[2 * e]), __uint_as_float(u[2 * e + 1]), p1[e], p2[e]);
             tmem_st16(trow + kColAU0 + 16 * hs, p1);
+            // part 1 goes over the first half of U^T: both halves have read it
+            tmem_fence_before_sync();
+            row_sync();
+            tmem_fence_after_sync();
             tmem_st16(trow + kColAU1 + 16 * hs, p2);
         }
         tmem_wait_st();
@@ -959,7 +982,7 @@ __device__ void row_role(const Params& p, const Maps& mp, unsigned char* smem, c
     write_outputs(p, mp, smem, trow, decs + ((n_chunks - 1) % 3) * 2 * T, b, h, row0, (n_chunks - 1) * T);
     const size_t base = (((size_t)b * p.Hv + h) * p.dv + row) * DK;
 #pragma unroll 1
-    for (int s = 0; s < 4; ++s) {
+    for (int s = 2 * half; s < 2 * half + 2; ++s) {
         uint32_t x[32];
         tmem_ld32(trow + kColS + 32 * s, x);
         if (row >= p.dv)
@@ -1012,7 +1035,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_chain_chunked(const Params p,
     // allocates all 512 columns
     pdl_wait_then_release();
     if (threadIdx.x == 0) {
-        const uint32_t counts[kNumBars] = {1, 1, 1, 128, 128, 128, 128, 128, 1, 128, 128, 1, 128, 128, 1, 1, 1, 129, 129};
+        const uint32_t counts[kNumBars] = {1, 1, 1, 128, 128, 128, 128, kRows, 1, kRows, 128, 1, kRows, 128, 1, 1, 1, 129, 129};
         for (int i = 0; i < kNumBars; ++i)
             mbar_init(bars + i, counts[i]);
         *abort_flag = 0;
@@ -1035,7 +1058,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_chain_chunked(const Params p,
     // Each TMA load is waited for by the thread that issued it before the CTA
     // can leave (a barrier has at most one phase outstanding: a buffer is
     // reloaded only after its previous load was used).
-    if (warp < 4) {
+    if (warp < 8) {
         int v_loads = 0;
         row_role(p, mp, smem, sy, tbase, b, h, row0, n_chunks, v_loads);
         if (threadIdx.x == 0) {
@@ -1043,10 +1066,10 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_chain_chunked(const Params p,
                 drain(bars + kVFull, (uint32_t)(v_loads - 1) & 1);
             asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
         }
-    } else if (warp < 8) {
+    } else if (warp < 12) {
         prep_role(p, smem, sy, tbase, b, h, n_chunks);
         asm volatile("cp.async.wait_all;" ::: "memory");
-    } else if (warp == 9) {
+    } else if (warp == 13) {
         if ((threadIdx.x & 31) == 0) {
             int kq_loads[2] = {0, 0};
             load_role(mp, smem, sy, b, hk, n_chunks, kq_loads);
