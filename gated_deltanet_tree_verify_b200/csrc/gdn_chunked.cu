@@ -48,7 +48,8 @@
 // the state rows (two threads per row, in warps w and w + 4, each with half
 // of the columns of the elementwise steps between the products), warps 8-11
 // prepare each chunk's S-independent operands one chunk ahead, warp 12
-// issues the MMAs, warp 13 the k/q loads.  k, q and v arrive by TMA (tensor maps over
+// issues the MMAs, warp 13 loads k, q, g and beta and computes the decays
+// two chunks ahead.  k, q and v arrive by TMA (tensor maps over
 // this GPU's q, k and v; one thread issues the copies, an mbarrier counts
 // the bytes), and each chunk's outputs leave as one TMA store of a 64-token
 // x 128-row tile staged in shared memory.  Hand-offs are mbarriers; every
@@ -73,7 +74,7 @@ namespace {
 constexpr int T = 64;           // tokens per chunk
 constexpr int DK = 128;         // d_k
 constexpr int TM = 128;         // state rows (d_v) per CTA: the MMAs' M
-constexpr int kThreads = 448;   // warps 0-7 rows, 8-11 preparation, 12 MMA issue, 13 k/q loads
+constexpr int kThreads = 448;   // warps 0-7 rows, 8-11 preparation, 12 MMA issue, 13 loads and decays
 constexpr int kRows = 256;      // row threads: two per state row, each with half of every step
 constexpr int kPrep0 = 256;     // first preparation thread
 
@@ -109,10 +110,9 @@ constexpr int kOffOut = kOffKT + kKTBytes;
 constexpr int kOffL = kOffOut + kOutBytes;         // L, f32 [T][LST]
 constexpr int kOffMf = kOffL + T * LST * 4;        // M, f32 [T][LST]
 constexpr int kOffAi = kOffMf + T * LST * 4;       // (I + L)^-1, f32 [T][AST]
-constexpr int kOffGB = kOffAi + T * AST * 4;       // [2][g | beta], f32
+constexpr int kOffGB = kOffAi + T * AST * 4;       // [2][a = exp(g) | beta], f32
 constexpr int kOffDec = kOffGB + 2 * 2 * T * 4;    // [3][Gamma | r], f32
-constexpr int kOffA = kOffDec + 3 * 2 * T * 4;     // a = exp(g), f32 [T]
-constexpr int kOffBar = kOffA + T * 4;             // mbarriers, tmem base, abort flag
+constexpr int kOffBar = kOffDec + 3 * 2 * T * 4;   // mbarriers, tmem base, abort flag
 constexpr int kSmem = kOffBar + 256;
 static_assert(kSmem <= 227 * 1024, "shared memory");
 
@@ -122,7 +122,7 @@ enum Bar {
     kKqFull1 = 1,
     kKqMma = 2,    // [K; Q] K^T done (MMA commit)
     kDkqFree = 3,  // [K; Q] K^T read out (128)
-    kDec0 = 4,     // decays of a chunk written, slots 0..2 (128)
+    kDec0 = 4,     // decays of a chunk written, slots 0..2 (1)
     kAsReady = 7,  // state parts written, previous outputs read (256 row threads)
     kXyDone = 8,   // X^T | Y^T done (commit)
     kApReady = 9,  // P^T parts written (256)
@@ -135,7 +135,9 @@ enum Bar {
     kVFull = 16,   // v of a chunk landed (TMA bytes)
     kKqBuf0 = 17,  // k/q buffer 0 / 1 no longer read: the chunk's MMAs (commit) and K^T (128)
     kKqBuf1 = 18,
-    kNumBars = 19
+    kGb0 = 19,     // a and beta of a chunk written, buffer 0 / 1 (1)
+    kGb1 = 20,
+    kNumBars = 21
 };
 
 struct Params {
@@ -318,11 +320,6 @@ __device__ __forceinline__ bool row_all(bool ok)
     return r != 0;
 }
 
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src)
-{
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
-}
-
 // ---- TMA -------------------------------------------------------------------------------------
 
 // The barrier's current phase also waits for `bytes` bytes of TMA data.
@@ -384,21 +381,6 @@ __device__ __forceinline__ void load_v(const Maps& mp, unsigned char* smem, uint
 {
     mbar_expect_tx(bar, kVBytes);
     tma_load(smem_addr(smem + kOffV), &mp.v, row0, h, c * T, b, bar);
-}
-
-// g and beta of chunk c into buffer buf (0 past the end: a = 1, beta = 0);
-// one element per thread.
-__device__ __forceinline__ void load_gb(const Params& p, unsigned char* smem, int buf, int c, int b, int h, int ptid)
-{
-    const int t = ptid & (T - 1), which = ptid >> 6;  // 0: g, 1: beta
-    const uint32_t dst = smem_addr(smem + kOffGB) + (buf * 2 * T + which * T + t) * 4;
-    if (c * T + t < p.N) {
-        const size_t gi = ((size_t)b * p.N + c * T + t) * p.Hv + h;
-        cp_async4(dst, (which == 0 ? p.g : p.beta) + gi);
-    } else {
-        asm volatile("st.shared.u32 [%0], %1;" ::"r"(dst), "r"(0u) : "memory");
-    }
-    asm volatile("cp.async.commit_group;" ::: "memory");
 }
 
 // Rows 16 I .. 16 I + 15 of block column J of (I + L)^-1, columns c0 ..
@@ -508,8 +490,7 @@ __device__ void invert_unit_lower(const float* L, float* Ai, int ptid)
     prep_sync();
 }
 
-__device__ void prep_role(const Params& p, unsigned char* smem, const Sync& sy, uint32_t tbase, int b, int h,
-                          int n_chunks)
+__device__ void prep_role(unsigned char* smem, const Sync& sy, uint32_t tbase, int n_chunks)
 {
     const int ptid = threadIdx.x - kPrep0;
     const int pw = ptid >> 5;                  // lane quarter of tensor memory
@@ -518,51 +499,19 @@ __device__ void prep_role(const Params& p, unsigned char* smem, const Sync& sy, 
     float* L = reinterpret_cast<float*>(smem + kOffL);
     float* Mf = reinterpret_cast<float*>(smem + kOffMf);
     float* Ai = reinterpret_cast<float*>(smem + kOffAi);
-    float* av = reinterpret_cast<float*>(smem + kOffA);
 
     for (int i = ptid; i < T * AST; i += 128)
         Ai[i] = 0.f;
-    load_gb(p, smem, 0, 0, b, h, ptid);
-    if (n_chunks > 1)
-        load_gb(p, smem, 1, 1, b, h, ptid);
 
     for (int c = 0; c < n_chunks; ++c) {
-        const int buf = c & 1, slot = c % 3;
+        const int buf = c & 1;
         const float* gb = reinterpret_cast<const float*>(smem + kOffGB) + buf * 2 * T;
-        float* Gam = reinterpret_cast<float*>(smem + kOffDec) + slot * 2 * T;
-        float* rv = Gam + T;
-        // 1. this chunk's g and beta; decays a = exp(g), then Gamma_t =
-        //    a_0 ... a_t and r_t = a_{t+1} ... a_{T-1} by thread t of the K rows
-        if (c == 0 && n_chunks > 1)
-            asm volatile("cp.async.wait_group 1;" ::: "memory");
-        else
-            asm volatile("cp.async.wait_group 0;" ::: "memory");
-        prep_sync();
-        if (ptid < T)
-            av[ptid] = expf(gb[ptid]);
-        prep_sync();
-        if (!qrow) {
-            float gm = 1.f, rr = 1.f;
-#pragma unroll
-            for (int e = 0; e < T / 4; ++e) {
-                const float4 a4 = reinterpret_cast<const float4*>(av)[e];
-                const float a[4] = {a4.x, a4.y, a4.z, a4.w};
-#pragma unroll
-                for (int f = 0; f < 4; ++f) {
-                    if (4 * e + f <= t)
-                        gm = __fmul_rn(gm, a[f]);
-                    else
-                        rr = __fmul_rn(rr, a[f]);
-                }
-            }
-            Gam[t] = gm;
-            rv[t] = rr;
-        }
-        sy.arrive(kDec0 + slot);
-        // 2. this thread's row of [K; Q] K^T times the row's decays
+        const float* av = gb;  // a = exp(g)
+        // 1. this chunk's a and beta (written by the load warp), then this
+        //    thread's row of [K; Q] K^T times the row's decays
         //    R[t][i] = a_{i+1} ... a_t, a running product over i from t down
         //    to 0: L (K rows) and M (Q rows)
-        if (!prep_all(sy.wait(kKqMma, c & 1)))
+        if (!prep_all(sy.wait(kGb0 + buf, (c >> 1) & 1) && sy.wait(kKqMma, c & 1)))
             return;
         tmem_fence_after_sync();
         {
@@ -600,16 +549,12 @@ __device__ void prep_role(const Params& p, unsigned char* smem, const Sync& sy, 
         tmem_fence_before_sync();
         sy.arrive(kDkqFree);
         prep_sync();
-        // 3. Ai = (I + L)^-1
+        // 2. Ai = (I + L)^-1
         invert_unit_lower(L, Ai, ptid);
-        // 4. once the previous chunk's U^T product is done with Ab: chunk
-        //    c + 1's g and beta start loading; Ab = Ai diag(beta) in 3 bf16 parts
-        if (c > 0) {
-            if (!prep_all(sy.wait(kUDone, (c - 1) & 1)))
-                return;
-            if (c + 1 < n_chunks)
-                load_gb(p, smem, (c + 1) & 1, c + 1, b, h, ptid);
-        }
+        // 3. Ab = Ai diag(beta) in 3 bf16 parts, once the previous chunk's
+        //    U^T product is done with them
+        if (c > 0 && !prep_all(sy.wait(kUDone, (c - 1) & 1)))
+            return;
 #pragma unroll 1
         for (int it = ptid; it < T * (T / 8); it += 128) {
             const int tt = it & (T - 1), pc = it >> 6;
@@ -636,7 +581,7 @@ __device__ void prep_role(const Params& p, unsigned char* smem, const Sync& sy, 
         }
         fence_proxy_async();
         sy.arrive(kAbReady);
-        // 5. M in 2 bf16 parts and K^T, once the previous chunk's update and
+        // 4. M in 2 bf16 parts and K^T, once the previous chunk's update and
         //    U^T M^T products are done with them (and this chunk's k is in)
         if (!prep_all((c == 0 || sy.wait(kCdDone, (c - 1) & 1)) && sy.wait(kKqFull0 + buf, (c >> 1) & 1)))
             return;
@@ -684,22 +629,86 @@ __device__ void prep_role(const Params& p, unsigned char* smem, const Sync& sy, 
     }
 }
 
-// ---- k/q loads ---------------------------------------------------------------------------
+// ---- loads and decays ----------------------------------------------------------------------
 
-// One thread: chunks 0 and 1, then chunk c + 2 into buffer c % 2 once chunk
-// c's MMAs and K^T are done with it.  kq_loads[j]: loads issued into buffer j.
-__device__ void load_role(const Maps& mp, unsigned char* smem, const Sync& sy, int b, int hk, int n_chunks,
-                          int (&kq_loads)[2])
+// Chunk c's a = exp(g) and beta into buffer buf, and its decays Gamma_t =
+// a_0 ... a_t and r_t = a_{t+1} ... a_{T-1} into slot c % 3: lane l holds
+// tokens 2 l and 2 l + 1; products across lanes by shuffle scans.  Tokens
+// past the end have a = 1, beta = 0.  One warp.
+__device__ __forceinline__ void decays(const Params& p, unsigned char* smem, int buf, int c, int b, int h, int lane)
 {
+    float a[2], bt[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+        const int t = c * T + 2 * lane + e;
+        float g = 0.f, be = 0.f;
+        if (t < p.N) {
+            const size_t gi = ((size_t)b * p.N + t) * p.Hv + h;
+            g = __ldg(p.g + gi);
+            be = __ldg(p.beta + gi);
+        }
+        a[e] = expf(g);
+        bt[e] = be;
+    }
+    // inclusive prefix and suffix products of the lanes' pair products
+    const float pr = __fmul_rn(a[0], a[1]);
+    float pre = pr, suf = pr;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const float up = __shfl_up_sync(0xffffffffu, pre, d);
+        const float dn = __shfl_down_sync(0xffffffffu, suf, d);
+        if (lane >= d)
+            pre = __fmul_rn(up, pre);
+        if (lane + d < 32)
+            suf = __fmul_rn(suf, dn);
+    }
+    float before = __shfl_up_sync(0xffffffffu, pre, 1);  // product of tokens < 2 lane
+    float after = __shfl_down_sync(0xffffffffu, suf, 1);  // product of tokens > 2 lane + 1
+    if (lane == 0)
+        before = 1.f;
+    if (lane == 31)
+        after = 1.f;
+    float* gb = reinterpret_cast<float*>(smem + kOffGB) + buf * 2 * T;
+    float* Gam = reinterpret_cast<float*>(smem + kOffDec) + (c % 3) * 2 * T;
+    *reinterpret_cast<float2*>(gb + 2 * lane) = make_float2(a[0], a[1]);
+    *reinterpret_cast<float2*>(gb + T + 2 * lane) = make_float2(bt[0], bt[1]);
+    const float g0 = __fmul_rn(before, a[0]);
+    *reinterpret_cast<float2*>(Gam + 2 * lane) = make_float2(g0, __fmul_rn(g0, a[1]));
+    *reinterpret_cast<float2*>(Gam + T + 2 * lane) = make_float2(__fmul_rn(a[1], after), after);
+}
+
+// One warp: chunks 0 and 1, then chunk c + 2 into buffer c % 2 once chunk c's
+// MMAs, K^T and preparation are done with it: k and q by TMA (lane 0),
+// a, beta and the decays.  kq_loads[j]: TMA loads issued into buffer j.
+__device__ void load_role(const Params& p, const Maps& mp, unsigned char* smem, const Sync& sy, int b, int h,
+                          int hk, int n_chunks, int (&kq_loads)[2])
+{
+    const int lane = threadIdx.x & 31;
     for (int c = 0; c < n_chunks && c < 2; ++c) {
-        load_kq(mp, smem, sy.bar + kKqFull0 + c, c, c, b, hk);
-        ++kq_loads[c];
+        if (lane == 0) {
+            load_kq(mp, smem, sy.bar + kKqFull0 + c, c, c, b, hk);
+            ++kq_loads[c];
+        }
+        decays(p, smem, c, c, b, h, lane);
+        __syncwarp();
+        if (lane == 0) {
+            sy.arrive(kGb0 + c);
+            sy.arrive(kDec0 + c);
+        }
     }
     for (int c = 0; c + 2 < n_chunks; ++c) {
-        if (!sy.wait(kKqBuf0 + (c & 1), (c >> 1) & 1))
+        if (!__all_sync(0xffffffffu, sy.wait(kKqBuf0 + (c & 1), (c >> 1) & 1)))
             return;
-        load_kq(mp, smem, sy.bar + kKqFull0 + (c & 1), c & 1, c + 2, b, hk);
-        ++kq_loads[c & 1];
+        if (lane == 0) {
+            load_kq(mp, smem, sy.bar + kKqFull0 + (c & 1), c & 1, c + 2, b, hk);
+            ++kq_loads[c & 1];
+        }
+        decays(p, smem, c & 1, c + 2, b, h, lane);
+        __syncwarp();
+        if (lane == 0) {
+            sy.arrive(kGb0 + (c & 1));
+            sy.arrive(kDec0 + (c + 2) % 3);
+        }
     }
 }
 
@@ -1035,7 +1044,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_chain_chunked(const Params p,
     // allocates all 512 columns
     pdl_wait_then_release();
     if (threadIdx.x == 0) {
-        const uint32_t counts[kNumBars] = {1, 1, 1, 128, 128, 128, 128, kRows, 1, kRows, 128, 1, kRows, 128, 1, 1, 1, 129, 129};
+        const uint32_t counts[kNumBars] = {1, 1, 1, 128, 1, 1, 1, kRows, 1, kRows, 128, 1, kRows, 128, 1, 1, 1, 129, 129, 1, 1};
         for (int i = 0; i < kNumBars; ++i)
             mbar_init(bars + i, counts[i]);
         *abort_flag = 0;
@@ -1067,12 +1076,11 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_chain_chunked(const Params p,
             asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
         }
     } else if (warp < 12) {
-        prep_role(p, smem, sy, tbase, b, h, n_chunks);
-        asm volatile("cp.async.wait_all;" ::: "memory");
+        prep_role(smem, sy, tbase, n_chunks);
     } else if (warp == 13) {
+        int kq_loads[2] = {0, 0};
+        load_role(p, mp, smem, sy, b, h, hk, n_chunks, kq_loads);
         if ((threadIdx.x & 31) == 0) {
-            int kq_loads[2] = {0, 0};
-            load_role(mp, smem, sy, b, hk, n_chunks, kq_loads);
             if (kq_loads[0] > 0)
                 drain(bars + kKqFull0, (uint32_t)(kq_loads[0] - 1) & 1);
             if (kq_loads[1] > 0)
