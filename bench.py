@@ -115,6 +115,32 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def bf16_tensor_peak():
+    """Measured dense bf16 tensor throughput (TFLOP/s, cuBLAS burst), else the
+    fallback of this pool's earlier measurement."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+# Tensor-core work of the chunked chain per (CTA, 64-token chunk): one CTA
+# holds 128 state rows; kind::f16 products of M = 128 rows, 2 * M * N * K
+# flops each, with operands split into bf16 parts (the issued work) and the
+# same products at one part each (the chunked form's own arithmetic).
+CHUNK_T, CHUNK_ROWS = 64, 128
+CHUNK_FLOPS_ISSUED = 2 * CHUNK_ROWS * (
+    3 * 2 * CHUNK_T * 128      # X^T | Y^T = S [K; Q]^T, S in 3 parts
+    + 2 * CHUNK_T * 128 // 2   # [K; Q] K^T (M = 2T rows of K and Q, N = T)
+    + 6 * CHUNK_T * CHUNK_T    # U^T = P^T Ab^T, 6 part products
+    + 3 * 128 * CHUNK_T        # S += (U^T diag(r)) K, 3 parts
+    + 3 * CHUNK_T * CHUNK_T)   # U^T M^T, 3 part products
+CHUNK_FLOPS_ALGO = 2 * CHUNK_ROWS * (
+    2 * CHUNK_T * 128 + 2 * CHUNK_T * 128 // 2 + CHUNK_T * CHUNK_T + 128 * CHUNK_T + CHUNK_T * CHUNK_T)
+
+
 def kernel_source_digest():
     """Digest of the sources the verify kernels are built from (the tree
     builder, chunked chain and commit kernels live in files of their own)."""
@@ -1086,6 +1112,18 @@ def _sweep_point(args, gdn, pt, peak, varlen_budgets, clocks):
                              "peak": alu_peak, "frac": flops / t / 1e12 / alu_peak,
                              "peak_source": f"148 SMs x 128 FP32 lanes x 2 x {args.sm_mhz:.0f} MHz"},
                 "hbm_gbps": io / t / 1e9}
+        if pt.get("chunked"):
+            # the tensor cores do the chain's work: issued bf16 flops against
+            # the measured dense bf16 peak, and the algorithmic share beside it
+            ctas = pt["batch"] * N_V_HEADS * -(-D // CHUNK_ROWS)
+            chunks = -(-n // CHUNK_T)
+            issued = ctas * chunks * CHUNK_FLOPS_ISSUED
+            tpeak, tkind = bf16_tensor_peak()
+            line["recurrence_tflops_equivalent"] = line.pop("roofline")["achieved"]
+            line["roofline"] = {"bound": "tensor", "achieved": issued / t / 1e12, "unit": "TFLOP/s",
+                                "peak": tpeak, "frac": issued / t / 1e12 / tpeak, "peak_source": tkind + " bf16",
+                                "algorithmic": ctas * chunks * CHUNK_FLOPS_ALGO / t / 1e12,
+                                "issued_gflop": issued / 1e9}
     else:
         tree = "ddtree" if pt["kind"] == "tree" else "chain"
         flags = 0 if pt["kind"] == "tree" else gdn.GDN_FLAG_CHAIN

@@ -96,8 +96,10 @@ enum {
      * d_k = 128, d_v a multiple of 64, no varlen or workspace): run the chain
      * in chunks of 64 tokens with tensor-core products (the chunked "WY" form
      * of the delta rule), for long prefill-style chains.  Same results up to
-     * f32 rounding (products in split tf32), not bit-identical to the
-     * token-by-token path.  Unsupported shapes: GDN_ERR_UNSUPPORTED. */
+     * f32 rounding (products of bf16 parts accumulated in f32), not
+     * bit-identical to the token-by-token path.  q, k, v and out are read and
+     * written through TMA tensor maps (the 16-byte alignment required above
+     * suffices).  Unsupported shapes: GDN_ERR_UNSUPPORTED. */
     GDN_FLAG_CHUNKED = 16,
     /* q and k are given raw; the kernel L2-normalises each (node, k-head)
      * row, x / |x| with no epsilon (a zero row gives inf/NaN), as the

@@ -43,6 +43,18 @@ def test_chunked_chain_matches_oracle(N, sd):
     assert r.max() <= (1e-5 if sd == "f32" else 2e-3)
 
 
+@pytest.mark.parametrize("sd", ["f32", "f16"])
+def test_chunked_partial_row_tile(sd):
+    """A CTA holds 128 state rows: d_v = 64 leaves half of its one tile
+    empty; rows past d_v are neither read nor written."""
+    prob = _chain(100, dv=64, gate="uniform_a")
+    res = run(prob, sd, flags=FLAGS | gdn.GDN_FLAG_CHUNKED)
+    assert res["status"] == 0
+    out, _, ex = oracle.verify_problem(prob, state_dtype=sd, want_exact=True, nthreads=8)
+    assert_out_close(res["out"], out)
+    assert_states_close(res["node_states"][:, 0], ex[:, -1], sd)
+
+
 def test_chunked_chain_reset_and_zero_beta():
     prob = _chain(150)
     prob.g[:, 70] = float("-inf")   # a = 0: the state restarts at token 70
