@@ -55,6 +55,17 @@ def test_chunked_partial_row_tile(sd):
     assert_states_close(res["node_states"][:, 0], ex[:, -1], sd)
 
 
+def test_chunked_one_v_head_per_k_head():
+    """G = 1: each v-head reads its own k-head (the grid's y index is the
+    v-head, the k/q tensor maps take h / G)."""
+    prob = _chain(130, B=3, Hk=4, Hv=4, seed=9)
+    res = run(prob, "f32", flags=FLAGS | gdn.GDN_FLAG_CHUNKED)
+    assert res["status"] == 0
+    out, _, ex = oracle.verify_problem(prob, state_dtype="f32", want_exact=True, nthreads=8)
+    assert_out_close(res["out"], out)
+    assert_states_close(res["node_states"][:, 0], ex[:, -1], "f32")
+
+
 def test_chunked_chain_reset_and_zero_beta():
     prob = _chain(150)
     prob.g[:, 70] = float("-inf")   # a = 0: the state restarts at token 70
