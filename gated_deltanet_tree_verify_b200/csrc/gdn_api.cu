@@ -537,12 +537,13 @@ gdn_status gdn_tree_verify_static_ws(const gdn_tree_desc* desc, const void* q, c
     gdn_status st = check_desc(desc, true);
     if (st != GDN_OK)
         return st;
+    // Descs whose walk needs no workspace, or more than the buffer holds, run
+    // as gdn_tree_verify does (stack slots in shared memory, or parent
+    // re-reads), which allocates nothing either.
     const size_t need = gdn_tree_verify_workspace_bytes(desc);
-    if (need == 0 || desc->batch == 0)
+    if (need == 0 || need > kStaticWorkspaceBytes || desc->batch == 0)
         return verify_impl(desc, nullptr, 0, q, k, v, g, beta, parent_idx, state_in, out, node_states, nullptr, 0,
                            stream, false);
-    if (need > kStaticWorkspaceBytes)
-        return fail(GDN_ERR_UNSUPPORTED, "workspace needed exceeds gdn_static_workspace_capacity()%s");
     void* ws = nullptr;
     st = static_ws_address(&ws);
     if (st != GDN_OK)

@@ -244,9 +244,9 @@ size_t gdn_tree_verify_workspace_bytes(const gdn_tree_desc* desc);
  * exists for callers that cannot allocate on the hot path.
  *
  * Same arguments, layouts and results as gdn_tree_verify.  When the desc
- * needs no workspace (gdn_tree_verify_workspace_bytes(desc) == 0) this is
- * gdn_tree_verify.  When it needs more than the capacity:
- * GDN_ERR_UNSUPPORTED, nothing launched.
+ * needs no workspace (gdn_tree_verify_workspace_bytes(desc) == 0), or more
+ * than the capacity, this is gdn_tree_verify (which allocates nothing either:
+ * its walks keep their branch states in shared memory or re-read parents).
  *
  * Races: the buffer is shared by every call in the process on that device.
  * Calls on one device must be ordered (one stream, or events between
