@@ -1,8 +1,9 @@
-"""Trees at the library's maximum size, GDN_MAX_TREE_NODES = 1024: random
-trees of 1024 nodes and a caterpillar 511 levels deep, in both persisted
+"""Inputs at the library's maximum sizes.  Trees of GDN_MAX_TREE_NODES =
+1024 nodes (random) and a caterpillar 511 levels deep, in both persisted
 dtypes, checked node by node against the oracle (outputs, every persisted
 state, and the commit of an accepted root-to-leaf path); one node more is
-refused before any launch.  These take the kernels' large-N routes (records
+refused before any launch.  A chain of 65535 tokens (the most a desc
+allows) by both chain paths.  These take the kernels' large-N routes (records
 streamed through the ring, stack slots or parent re-reads) that the
 budget-sized workloads never reach."""
 import numpy as np
@@ -60,3 +61,25 @@ def test_deep_caterpillar(sd):
     prob = make_problem(batch=1, n_nodes=par.shape[0], n_k_heads=1, n_v_heads=3, d_k=128, d_v=128,
                         tree="given", parents=par[None], seed=811, qkv_dtype="bf16")
     _check(prob, sd)
+
+
+@pytest.mark.parametrize("chunked", [False, True])
+def test_longest_chain_last_state(chunked):
+    """A chain of 65535 tokens, the most a desc allows, last state only, by
+    the token-by-token walk and by the chunked tensor-core form: every
+    output and the last state of 8 rows at each end of d_v against the
+    oracle (rows of S evolve independently given k)."""
+    N = 0xFFFF
+    prob = make_problem(batch=1, n_nodes=N, n_k_heads=1, n_v_heads=1, d_k=128, d_v=128, tree="chain",
+                        seed=703, qkv_dtype="bf16", gate="uniform_a", accept="root")
+    prob.accept_path = torch.arange(N, dtype=torch.int32)[None].contiguous()
+    prob.accept_len = torch.full((1,), N, dtype=torch.int32)
+    flags = gdn.GDN_FLAG_CHAIN | gdn.GDN_FLAG_PERSIST_LAST | (gdn.GDN_FLAG_CHUNKED if chunked else 0)
+    res = run(prob, "f32", flags=flags)
+    assert res["status"] == 0
+    for rows in (slice(0, 8), slice(120, 128)):
+        out, _, ex = oracle.verify(prob.q, prob.k, prob.v[..., rows], prob.g, prob.beta, prob.parent,
+                                   prob.state_in[:, :, rows], prob.scale, want_exact=True)
+        assert_out_close(res["out"][..., rows], out)
+        assert_states_close(res["node_states"][:, 0, :, rows], ex[:, -1], "f32")
+        del out, ex
