@@ -153,6 +153,7 @@ struct Params {
     int N, Hk, Hv, dv, G;
     float scale;
     int state_f16;
+    int gates;  // GDN_FLAG_GATES: g and beta hold the gates' pre-activations
 };
 
 // ---- tcgen05 ----------------------------------------------------------------
@@ -633,22 +634,29 @@ __device__ void prep_role(unsigned char* smem, const Sync& sy, uint32_t tbase, i
 
 // Chunk c's a = exp(g) and beta into buffer buf, and its decays Gamma_t =
 // a_0 ... a_t and r_t = a_{t+1} ... a_{T-1} into slot c % 3: lane l holds
-// tokens 2 l and 2 l + 1; products across lanes by shuffle scans.  Tokens
-// past the end have a = 1, beta = 0.  One warp.
+// tokens 2 l and 2 l + 1; products across lanes by shuffle scans.  With raw
+// gates, g = x and beta = y stand for g = -softplus(x) and beta = sigmoid(y):
+// a = 1 / (1 + e^x), beta = 1 / (1 + e^-y) (the walk kernels' expressions,
+// so x = +inf resets).  Tokens past the end have a = 1, beta = 0.  One warp.
 __device__ __forceinline__ void decays(const Params& p, unsigned char* smem, int buf, int c, int b, int h, int lane)
 {
     float a[2], bt[2];
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
         const int t = c * T + 2 * lane + e;
-        float g = 0.f, be = 0.f;
+        a[e] = 1.f;
+        bt[e] = 0.f;
         if (t < p.N) {
             const size_t gi = ((size_t)b * p.N + t) * p.Hv + h;
-            g = __ldg(p.g + gi);
-            be = __ldg(p.beta + gi);
+            const float g = __ldg(p.g + gi), be = __ldg(p.beta + gi);
+            if (p.gates) {
+                a[e] = __fdiv_rn(1.f, __fadd_rn(1.f, expf(g)));
+                bt[e] = __fdiv_rn(1.f, __fadd_rn(1.f, expf(-be)));
+            } else {
+                a[e] = expf(g);
+                bt[e] = be;
+            }
         }
-        a[e] = expf(g);
-        bt[e] = be;
     }
     // inclusive prefix and suffix products of the lanes' pair products
     const float pr = __fmul_rn(a[0], a[1]);
@@ -1168,6 +1176,7 @@ cudaError_t launch_chunked(const VerifyArgs& a, cudaStream_t stream)
     p.G = a.n_v_heads / a.n_k_heads;
     p.scale = a.scale;
     p.state_f16 = a.state_dtype == GDN_F16 ? 1 : 0;
+    p.gates = (a.flags & GDN_FLAG_GATES) ? 1 : 0;
     const EncodeTiledFn fn = encode_tiled_fn();
     if (fn == nullptr)
         return cudaErrorNotSupported;

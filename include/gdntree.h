@@ -110,7 +110,7 @@ enum {
      * gates g = -softplus(x) = -log(1 + e^x) and beta = sigmoid(y), the
      * workloads' gate recipe, and the kernels apply both (as
      * a = exp(g) = 1 / (1 + e^x) and beta = 1 / (1 + e^-y), in f32, once per
-     * node).  x = +inf gives a = 0 (a reset).  Not with GDN_FLAG_CHUNKED. */
+     * node).  x = +inf gives a = 0 (a reset).  Also with GDN_FLAG_CHUNKED. */
     GDN_FLAG_GATES = 64
 };
 

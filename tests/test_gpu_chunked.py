@@ -66,6 +66,25 @@ def test_chunked_one_v_head_per_k_head():
     assert_states_close(res["node_states"][:, 0], ex[:, -1], "f32")
 
 
+@pytest.mark.parametrize("sd", ["f32", "f16"])
+def test_chunked_raw_gates(sd):
+    """GDN_FLAG_GATES: g and beta given as the pre-activations x, y; the
+    chunked form applies a = 1 / (1 + e^x), beta = sigmoid(y) per token, x =
+    +inf resets, and tokens past the end stay a = 1, beta = 0."""
+    prob = make_problem(batch=2, n_nodes=150, n_k_heads=2, n_v_heads=6, d_k=128, d_v=128, tree="chain",
+                        seed=21, qkv_dtype="bf16", raw_gates=True, accept="prefix")
+    prob.g[:, 77] = float("inf")  # a = 0: the state restarts at token 77
+    prob.accept_path = torch.arange(150, dtype=torch.int32).repeat(2, 1).contiguous()
+    prob.accept_len = torch.full((2,), 150, dtype=torch.int32)
+    res = run(prob, sd, flags=FLAGS | gdn.GDN_FLAG_CHUNKED | gdn.GDN_FLAG_GATES)
+    assert res["status"] == 0
+    out, _, ex = oracle.verify_problem(prob, state_dtype=sd, want_exact=True, nthreads=8, raw_gates=True)
+    assert_out_close(res["out"], out)
+    assert_states_close(res["node_states"][:, 0], ex[:, -1], sd)
+    ref = run(prob, sd, flags=FLAGS | gdn.GDN_FLAG_GATES)
+    assert (res["out"] - ref["out"]).abs().max() <= 1e-4
+
+
 def test_chunked_chain_reset_and_zero_beta():
     prob = _chain(150)
     prob.g[:, 70] = float("-inf")   # a = 0: the state restarts at token 70
