@@ -197,10 +197,9 @@ gdn_status verify_impl(const gdn_tree_desc* desc, const int32_t* cu, int32_t tot
     a.cu_nodes = varlen ? cu : nullptr;
     a.total_nodes = varlen ? total : 0;
     if (d.flags & GDN_FLAG_CHUNKED) {
-        if (varlen || workspace != nullptr || (d.flags & GDN_FLAG_QK_L2NORM) || !gdn::chunked_supported(a))
+        if (varlen || workspace != nullptr || !gdn::chunked_supported(a))
             return fail(GDN_ERR_UNSUPPORTED,
-                        "GDN_FLAG_CHUNKED needs CHAIN + PERSIST_LAST, bf16 q/k/v, d_k = 128, d_v %% 64 == 0, no "
-                        "QK_L2NORM%s");
+                        "GDN_FLAG_CHUNKED needs CHAIN + PERSIST_LAST, bf16 q/k/v, d_k = 128, d_v %% 64 == 0%s");
         const size_t B = d.batch, N = d.n_nodes, Hk = d.n_k_heads, Hv = d.n_v_heads, dk = d.d_k, dv = d.d_v;
         const Range ins[] = {{q, B * N * Hk * dk * 2, "q"}, {k, B * N * Hk * dk * 2, "k"},
                              {v, B * N * Hv * dv * 2, "v"}, {g, B * N * Hv * 4, "g"},

@@ -110,9 +110,16 @@ constexpr int kOffOut = kOffKT + kKTBytes;
 constexpr int kOffL = kOffOut + kOutBytes;         // L, f32 [T][LST]
 constexpr int kOffMf = kOffL + T * LST * 4;        // M, f32 [T][LST]
 constexpr int kOffAi = kOffMf + T * LST * 4;       // (I + L)^-1, f32 [T][AST]
-constexpr int kOffGB = kOffAi + T * AST * 4;       // [2][a = exp(g) | beta], f32
-constexpr int kOffDec = kOffGB + 2 * 2 * T * 4;    // [3][Gamma | r], f32
-constexpr int kOffBar = kOffDec + 3 * 2 * T * 4;   // mbarriers, tmem base, abort flag
+// Per-token scalars of a chunk: for the preparation warps a = exp(g), beta
+// and the inverse norms n_t = 1 / |k_t|, m_t = 1 / |q_t| (1 without
+// GDN_FLAG_QK_L2NORM); for the row threads the decays as they use them,
+// Gamma_t n_t (against X^T), r_t n_t (the update), Gamma_t m_t (against
+// Y^T), and Gamma_{T-1}.
+constexpr int kGB = 4 * T;                         // floats per buffer: a | beta | n | m
+constexpr int kDec = 3 * T + 4;                    // floats per slot: Gamma n | r n | Gamma m | Gamma_{T-1}
+constexpr int kOffGB = kOffAi + T * AST * 4;       // [2][kGB], f32
+constexpr int kOffDec = kOffGB + 2 * kGB * 4;      // [3][kDec], f32
+constexpr int kOffBar = kOffDec + 3 * kDec * 4;    // mbarriers, tmem base, abort flag
 constexpr int kSmem = kOffBar + 256;
 static_assert(kSmem <= 227 * 1024, "shared memory");
 
@@ -153,7 +160,8 @@ struct Params {
     int N, Hk, Hv, dv, G;
     float scale;
     int state_f16;
-    int gates;  // GDN_FLAG_GATES: g and beta hold the gates' pre-activations
+    int gates;    // GDN_FLAG_GATES: g and beta hold the gates' pre-activations
+    int qk_norm;  // GDN_FLAG_QK_L2NORM: q and k rows are normalised inside
 };
 
 // ---- tcgen05 ----------------------------------------------------------------
@@ -491,7 +499,51 @@ __device__ void invert_unit_lower(const float* L, float* Ai, int ptid)
     prep_sync();
 }
 
-__device__ void prep_role(unsigned char* smem, const Sync& sy, uint32_t tbase, int n_chunks)
+// This thread's row t of [K; Q] K^T (tensor memory at ta) times the row's
+// decays R[t][i] = a_{i+1} ... a_t, a running product over i from t down to
+// 0: row t of L = diag(beta) (K K^T o R) below the diagonal (K rows) or of
+// M = Q K^T o R on and below it (Q rows).  NORM: the products are of the
+// normalised rows, (x_t . k_i) / (|x_t| |k_i|), from the inverse norms in gb.
+template <bool NORM>
+__device__ __forceinline__ void lm_row(const float* gb, float* out, bool qrow, int t, uint32_t ta)
+{
+    const float bt = gb[T + t];
+    const float nt = NORM ? gb[(qrow ? 3 : 2) * T + t] : 1.f;  // this row's 1 / |q_t| or 1 / |k_t|
+    float* rowp = out + t * LST;
+    float run = 1.f;
+#pragma unroll 1
+    for (int hs = 1; hs >= 0; --hs) {
+        uint32_t d[32];
+        float a[32], nn[32];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float4 x = reinterpret_cast<const float4*>(gb + 32 * hs)[e];
+            a[4 * e] = x.x, a[4 * e + 1] = x.y, a[4 * e + 2] = x.z, a[4 * e + 3] = x.w;
+            if (NORM) {
+                const float4 y = reinterpret_cast<const float4*>(gb + 2 * T + 32 * hs)[e];
+                nn[4 * e] = y.x, nn[4 * e + 1] = y.y, nn[4 * e + 2] = y.z, nn[4 * e + 3] = y.w;
+            }
+        }
+        tmem_ld32(ta + 32 * hs, d);
+        float val[32];
+#pragma unroll
+        for (int e = 31; e >= 0; --e) {
+            const int i = 32 * hs + e;
+            const float kk = NORM ? __fmul_rn(__uint_as_float(d[e]), __fmul_rn(nt, nn[e])) : __uint_as_float(d[e]);
+            if (qrow)
+                val[e] = i <= t ? __fmul_rn(kk, run) : 0.f;
+            else
+                val[e] = i < t ? __fmul_rn(bt, __fmul_rn(kk, run)) : 0.f;
+            if (i <= t)
+                run = __fmul_rn(run, a[e]);
+        }
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+            rowp[32 * hs + e] = val[e];
+    }
+}
+
+__device__ void prep_role(unsigned char* smem, const Sync& sy, uint32_t tbase, int n_chunks, int p_qk_norm)
 {
     const int ptid = threadIdx.x - kPrep0;
     const int pw = ptid >> 5;                  // lane quarter of tensor memory
@@ -506,8 +558,7 @@ __device__ void prep_role(unsigned char* smem, const Sync& sy, uint32_t tbase, i
 
     for (int c = 0; c < n_chunks; ++c) {
         const int buf = c & 1;
-        const float* gb = reinterpret_cast<const float*>(smem + kOffGB) + buf * 2 * T;
-        const float* av = gb;  // a = exp(g)
+        const float* gb = reinterpret_cast<const float*>(smem + kOffGB) + buf * kGB;
         // 1. this chunk's a and beta (written by the load warp), then this
         //    thread's row of [K; Q] K^T times the row's decays
         //    R[t][i] = a_{i+1} ... a_t, a running product over i from t down
@@ -515,38 +566,10 @@ __device__ void prep_role(unsigned char* smem, const Sync& sy, uint32_t tbase, i
         if (!prep_all(sy.wait(kGb0 + buf, (c >> 1) & 1) && sy.wait(kKqMma, c & 1)))
             return;
         tmem_fence_after_sync();
-        {
-            const float bt = gb[T + t];
-            float* rowp = (qrow ? Mf : L) + t * LST;
-            const uint32_t ta = tbase + ((uint32_t)(32 * pw) << 16) + kColKQ;
-            float run = 1.f;
-#pragma unroll 1
-            for (int hs = 1; hs >= 0; --hs) {
-                uint32_t d[32];
-                float a[32];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float4 x = reinterpret_cast<const float4*>(av + 32 * hs)[e];
-                    a[4 * e] = x.x, a[4 * e + 1] = x.y, a[4 * e + 2] = x.z, a[4 * e + 3] = x.w;
-                }
-                tmem_ld32(ta + 32 * hs, d);
-                float val[32];
-#pragma unroll
-                for (int e = 31; e >= 0; --e) {
-                    const int i = 32 * hs + e;
-                    const float kk = __uint_as_float(d[e]);
-                    if (qrow)
-                        val[e] = i <= t ? __fmul_rn(kk, run) : 0.f;
-                    else
-                        val[e] = i < t ? __fmul_rn(bt, __fmul_rn(kk, run)) : 0.f;
-                    if (i <= t)
-                        run = __fmul_rn(run, a[e]);
-                }
-#pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    rowp[32 * hs + e] = val[e];
-            }
-        }
+        if (p_qk_norm)
+            lm_row<true>(gb, qrow ? Mf : L, qrow, t, tbase + ((uint32_t)(32 * pw) << 16) + kColKQ);
+        else
+            lm_row<false>(gb, qrow ? Mf : L, qrow, t, tbase + ((uint32_t)(32 * pw) << 16) + kColKQ);
         tmem_fence_before_sync();
         sy.arrive(kDkqFree);
         prep_sync();
@@ -632,12 +655,15 @@ __device__ void prep_role(unsigned char* smem, const Sync& sy, uint32_t tbase, i
 
 // ---- loads and decays ----------------------------------------------------------------------
 
-// Chunk c's a = exp(g) and beta into buffer buf, and its decays Gamma_t =
-// a_0 ... a_t and r_t = a_{t+1} ... a_{T-1} into slot c % 3: lane l holds
-// tokens 2 l and 2 l + 1; products across lanes by shuffle scans.  With raw
-// gates, g = x and beta = y stand for g = -softplus(x) and beta = sigmoid(y):
-// a = 1 / (1 + e^x), beta = 1 / (1 + e^-y) (the walk kernels' expressions,
-// so x = +inf resets).  Tokens past the end have a = 1, beta = 0.  One warp.
+// Chunk c's per-token scalars (kGB floats into buffer buf, kDec into slot
+// c % 3): a = exp(g) and beta; with raw gates, g = x and beta = y stand for
+// g = -softplus(x) and beta = sigmoid(y), so a = 1 / (1 + e^x) and
+// beta = 1 / (1 + e^-y) (the walk kernels' expressions; x = +inf resets);
+// tokens past the end have a = 1, beta = 0.  The decays Gamma_t = a_0 ...
+// a_t and r_t = a_{t+1} ... a_{T-1} by shuffle scans (lane l holds tokens
+// 2 l and 2 l + 1).  With qk_norm the inverse norms of the chunk's k and q
+// rows, read from its [K; Q] buffer (which must have landed), else 1 (and 1
+// for tokens past the end).  One warp.
 __device__ __forceinline__ void decays(const Params& p, unsigned char* smem, int buf, int c, int b, int h, int lane)
 {
     float a[2], bt[2];
@@ -658,6 +684,33 @@ __device__ __forceinline__ void decays(const Params& p, unsigned char* smem, int
             }
         }
     }
+    // inverse norms of K rows (n) and Q rows (m) 2 lane and 2 lane + 1
+    float nk[2] = {1.f, 1.f}, nq[2] = {1.f, 1.f};
+    if (p.qk_norm) {
+        const unsigned char* kq = smem + kOffKQ + buf * kKQBytes;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int n = (e >> 1) * T + 2 * lane + (e & 1);  // row of [K; Q]
+            float ss = 0.f;
+#pragma unroll 4
+            for (int pc = 0; pc < DK / 8; ++pc) {
+                const uint4 u = *reinterpret_cast<const uint4*>(kq + pc * (2 * T * 16) + (n >> 3) * 128 + (n & 7) * 16);
+                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int f = 0; f < 4; ++f) {
+                    const float2 x = bf16x2_to_float2(w[f]);
+                    ss = __fmaf_rn(x.x, x.x, ss);
+                    ss = __fmaf_rn(x.y, x.y, ss);
+                }
+            }
+            // tokens past the end are zero rows: they keep 1 (no 0 * inf)
+            const float inv = c * T + 2 * lane + (e & 1) < p.N ? __fdiv_rn(1.f, __fsqrt_rn(ss)) : 1.f;
+            if (e < 2)
+                nk[e] = inv;
+            else
+                nq[e - 2] = inv;
+        }
+    }
     // inclusive prefix and suffix products of the lanes' pair products
     const float pr = __fmul_rn(a[0], a[1]);
     float pre = pr, suf = pr;
@@ -676,13 +729,19 @@ __device__ __forceinline__ void decays(const Params& p, unsigned char* smem, int
         before = 1.f;
     if (lane == 31)
         after = 1.f;
-    float* gb = reinterpret_cast<float*>(smem + kOffGB) + buf * 2 * T;
-    float* Gam = reinterpret_cast<float*>(smem + kOffDec) + (c % 3) * 2 * T;
+    const float g0 = __fmul_rn(before, a[0]), g1 = __fmul_rn(g0, a[1]);  // Gamma
+    const float r0 = __fmul_rn(a[1], after), r1 = after;                  // r
+    float* gb = reinterpret_cast<float*>(smem + kOffGB) + buf * kGB;
+    float* dec = reinterpret_cast<float*>(smem + kOffDec) + (c % 3) * kDec;
     *reinterpret_cast<float2*>(gb + 2 * lane) = make_float2(a[0], a[1]);
     *reinterpret_cast<float2*>(gb + T + 2 * lane) = make_float2(bt[0], bt[1]);
-    const float g0 = __fmul_rn(before, a[0]);
-    *reinterpret_cast<float2*>(Gam + 2 * lane) = make_float2(g0, __fmul_rn(g0, a[1]));
-    *reinterpret_cast<float2*>(Gam + T + 2 * lane) = make_float2(__fmul_rn(a[1], after), after);
+    *reinterpret_cast<float2*>(gb + 2 * T + 2 * lane) = make_float2(nk[0], nk[1]);
+    *reinterpret_cast<float2*>(gb + 3 * T + 2 * lane) = make_float2(nq[0], nq[1]);
+    *reinterpret_cast<float2*>(dec + 2 * lane) = make_float2(__fmul_rn(g0, nk[0]), __fmul_rn(g1, nk[1]));
+    *reinterpret_cast<float2*>(dec + T + 2 * lane) = make_float2(__fmul_rn(r0, nk[0]), __fmul_rn(r1, nk[1]));
+    *reinterpret_cast<float2*>(dec + 2 * T + 2 * lane) = make_float2(__fmul_rn(g0, nq[0]), __fmul_rn(g1, nq[1]));
+    if (lane == 31)
+        dec[3 * T] = g1;  // Gamma_{T-1}
 }
 
 // One warp: chunks 0 and 1, then chunk c + 2 into buffer c % 2 once chunk c's
@@ -697,6 +756,8 @@ __device__ void load_role(const Params& p, const Maps& mp, unsigned char* smem, 
             load_kq(mp, smem, sy.bar + kKqFull0 + c, c, c, b, hk);
             ++kq_loads[c];
         }
+        if (p.qk_norm && !__all_sync(0xffffffffu, sy.wait(kKqFull0 + c, 0)))
+            return;
         decays(p, smem, c, c, b, h, lane);
         __syncwarp();
         if (lane == 0) {
@@ -711,6 +772,8 @@ __device__ void load_role(const Params& p, const Maps& mp, unsigned char* smem, 
             load_kq(mp, smem, sy.bar + kKqFull0 + (c & 1), c & 1, c + 2, b, hk);
             ++kq_loads[c & 1];
         }
+        if (p.qk_norm && !__all_sync(0xffffffffu, sy.wait(kKqFull0 + (c & 1), ((c + 2) >> 1) & 1)))
+            return;
         decays(p, smem, c & 1, c + 2, b, h, lane);
         __syncwarp();
         if (lane == 0) {
@@ -814,7 +877,8 @@ __device__ void mma_role(unsigned char* smem, const Sync& sy, uint32_t tbase, in
 
 // ---- row warps ----------------------------------------------------------------------------------
 
-// The previous chunk's outputs, scale (Gamma_t Y^T + U^T M^T): each thread
+// The previous chunk's outputs, scale (Gamma_t Y^T + U^T M^T) (Gam holds
+// Gamma_t / |q_t| with q/k normalisation, Gamma_t without): each thread
 // writes its row of the [t][row] tile in shared memory, then one thread
 // stores the tile with TMA (after the previous store has read it).
 __device__ __forceinline__ void write_outputs(const Params& p, const Maps& mp, unsigned char* smem, uint32_t trow,
@@ -863,18 +927,18 @@ __device__ void row_role(const Params& p, const Maps& mp, unsigned char* smem, c
 
     for (int c = 0; c < n_chunks; ++c) {
         const int slot = c % 3;
-        const float* Gam = decs + slot * 2 * T;
-        const float* rv = Gam + T;
+        const float* Gam = decs + slot * kDec;  // Gamma_t / |k_t|
+        const float* rv = Gam + T;              // r_t / |k_t|
         if (!row_all(sy.wait(kDec0 + slot, (c / 3) & 1)))
             return;
-        const float gT = Gam[T - 1];
+        const float gT = Gam[3 * T];            // Gamma_{T-1}
         // 0. the previous chunk's outputs; S into 3 bf16 parts (A of X^T | Y^T),
         //    and Gamma_{T-1} S back as the update's accumulator
         if (c > 0) {
             if (!row_all(sy.wait(kCdDone, (c - 1) & 1)))
                 return;
             tmem_fence_after_sync();
-            write_outputs(p, mp, smem, trow, decs + ((c - 1) % 3) * 2 * T, b, h, row0, (c - 1) * T);
+            write_outputs(p, mp, smem, trow, decs + ((c - 1) % 3) * kDec + 2 * T, b, h, row0, (c - 1) * T);
         }
 #pragma unroll 1
         for (int s = 2 * half; s < 2 * half + 2; ++s) {
@@ -996,7 +1060,7 @@ __device__ void row_role(const Params& p, const Maps& mp, unsigned char* smem, c
     if (!row_all(sy.wait(kCdDone, (n_chunks - 1) & 1)))
         return;
     tmem_fence_after_sync();
-    write_outputs(p, mp, smem, trow, decs + ((n_chunks - 1) % 3) * 2 * T, b, h, row0, (n_chunks - 1) * T);
+    write_outputs(p, mp, smem, trow, decs + ((n_chunks - 1) % 3) * kDec + 2 * T, b, h, row0, (n_chunks - 1) * T);
     const size_t base = (((size_t)b * p.Hv + h) * p.dv + row) * DK;
 #pragma unroll 1
     for (int s = 2 * half; s < 2 * half + 2; ++s) {
@@ -1084,7 +1148,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_chain_chunked(const Params p,
             asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
         }
     } else if (warp < 12) {
-        prep_role(smem, sy, tbase, n_chunks);
+        prep_role(smem, sy, tbase, n_chunks, p.qk_norm);
     } else if (warp == 13) {
         int kq_loads[2] = {0, 0};
         load_role(p, mp, smem, sy, b, h, hk, n_chunks, kq_loads);
@@ -1177,6 +1241,7 @@ cudaError_t launch_chunked(const VerifyArgs& a, cudaStream_t stream)
     p.scale = a.scale;
     p.state_f16 = a.state_dtype == GDN_F16 ? 1 : 0;
     p.gates = (a.flags & GDN_FLAG_GATES) ? 1 : 0;
+    p.qk_norm = (a.flags & GDN_FLAG_QK_L2NORM) ? 1 : 0;
     const EncodeTiledFn fn = encode_tiled_fn();
     if (fn == nullptr)
         return cudaErrorNotSupported;

@@ -104,7 +104,7 @@ enum {
     /* q and k are given raw; the kernel L2-normalises each (node, k-head)
      * row, x / |x| with no epsilon (a zero row gives inf/NaN), as the
      * workloads' input preparation does.  Folded into per-node scalars, so
-     * the node loop does the same work.  Not with GDN_FLAG_CHUNKED. */
+     * the node loop does the same work.  Also with GDN_FLAG_CHUNKED. */
     GDN_FLAG_QK_L2NORM = 32,
     /* g and beta are given raw: they hold the pre-activations x and y of the
      * gates g = -softplus(x) = -log(1 + e^x) and beta = sigmoid(y), the

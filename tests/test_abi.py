@@ -81,8 +81,7 @@ def test_verify_batch_zero_is_a_noop(lib):
     (dict(qkv_dtype=gdn.GDN_F16), gdn.GDN_ERR_UNSUPPORTED),
     (dict(state_dtype=gdn.GDN_BF16), gdn.GDN_ERR_UNSUPPORTED),
     (dict(flags=128), gdn.GDN_ERR_INVALID_ARG),     # no such flag
-    (dict(flags=16 | 1 | 2 | 32), gdn.GDN_ERR_UNSUPPORTED),  # chunked + fused normalisation
-    (dict(flags=16 | 1 | 2 | 64 | 32), gdn.GDN_ERR_UNSUPPORTED),  # chunked + gates + normalisation
+    (dict(flags=16 | 2 | 32 | 64), gdn.GDN_ERR_UNSUPPORTED),  # chunked with the fused steps, no CHAIN
     (dict(flags=16), gdn.GDN_ERR_UNSUPPORTED),      # chunked needs CHAIN + PERSIST_LAST
     (dict(flags=16 | 1 | 2, d_v=32), gdn.GDN_ERR_UNSUPPORTED),
     (dict(scale=float("nan")), gdn.GDN_ERR_INVALID_ARG),

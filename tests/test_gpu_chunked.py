@@ -85,6 +85,29 @@ def test_chunked_raw_gates(sd):
     assert (res["out"] - ref["out"]).abs().max() <= 1e-4
 
 
+@pytest.mark.parametrize("sd", ["f32", "f16"])
+def test_chunked_fused_normalisation_and_gates(sd):
+    """GDN_FLAG_QK_L2NORM (+ GATES): q and k given raw, each token's rows
+    normalised inside, folded into per-token scalars (1 / |k_t| into the
+    decays and K K^T, 1 / |q_t| into Q K^T and the outputs)."""
+    prob = make_problem(batch=2, n_nodes=150, n_k_heads=2, n_v_heads=6, d_k=128, d_v=128, tree="chain",
+                        seed=23, qkv_dtype="bf16", raw_gates=True, accept="prefix")
+    gen = torch.Generator().manual_seed(24)
+    prob.q = (prob.q.float() * (0.5 + 3 * torch.rand(prob.q.shape[:3] + (1,), generator=gen))).to(torch.bfloat16)
+    prob.k = (prob.k.float() * (0.5 + 3 * torch.rand(prob.k.shape[:3] + (1,), generator=gen))).to(torch.bfloat16)
+    prob.accept_path = torch.arange(150, dtype=torch.int32).repeat(2, 1).contiguous()
+    prob.accept_len = torch.full((2,), 150, dtype=torch.int32)
+    flags = FLAGS | gdn.GDN_FLAG_QK_L2NORM | gdn.GDN_FLAG_GATES
+    res = run(prob, sd, flags=flags | gdn.GDN_FLAG_CHUNKED)
+    assert res["status"] == 0
+    out, _, ex = oracle.verify_problem(prob, state_dtype=sd, want_exact=True, nthreads=8, qk_l2norm=True,
+                                       raw_gates=True)
+    assert_out_close(res["out"], out)
+    assert_states_close(res["node_states"][:, 0], ex[:, -1], sd)
+    ref = run(prob, sd, flags=flags)
+    assert (res["out"] - ref["out"]).abs().max() <= 1e-4
+
+
 def test_chunked_chain_reset_and_zero_beta():
     prob = _chain(150)
     prob.g[:, 70] = float("-inf")   # a = 0: the state restarts at token 70
