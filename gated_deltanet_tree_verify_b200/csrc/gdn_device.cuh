@@ -154,6 +154,12 @@ __device__ __forceinline__ void pdl_wait_then_release()
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// A hint that the 128-byte line holding p should be brought into L2.
+__device__ __forceinline__ void prefetch_l2(const void* p)
+{
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // ---- 256-bit global accesses ---------------------------------------------------
 
 // 8 floats at a 32-byte-aligned global address in one access.  The load is a

@@ -127,6 +127,7 @@ struct KParams {
     float scale;
     int rows, warps, slots;
     int persist_last, validate, early_tree;
+    int prefetch;        // early_tree on a small layer: L2 prefetch of the records before the wait
     int qk_norm;         // GDN_FLAG_QK_L2NORM: k and q normalised per node inside the kernel
     int gates;           // GDN_FLAG_GATES: g and beta are raw (gate_scalars)
     float* ws;           // global stack slots (kTreeGlobal kinds): slots x rows x d_k per CTA
@@ -1492,6 +1493,30 @@ __device__ __forceinline__ void staged_body(const KParams& p, uint32_t tbase)
     const int32_t* prow = p.parent + sq.n0;
     const int per_node = p.raw_bytes / 16;  // 16-byte chunks per node
     constexpr int LR = LaneMap<DK, C, RL>::LR;
+    if (p.prefetch) {
+        // Ahead of the wait, bring this CTA's records into L2 so that the
+        // copies after it start from there (small layers, where the first
+        // records' latency is exposed; on large ones the prefetched lines
+        // would compete for L2 with the running layer's states).  Only a
+        // hint: global writes land in L2, so a line the preceding kernel
+        // rewrites is read new after the wait.
+        const char* kg = static_cast<const char*>(p.k);
+        const char* qg = static_cast<const char*>(p.q);
+        const char* vg = static_cast<const char*>(p.v);
+        constexpr int kRowBytes = DK * (int)sizeof(QT);
+        for (int n = tid; n < N; n += blockDim.x) {
+            const size_t node = (size_t)sq.n0 + n;
+            const size_t kq = (node * p.Hk + hk) * kRowBytes;
+#pragma unroll
+            for (int off = 0; off < kRowBytes; off += 128) {
+                prefetch_l2(kg + kq + off);
+                prefetch_l2(qg + kq + off);
+            }
+            prefetch_l2(vg + ((node * p.Hv + h) * p.dv + row0) * sizeof(QT));
+            prefetch_l2(p.g + node * p.Hv + h);
+            prefetch_l2(p.beta + node * p.Hv + h);
+        }
+    }
     auto stage = [&]() {
         const QT* kg = static_cast<const QT*>(p.k);
         const QT* qg = static_cast<const QT*>(p.q);
