@@ -132,7 +132,7 @@ def bf16_tensor_peak():
 # same products at one part each (the chunked form's own arithmetic).
 CHUNK_T, CHUNK_ROWS = 64, 128
 CHUNK_FLOPS_ISSUED = 2 * CHUNK_ROWS * (
-    3 * 2 * CHUNK_T * 128      # X^T | Y^T = S [K; Q]^T, S in 3 parts
+    2 * 2 * CHUNK_T * 128      # X^T | Y^T = S [K; Q]^T, S in 2 parts
     + 2 * CHUNK_T * 128 // 2   # [K; Q] K^T (M = 2T rows of K and Q, N = T)
     + 6 * CHUNK_T * CHUNK_T    # U^T = P^T Ab^T, 6 part products
     + 3 * 128 * CHUNK_T        # S += (U^T diag(r)) K, 3 parts

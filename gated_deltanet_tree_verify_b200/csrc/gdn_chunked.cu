@@ -29,12 +29,14 @@
 //
 // Every product is a tcgen05.mma (kind::f16, bf16 operands, f32 accumulation
 // in tensor memory), issued by one thread.  Operands that are not exact in
-// bf16 (the state, U, Ab, M) are split into bf16 parts, x = x1 + x2 + x3
-// (x2 = bf16(x - x1), x3 = bf16(x - x1 - x2): 24 bits), and each product is
-// formed from the part products down to ~2^-24 relative (S and U parts
-// against the exact bf16 K and Q; 6 of the 9 part products for U^T Ab^T;
-// 3 of 4 two-part products for the output-only U^T M^T), which keeps the
-// chunked form at f32 accuracy.  Layout: the A operands (the state, P^T,
+// bf16 (the state, U, Ab, M) are split into bf16 parts, x = x1 + x2 (+ x3)
+// (x2 = bf16(x - x1), x3 = bf16(x - x1 - x2): 16 or 24 bits).  The update
+// adds U^T diag(r) in 3 parts against the exact bf16 K, and U^T Ab^T takes 6
+// of the 9 part products (down to ~2^-16 relative); the state enters
+// X^T | Y^T in 2 parts against the exact K and Q (its rounding there reaches
+// the state only through U), and the output-only U^T M^T takes 3 of 4
+// two-part products.  Over long chains the chunked form stays within a few
+// times the f32 token walk's own rounding error.  Layout: the A operands (the state, P^T,
 // U^T) live in tensor memory, written by the thread that owns the row
 // (bf16 pairs per 32-bit column, the even element in the low half); the B
 // operands (K, Q, K^T, Ab, M) in shared memory in the canonical K-major
@@ -81,7 +83,7 @@ constexpr int kPrep0 = 256;     // first preparation thread
 // Tensor-memory columns (128 lanes x 512 columns of 32 bits, all of it).
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;     // state S, f32 [d_v x d_k]
-constexpr uint32_t kColAS = 128;  // S in 3 bf16 parts, 64 columns each (A of X^T | Y^T)
+constexpr uint32_t kColAS = 128;  // S in 2 bf16 parts, 64 columns each (A of X^T | Y^T)
 constexpr uint32_t kColAP = 128;  //   after that product: P^T in 3 parts of 32 columns
 constexpr uint32_t kColU = 224;   //   and U^T, f32 [d_v x T]
 constexpr uint32_t kColAUr = 128; //   after that: U^T diag(r) in 3 parts (A of the update)
@@ -130,21 +132,23 @@ enum Bar {
     kKqMma = 2,    // [K; Q] K^T done (MMA commit)
     kDkqFree = 3,  // [K; Q] K^T read out (128)
     kDec0 = 4,     // decays of a chunk written, slots 0..2 (1)
-    kAsReady = 7,  // state parts written, previous outputs read (256 row threads)
+    kAsReady = 7,  // state parts of d_k 0-31 and 64-95 written, previous outputs read (256 row threads)
     kXyDone = 8,   // X^T | Y^T done (commit)
     kApReady = 9,  // P^T parts written (256)
     kAbReady = 10, // Ab parts written (128)
     kUDone = 11,   // U^T done (commit)
     kAuReady = 12, // U^T parts written (256)
     kMktReady = 13,// M parts and K^T written (128)
-    kCdDone = 14,  // update and U^T M^T done (commit)
+    kCdDone = 14,  // update done, and U^T M^T before it (commit)
     kFin = 15,     // all MMAs retired (commit)
     kVFull = 16,   // v of a chunk landed (TMA bytes)
     kKqBuf0 = 17,  // k/q buffer 0 / 1 no longer read: the chunk's MMAs (commit) and K^T (128)
     kKqBuf1 = 18,
     kGb0 = 19,     // a and beta of a chunk written, buffer 0 / 1 (1)
     kGb1 = 20,
-    kNumBars = 21
+    kOutDone = 21, // U^T M^T done (commit): the chunk's outputs can be formed
+    kAsReady2 = 22,// state parts of d_k 32-63 and 96-127 written (256)
+    kNumBars = 23
 };
 
 struct Params {
@@ -810,15 +814,19 @@ __device__ void mma_role(unsigned char* smem, const Sync& sy, uint32_t tbase, in
     kq_product(0);
     for (int c = 0; c < n_chunks; ++c) {
         const uint32_t kq = kq0 + (c & 1) * kKQBytes;
-        // X^T | Y^T = S [K; Q]^T, S in 3 parts
-        if (!sy.wait(kAsReady, c & 1))
-            return;
-        tmem_fence_after_sync();
+        // X^T | Y^T = S [K; Q]^T, S in 2 parts, in two stages of d_k as the
+        // row threads write the parts: k-steps 0, 1, 4, 5, then 2, 3, 6, 7
 #pragma unroll
-        for (int q = 0; q < 3 * (DK / 16); ++q) {
-            const int part = q >> 3, ks = q & 7;
-            mma_ts(tbase + kColX, tbase + kColAS + 64 * part + 8 * ks, kdesc(kq + ks * 2 * kKQLbo, kKQLbo),
-                   idesc_bf16(2 * T), q != 0 ? 1u : 0u);
+        for (int stage = 0; stage < 2; ++stage) {
+            if (!sy.wait(stage == 0 ? kAsReady : kAsReady2, c & 1))
+                return;
+            tmem_fence_after_sync();
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int part = q >> 2, ks = (q & 1) + ((q & 2) << 1) + 2 * stage;
+                mma_ts(tbase + kColX, tbase + kColAS + 64 * part + 8 * ks, kdesc(kq + ks * 2 * kKQLbo, kKQLbo),
+                       idesc_bf16(2 * T), stage + q != 0 ? 1u : 0u);
+            }
         }
         mma_commit(sy.bar + kXyDone);
         mma_commit(sy.bar + kKqBuf0 + (c & 1));  // with [K; Q] K^T of c, issued before
@@ -827,18 +835,21 @@ __device__ void mma_role(unsigned char* smem, const Sync& sy, uint32_t tbase, in
         // (P, Ab) of weight at least 2^-16
         bool kq_done = c + 1 >= n_chunks, u_done = false;
         const long long t0 = clock64();
-        while (!(kq_done && u_done)) {
-            __nanosleep(32);  // leave the issue slots to the warps being waited for
-            if (*sy.abort || clock64() - t0 > (1ll << 31)) {
-                *sy.abort = 1;
-                report_status(sy.status, kStatusTimeout);
-                return;
+        for (bool issued = true; !(kq_done && u_done); ) {
+            if (!issued) {
+                __nanosleep(32);  // leave the issue slots to the warps being waited for
+                if (*sy.abort || clock64() - t0 > (1ll << 31)) {
+                    *sy.abort = 1;
+                    report_status(sy.status, kStatusTimeout);
+                    return;
+                }
             }
+            issued = false;
             if (!kq_done && mbar_test(sy.bar + kKqFull0 + ((c + 1) & 1), ((c + 1) >> 1) & 1) &&
                 mbar_test(sy.bar + kDkqFree, c & 1)) {
                 tmem_fence_after_sync();
                 kq_product(c + 1);
-                kq_done = true;
+                kq_done = issued = true;
             }
             if (!u_done && mbar_test(sy.bar + kApReady, c & 1) && mbar_test(sy.bar + kAbReady, c & 1)) {
                 tmem_fence_after_sync();
@@ -851,25 +862,27 @@ __device__ void mma_role(unsigned char* smem, const Sync& sy, uint32_t tbase, in
                            kdesc(ab + pa * kTTBytes + ks * 2 * kTTLbo, kTTLbo), idesc_bf16(T), q != 0 ? 1u : 0u);
                 }
                 mma_commit(sy.bar + kUDone);
-                u_done = true;
+                u_done = issued = true;
             }
         }
-        // S += (U^T diag(r)) K and U^T M^T
+        // U^T M^T, then S += (U^T diag(r)) K: the row threads form this
+        // chunk's outputs while the update runs
         if (!sy.wait(kAuReady, c & 1) || !sy.wait(kMktReady, c & 1))
             return;
         tmem_fence_after_sync();
-#pragma unroll
-        for (int q = 0; q < 3 * (T / 16); ++q) {
-            const int part = q >> 2, ks = q & 3;
-            mma_ts(tbase + kColS, tbase + kColAUr + 32 * part + 8 * ks, kdesc(kt + ks * 2 * kKTLbo, kKTLbo),
-                   idesc_bf16(DK), 1u);
-        }
 #pragma unroll
         for (int q = 0; q < 3 * (T / 16); ++q) {
             const int pr = q >> 2, ks = q & 3;  // (U, M) parts: (0,0) (0,1) (1,0)
             const uint32_t au = pr == 2 ? kColAU1 : kColAU0;
             mma_ts(tbase + kColX, tbase + au + 8 * ks, kdesc(mm + (pr == 1 ? kTTBytes : 0) + ks * 2 * kTTLbo, kTTLbo),
                    idesc_bf16(T), q != 0 ? 1u : 0u);
+        }
+        mma_commit(sy.bar + kOutDone);
+#pragma unroll
+        for (int q = 0; q < 3 * (T / 16); ++q) {
+            const int part = q >> 2, ks = q & 3;
+            mma_ts(tbase + kColS, tbase + kColAUr + 32 * part + 8 * ks, kdesc(kt + ks * 2 * kKTLbo, kKTLbo),
+                   idesc_bf16(DK), 1u);
         }
         mma_commit(sy.bar + kCdDone);
     }
@@ -932,13 +945,16 @@ __device__ void row_role(const Params& p, const Maps& mp, unsigned char* smem, c
         if (!row_all(sy.wait(kDec0 + slot, (c / 3) & 1)))
             return;
         const float gT = Gam[3 * T];            // Gamma_{T-1}
-        // 0. the previous chunk's outputs; S into 3 bf16 parts (A of X^T | Y^T),
+        // 0. the previous chunk's outputs; S into 2 bf16 parts (A of X^T | Y^T),
         //    and Gamma_{T-1} S back as the update's accumulator
         if (c > 0) {
-            if (!row_all(sy.wait(kCdDone, (c - 1) & 1)))
+            if (!row_all(sy.wait(kOutDone, (c - 1) & 1)))
                 return;
             tmem_fence_after_sync();
             write_outputs(p, mp, smem, trow, decs + ((c - 1) % 3) * kDec + 2 * T, b, h, row0, (c - 1) * T);
+            if (!row_all(sy.wait(kCdDone, (c - 1) & 1)))
+                return;
+            tmem_fence_after_sync();
         }
 #pragma unroll 1
         for (int s = 2 * half; s < 2 * half + 2; ++s) {
@@ -963,21 +979,20 @@ __device__ void row_role(const Params& p, const Maps& mp, unsigned char* smem, c
             } else {
                 tmem_ld32(trow + kColS + 32 * s, x);
             }
-            uint32_t p1[16], p2[16], p3[16];
+            uint32_t p1[16], p2[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e)
-                split3(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1]), p1[e], p2[e], p3[e]);
+                split2(__uint_as_float(x[2 * e]), __uint_as_float(x[2 * e + 1]), p1[e], p2[e]);
             tmem_st16(trow + kColAS + 16 * s, p1);
             tmem_st16(trow + kColAS + 64 + 16 * s, p2);
-            tmem_st16(trow + kColAS + 128 + 16 * s, p3);
 #pragma unroll
             for (int e = 0; e < 32; ++e)
                 x[e] = __float_as_uint(__fmul_rn(gT, __uint_as_float(x[e])));
             tmem_st32(trow + kColS + 32 * s, x);
+            tmem_wait_st();
+            tmem_fence_before_sync();
+            sy.arrive(s == 2 * half ? kAsReady : kAsReady2);
         }
-        tmem_wait_st();
-        tmem_fence_before_sync();
-        sy.arrive(kAsReady);
 
         // 1. P^T = V^T - X^T diag(Gamma) into 3 bf16 parts (A of U^T)
         if (!row_all(sy.wait(kXyDone, c & 1) && sy.wait(kVFull, c & 1)))
@@ -1116,7 +1131,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_chain_chunked(const Params p,
     // allocates all 512 columns
     pdl_wait_then_release();
     if (threadIdx.x == 0) {
-        const uint32_t counts[kNumBars] = {1, 1, 1, 128, 1, 1, 1, kRows, 1, kRows, 128, 1, kRows, 128, 1, 1, 1, 129, 129, 1, 1};
+        const uint32_t counts[kNumBars] = {1, 1, 1, 128, 1, 1, 1, kRows, 1, kRows, 128, 1, kRows, 128, 1, 1, 1, 129, 129, 1, 1, 1, kRows};
         for (int i = 0; i < kNumBars; ++i)
             mbar_init(bars + i, counts[i]);
         *abort_flag = 0;
