@@ -95,9 +95,9 @@ enum {
     /* Chains only (with GDN_FLAG_CHAIN and GDN_FLAG_PERSIST_LAST, bf16 q/k/v,
      * d_k = 128, d_v a multiple of 64, no varlen or workspace): run the chain
      * in chunks of 64 tokens with tensor-core products (the chunked "WY" form
-     * of the delta rule), for long prefill-style chains.  Same results up to
-     * f32 rounding (products of bf16 parts accumulated in f32), not
-     * bit-identical to the token-by-token path.  q, k, v and out are read and
+     * of the delta rule), for long prefill-style chains.  Results agree with
+     * the token-by-token path to within a few times its f32 rounding error
+     * (products of bf16 parts accumulated in f32), not bit-identically.  q, k, v and out are read and
      * written through TMA tensor maps (the 16-byte alignment required above
      * suffices).  Unsupported shapes: GDN_ERR_UNSUPPORTED. */
     GDN_FLAG_CHUNKED = 16,
