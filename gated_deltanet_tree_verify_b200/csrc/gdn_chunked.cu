@@ -469,8 +469,9 @@ __device__ __forceinline__ void block_column(const float* L, float* Ai, int J, i
 // (I + L)^-1 for the unit lower triangular I + L (L strictly lower, f32
 // [T][LST]) into Ai (f32 [T][AST], whose entries above the diagonal stay 0).
 // Warp w inverts diagonal block w (one column per lane); then the block
-// columns, each by its own warp (block column 0 split over warps 0 and 1),
-// with no barrier between warps until the end.
+// columns, in halves of 8 columns: warps 0 and 1 take block column 0 (three
+// block rows), warps 2 and 3 block columns 1 and 2 (two and one), with no
+// barrier between warps until the end.
 __device__ void invert_unit_lower(const float* L, float* Ai, int ptid)
 {
     const int pw = ptid >> 5, lane = ptid & 31;
@@ -496,10 +497,12 @@ __device__ void invert_unit_lower(const float* L, float* Ai, int ptid)
             Ac[i * AST] = d[i];
     }
     prep_sync();
-    if (pw < 2)
+    if (pw < 2) {
         block_column<8>(L, Ai, 0, 8 * pw, lane);
-    else
-        block_column<16>(L, Ai, pw - 1, 16 * (pw - 1), lane);
+    } else {
+        block_column<8>(L, Ai, 1, 16 + 8 * (pw - 2), lane);
+        block_column<8>(L, Ai, 2, 32 + 8 * (pw - 2), lane);
+    }
     prep_sync();
 }
 
