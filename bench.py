@@ -21,6 +21,7 @@ Under torchrun (N > 1) every rank runs a replica; rank 0 prints the line.
 from __future__ import annotations
 
 import argparse
+import contextlib
 import datetime
 import hashlib
 import json
@@ -139,6 +140,21 @@ CHUNK_FLOPS_ISSUED = 2 * CHUNK_ROWS * (
     + 3 * CHUNK_T * CHUNK_T)   # U^T M^T, 3 part products
 CHUNK_FLOPS_ALGO = 2 * CHUNK_ROWS * (
     2 * CHUNK_T * 128 + 2 * CHUNK_T * 128 // 2 + CHUNK_T * CHUNK_T + 128 * CHUNK_T + CHUNK_T * CHUNK_T)
+
+
+def chunked_tensor_roofline(t: float, batch: int, n_tokens: int) -> dict:
+    """Tensor roofline of one GDN_FLAG_CHUNKED launch over ``batch`` chains of
+    ``n_tokens`` (48 v-heads, d = 128) that took ``t`` seconds: the issued
+    bf16 flops (bf16 parts included) against the measured dense bf16 peak
+    (the burst figure: the launch is timed on its own), and the chunked
+    form's own flops beside them."""
+    ctas = batch * N_V_HEADS * -(-D // CHUNK_ROWS)
+    chunks = -(-n_tokens // CHUNK_T)
+    issued = ctas * chunks * CHUNK_FLOPS_ISSUED
+    tpeak, tkind = bf16_tensor_peak()
+    return {"bound": "tensor", "achieved": issued / t / 1e12, "unit": "TFLOP/s", "peak": tpeak,
+            "frac": issued / t / 1e12 / tpeak, "peak_source": tkind + " bf16",
+            "algorithmic": ctas * chunks * CHUNK_FLOPS_ALGO / t / 1e12, "issued_gflop": issued / 1e9}
 
 
 def kernel_source_digest():
@@ -441,6 +457,16 @@ def run_ours(args, ws, rank, local):
         torch.cuda.nvtx.range_push("target points")
         result["target"] = run_target(args, device, stream, local)
         torch.cuda.nvtx.range_pop()
+    if not args.no_chunked:
+        # the chunked tensor-core chain on the long-chain workload; a failure
+        # here is reported in its key and does not cost the line
+        stage("chunked chain point")
+        torch.cuda.nvtx.range_push("chunked chain")
+        try:
+            result["chunked_chain"] = run_chunked_point(local)
+        except Exception as exc:  # noqa: BLE001
+            result["chunked_chain"] = {"error": f"{type(exc).__name__}: {exc}"}
+        torch.cuda.nvtx.range_pop()
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         stage("cpu baseline (oracle)")
         result["cpu_baseline"] = cpu_baseline(args, stack)
@@ -565,6 +591,29 @@ def _target_point(budget, batch, state_dtype, *, layers, device, stream, local, 
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
     return point
+
+
+CHUNKED_POINT = dict(batch=8, n_tokens=4096, reps=40)
+
+
+def run_chunked_point(local: int) -> dict:
+    """The long-chain workload (8 chains of 4096 tokens, 48 v-heads / 16
+    k-heads, d = 128, bf16 q/k/v, a = exp(g) in [0.5, 1], last-only f32
+    state) through GDN_FLAG_CHUNKED: the mean time of one launch over graph
+    replays on two distinct buffer sets (each larger than L2), with its
+    tensor roofline and its own clock record."""
+    import gated_deltanet_tree_verify_b200 as gdn
+    batch, n, reps = CHUNKED_POINT["batch"], CHUNKED_POINT["n_tokens"], CHUNKED_POINT["reps"]
+    flags = gdn.GDN_FLAG_CHAIN | gdn.GDN_FLAG_PERSIST_LAST | gdn.GDN_FLAG_CHUNKED
+    sampler = ClockSampler(local, period_s=0.01)
+    t, R = _verify_point(batch=batch, n_nodes=n, tree="chain", state_dtype="f32", flags=flags, gate="uniform_a",
+                         reps=reps, min_bytes=0, sampler=sampler)
+    return {"workload": f"long_chain{n}_b{batch}_persist_last_f32", "flags": "GDN_FLAG_CHUNKED",
+            "batch": batch, "tokens_per_chain": n, "ms_per_launch": t * 1e3, "tokens_per_s": batch * n / t,
+            "buffer_sets": R, "reps": reps, "roofline": chunked_tensor_roofline(t, batch, n),
+            "clocks": sampler.summary(),
+            "timing": "CUDA graph of one launch per buffer set, replayed back to back; CUDA events around "
+                      "the replays"}
 
 
 def run_target(args, device, stream, local):
@@ -819,12 +868,13 @@ FP32_LANES_PER_SM = 128  # FP32 CUDA-core lanes per SM (B200); 148 SMs
 
 
 def _verify_point(*, batch, n_nodes, tree, state_dtype, flags=0, gate="softplus", reps=20,
-                  min_bytes=512 << 20, seed=11, workspace=False, planned=False):
+                  min_bytes=512 << 20, seed=11, workspace=False, planned=False, sampler=None):
     """Mean time of one verify launch, over graph replays of R launches on R
     distinct buffer sets (R sized so the sets together exceed min_bytes).
     With ``workspace``, through gdn_tree_verify_ws (one workspace per set);
     with ``planned``, through gdn_tree_verify_planned with each set's plan
-    built beforehand (a step builds it once for all its layers)."""
+    built beforehand (a step builds it once for all its layers).  A
+    ``sampler`` (ClockSampler) runs around the timed replays only."""
     import gated_deltanet_tree_verify_b200 as gdn
     persist_last = bool(flags & gdn.GDN_FLAG_PERSIST_LAST)
     tdt = torch.float32 if state_dtype == "f32" else torch.float16
@@ -881,11 +931,12 @@ def _verify_point(*, batch, n_nodes, tree, state_dtype, flags=0, gate="softplus"
         graph.replay()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(reps):
-        graph.replay()
-    e1.record()
-    torch.cuda.synchronize()
+    with (sampler if sampler is not None else contextlib.nullcontext()):
+        e0.record()
+        for _ in range(reps):
+            graph.replay()
+        e1.record()
+        torch.cuda.synchronize()
     per_launch_s = e0.elapsed_time(e1) / 1e3 / (reps * R)
     del graph
     return per_launch_s, R
@@ -1115,15 +1166,8 @@ def _sweep_point(args, gdn, pt, peak, varlen_budgets, clocks):
         if pt.get("chunked"):
             # the tensor cores do the chain's work: issued bf16 flops against
             # the measured dense bf16 peak, and the algorithmic share beside it
-            ctas = pt["batch"] * N_V_HEADS * -(-D // CHUNK_ROWS)
-            chunks = -(-n // CHUNK_T)
-            issued = ctas * chunks * CHUNK_FLOPS_ISSUED
-            tpeak, tkind = bf16_tensor_peak()
             line["recurrence_tflops_equivalent"] = line.pop("roofline")["achieved"]
-            line["roofline"] = {"bound": "tensor", "achieved": issued / t / 1e12, "unit": "TFLOP/s",
-                                "peak": tpeak, "frac": issued / t / 1e12 / tpeak, "peak_source": tkind + " bf16",
-                                "algorithmic": ctas * chunks * CHUNK_FLOPS_ALGO / t / 1e12,
-                                "issued_gflop": issued / 1e9}
+            line["roofline"] = chunked_tensor_roofline(t, pt["batch"], n)
     else:
         tree = "ddtree" if pt["kind"] == "tree" else "chain"
         flags = 0 if pt["kind"] == "tree" else gdn.GDN_FLAG_CHAIN
@@ -1154,6 +1198,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-target", action="store_true",
                     help="skip the batched-tree target points (budget 22-128, batch 8 and 32, f32 and f16)")
+    ap.add_argument("--no-chunked", action="store_true",
+                    help="skip the chunked tensor-core chain point (8 chains x 4096 tokens)")
     ap.add_argument("--sweep", action="store_true",
                     help="single-layer verify timings over budgets, batches, dtypes and the long chain "
                          "(one JSON line per point; not the benchmark line)")
