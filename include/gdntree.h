@@ -24,7 +24,12 @@
  * Conventions shared by every entry point:
  *   - Every data pointer is a caller-owned DEVICE pointer (cudaMalloc'd, or a
  *     framework tensor's storage).  The library allocates nothing, keeps no
- *     state between calls and never synchronises the stream.
+ *     data between calls and never synchronises the stream.  It does remember,
+ *     per device for the life of the process, that it has raised a kernel's
+ *     dynamic shared-memory limit (once per kernel and device): after a
+ *     cudaDeviceReset in the same process, a launch that needs more than the
+ *     default 48 KB of shared memory returns GDN_ERR_CUDA instead of running
+ *     (nothing is written); a new process starts afresh.
  *   - Layouts are row-major with the last index contiguous.  B = batch
  *     (independent sequences), N = n_nodes, H_k / H_v = k-heads / v-heads with
  *     G = H_v / H_k; v-head h reads k-head h / G (contiguous groups).
